@@ -1,0 +1,145 @@
+"""fp64 CPU oracle for the KDA forward -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and the bench's CPU-baseline leg may
+import this package. The product (the CUDA library and its Python binding)
+never imports it, and it imports nothing from the product.
+
+Python side: ctypes marshalling around ``kda_oracle.cpp`` (the arithmetic lives
+there, in plain fp64 C++). ``build()`` compiles it with g++ into
+``liboracle.so`` next to the source.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kda_oracle.cpp")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle (portable x86-64/aarch64 code, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["g++", "-O2", "-std=c++17", "-fPIC", "-shared", "-pthread", "-fno-fast-math",
+               "-ffp-contract=off", "-o", tmp, _SRC]
+        subprocess.check_call(cmd)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            try:
+                lib = ctypes.CDLL(build())
+            except OSError:
+                lib = ctypes.CDLL(build(force=True))
+            P = ctypes.c_void_p
+            i32, i64, f64 = ctypes.c_int32, ctypes.c_int64, ctypes.c_double
+            scan_args = [P, P, P, P, P, i64, i32, i32, i32, P, i32, f64, P, P, P, i32, i32, i32, i32, i32]
+            lib.kda_oracle_scan_bf16.argtypes = scan_args
+            lib.kda_oracle_scan_bf16.restype = ctypes.c_int
+            lib.kda_oracle_scan_f64.argtypes = scan_args
+            lib.kda_oracle_scan_f64.restype = ctypes.c_int
+            lib.kda_oracle_chunked_f64.argtypes = [P, P, P, P, P, i64, i32, i32, i32, P, i32, f64, P, P, P, i32, i32]
+            lib.kda_oracle_chunked_f64.restype = ctypes.c_int
+            lib.kda_oracle_unit_lower_inverse.argtypes = [P, i32, P, i32]
+            lib.kda_oracle_unit_lower_inverse.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return None if a is None else np.ascontiguousarray(a, dtype=dtype)
+
+
+def scan(q, k, v, g, beta, cu_seqlens, scale, initial_state=None, *, erase=True,
+         want_out=True, want_final=True, col_begin=0, col_end=None, col_block=16, nthreads=0):
+    """Token-by-token fp64 recurrence.
+
+    ``q``/``k``/``v`` are either uint16 bf16 bit patterns (library format, with
+    float32 ``g``/``beta``/``initial_state``) or float64 arrays (all inputs
+    float64). Returns ``(out, final_state)`` as float64 arrays (or ``None``
+    where not requested); only value columns ``[col_begin, col_end)`` are
+    filled, the rest is NaN.
+    """
+    lib = _load()
+    bf16 = np.asarray(q).dtype == np.uint16
+    vt = np.uint16 if bf16 else np.float64
+    gt = np.float32 if bf16 else np.float64
+    q, k, v = _c(q, vt), _c(k, vt), _c(v, vt)
+    g, beta = _c(g, gt), _c(beta, gt)
+    init = _c(initial_state, gt)
+    cu = _c(cu_seqlens, np.int32)
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    nseq = cu.shape[0] - 1
+    if col_end is None:
+        col_end = dv
+    out = np.full((T, H, dv), np.nan) if want_out else None
+    fin = np.full((nseq, H, dk, dv), np.nan) if want_final else None
+    fn = lib.kda_oracle_scan_bf16 if bf16 else lib.kda_oracle_scan_f64
+    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), T, H, dk, dv, _ptr(cu), nseq, float(scale),
+            _ptr(init), _ptr(out), _ptr(fin), 1 if erase else 0, int(col_begin), int(col_end),
+            int(col_block), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle scan rejected its arguments (code {rc})")
+    return out, fin
+
+
+def chunked(q, k, v, g, beta, cu_seqlens, scale, initial_state=None, *, chunk=16, nthreads=0):
+    """Naive fp64 chunked (WY-form) rewrite; all inputs converted to float64."""
+    lib = _load()
+    from kda_inputs import bf16_bits_to_f32  # input-format widening only
+
+    def f64(a):
+        a = np.asarray(a)
+        if a.dtype == np.uint16:
+            a = bf16_bits_to_f32(a)
+        return np.ascontiguousarray(a, dtype=np.float64)
+
+    q, k, v, g, beta = map(f64, (q, k, v, g, beta))
+    init = None if initial_state is None else f64(initial_state)
+    cu = _c(cu_seqlens, np.int32)
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    nseq = cu.shape[0] - 1
+    out = np.full((T, H, dv), np.nan)
+    fin = np.full((nseq, H, dk, dv), np.nan)
+    rc = lib.kda_oracle_chunked_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), T, H, dk, dv, _ptr(cu),
+                                    nseq, float(scale), _ptr(init), _ptr(out), _ptr(fin), int(chunk), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle chunked rejected its arguments (code {rc})")
+    return out, fin
+
+
+def unit_lower_inverse(L: np.ndarray, method: str = "substitution") -> np.ndarray:
+    """(I + L)^{-1} for strictly lower-triangular L (upper part ignored)."""
+    lib = _load()
+    L = np.ascontiguousarray(L, dtype=np.float64)
+    n = L.shape[0]
+    X = np.empty((n, n), dtype=np.float64)
+    m = {"substitution": 0, "doubling": 1}[method]
+    rc = lib.kda_oracle_unit_lower_inverse(_ptr(L), n, _ptr(X), m)
+    if rc != 0:
+        raise ValueError(f"oracle inverse rejected its arguments (code {rc})")
+    return X
+
+
+def scan_inputs(inp, **kw):
+    """Run the scan on a ``kda_inputs.KDAInputs`` batch."""
+    return scan(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens, inp.scale, inp.initial_state, **kw)
