@@ -1,0 +1,424 @@
+#!/usr/bin/env python
+"""Bench: KDA forward (prefill) throughput on B200, in Mtok*head/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl kda|reference]
+
+A step is one kda_fwd call over the whole workload (every (sequence, head)
+chain of the batch), i.e. the full hot path. The default workload is the
+Kimi-Linear-shaped fixed-length batch (T = 8192, H = 32, d = 128, zero initial
+state, final state returned). Inputs are seeded synthetic data of that shape
+(kda_inputs). For N > 1 (torchrun) every rank runs its own independent batch
+(weak scaling, no data-path collective); the time is the max over ranks.
+
+Output: one JSON line on rank 0 (see the keys in ``main``).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import kda_inputs  # noqa: E402
+
+METRIC = "KDA fwd prefill Mtok·head/s at d=128 on 1 B200; % of TC/HBM roofline"
+UNIT = "Mtok·head/s"
+D = 128
+# Counted work per token*head (d = 128): q, k, v, o bf16 + g fp32 + beta fp32.
+BYTES_PER_TOKHEAD = 3 * D * 2 + D * 4 + 4 + D * 2          # 1540 B
+FLOPS_PER_TOKHEAD = 6 * D * D + 10 * 16 * D                # 118784 FLOP
+STATE_BYTES = D * D * 4                                    # one (sequence, head) state
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+KERNEL_SOURCES = [os.path.join(ROOT, "kimi_delta_attention_26_b200", "csrc", "kda_fwd.cu")]
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), float(j["bf16_tflops"]), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def recorded_traffic(workload_name: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", f"kda_fwd_{workload_name}.md")
+    if not os.path.exists(p):
+        return None
+    txt = open(p).read()
+    m_b = re.search(r"traffic_bytes_per_launch\s*=\s*([0-9.eE+]+)", txt)
+    m_s = re.search(r"kernel_source_sha256\s*=\s*([0-9a-f]{64})", txt)
+    if not m_b or not m_s or m_s.group(1) != kernel_source_sha():
+        return None
+    return float(m_b.group(1))
+
+
+def work_units(inp) -> int:
+    return inp.total_tokens * inp.num_heads
+
+
+def algorithmic_bytes(inp, with_init: bool, with_final: bool) -> int:
+    n = work_units(inp) * BYTES_PER_TOKHEAD
+    states = inp.num_seqs * inp.num_heads * STATE_BYTES
+    return n + (states if with_init else 0) + (states if with_final else 0)
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples = []
+        self.reasons = 0
+        self.ok = False
+        self.max_mhz = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            bus = None
+            try:
+                import torch
+
+                props = torch.cuda.get_device_properties(device_index)
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report nothing rather than guess
+            log(f"clock sampling unavailable: {e}")
+        self.period = period_s
+        self._t = None
+
+    def _sample(self):
+        nv = self._nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        except Exception:
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+        self.reasons |= int(r)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+            try:
+                self._sample()
+            except Exception:
+                pass
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return None
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": float(self.max_mhz),
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------ CPU (oracle) leg
+def cpu_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_prefix_run(inp, ntok: int, nthreads: int) -> float:
+    """Run the oracle (as it stands) on the first ntok tokens of every sequence
+    prefix of the packed batch; returns seconds."""
+    import oracle  # test infrastructure; only this leg of the bench executes it
+
+    ntok = max(1, min(ntok, inp.total_tokens))
+    cu = np.minimum(inp.cu_seqlens, ntok).astype(np.int32)
+    init = inp.initial_state
+    t = time.perf_counter()
+    oracle.scan(inp.q[:ntok], inp.k[:ntok], inp.v[:ntok], inp.g[:ntok], inp.beta[:ntok], cu, inp.scale, init,
+                nthreads=nthreads)
+    return time.perf_counter() - t
+
+
+def cpu_baseline(inp, target_s: float):
+    nthreads = cpu_threads()
+    probe = min(inp.total_tokens, 64)
+    t_probe = oracle_prefix_run(inp, probe, nthreads)
+    ntok = int(min(inp.total_tokens, max(probe, probe * target_s / max(t_probe, 1e-6))))
+    dt = oracle_prefix_run(inp, ntok, nthreads)
+    units = ntok * inp.num_heads
+    return {"value": units / dt / 1e6, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+            "sample": f"fp64 token scan on the first {ntok} of {inp.total_tokens} tokens, all "
+                      f"{inp.num_heads} heads ({units} tok*head, {dt:.1f} s, {nthreads} threads)"}
+
+
+# ----------------------------------------------------------------- dist utils
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def aggregate(times_ms, units):
+    """Whole-job throughput: all ranks' units over the slowest rank's time."""
+    t = max(times_ms)
+    return sum(units) / (t * 1e-3) / 1e6, t
+
+
+# ---------------------------------------------------------------- reference
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0  # the CPU oracle arm runs on rank 0 only
+    wl = kda_inputs.workload(args.config)
+    inp = wl.make()
+    nthreads = cpu_threads()
+    budget = min(10.0, 150.0 / max(1, args.steps + args.warmup))
+    probe = min(inp.total_tokens, 64)
+    t_probe = oracle_prefix_run(inp, probe, nthreads)
+    ntok = int(min(inp.total_tokens, max(probe, probe * budget / max(t_probe, 1e-6))))
+    for _ in range(args.warmup):
+        oracle_prefix_run(inp, ntok, nthreads)
+    dts = [oracle_prefix_run(inp, ntok, nthreads) for _ in range(args.steps)]
+    dt = sum(dts) / len(dts)
+    units = ntok * inp.num_heads
+    value = units / dt / 1e6
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "seq_lens": list(wl.seqlens), "num_heads": wl.num_heads, "head_dim": D,
+                   "sample_tokens": ntok},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+                         "sample": f"fp64 token scan on the first {ntok} of {inp.total_tokens} tokens, "
+                                   f"all {inp.num_heads} heads, per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------- kda
+def run_kda(args):
+    import torch
+    import torch.distributed as dist
+
+    ws, rank, local = dist_env()
+    if ws != args.gpus:
+        log(f"note: --gpus {args.gpus} but WORLD_SIZE={ws}; using WORLD_SIZE")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    import kimi_delta_attention_26_b200 as kda
+
+    wl = kda_inputs.workload(args.config)
+    inp = wl.make(seed=wl.seed + rank)  # an independent batch per rank
+    with_init = inp.initial_state is not None
+    stream = torch.cuda.current_stream(dev)
+
+    # pinned host copies (for the end-to-end leg) and device-resident inputs
+    def pinned(a):
+        return torch.from_numpy(a).pin_memory()
+
+    h = {"q": pinned(inp.q).view(torch.bfloat16), "k": pinned(inp.k).view(torch.bfloat16),
+         "v": pinned(inp.v).view(torch.bfloat16), "g": pinned(inp.g), "beta": pinned(inp.beta),
+         "cu": pinned(inp.cu_seqlens)}
+    if with_init:
+        h["init"] = pinned(inp.initial_state)
+    d = {key: t.to(dev, non_blocking=False) for key, t in h.items()}
+    T, H, N = inp.total_tokens, inp.num_heads, inp.num_seqs
+    out = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+    fin = torch.empty((N, H, D, D), dtype=torch.float32, device=dev)
+    h_out = torch.empty((T, H, D), dtype=torch.bfloat16).pin_memory()
+    h_fin = torch.empty((N, H, D, D), dtype=torch.float32).pin_memory()
+
+    in_bytes = sum(t.numel() * t.element_size() for t in d.values())
+    flush = None
+    if in_bytes < 2 * L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        kda.kda_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], inp.scale, d["cu"], d.get("init"),
+                    out=out, final_state=fin, stream=stream)
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+
+    # ---- device-resident timing: per-launch CUDA events on the launch stream
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(local)
+    sampler.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        if flush is not None:
+            flush.add_(1.0)  # evict the previous launch's working set from L2
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.stop()
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    ms = sum(launch_ms) / len(launch_ms)
+
+    # ---- end-to-end through the public API with host buffers
+    def e2e_step():
+        for key in d:
+            d[key].copy_(h[key], non_blocking=True)
+        step()
+        h_out.copy_(out, non_blocking=True)
+        h_fin.copy_(fin, non_blocking=True)
+
+    for _ in range(max(1, min(args.warmup, 3))):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, min(args.steps, 10))
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    h2d = in_bytes
+    d2h = h_out.numel() * h_out.element_size() + h_fin.numel() * h_fin.element_size()
+
+    # ---- max over ranks
+    units = work_units(inp)
+    if ws > 1:
+        tt = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(tt[0]), float(tt[1])
+        uu = torch.tensor([units], dtype=torch.float64, device=dev)
+        dist.all_reduce(uu)
+        total_units = float(uu[0])
+    else:
+        total_units = float(units)
+    value = total_units / (ms * 1e-3) / 1e6
+    e2e_value = total_units / (e2e_ms * 1e-3) / 1e6
+
+    if rank == 0:
+        hbm_peak, tc_peak, peak_kind = measured_peaks()
+        bytes_launch = algorithmic_bytes(inp, with_init, True)
+        flops_launch = units * FLOPS_PER_TOKHEAD
+        gbs = bytes_launch / (ms * 1e-3) / 1e9
+        tflops = flops_launch / (ms * 1e-3) / 1e12
+        t_hbm = bytes_launch / (hbm_peak * 1e9)
+        t_tc = flops_launch / (tc_peak * 1e12)
+        bound = "hbm" if t_hbm >= t_tc else "tensor"
+        roof = {"bound": bound,
+                "achieved": gbs if bound == "hbm" else tflops,
+                "peak": hbm_peak if bound == "hbm" else tc_peak,
+                "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+                "peak_source": f"{peak_kind} ({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'recipe fallback'})",
+                "traffic": recorded_traffic(wl.name),
+                "algorithmic_bytes_per_launch": bytes_launch,
+                "tflops_counted": tflops}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "seq_lens": list(wl.seqlens) if len(wl.seqlens) <= 16 else None,
+                       "total_tokens": T, "num_heads": H, "head_dim": D, "num_seqs": N,
+                       "initial_state": "random" if with_init else "zero", "final_state": True,
+                       "global_batch": N * ws, "seq_len": T,
+                       "l2": "flushed between launches" if flush is not None
+                             else f"inputs larger than L2 ({in_bytes / 2**20:.0f} MiB)",
+                       "parallelism": f"dp{ws} (independent batch per GPU)", "seed": wl.seed},
+            "roofline": roof,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": args.steps,
+            "launch_ms": {"min": min(launch_ms), "median": statistics.median(launch_ms), "max": max(launch_ms)},
+            "clocks": sampler.summary(),
+        }
+        if ws == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(inp, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=2, choices=sorted(kda_inputs.WORKLOADS))
+    ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        log("note: raising --warmup to 3 (minimum)")
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_kda(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

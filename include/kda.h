@@ -1,0 +1,101 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention prefill library.
+ *
+ * The library computes the chunked forward (prefill) of Kimi Delta Attention
+ * (KDA) for head dimension dk = dv = 128 on one GPU. Per sequence and head:
+ *
+ *   S_t = (I - beta_t k_t k_t^T) Diag(exp g_t) S_{t-1} + beta_t k_t v_t^T
+ *   o_t = scale * S_t^T q_t
+ *
+ * with S a 128 x 128 fp32 state (rows: key channels, columns: value
+ * channels), g_t a natural-log decay per key channel and beta_t a scalar.
+ * KDA is Gated DeltaNet with one decay per channel instead of one scalar
+ * decay for the whole state, keeping the history in a fixed-size state
+ * (page "Kimi K3 开源满月…", section "KDA 内核到底难在哪"; page
+ * "FlashKDA: CUTLASS Kernel من Moonshot لـ Kimi", section "سياق Kimi Linear").
+ * Head dimension 128 only and forward only, as for FlashKDA (same FlashKDA
+ * page, section "المتطلبات الأساسية"; page "Moonshot AI … FlashKDA …
+ * (kucoin)"). Sequences of different lengths are packed along the token axis
+ * and described by cu_seqlens in the FlashAttention convention (FlashKDA page,
+ * section "تكامل مباشر مع flash-linear-attention").
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device.
+ *   - The caller owns all memory; kda_fwd allocates nothing.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and the call returns without synchronising.
+ *   - Argument errors are reported synchronously through the return code and
+ *     nothing is enqueued; the functions never abort the process.
+ *   - Results are deterministic: no atomics, no split reductions, and each
+ *     (sequence, head) is computed independently of the rest of the batch, so
+ *     a sequence gives bit-identical results alone or inside any batch.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KDA_HEAD_DIM 128
+#define KDA_ABI_VERSION 1
+
+typedef enum kda_status {
+  KDA_OK = 0,
+  KDA_ERR_NULL = 1,        /* a required pointer is NULL */
+  KDA_ERR_SHAPE = 2,       /* invalid sizes (negative T, H < 1, num_seqs < 1,
+                              cu_seqlens NULL with num_seqs != 1, int overflow) */
+  KDA_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned */
+  KDA_ERR_UNSUPPORTED = 4, /* the current device is not sm_100 (B200) */
+  KDA_ERR_CUDA = 5         /* a CUDA runtime call or the launch failed */
+} kda_status_t;
+
+/*
+ * kda_fwd -- chunked KDA forward (prefill) for a packed batch.
+ *
+ * Layouts (row-major, contiguous, T = total_tokens, H = num_heads, N = num_seqs):
+ *   q, k, v, out   bf16  [T, H, 128]
+ *   g              fp32  [T, H, 128]   natural-log decay per key channel.
+ *                  Precondition: -5 <= g <= 0 (the gate lower bound of
+ *                  FlashKDA, page "Kimi K3 开源满月…", section
+ *                  "KDA 内核到底难在哪"); outside it results are undefined
+ *                  (may be inf/NaN), never an out-of-bounds access.
+ *   beta           fp32  [T, H]
+ *   initial_state  fp32  [N, H, 128 (key), 128 (value)] or NULL (zero state)
+ *   final_state    fp32  [N, H, 128, 128] or NULL (not written); may alias
+ *                  initial_state (each (sequence, head) reads its slice before
+ *                  writing it).
+ *   cu_seqlens     int32 [N + 1] on the device, cu[0] = 0, non-decreasing,
+ *                  cu[N] = T; or NULL, meaning one sequence of T tokens
+ *                  (then num_seqs must be 1). Its contents are not checked on
+ *                  the host (that would need a synchronisation); the kernel
+ *                  clamps every boundary into [0, T], so bad contents give
+ *                  wrong results, never an out-of-bounds access.
+ *   scale          the output scale (usually 1/sqrt(128)).
+ * Alignment: every tensor pointer must be 16-byte aligned.
+ * Zero-length sequences are allowed: their final state equals their initial
+ * state (or zeros). T = 0 is allowed.
+ * Returns KDA_OK once the work is enqueued.
+ */
+kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                     float scale, const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                     int32_t num_heads, const float* initial_state, void* out, float* final_state,
+                     void* stream);
+
+/* Human-readable text of a status code (static storage, never NULL). */
+const char* kda_status_string(kda_status_t status);
+
+/* Text of the last CUDA error seen by this thread inside the library
+ * (static thread-local storage; "" if none). */
+const char* kda_last_cuda_error(void);
+
+/* KDA_ABI_VERSION of the loaded library. */
+int32_t kda_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

@@ -1,0 +1,117 @@
+"""B200 (sm_100a) Kimi Delta Attention prefill -- Python binding of ``libkda.so``.
+
+This module only marshals arguments: it checks torch tensors, allocates
+outputs with torch (device memory), and calls the C ABI declared in
+``include/kda.h`` on the current CUDA stream. Every step of the computation
+runs in the library's CUDA kernels; there is no fallback. Importing the
+module fails loudly if ``libkda.so`` has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = ["kda_fwd", "library_path", "KDAError", "HEAD_DIM"]
+
+HEAD_DIM = 128
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libkda.so")
+
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"{_LIB_PATH} is missing: build the CUDA library first "
+        "(python -m kimi_delta_attention_26_b200.build or __graft_entry__.build())")
+
+_lib = ctypes.CDLL(_LIB_PATH)
+_P = ctypes.c_void_p
+_lib.kda_fwd.argtypes = [_P, _P, _P, _P, _P, ctypes.c_float, _P, ctypes.c_int32, ctypes.c_int64,
+                         ctypes.c_int32, _P, _P, _P, _P]
+_lib.kda_fwd.restype = ctypes.c_int
+_lib.kda_status_string.argtypes = [ctypes.c_int]
+_lib.kda_status_string.restype = ctypes.c_char_p
+_lib.kda_last_cuda_error.argtypes = []
+_lib.kda_last_cuda_error.restype = ctypes.c_char_p
+_lib.kda_abi_version.argtypes = []
+_lib.kda_abi_version.restype = ctypes.c_int32
+
+
+class KDAError(RuntimeError):
+    def __init__(self, code: int):
+        msg = _lib.kda_status_string(code).decode()
+        cuda = _lib.kda_last_cuda_error().decode()
+        super().__init__(f"kda_fwd failed ({code}): {msg}" + (f" [{cuda}]" if cuda else ""))
+        self.code = code
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _check(t: torch.Tensor, name: str, dtype: torch.dtype, shape: Tuple[int, ...], device) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def kda_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, beta: torch.Tensor,
+            scale: Optional[float] = None, cu_seqlens: Optional[torch.Tensor] = None,
+            initial_state: Optional[torch.Tensor] = None, output_final_state: bool = True,
+            out: Optional[torch.Tensor] = None, final_state: Optional[torch.Tensor] = None,
+            stream: Optional[torch.cuda.Stream] = None):
+    """Chunked KDA forward on packed sequences (see ``include/kda.h``).
+
+    q, k, v: bf16 [T, H, 128]; g: fp32 [T, H, 128] (log decay, in [-5, 0]);
+    beta: fp32 [T, H]; cu_seqlens: int32 [N + 1] on the device (None: one
+    sequence); initial_state: fp32 [N, H, 128, 128] or None.
+    Returns ``(out, final_state)``; ``final_state`` is None unless requested.
+    """
+    if q.dim() != 3:
+        raise ValueError("q must be [T, H, 128]")
+    T, H, d = q.shape
+    if d != HEAD_DIM:
+        raise ValueError(f"head dimension must be {HEAD_DIM}")
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("kda_fwd runs on CUDA tensors only")
+    N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    _check(q, "q", torch.bfloat16, (T, H, d), dev)
+    _check(k, "k", torch.bfloat16, (T, H, d), dev)
+    _check(v, "v", torch.bfloat16, (T, H, d), dev)
+    _check(g, "g", torch.float32, (T, H, d), dev)
+    _check(beta, "beta", torch.float32, (T, H), dev)
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32, (N + 1,), dev)
+    if initial_state is not None:
+        _check(initial_state, "initial_state", torch.float32, (N, H, d, d), dev)
+    if out is None:
+        out = torch.empty((T, H, d), dtype=torch.bfloat16, device=dev)
+    _check(out, "out", torch.bfloat16, (T, H, d), dev)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((N, H, d, d), dtype=torch.float32, device=dev)
+    if final_state is not None:
+        _check(final_state, "final_state", torch.float32, (N, H, d, d), dev)
+    if scale is None:
+        scale = d ** -0.5
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    with torch.cuda.device(dev):
+        rc = _lib.kda_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), ctypes.c_float(scale),
+                          _ptr(cu_seqlens), N, T, H, _ptr(initial_state), _ptr(out), _ptr(final_state),
+                          ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise KDAError(rc)
+    return out, final_state

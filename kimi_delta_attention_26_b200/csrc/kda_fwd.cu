@@ -1,0 +1,622 @@
+// kda_fwd.cu -- chunked Kimi Delta Attention forward for sm_100a.
+//
+// One CTA owns one (sequence, head, value-column slice) work item and walks the
+// sequence chunk by chunk, carrying the fp32 state slice in registers.
+// Columns of the state evolve independently (the recurrence multiplies S only
+// from the left), so slicing the value columns needs no exchange between CTAs.
+//
+// Per chunk of C tokens (chunk-local cumulative log-decay G_i, inclusive):
+//   A[i][j]   = sum_c k_i[c] k_j[c] exp(G_i[c] - G_j[c])     (j < i)
+//   T         = (I + diag(beta) A)^{-1}
+//   W         = T diag(beta) (k * exp G)          U = T diag(beta) V
+//   Vnew      = U - W S
+//   Aqk[i][j] = sum_c q_i[c] k_j[c] exp(G_i[c] - G_j[c])     (j <= i)
+//   O         = scale (Qd S + Aqk Vnew)           Qd = q * exp G
+//   S        <- Diag(exp G_last) S + Kend^T Vnew  Kend_j = k_j * exp(G_last - G_j)
+// Chunking a delta-rule recurrence into small dense products with one state
+// chain across chunks follows the FlashKDA description (page "Kimi K3 开源满月…",
+// section "KDA 内核到底难在哪"); the chunk is 64 tokens here.
+//
+// Exponent range. With -5 <= g <= 0 a 16-token sub-block spans at most a
+// factor e^80 (< FLT_MAX ~ e^88.7), the bound that lets FlashKDA keep every
+// causal block on dense tensor-core products (same page and section:
+// lower_bound = -5). Factors are therefore anchored per 16-token sub-block:
+// with R_b the cumulative log-decay at the start of sub-block b,
+//   E_i = exp(G_i - R_I)       in [e^-80, 1]     (row i in sub-block I)
+//   F_j = exp(R_{J+1} - G_j)   in [e^-80, 1]     (row j in sub-block J)
+//   exp(G_i - G_j) = E_i * exp(R_I - R_{J+1}) * F_j   for J <= I,
+// where the middle per-channel factor is <= 1 for J < I and <= e^80 for J = I.
+// Masked (upper) entries are removed by selection, never by multiplying by 0.
+// A chunk-wide anchor plays the same role in the B200 kernel described on the
+// same page (section "反转二", chunk 32 with an anchor scalar).
+//
+// Tensor-core work uses mma.sync m16n8k16 (bf16 in, fp32 accumulate); the
+// unit-lower inverse is fp32 on the CUDA cores (forward substitution on the
+// 16 x 16 diagonal blocks, block substitution for the rest).
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/kda.h"
+
+namespace kda {
+
+constexpr int D = KDA_HEAD_DIM;  // dk = dv = 128
+constexpr int C = 64;            // chunk length (tokens)
+constexpr int BS = 16;           // anchoring sub-block (tokens)
+constexpr int NB = C / BS;       // sub-blocks per chunk
+constexpr int NS = 64;           // value columns per CTA
+constexpr int NSLICE = D / NS;   // CTAs per (sequence, head)
+constexpr int NTHREADS = 256;
+constexpr int NWARPS = NTHREADS / 32;
+
+// Padded row strides (elements). Row pitches of 272 / 144 bytes shift
+// successive rows by 4 banks, so 8-row ldmatrix reads are conflict-free.
+constexpr int LDK = D + 8;   // bf16 [C][D] tiles
+constexpr int LDN = NS + 8;  // bf16 [*][NS] tiles
+constexpr int LDC = C + 8;   // bf16 [C][C] tiles
+constexpr int LDF = C + 4;   // fp32 [C][C] tiles
+
+static_assert(NWARPS == 8, "warp roles below assume 8 warps");
+static_assert(NB == 4 && C == 64 && NS == 64, "tile mapping below assumes C = NS = 64");
+
+// Shared-memory plan (bytes). Buffers whose lifetimes do not overlap share
+// storage: W reuses KL, L reuses QL, T reuses KF.
+struct Smem {
+  static constexpr int kTileK = C * LDK * 2;       // 17408
+  static constexpr int kTileCF = C * LDF * 4;      // 17408
+  static constexpr int kTileC = C * LDC * 2;       // 9216
+  static constexpr int kTileN = C * LDN * 2;       // 9216
+  static constexpr int kS = D * LDN * 2;           // 18432
+  static constexpr int oKL = 0;                    // bf16 k*E        -> W
+  static constexpr int oQL = oKL + kTileK;         // bf16 q*E        -> L (fp32)
+  static constexpr int oKF = oQL + kTileK;         // bf16 k*F        -> T (fp32)
+  static constexpr int oKd = oKF + kTileK;         // bf16 k*exp(G)
+  static constexpr int oQd = oKd + kTileK;         // bf16 q*exp(G)
+  static constexpr int oKe = oQd + kTileK;         // bf16 k*exp(G_last - G)
+  static constexpr int oTb = oKe + kTileK;         // bf16 T diag(beta)
+  static constexpr int oAqk = oTb + kTileC;        // bf16 masked Aqk
+  static constexpr int oV = oAqk + kTileC;         // bf16 V slice
+  static constexpr int oVn = oV + kTileN;          // bf16 Vnew slice
+  static constexpr int oS = oVn + kTileN;          // bf16 copy of the state slice
+  static constexpr int oPf = oS + kS;              // fp32 [NB][NB][D] pair factors
+  static constexpr int oTmp = oPf + NB * NB * D * 4;  // fp32 [3][16][16] block products
+  static constexpr int oGam = oTmp + 3 * 16 * 16 * 4; // fp32 [D] chunk decay
+  static constexpr int oBeta = oGam + D * 4;       // fp32 [C]
+  static constexpr int kBytes = oBeta + C * 4;
+};
+static_assert(Smem::kBytes <= 227 * 1024, "shared memory budget");
+
+// ---------------------------------------------------------------- primitives
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
+}
+
+// D += A(16x16, row) * B(16x8, col); bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  uint32_t u;
+  memcpy(&u, &h, 4);
+  return u;
+}
+
+__device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
+  __nv_bfloat162 h;
+  memcpy(&h, &u, 4);
+  return __bfloat1622float2(h);
+}
+
+__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t u, float s0, float s1) {
+  float2 f = unpack_bf16(u);
+  return pack_bf16(f.x * s0, f.y * s1);
+}
+
+__device__ __forceinline__ float bf16_to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// ---------------------------------------------------------------- the kernel
+struct Params {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const float* g;
+  const float* beta;
+  const int32_t* cu;       // may be null: one sequence [0, T)
+  const float* init;       // may be null
+  __nv_bfloat16* out;
+  float* fin;              // may be null
+  int64_t T;
+  int32_t H;
+  int32_t nseq;
+  float scale;
+};
+
+__global__ void __launch_bounds__(NTHREADS, 1) kda_fwd_chunked_kernel(const Params p) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __nv_bfloat16* sKL = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oKL);
+  __nv_bfloat16* sW = sKL;
+  __nv_bfloat16* sQL = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oQL);
+  float* sL = reinterpret_cast<float*>(smem + Smem::oQL);
+  __nv_bfloat16* sKF = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oKF);
+  float* sT = reinterpret_cast<float*>(smem + Smem::oKF);
+  __nv_bfloat16* sKd = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oKd);
+  __nv_bfloat16* sQd = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oQd);
+  __nv_bfloat16* sKe = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oKe);
+  __nv_bfloat16* sTb = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oTb);
+  __nv_bfloat16* sAqk = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oAqk);
+  __nv_bfloat16* sV = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oV);
+  __nv_bfloat16* sVn = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oVn);
+  __nv_bfloat16* sS = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oS);
+  float* sPf = reinterpret_cast<float*>(smem + Smem::oPf);
+  float* sTmp = reinterpret_cast<float*>(smem + Smem::oTmp);
+  float* sGam = reinterpret_cast<float*>(smem + Smem::oGam);
+  float* sBeta = reinterpret_cast<float*>(smem + Smem::oBeta);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int gq = lane >> 2;  // mma fragment row group
+  const int tq = lane & 3;   // mma fragment column pair
+
+  const int slice = blockIdx.x;
+  const int h = blockIdx.y;
+  const int seq = blockIdx.z;
+  const int dv0 = slice * NS;
+  const int H = p.H;
+  const int64_t T = p.T;
+
+  int64_t t0 = 0, t1 = T;
+  if (p.cu) {
+    t0 = p.cu[seq];
+    t1 = p.cu[seq + 1];
+    t0 = t0 < 0 ? 0 : (t0 > T ? T : t0);
+    t1 = t1 < t0 ? t0 : (t1 > T ? T : t1);
+  }
+
+  // ---- state slice: fp32 master in registers (mma accumulator layout of the
+  // rows 16*warp..16*warp+15 x all NS columns), bf16 copy in shared memory.
+  float sreg[NS / 8][4];
+  {
+    const size_t sbase = (static_cast<size_t>(seq) * H + h) * D * D;
+#pragma unroll
+    for (int nt = 0; nt < NS / 8; ++nt) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int r = 16 * warp + gq + 8 * half;
+        const int c = 8 * nt + 2 * tq;
+        float2 x = make_float2(0.f, 0.f);
+        if (p.init) x = *reinterpret_cast<const float2*>(p.init + sbase + static_cast<size_t>(r) * D + dv0 + c);
+        sreg[nt][2 * half] = x.x;
+        sreg[nt][2 * half + 1] = x.y;
+        *reinterpret_cast<uint32_t*>(sS + r * LDN + c) = pack_bf16(x.x, x.y);
+      }
+    }
+  }
+  __syncthreads();
+
+  const size_t row_stride = static_cast<size_t>(H) * D;  // elements between tokens
+
+  for (int64_t cs = t0; cs < t1; cs += C) {
+    const int m = static_cast<int>((t1 - cs) < C ? (t1 - cs) : C);  // valid rows
+
+    // ================= phase 1: gates, anchored factors, operands; V slice
+    if (tid < D) {
+      const int c = tid;
+      float gl[C];
+#pragma unroll
+      for (int i = 0; i < C; ++i)
+        gl[i] = (i < m) ? __ldg(p.g + (cs + i) * row_stride + static_cast<size_t>(h) * D + c) : 0.f;
+      float R[NB + 1];
+      R[0] = 0.f;
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < BS; ++i) {
+          s += gl[BS * b + i];
+          gl[BS * b + i] = s;  // now: cumulative log-decay within the sub-block
+        }
+        R[b + 1] = R[b] + s;
+      }
+#pragma unroll
+      for (int I = 0; I < NB; ++I)
+#pragma unroll
+        for (int J = 0; J <= I; ++J) sPf[(I * NB + J) * D + c] = __expf(R[I] - R[J + 1]);
+      sGam[c] = __expf(R[NB]);
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const float eR = __expf(R[b]);
+        const float eEnd = __expf(R[NB] - R[b + 1]);
+        const float bsum = R[b + 1] - R[b];
+#pragma unroll
+        for (int i = 0; i < BS; ++i) {
+          const int row = BS * b + i;
+          float kv = 0.f, qv = 0.f;
+          if (row < m) {
+            const size_t off = (cs + row) * row_stride + static_cast<size_t>(h) * D + c;
+            kv = bf16_to_f32(p.k[off]);
+            qv = bf16_to_f32(p.q[off]);
+          }
+          const float E = __expf(gl[row]);
+          const float F = __expf(bsum - gl[row]);
+          sKL[row * LDK + c] = __float2bfloat16_rn(kv * E);
+          sQL[row * LDK + c] = __float2bfloat16_rn(qv * E);
+          sKF[row * LDK + c] = __float2bfloat16_rn(kv * F);
+          sKd[row * LDK + c] = __float2bfloat16_rn(kv * (E * eR));
+          sQd[row * LDK + c] = __float2bfloat16_rn(qv * (E * eR));
+          sKe[row * LDK + c] = __float2bfloat16_rn(kv * (F * eEnd));
+        }
+      }
+    } else {
+      const int t = tid - D;  // 128 threads: V slice (C x NS bf16, 16-byte pieces) and beta
+      constexpr int kPieces = C * NS / 8;
+      for (int idx = t; idx < kPieces; idx += NTHREADS - D) {
+        const int row = idx / (NS / 8);
+        const int col = (idx % (NS / 8)) * 8;
+        uint4 x = make_uint4(0, 0, 0, 0);
+        if (row < m)
+          x = __ldg(reinterpret_cast<const uint4*>(p.v + (cs + row) * row_stride + static_cast<size_t>(h) * D + dv0 + col));
+        *reinterpret_cast<uint4*>(sV + row * LDN + col) = x;
+      }
+      if (t < C) sBeta[t] = (t < m) ? __ldg(p.beta + (cs + t) * H + h) : 0.f;
+    }
+    __syncthreads();
+
+    // ================= phase 2: masked A (-> L = diag(beta) A) and Aqk blocks
+    for (int pr = warp; pr < NB * (NB + 1) / 2; pr += NWARPS) {
+      int I = 0, J = pr;
+      while (J > I) {
+        ++I;
+        J -= I;
+      }
+      // now pr = I*(I+1)/2 + J with J <= I
+      float accA[2][4] = {}, accQ[2][4] = {};
+      const float* pf = sPf + (I * NB + J) * D;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        uint32_t a[4], aq[4], b[4];
+        ldsm_x4(a, sKL + (16 * I + (lane & 15)) * LDK + 16 * kk + (lane >> 4) * 8);
+        ldsm_x4(aq, sQL + (16 * I + (lane & 15)) * LDK + 16 * kk + (lane >> 4) * 8);
+        ldsm_x4(b, sKF + (16 * J + (lane & 7) + ((lane >> 4) << 3)) * LDK + 16 * kk + ((lane >> 3) & 1) * 8);
+        const float2 f01 = *reinterpret_cast<const float2*>(pf + 16 * kk + 2 * tq);
+        const float2 f23 = *reinterpret_cast<const float2*>(pf + 16 * kk + 8 + 2 * tq);
+        a[0] = scale_bf16x2(a[0], f01.x, f01.y);
+        a[1] = scale_bf16x2(a[1], f01.x, f01.y);
+        a[2] = scale_bf16x2(a[2], f23.x, f23.y);
+        a[3] = scale_bf16x2(a[3], f23.x, f23.y);
+        aq[0] = scale_bf16x2(aq[0], f01.x, f01.y);
+        aq[1] = scale_bf16x2(aq[1], f01.x, f01.y);
+        aq[2] = scale_bf16x2(aq[2], f23.x, f23.y);
+        aq[3] = scale_bf16x2(aq[3], f23.x, f23.y);
+        mma_bf16(accA[0], a, b[0], b[1]);
+        mma_bf16(accA[1], a, b[2], b[3]);
+        mma_bf16(accQ[0], aq, b[0], b[1]);
+        mma_bf16(accQ[1], aq, b[2], b[3]);
+      }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = 16 * I + gq + (e >> 1) * 8;
+          const int j = 16 * J + 8 * nt + 2 * tq + (e & 1);
+          sL[i * LDF + j] = (j < i) ? sBeta[i] * accA[nt][e] : 0.f;
+          sAqk[i * LDC + j] = __float2bfloat16_rn((j <= i) ? accQ[nt][e] : 0.f);
+        }
+    }
+    __syncthreads();
+
+    // ================= phase 3: T = (I + L)^{-1}, then Tb = T diag(beta)
+    if (warp < 2) {
+      // diagonal 16 x 16 blocks: one half-warp per block, one lane per column
+      const int I = 2 * warp + (lane >> 4);
+      const int col = lane & 15;
+      const float* Lb = sL + (16 * I) * LDF + 16 * I;
+      float x[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) x[i] = (i == col) ? 1.f : 0.f;
+#pragma unroll
+      for (int mm = 0; mm < 16; ++mm) {
+        const float xm = x[mm];
+#pragma unroll
+        for (int i = mm + 1; i < 16; ++i) x[i] = fmaf(-Lb[i * LDF + mm], xm, x[i]);
+      }
+      float* Tb = sT + (16 * I) * LDF + 16 * I;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) Tb[i * LDF + col] = x[i];
+    }
+    __syncthreads();
+    {
+      // off-diagonal blocks by distance d = I - J:
+      //   T_IJ = -T_II * sum_{K=J}^{I-1} L_IK T_KJ
+      const int r = tid >> 4, cc = tid & 15;
+      for (int d = 1; d < NB; ++d) {
+        for (int J = 0; J + d < NB; ++J) {
+          const int I = J + d;
+          float acc = 0.f;
+          for (int K = J; K < I; ++K) {
+            const float* Lr = sL + (16 * I + r) * LDF + 16 * K;
+            const float* Tc = sT + (16 * K) * LDF + 16 * J + cc;
+#pragma unroll
+            for (int mm = 0; mm < 16; ++mm) acc = fmaf(Lr[mm], Tc[mm * LDF], acc);
+          }
+          sTmp[J * 256 + r * 16 + cc] = acc;
+        }
+        __syncthreads();
+        for (int J = 0; J + d < NB; ++J) {
+          const int I = J + d;
+          const float* Tr = sT + (16 * I + r) * LDF + 16 * I;
+          float acc = 0.f;
+#pragma unroll
+          for (int mm = 0; mm < 16; ++mm) acc = fmaf(Tr[mm], sTmp[J * 256 + mm * 16 + cc], acc);
+          sT[(16 * I + r) * LDF + 16 * J + cc] = -acc;
+        }
+        __syncthreads();
+      }
+      // Tb = T diag(beta) in bf16, lower blocks only (the products below skip J > I)
+      for (int idx = tid; idx < C * C; idx += NTHREADS) {
+        const int i = idx / C, j = idx % C;
+        if ((j >> 4) <= (i >> 4)) sTb[i * LDC + j] = __float2bfloat16_rn(sT[i * LDF + j] * sBeta[j]);
+      }
+    }
+    __syncthreads();
+
+    // ================= phase 4: W = Tb Kd (all 128 channels), U = Tb V (slice)
+    const int I4 = warp >> 1;       // row sub-block of this warp (phases 4 and 5a/5b)
+    float uacc[4][4] = {};          // U tile: rows 16*I4.., columns (warp&1)*32 + 8*nt
+    {
+      const int ch = (warp & 1) * 64;
+      float acc[8][4] = {};
+      for (int J = 0; J <= I4; ++J) {
+        uint32_t a[4];
+        ldsm_x4(a, sTb + (16 * I4 + (lane & 15)) * LDC + 16 * J + (lane >> 4) * 8);
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {
+          uint32_t b[4];
+          ldsm_x4_t(b, sKd + (16 * J + (lane & 7) + ((lane >> 3) & 1) * 8) * LDK + ch + 16 * np + (lane >> 4) * 8);
+          mma_bf16(acc[2 * np], a, b[0], b[1]);
+          mma_bf16(acc[2 * np + 1], a, b[2], b[3]);
+        }
+        const int nh = (warp & 1) * 32;
+#pragma unroll
+        for (int np = 0; np < 2; ++np) {
+          uint32_t b[4];
+          ldsm_x4_t(b, sV + (16 * J + (lane & 7) + ((lane >> 3) & 1) * 8) * LDN + nh + 16 * np + (lane >> 4) * 8);
+          mma_bf16(uacc[2 * np], a, b[0], b[1]);
+          mma_bf16(uacc[2 * np + 1], a, b[2], b[3]);
+        }
+      }
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int i = 16 * I4 + gq + 8 * half;
+          const int c = ch + 8 * nt + 2 * tq;
+          *reinterpret_cast<uint32_t*>(sW + i * LDK + c) = pack_bf16(acc[nt][2 * half], acc[nt][2 * half + 1]);
+        }
+    }
+    __syncthreads();
+
+    // ================= phase 5a: Vnew = U - W S ; O = Qd S (same B fragments)
+    const int nh = (warp & 1) * 32;
+    float oacc[4][4] = {};
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      uint32_t aw[4], aqd[4];
+      ldsm_x4(aw, sW + (16 * I4 + (lane & 15)) * LDK + 16 * kk + (lane >> 4) * 8);
+      ldsm_x4(aqd, sQd + (16 * I4 + (lane & 15)) * LDK + 16 * kk + (lane >> 4) * 8);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) aw[e] ^= 0x80008000u;  // -W (exact sign flip)
+#pragma unroll
+      for (int np = 0; np < 2; ++np) {
+        uint32_t b[4];
+        ldsm_x4_t(b, sS + (16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8) * LDN + nh + 16 * np + (lane >> 4) * 8);
+        mma_bf16(uacc[2 * np], aw, b[0], b[1]);
+        mma_bf16(uacc[2 * np + 1], aw, b[2], b[3]);
+        mma_bf16(oacc[2 * np], aqd, b[0], b[1]);
+        mma_bf16(oacc[2 * np + 1], aqd, b[2], b[3]);
+      }
+    }
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int i = 16 * I4 + gq + 8 * half;
+        const int c = nh + 8 * nt + 2 * tq;
+        *reinterpret_cast<uint32_t*>(sVn + i * LDN + c) = pack_bf16(uacc[nt][2 * half], uacc[nt][2 * half + 1]);
+      }
+    __syncthreads();
+
+    // ================= phase 5b: O += Aqk Vnew ; store O
+    for (int J = 0; J <= I4; ++J) {
+      uint32_t a[4];
+      ldsm_x4(a, sAqk + (16 * I4 + (lane & 15)) * LDC + 16 * J + (lane >> 4) * 8);
+#pragma unroll
+      for (int np = 0; np < 2; ++np) {
+        uint32_t b[4];
+        ldsm_x4_t(b, sVn + (16 * J + (lane & 7) + ((lane >> 3) & 1) * 8) * LDN + nh + 16 * np + (lane >> 4) * 8);
+        mma_bf16(oacc[2 * np], a, b[0], b[1]);
+        mma_bf16(oacc[2 * np + 1], a, b[2], b[3]);
+      }
+    }
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int i = 16 * I4 + gq + 8 * half;
+        if (i < m) {
+          const int c = dv0 + nh + 8 * nt + 2 * tq;
+          *reinterpret_cast<uint32_t*>(p.out + (cs + i) * row_stride + static_cast<size_t>(h) * D + c) =
+              pack_bf16(p.scale * oacc[nt][2 * half], p.scale * oacc[nt][2 * half + 1]);
+        }
+      }
+
+    // ================= phase 5c: S <- Diag(gamma) S + Kend^T Vnew (rows 16*warp..)
+    {
+      const float g0 = sGam[16 * warp + gq], g1 = sGam[16 * warp + gq + 8];
+#pragma unroll
+      for (int nt = 0; nt < NS / 8; ++nt) {
+        sreg[nt][0] *= g0;
+        sreg[nt][1] *= g0;
+        sreg[nt][2] *= g1;
+        sreg[nt][3] *= g1;
+      }
+#pragma unroll
+      for (int J = 0; J < NB; ++J) {
+        uint32_t a[4];
+        ldsm_x4_t(a, sKe + (16 * J + (lane & 7) + ((lane >> 4) << 3)) * LDK + 16 * warp + ((lane >> 3) & 1) * 8);
+#pragma unroll
+        for (int np = 0; np < NS / 16; ++np) {
+          uint32_t b[4];
+          ldsm_x4_t(b, sVn + (16 * J + (lane & 7) + ((lane >> 3) & 1) * 8) * LDN + 16 * np + (lane >> 4) * 8);
+          mma_bf16(sreg[2 * np], a, b[0], b[1]);
+          mma_bf16(sreg[2 * np + 1], a, b[2], b[3]);
+        }
+      }
+#pragma unroll
+      for (int nt = 0; nt < NS / 8; ++nt)
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int r = 16 * warp + gq + 8 * half;
+          *reinterpret_cast<uint32_t*>(sS + r * LDN + 8 * nt + 2 * tq) = pack_bf16(sreg[nt][2 * half], sreg[nt][2 * half + 1]);
+        }
+    }
+    __syncthreads();
+  }
+
+  if (p.fin) {
+    const size_t sbase = (static_cast<size_t>(seq) * H + h) * D * D;
+#pragma unroll
+    for (int nt = 0; nt < NS / 8; ++nt)
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int r = 16 * warp + gq + 8 * half;
+        const int c = 8 * nt + 2 * tq;
+        *reinterpret_cast<float2*>(p.fin + sbase + static_cast<size_t>(r) * D + dv0 + c) =
+            make_float2(sreg[nt][2 * half], sreg[nt][2 * half + 1]);
+      }
+  }
+}
+
+}  // namespace kda
+
+// =================================================================== C ABI
+namespace {
+
+thread_local char g_last_cuda_error[256] = "";
+
+kda_status_t cuda_fail(cudaError_t e) {
+  std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(e),
+                cudaGetErrorString(e));
+  return KDA_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kMaxDevices = 64;
+int g_device_ready[kMaxDevices];  // 0 unknown, 1 ready, -1 unsupported
+
+kda_status_t prepare_device(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return KDA_ERR_UNSUPPORTED;
+  if (g_device_ready[dev] == 1) return KDA_OK;
+  if (g_device_ready[dev] == -1) return KDA_ERR_UNSUPPORTED;
+  int major = 0, minor = 0;
+  cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (major != 10 || minor != 0) {
+    g_device_ready[dev] = -1;
+    return KDA_ERR_UNSUPPORTED;
+  }
+  e = cudaFuncSetAttribute(kda::kda_fwd_chunked_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kda::Smem::kBytes);
+  if (e != cudaSuccess) return cuda_fail(e);
+  g_device_ready[dev] = 1;
+  return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                     float scale, const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                     int32_t num_heads, const float* initial_state, void* out, float* final_state,
+                     void* stream) {
+  g_last_cuda_error[0] = '\0';
+  if (!q || !k || !v || !g || !beta || !out) return KDA_ERR_NULL;
+  if (total_tokens < 0 || num_heads < 1 || num_seqs < 1) return KDA_ERR_SHAPE;
+  if (!cu_seqlens && num_seqs != 1) return KDA_ERR_SHAPE;
+  if (num_heads > 65535 || num_seqs > 65535) return KDA_ERR_SHAPE;  // grid.y / grid.z limits
+  if (total_tokens > (int64_t(1) << 40) / (int64_t(num_heads) * KDA_HEAD_DIM)) return KDA_ERR_SHAPE;
+  const void* ptrs[] = {q, k, v, g, beta, out, initial_state, final_state, cu_seqlens};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
+
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  kda_status_t st = prepare_device(dev);
+  if (st != KDA_OK) return st;
+
+  kda::Params p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.g = g;
+  p.beta = beta;
+  p.cu = cu_seqlens;
+  p.init = initial_state;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.fin = final_state;
+  p.T = total_tokens;
+  p.H = num_heads;
+  p.nseq = num_seqs;
+  p.scale = scale;
+  dim3 grid(kda::NSLICE, num_heads, num_seqs);
+  kda::kda_fwd_chunked_kernel<<<grid, kda::NTHREADS, kda::Smem::kBytes, static_cast<cudaStream_t>(stream)>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return KDA_OK;
+}
+
+const char* kda_status_string(kda_status_t s) {
+  switch (s) {
+    case KDA_OK: return "ok";
+    case KDA_ERR_NULL: return "a required pointer is NULL";
+    case KDA_ERR_SHAPE: return "invalid sizes";
+    case KDA_ERR_ALIGN: return "a tensor pointer is not 16-byte aligned";
+    case KDA_ERR_UNSUPPORTED: return "the current device is not sm_100 (B200)";
+    case KDA_ERR_CUDA: return "a CUDA call failed (see kda_last_cuda_error)";
+  }
+  return "unknown status";
+}
+
+const char* kda_last_cuda_error(void) { return g_last_cuda_error; }
+
+int32_t kda_abi_version(void) { return KDA_ABI_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,70 @@
+"""The C-ABI library loads, exports every declared symbol, and rejects bad
+arguments on the host before touching the GPU (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from kimi_delta_attention_26_b200 import build
+
+    build.build()
+    return ctypes.CDLL(build.LIB)
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "kda.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared_functions()
+    assert "kda_fwd" in names and len(names) >= 4
+    for n in names:
+        assert hasattr(lib, n), f"libkda.so does not export {n}"
+
+
+def test_abi_version_and_status_strings(lib):
+    lib.kda_abi_version.restype = ctypes.c_int32
+    assert lib.kda_abi_version() == 1
+    lib.kda_status_string.restype = ctypes.c_char_p
+    lib.kda_status_string.argtypes = [ctypes.c_int]
+    for code in range(6):
+        assert len(lib.kda_status_string(code)) > 0
+    assert lib.kda_status_string(99) == b"unknown status"
+
+
+def _call(lib, q=0x1000, k=0x2000, v=0x3000, g=0x4000, beta=0x5000, scale=1.0, cu=0x6000, nseq=1,
+          T=4, H=1, init=None, out=0x7000, fin=None):
+    P = ctypes.c_void_p
+    lib.kda_fwd.argtypes = [P, P, P, P, P, ctypes.c_float, P, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32,
+                            P, P, P, P]
+    lib.kda_fwd.restype = ctypes.c_int
+    return lib.kda_fwd(q, k, v, g, beta, scale, cu, nseq, T, H, init, out, fin, None)
+
+
+# These calls fail validation before any CUDA call, so the fake addresses are
+# never dereferenced or handed to the driver.
+def test_rejects_null_pointers(lib):
+    for name in ("q", "k", "v", "g", "beta", "out"):
+        assert _call(lib, **{name: None}) == 1, name
+
+
+def test_rejects_bad_shapes(lib):
+    assert _call(lib, T=-1) == 2
+    assert _call(lib, H=0) == 2
+    assert _call(lib, nseq=0) == 2
+    assert _call(lib, cu=None, nseq=2) == 2
+    assert _call(lib, H=70000) == 2
+    assert _call(lib, T=1 << 40, H=32) == 2
+
+
+def test_rejects_misaligned_pointers(lib):
+    for name in ("q", "k", "v", "g", "beta", "out", "init", "fin", "cu"):
+        assert _call(lib, **{name: 0x8008}) == 3, name

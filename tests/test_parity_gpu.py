@@ -1,0 +1,179 @@
+"""GPU parity: the CUDA path against the fp64 oracle on the same seeded inputs.
+
+All calls go through the C ABI (``libkda.so``) via the thin Python binding.
+Bars: o max-abs <= 3e-2 and rel-RMS <= 5e-3; final state rel-RMS <= 5e-3;
+segment handling bit-exact (a sequence gives the same bits alone or packed).
+"""
+import numpy as np
+import pytest
+
+import kda_inputs
+from tests import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kda():
+    import torch
+
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import kimi_delta_attention_26_b200 as m
+
+    return m
+
+
+def _check(oracle_mod, inp, label, cols=None, **kw):
+    out, fin = H.run_gpu(inp, **kw)
+    if cols is None:
+        o_ref, f_ref = oracle_mod.scan_inputs(inp)
+        return H.assert_parity(out, fin, o_ref, f_ref, label=label)
+    o_ref, f_ref = oracle_mod.scan_inputs(inp, col_begin=cols.start, col_end=cols.stop)
+    return H.assert_parity(out, fin, o_ref, f_ref, cols=cols, label=label)
+
+
+def test_tiny_config(kda, oracle_mod):
+    inp = kda_inputs.workload(1).make()
+    mo, ms = _check(oracle_mod, inp, "tiny T=256 H=2")
+    print("tiny", mo, ms)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_ragged_varlen_small(kda, oracle_mod, seed):
+    # lengths around the 16-token anchor blocks and 64-token chunks, an empty
+    # sequence, several chunks, random initial states
+    lens = [1, 15, 16, 17, 63, 64, 65, 200, 0, 129, 300]
+    inp = kda_inputs.make_inputs(lens, 3, seed=50 + seed, random_initial_state=True)
+    _check(oracle_mod, inp, f"ragged seed={seed}")
+
+
+def test_zero_initial_state_null_equals_zeros(kda):
+    import torch
+
+    inp = kda_inputs.make_inputs([100, 37], 2, seed=3)
+    out_a, fin_a = H.run_gpu(inp)
+    inp.initial_state = np.zeros((2, 2, 128, 128), np.float32)
+    out_b, fin_b = H.run_gpu(inp)
+    assert torch.equal(out_a, out_b) and torch.equal(fin_a, fin_b)
+
+
+def test_gate_extremes(kda, oracle_mod):
+    # g at the lower bound everywhere (fastest decay) and g = 0 (no decay)
+    for fill in (-5.0, 0.0):
+        inp = kda_inputs.make_inputs([150, 70], 2, seed=8, random_initial_state=True)
+        inp.g[:] = fill
+        _check(oracle_mod, inp, f"g={fill}")
+
+
+def test_single_token_and_all_empty(kda, oracle_mod):
+    import torch
+
+    inp = kda_inputs.make_inputs([1], 4, seed=9, random_initial_state=True)
+    _check(oracle_mod, inp, "T=1")
+    inp = kda_inputs.make_inputs([0, 0, 0], 2, seed=10, random_initial_state=True)
+    out, fin = H.run_gpu(inp)
+    assert out.numel() == 0
+    assert torch.equal(fin.cpu(), torch.from_numpy(inp.initial_state))
+
+
+def test_segments_bit_exact(kda):
+    """A packed batch restricted to one sequence equals that sequence run alone, bitwise."""
+    import torch
+
+    lens = [5, 64, 0, 130, 77, 1]
+    inp = kda_inputs.make_inputs(lens, 2, seed=11, random_initial_state=True)
+    out, fin = H.run_gpu(inp)
+    cu = inp.cu_seqlens
+    for i, L in enumerate(lens):
+        sub = kda_inputs.KDAInputs(
+            q=inp.q[cu[i]:cu[i + 1]], k=inp.k[cu[i]:cu[i + 1]], v=inp.v[cu[i]:cu[i + 1]],
+            g=inp.g[cu[i]:cu[i + 1]], beta=inp.beta[cu[i]:cu[i + 1]],
+            cu_seqlens=np.array([0, L], np.int32), initial_state=inp.initial_state[i:i + 1].copy(),
+            scale=inp.scale, seed=inp.seed)
+        o_i, f_i = H.run_gpu(sub)
+        assert torch.equal(out[cu[i]:cu[i + 1]], o_i), f"segment {i}: output bits differ"
+        assert torch.equal(fin[i], f_i[0]), f"segment {i}: state bits differ"
+
+
+def test_no_cu_seqlens_equals_single_sequence(kda):
+    import torch
+
+    inp = kda_inputs.make_inputs([333], 2, seed=12, random_initial_state=True)
+    d = H.to_device(inp)
+    a = kda.kda_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], inp.scale, d["cu_seqlens"], d["initial_state"])
+    b = kda.kda_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], inp.scale, None, d["initial_state"])
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("t1", [64, 100])
+def test_resume_from_final_state(kda, oracle_mod, t1):
+    import torch
+
+    inp = kda_inputs.make_inputs([257], 2, seed=13, random_initial_state=True)
+    d = H.to_device(inp)
+    full_o, full_f = kda.kda_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], inp.scale, None, d["initial_state"])
+    a_o, a_f = kda.kda_fwd(d["q"][:t1].contiguous(), d["k"][:t1].contiguous(), d["v"][:t1].contiguous(),
+                           d["g"][:t1].contiguous(), d["beta"][:t1].contiguous(), inp.scale, None, d["initial_state"])
+    b_o, b_f = kda.kda_fwd(d["q"][t1:].contiguous(), d["k"][t1:].contiguous(), d["v"][t1:].contiguous(),
+                           d["g"][t1:].contiguous(), d["beta"][t1:].contiguous(), inp.scale, None, a_f)
+    torch.cuda.synchronize()
+    o_ref, f_ref = oracle_mod.scan_inputs(inp)
+    H.assert_parity(torch.cat([a_o, b_o]), b_f, o_ref, f_ref, label=f"resume t1={t1}")
+    if t1 % 64 == 0:
+        # splitting on a chunk boundary changes nothing but the state's fp32 round trip
+        assert torch.equal(torch.cat([a_o, b_o]), full_o)
+        assert torch.equal(b_f, full_f)
+
+
+def test_in_place_state_update(kda):
+    import torch
+
+    inp = kda_inputs.make_inputs([90, 10], 2, seed=14, random_initial_state=True)
+    d = H.to_device(inp)
+    o1, f1 = kda.kda_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], inp.scale, d["cu_seqlens"], d["initial_state"])
+    st = d["initial_state"].clone()
+    o2, f2 = kda.kda_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], inp.scale, d["cu_seqlens"], st, final_state=st)
+    torch.cuda.synchronize()
+    assert f2.data_ptr() == st.data_ptr()
+    assert torch.equal(o1, o2) and torch.equal(f1, st)
+
+
+def test_deterministic(kda):
+    import torch
+
+    inp = kda_inputs.make_inputs([500, 3, 260], 4, seed=15, random_initial_state=True)
+    a = H.run_gpu(inp)
+    b = H.run_gpu(inp)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_no_writes_outside_outputs(kda):
+    """Guard regions around out and final_state keep their sentinel values."""
+    import torch
+
+    inp = kda_inputs.make_inputs([70, 0, 33], 2, seed=16, random_initial_state=True)
+    d = H.to_device(inp)
+    T, nh = inp.total_tokens, inp.num_heads
+    guard = 4096
+    ob = torch.full((T * nh * 128 + 2 * guard,), 7.0, dtype=torch.bfloat16, device="cuda")
+    fb = torch.full((3 * nh * 128 * 128 + 2 * guard,), 7.0, dtype=torch.float32, device="cuda")
+    out = ob[guard:guard + T * nh * 128].view(T, nh, 128)
+    fin = fb[guard:guard + 3 * nh * 128 * 128].view(3, nh, 128, 128)
+    kda.kda_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], inp.scale, d["cu_seqlens"], d["initial_state"],
+                out=out, final_state=fin)
+    torch.cuda.synchronize()
+    for buf in (ob, fb):
+        assert bool((buf[:guard] == 7.0).all()) and bool((buf[-guard:] == 7.0).all())
+
+
+# --------------------------------------------------------------- full sizes
+# The five workloads at their full sizes, in the launch configuration the
+# bench times; the oracle computes a sample of value columns (columns evolve
+# independently, so a column subset is exact) for every token and head.
+@pytest.mark.parametrize("cfg", [2, 3, 4, 5])
+def test_full_size_workloads_sampled_columns(kda, oracle_mod, cfg):
+    inp = kda_inputs.workload(cfg).make()
+    cols = slice(40, 56) if cfg != 5 else slice(100, 108)
+    mo, ms = _check(oracle_mod, inp, f"config {cfg}", cols=cols)
+    print(f"config {cfg}", mo, ms)
