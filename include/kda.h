@@ -76,7 +76,8 @@ typedef enum kda_status {
  *   scale          the output scale (usually 1/sqrt(128)).
  * Alignment: every tensor pointer must be 16-byte aligned.
  * Zero-length sequences are allowed: their final state equals their initial
- * state (or zeros). T = 0 is allowed.
+ * state (or zeros). T = 0 is allowed; then q, k, v, g, beta and out may be
+ * NULL (they are never read or written).
  * Returns KDA_OK once the work is enqueued.
  */
 kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,

@@ -286,45 +286,66 @@ __global__ void __launch_bounds__(NTHREADS, 1) kda_fwd_chunked_kernel(const Para
     __syncthreads();
 
     // ================= phase 2: masked A (-> L = diag(beta) A) and Aqk blocks
-    for (int pr = warp; pr < NB * (NB + 1) / 2; pr += NWARPS) {
-      int I = 0, J = pr;
-      while (J > I) {
-        ++I;
-        J -= I;
-      }
-      // now pr = I*(I+1)/2 + J with J <= I
-      float accA[2][4] = {}, accQ[2][4] = {};
-      const float* pf = sPf + (I * NB + J) * D;
+    // Each warp owns at most two of the NB*(NB+1)/2 lower block pairs. L lives
+    // in the storage of QL, which other warps may still be reading, so every
+    // warp keeps its products in registers until all reads are done.
+    {
+      constexpr int kPairs = NB * (NB + 1) / 2;
+      float accA[2][2][4] = {}, accQ[2][2][4] = {};
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        uint32_t a[4], aq[4], b[4];
-        ldsm_x4(a, sKL + (16 * I + (lane & 15)) * LDK + 16 * kk + (lane >> 4) * 8);
-        ldsm_x4(aq, sQL + (16 * I + (lane & 15)) * LDK + 16 * kk + (lane >> 4) * 8);
-        ldsm_x4(b, sKF + (16 * J + (lane & 7) + ((lane >> 4) << 3)) * LDK + 16 * kk + ((lane >> 3) & 1) * 8);
-        const float2 f01 = *reinterpret_cast<const float2*>(pf + 16 * kk + 2 * tq);
-        const float2 f23 = *reinterpret_cast<const float2*>(pf + 16 * kk + 8 + 2 * tq);
-        a[0] = scale_bf16x2(a[0], f01.x, f01.y);
-        a[1] = scale_bf16x2(a[1], f01.x, f01.y);
-        a[2] = scale_bf16x2(a[2], f23.x, f23.y);
-        a[3] = scale_bf16x2(a[3], f23.x, f23.y);
-        aq[0] = scale_bf16x2(aq[0], f01.x, f01.y);
-        aq[1] = scale_bf16x2(aq[1], f01.x, f01.y);
-        aq[2] = scale_bf16x2(aq[2], f23.x, f23.y);
-        aq[3] = scale_bf16x2(aq[3], f23.x, f23.y);
-        mma_bf16(accA[0], a, b[0], b[1]);
-        mma_bf16(accA[1], a, b[2], b[3]);
-        mma_bf16(accQ[0], aq, b[0], b[1]);
-        mma_bf16(accQ[1], aq, b[2], b[3]);
-      }
+      for (int slot = 0; slot < 2; ++slot) {
+        const int pr = warp + slot * NWARPS;
+        if (pr < kPairs) {
+          int I = 0, J = pr;  // pr = I*(I+1)/2 + J with J <= I
+          while (J > I) {
+            ++I;
+            J -= I;
+          }
+          const float* pf = sPf + (I * NB + J) * D;
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = 16 * I + gq + (e >> 1) * 8;
-          const int j = 16 * J + 8 * nt + 2 * tq + (e & 1);
-          sL[i * LDF + j] = (j < i) ? sBeta[i] * accA[nt][e] : 0.f;
-          sAqk[i * LDC + j] = __float2bfloat16_rn((j <= i) ? accQ[nt][e] : 0.f);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            uint32_t a[4], aq[4], b[4];
+            ldsm_x4(a, sKL + (16 * I + (lane & 15)) * LDK + 16 * kk + (lane >> 4) * 8);
+            ldsm_x4(aq, sQL + (16 * I + (lane & 15)) * LDK + 16 * kk + (lane >> 4) * 8);
+            ldsm_x4(b, sKF + (16 * J + (lane & 7) + ((lane >> 4) << 3)) * LDK + 16 * kk + ((lane >> 3) & 1) * 8);
+            const float2 f01 = *reinterpret_cast<const float2*>(pf + 16 * kk + 2 * tq);
+            const float2 f23 = *reinterpret_cast<const float2*>(pf + 16 * kk + 8 + 2 * tq);
+            a[0] = scale_bf16x2(a[0], f01.x, f01.y);
+            a[1] = scale_bf16x2(a[1], f01.x, f01.y);
+            a[2] = scale_bf16x2(a[2], f23.x, f23.y);
+            a[3] = scale_bf16x2(a[3], f23.x, f23.y);
+            aq[0] = scale_bf16x2(aq[0], f01.x, f01.y);
+            aq[1] = scale_bf16x2(aq[1], f01.x, f01.y);
+            aq[2] = scale_bf16x2(aq[2], f23.x, f23.y);
+            aq[3] = scale_bf16x2(aq[3], f23.x, f23.y);
+            mma_bf16(accA[slot][0], a, b[0], b[1]);
+            mma_bf16(accA[slot][1], a, b[2], b[3]);
+            mma_bf16(accQ[slot][0], aq, b[0], b[1]);
+            mma_bf16(accQ[slot][1], aq, b[2], b[3]);
+          }
         }
+      }
+      __syncthreads();
+#pragma unroll
+      for (int slot = 0; slot < 2; ++slot) {
+        const int pr = warp + slot * NWARPS;
+        if (pr < kPairs) {
+          int I = 0, J = pr;
+          while (J > I) {
+            ++I;
+            J -= I;
+          }
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int i = 16 * I + gq + (e >> 1) * 8;
+              const int j = 16 * J + 8 * nt + 2 * tq + (e & 1);
+              sL[i * LDF + j] = (j < i) ? sBeta[i] * accA[slot][nt][e] : 0.f;
+              sAqk[i * LDC + j] = __float2bfloat16_rn((j <= i) ? accQ[slot][nt][e] : 0.f);
+            }
+        }
+      }
     }
     __syncthreads();
 
@@ -567,8 +588,8 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* g
                      int32_t num_heads, const float* initial_state, void* out, float* final_state,
                      void* stream) {
   g_last_cuda_error[0] = '\0';
-  if (!q || !k || !v || !g || !beta || !out) return KDA_ERR_NULL;
   if (total_tokens < 0 || num_heads < 1 || num_seqs < 1) return KDA_ERR_SHAPE;
+  if (total_tokens > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_NULL;
   if (!cu_seqlens && num_seqs != 1) return KDA_ERR_SHAPE;
   if (num_heads > 65535 || num_seqs > 65535) return KDA_ERR_SHAPE;  // grid.y / grid.z limits
   if (total_tokens > (int64_t(1) << 40) / (int64_t(num_heads) * KDA_HEAD_DIM)) return KDA_ERR_SHAPE;

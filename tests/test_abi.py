@@ -54,6 +54,9 @@ def _call(lib, q=0x1000, k=0x2000, v=0x3000, g=0x4000, beta=0x5000, scale=1.0, c
 def test_rejects_null_pointers(lib):
     for name in ("q", "k", "v", "g", "beta", "out"):
         assert _call(lib, **{name: None}) == 1, name
+        # with T = 0 the token tensors are never touched, so NULL is fine; the
+        # call then goes on to a misaligned init pointer and stops there
+        assert _call(lib, T=0, init=0x8008, **{name: None}) == 3, name
 
 
 def test_rejects_bad_shapes(lib):
