@@ -1,38 +1,45 @@
-// kda_fwd.cu -- chunked Kimi Delta Attention forward for sm_100a.
+// kda_fwd.cu -- chunked Kimi Delta Attention forward (prefill) for sm_100a.
 //
-// One CTA owns one (sequence, head, value-column slice) work item and walks the
-// sequence chunk by chunk, carrying the fp32 state slice in registers.
-// Columns of the state evolve independently (the recurrence multiplies S only
-// from the left), so slicing the value columns needs no exchange between CTAs.
+// Work decomposition
+//   One CTA per (sequence, head, 32-column value slice). Columns of the state
+//   evolve independently (the recurrence multiplies S only from the left), so
+//   slices never exchange data. Inside a CTA, warps specialise:
+//     warps 0-3  "chain":  the serial state recurrence. Warp w owns the state
+//                transpose S^T[16 value rows x 64 key columns]: value block
+//                w>>1 (16 of the 32 columns) and key half w&1. The state lives
+//                in mma.sync accumulator registers (fp32) for the whole sequence
+//                and doubles, after a bf16 conversion, as the A operand of the
+//                next chunk's products, so it never touches shared memory.
+//     warps 4-7  "gate":   one key channel per thread. Per chunk they turn the
+//                gates into decay factors and write the chunk operands; then
+//                each warp computes one 16x8 block of A or Aqk.
+//     warp  8    "solver": (I + L)^{-1} by forward substitution, T diag(beta),
+//                and the value-slice tile.
+//   Producers run up to NSTAGE chunks ahead of the chain through a ring of
+//   shared-memory stages guarded by mbarriers.
 //
-// Per chunk of C tokens (chunk-local cumulative log-decay G_i, inclusive):
-//   A[i][j]   = sum_c k_i[c] k_j[c] exp(G_i[c] - G_j[c])     (j < i)
-//   T         = (I + diag(beta) A)^{-1}
-//   W         = T diag(beta) (k * exp G)          U = T diag(beta) V
-//   Vnew      = U - W S
-//   Aqk[i][j] = sum_c q_i[c] k_j[c] exp(G_i[c] - G_j[c])     (j <= i)
-//   O         = scale (Qd S + Aqk Vnew)           Qd = q * exp G
-//   S        <- Diag(exp G_last) S + Kend^T Vnew  Kend_j = k_j * exp(G_last - G_j)
-// Chunking a delta-rule recurrence into small dense products with one state
-// chain across chunks follows the FlashKDA description (page "Kimi K3 开源满月…",
-// section "KDA 内核到底难在哪"); the chunk is 64 tokens here.
+// Per chunk of C = 16 tokens, with Gamma_i the inclusive cumulative log-decay
+// inside the chunk (e_i = exp(g_i) per channel):
+//   E_i = prod_{s<=i} e_s = exp(Gamma_i),  F_i = prod_{s>i} e_s = exp(Gamma_last - Gamma_i)
+//   Kd = k*E,  Qd = q*E,  KR = k*F/gamma = k*exp(-Gamma),  Kend = k*F,  gamma = E_last
+//   A   = tril(Kd KR^T, -1),  L = diag(beta) A,  Aqk = tril(Qd KR^T)
+//   Tb  = (I + L)^{-1} diag(beta)
+//   X   = V - Kd S,   Vnew = Tb X          (the chunk's delta-rule writes)
+//   O   = scale (Qd S + Aqk Vnew)
+//   S  <- Diag(gamma) S + Kend^T Vnew
+// All factors stay in [e^-80, e^80] because -5 <= g <= 0 and a chunk has 16
+// tokens; this is the bound that lets FlashKDA keep 16-token causal blocks on
+// dense tensor-core products (page "Kimi K3 开源满月…", section
+// "KDA 内核到底难在哪": 16-token chunks, lower_bound = -5). The chain works
+// on S^T so that every product on it takes the register-resident state as
+// its A operand: X^T = V^T - S^T Kd^T, Vnew^T = X^T Tb^T,
+// S^T <- S^T Diag(gamma) + Vnew^T Kend.
 //
-// Exponent range. With -5 <= g <= 0 a 16-token sub-block spans at most a
-// factor e^80 (< FLT_MAX ~ e^88.7), the bound that lets FlashKDA keep every
-// causal block on dense tensor-core products (same page and section:
-// lower_bound = -5). Factors are therefore anchored per 16-token sub-block:
-// with R_b the cumulative log-decay at the start of sub-block b,
-//   E_i = exp(G_i - R_I)       in [e^-80, 1]     (row i in sub-block I)
-//   F_j = exp(R_{J+1} - G_j)   in [e^-80, 1]     (row j in sub-block J)
-//   exp(G_i - G_j) = E_i * exp(R_I - R_{J+1}) * F_j   for J <= I,
-// where the middle per-channel factor is <= 1 for J < I and <= e^80 for J = I.
-// Masked (upper) entries are removed by selection, never by multiplying by 0.
-// A chunk-wide anchor plays the same role in the B200 kernel described on the
-// same page (section "反转二", chunk 32 with an anchor scalar).
-//
-// Tensor-core work uses mma.sync m16n8k16 (bf16 in, fp32 accumulate); the
-// unit-lower inverse is fp32 on the CUDA cores (forward substitution on the
-// 16 x 16 diagonal blocks, block substitution for the rest).
+// Tensor cores: mma.sync m16n8k16 (bf16 in, fp32 accumulate). On this part a
+// dependent m16n8k16 completes in ~21 cycles while a tcgen05.mma of the shapes
+// this recurrence has (M <= 128, N <= 128, K = 16) costs ~90 cycles of issue
+// plus a ~250-cycle commit/mbarrier round trip; the chain is a serial sequence
+// of such small products, so it stays on the synchronous path.
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -45,76 +52,120 @@
 
 namespace kda {
 
-constexpr int D = KDA_HEAD_DIM;  // dk = dv = 128
-constexpr int C = 64;            // chunk length (tokens)
-constexpr int BS = 16;           // anchoring sub-block (tokens)
-constexpr int NB = C / BS;       // sub-blocks per chunk
-constexpr int NS = 64;           // value columns per CTA
-constexpr int NSLICE = D / NS;   // CTAs per (sequence, head)
-constexpr int NTHREADS = 256;
-constexpr int NWARPS = NTHREADS / 32;
+constexpr int D = KDA_HEAD_DIM;   // dk = dv = 128
+constexpr int C = 16;             // chunk length (tokens)
+constexpr int NS = 32;            // value columns per CTA
+constexpr int NSLICE = D / NS;    // CTAs per (sequence, head)
+constexpr int NSTAGE = 4;         // producer look-ahead (chunks)
+constexpr int NCHAIN = 4;         // chain warps
+constexpr int NGATE = 4;          // gate warps (one key channel per thread)
+constexpr int NTHREADS = (NCHAIN + NGATE + 1) * 32;
+constexpr int GATE_T0 = NCHAIN * 32;  // first gate thread
 
-// Padded row strides (elements). Row pitches of 272 / 144 bytes shift
-// successive rows by 4 banks, so 8-row ldmatrix reads are conflict-free.
-constexpr int LDK = D + 8;   // bf16 [C][D] tiles
-constexpr int LDN = NS + 8;  // bf16 [*][NS] tiles
-constexpr int LDC = C + 8;   // bf16 [C][C] tiles
-constexpr int LDF = C + 4;   // fp32 [C][C] tiles
+// Padded row pitches: 272 B, 48 B and 80 B rows keep 8-row ldmatrix reads on
+// distinct banks.
+constexpr int LDK = D + 8;
+constexpr int LDC = C + 8;
+constexpr int LDV = NS + 8;
 
-static_assert(NWARPS == 8, "warp roles below assume 8 warps");
-static_assert(NB == 4 && C == 64 && NS == 64, "tile mapping below assumes C = NS = 64");
-
-// Shared-memory plan (bytes). Buffers whose lifetimes do not overlap share
-// storage: W reuses KL, L reuses QL, T reuses KF.
-struct Smem {
-  static constexpr int kTileK = C * LDK * 2;       // 17408
-  static constexpr int kTileCF = C * LDF * 4;      // 17408
-  static constexpr int kTileC = C * LDC * 2;       // 9216
-  static constexpr int kTileN = C * LDN * 2;       // 9216
-  static constexpr int kS = D * LDN * 2;           // 18432
-  static constexpr int oKL = 0;                    // bf16 k*E        -> W
-  static constexpr int oQL = oKL + kTileK;         // bf16 q*E        -> L (fp32)
-  static constexpr int oKF = oQL + kTileK;         // bf16 k*F        -> T (fp32)
-  static constexpr int oKd = oKF + kTileK;         // bf16 k*exp(G)
-  static constexpr int oQd = oKd + kTileK;         // bf16 q*exp(G)
-  static constexpr int oKe = oQd + kTileK;         // bf16 k*exp(G_last - G)
-  static constexpr int oTb = oKe + kTileK;         // bf16 T diag(beta)
-  static constexpr int oAqk = oTb + kTileC;        // bf16 masked Aqk
-  static constexpr int oV = oAqk + kTileC;         // bf16 V slice
-  static constexpr int oVn = oV + kTileN;          // bf16 Vnew slice
-  static constexpr int oS = oVn + kTileN;          // bf16 copy of the state slice
-  static constexpr int oPf = oS + kS;              // fp32 [NB][NB][D] pair factors
-  static constexpr int oTmp = oPf + NB * NB * D * 4;  // fp32 [3][16][16] block products
-  static constexpr int oGam = oTmp + 3 * 16 * 16 * 4; // fp32 [D] chunk decay
-  static constexpr int oBeta = oGam + D * 4;       // fp32 [C]
-  static constexpr int kBytes = oBeta + C * 4;
+struct __align__(16) Stage {
+  __nv_bfloat16 kd[C][LDK];
+  __nv_bfloat16 qd[C][LDK];
+  __nv_bfloat16 kr[C][LDK];
+  __nv_bfloat16 ke[C][LDK];
+  __nv_bfloat16 tb[C][LDC];
+  __nv_bfloat16 aqk[C][LDC];
+  __nv_bfloat16 v[C][LDV];
+  float L[C][C + 1];
+  float gam[D];
+  float beta[C];
 };
-static_assert(Smem::kBytes <= 227 * 1024, "shared memory budget");
+
+struct __align__(16) Shared {
+  Stage st[NSTAGE];
+  float xbuf[2][2][32][8];   // X^T partial sums exchanged inside a chain-warp pair
+  float obuf[2][2][32][4];   // O^T partial sums exchanged inside a chain-warp pair
+  unsigned long long full[NSTAGE];       // solver -> chain
+  unsigned long long gate_done[NSTAGE];  // gate -> solver
+  unsigned long long empty[NSTAGE];      // chain -> gate
+};
+static_assert(sizeof(Stage) % 16 == 0, "stage alignment");
+static_assert(sizeof(Shared) <= 227 * 1024, "shared memory budget");
+
+// Wait budget for every mbarrier wait (cycles). A wait that runs out records
+// a timeout and lets the thread continue, so no barrier is ever left waiting.
+constexpr long long kWaitCycles = 4ll << 30;
+__device__ unsigned int g_wait_timeouts = 0;
 
 // ---------------------------------------------------------------- primitives
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+__device__ __forceinline__ void mbar_init(unsigned long long* m, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(m)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(unsigned long long* m) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(m)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(unsigned long long* m, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(smem_u32(m)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ void mbar_wait(unsigned long long* m, uint32_t parity) {
+  if (mbar_try_wait(m, parity)) return;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(m, parity)) {
+    if (clock64() - t0 > kWaitCycles) {
+      atomicAdd(&g_wait_timeouts, 1u);
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
+}
+
+__device__ __forceinline__ void ldsm_x2(uint32_t (&r)[2], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
                : "r"(smem_u32(p)));
 }
 
 __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(smem_u32(p)));
 }
 
-// D += A(16x16, row) * B(16x8, col); bf16 inputs, fp32 accumulate.
-__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+// D += A(16x16 row-major fragment) * B(16x8 column fragment); bf16 in, fp32 acc.
+__device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};\n"
+      "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -124,18 +175,14 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return u;
 }
 
-__device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
-  __nv_bfloat162 h;
-  memcpy(&h, &u, 4);
-  return __bfloat1622float2(h);
+// A fragment (16 rows x 16 k) from two accumulator tiles (16 rows x 8 cols each)
+// holding k columns [0, 8) and [8, 16).
+__device__ __forceinline__ void acc_to_afrag(uint32_t (&a)[4], const float (&lo)[4], const float (&hi)[4]) {
+  a[0] = pack_bf16(lo[0], lo[1]);
+  a[1] = pack_bf16(lo[2], lo[3]);
+  a[2] = pack_bf16(hi[0], hi[1]);
+  a[3] = pack_bf16(hi[2], hi[3]);
 }
-
-__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t u, float s0, float s1) {
-  float2 f = unpack_bf16(u);
-  return pack_bf16(f.x * s0, f.y * s1);
-}
-
-__device__ __forceinline__ float bf16_to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 
 // ---------------------------------------------------------------- the kernel
 struct Params {
@@ -144,42 +191,26 @@ struct Params {
   const __nv_bfloat16* v;
   const float* g;
   const float* beta;
-  const int32_t* cu;       // may be null: one sequence [0, T)
-  const float* init;       // may be null
+  const int32_t* cu;   // may be null: one sequence [0, T)
+  const float* init;   // may be null
   __nv_bfloat16* out;
-  float* fin;              // may be null
+  float* fin;          // may be null
   int64_t T;
   int32_t H;
-  int32_t nseq;
   float scale;
 };
 
-__global__ void __launch_bounds__(NTHREADS, 1) kda_fwd_chunked_kernel(const Params p) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  __nv_bfloat16* sKL = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oKL);
-  __nv_bfloat16* sW = sKL;
-  __nv_bfloat16* sQL = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oQL);
-  float* sL = reinterpret_cast<float*>(smem + Smem::oQL);
-  __nv_bfloat16* sKF = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oKF);
-  float* sT = reinterpret_cast<float*>(smem + Smem::oKF);
-  __nv_bfloat16* sKd = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oKd);
-  __nv_bfloat16* sQd = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oQd);
-  __nv_bfloat16* sKe = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oKe);
-  __nv_bfloat16* sTb = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oTb);
-  __nv_bfloat16* sAqk = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oAqk);
-  __nv_bfloat16* sV = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oV);
-  __nv_bfloat16* sVn = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oVn);
-  __nv_bfloat16* sS = reinterpret_cast<__nv_bfloat16*>(smem + Smem::oS);
-  float* sPf = reinterpret_cast<float*>(smem + Smem::oPf);
-  float* sTmp = reinterpret_cast<float*>(smem + Smem::oTmp);
-  float* sGam = reinterpret_cast<float*>(smem + Smem::oGam);
-  float* sBeta = reinterpret_cast<float*>(smem + Smem::oBeta);
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
+
+__global__ void __launch_bounds__(NTHREADS, 1) kda_fwd_kernel(const Params p) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  Shared& sh = *reinterpret_cast<Shared*>(smem_raw);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int gq = lane >> 2;  // mma fragment row group
-  const int tq = lane & 3;   // mma fragment column pair
+  const int gq = lane >> 2;  // fragment row group
+  const int tq = lane & 3;   // fragment column pair
 
   const int slice = blockIdx.x;
   const int h = blockIdx.y;
@@ -187,6 +218,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) kda_fwd_chunked_kernel(const Para
   const int dv0 = slice * NS;
   const int H = p.H;
   const int64_t T = p.T;
+  const size_t row_stride = static_cast<size_t>(H) * D;  // elements between tokens of q/k/v/g/out
 
   int64_t t0 = 0, t1 = T;
   if (p.cu) {
@@ -195,349 +227,286 @@ __global__ void __launch_bounds__(NTHREADS, 1) kda_fwd_chunked_kernel(const Para
     t0 = t0 < 0 ? 0 : (t0 > T ? T : t0);
     t1 = t1 < t0 ? t0 : (t1 > T ? T : t1);
   }
+  const int nch = static_cast<int>((t1 - t0 + C - 1) / C);
 
-  // ---- state slice: fp32 master in registers (mma accumulator layout of the
-  // rows 16*warp..16*warp+15 x all NS columns), bf16 copy in shared memory.
-  float sreg[NS / 8][4];
-  {
-    const size_t sbase = (static_cast<size_t>(seq) * H + h) * D * D;
-#pragma unroll
-    for (int nt = 0; nt < NS / 8; ++nt) {
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int r = 16 * warp + gq + 8 * half;
-        const int c = 8 * nt + 2 * tq;
-        float2 x = make_float2(0.f, 0.f);
-        if (p.init) x = *reinterpret_cast<const float2*>(p.init + sbase + static_cast<size_t>(r) * D + dv0 + c);
-        sreg[nt][2 * half] = x.x;
-        sreg[nt][2 * half + 1] = x.y;
-        *reinterpret_cast<uint32_t*>(sS + r * LDN + c) = pack_bf16(x.x, x.y);
-      }
+  if (tid == 0) {
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(&sh.full[s], 32);
+      mbar_init(&sh.gate_done[s], NGATE * 32);
+      mbar_init(&sh.empty[s], NCHAIN * 32);
     }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
 
-  const size_t row_stride = static_cast<size_t>(H) * D;  // elements between tokens
-
-  for (int64_t cs = t0; cs < t1; cs += C) {
-    const int m = static_cast<int>((t1 - cs) < C ? (t1 - cs) : C);  // valid rows
-
-    // ================= phase 1: gates, anchored factors, operands; V slice
-    if (tid < D) {
-      const int c = tid;
-      float gl[C];
+  if (warp < NCHAIN) {
+    // =========================================================== chain warps
+    const int pr = warp >> 1;          // value block (16 columns) inside the slice
+    const int dh = warp & 1;           // key half
+    const int k0 = 64 * dh;            // first key channel of this warp
+    const int vrow = 16 * pr;          // first value column (slice-local)
+    // S^T fragment: rows = value columns vrow + gq (+8), cols = key channels
+    // k0 + 8*nt + 2*tq (+1), nt = 0..7.
+    float sT[8][4];
+    const size_t sbase = (static_cast<size_t>(seq) * H + h) * D * D;
 #pragma unroll
-      for (int i = 0; i < C; ++i)
-        gl[i] = (i < m) ? __ldg(p.g + (cs + i) * row_stride + static_cast<size_t>(h) * D + c) : 0.f;
-      float R[NB + 1];
-      R[0] = 0.f;
+    for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        float s = 0.f;
-#pragma unroll
-        for (int i = 0; i < BS; ++i) {
-          s += gl[BS * b + i];
-          gl[BS * b + i] = s;  // now: cumulative log-decay within the sub-block
-        }
-        R[b + 1] = R[b] + s;
+      for (int e = 0; e < 4; ++e) {
+        const int dv = dv0 + vrow + gq + 8 * (e >> 1);
+        const int dk = k0 + 8 * nt + 2 * tq + (e & 1);
+        sT[nt][e] = p.init ? __ldg(p.init + sbase + static_cast<size_t>(dk) * D + dv) : 0.f;
       }
-#pragma unroll
-      for (int I = 0; I < NB; ++I)
-#pragma unroll
-        for (int J = 0; J <= I; ++J) sPf[(I * NB + J) * D + c] = __expf(R[I] - R[J + 1]);
-      sGam[c] = __expf(R[NB]);
-#pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        const float eR = __expf(R[b]);
-        const float eEnd = __expf(R[NB] - R[b + 1]);
-        const float bsum = R[b + 1] - R[b];
-#pragma unroll
-        for (int i = 0; i < BS; ++i) {
-          const int row = BS * b + i;
-          float kv = 0.f, qv = 0.f;
-          if (row < m) {
-            const size_t off = (cs + row) * row_stride + static_cast<size_t>(h) * D + c;
-            kv = bf16_to_f32(p.k[off]);
-            qv = bf16_to_f32(p.q[off]);
-          }
-          const float E = __expf(gl[row]);
-          const float F = __expf(bsum - gl[row]);
-          sKL[row * LDK + c] = __float2bfloat16_rn(kv * E);
-          sQL[row * LDK + c] = __float2bfloat16_rn(qv * E);
-          sKF[row * LDK + c] = __float2bfloat16_rn(kv * F);
-          sKd[row * LDK + c] = __float2bfloat16_rn(kv * (E * eR));
-          sQd[row * LDK + c] = __float2bfloat16_rn(qv * (E * eR));
-          sKe[row * LDK + c] = __float2bfloat16_rn(kv * (F * eEnd));
-        }
-      }
-    } else {
-      const int t = tid - D;  // 128 threads: V slice (C x NS bf16, 16-byte pieces) and beta
-      constexpr int kPieces = C * NS / 8;
-      for (int idx = t; idx < kPieces; idx += NTHREADS - D) {
-        const int row = idx / (NS / 8);
-        const int col = (idx % (NS / 8)) * 8;
-        uint4 x = make_uint4(0, 0, 0, 0);
-        if (row < m)
-          x = __ldg(reinterpret_cast<const uint4*>(p.v + (cs + row) * row_stride + static_cast<size_t>(h) * D + dv0 + col));
-        *reinterpret_cast<uint4*>(sV + row * LDN + col) = x;
-      }
-      if (t < C) sBeta[t] = (t < m) ? __ldg(p.beta + (cs + t) * H + h) : 0.f;
-    }
-    __syncthreads();
 
-    // ================= phase 2: masked A (-> L = diag(beta) A) and Aqk blocks
-    // Each warp owns at most two of the NB*(NB+1)/2 lower block pairs. L lives
-    // in the storage of QL, which other warps may still be reading, so every
-    // warp keeps its products in registers until all reads are done.
-    {
-      constexpr int kPairs = NB * (NB + 1) / 2;
-      float accA[2][2][4] = {}, accQ[2][2][4] = {};
+    for (int n = 0; n < nch; ++n) {
+      const int s = n % NSTAGE;
+      const uint32_t ph = static_cast<uint32_t>(n / NSTAGE) & 1u;
+      const int64_t cs = t0 + static_cast<int64_t>(n) * C;
+      const int m = static_cast<int>((t1 - cs) < C ? (t1 - cs) : C);
+      Stage& st = sh.st[s];
+      mbar_wait(&sh.full[s], ph);
+
+      // ---- X^T = V^T - S^T Kd^T and O^T = S^T Qd^T over this warp's key half
+      float x[2][4], o[2][4];
 #pragma unroll
-      for (int slot = 0; slot < 2; ++slot) {
-        const int pr = warp + slot * NWARPS;
-        if (pr < kPairs) {
-          int I = 0, J = pr;  // pr = I*(I+1)/2 + J with J <= I
-          while (J > I) {
-            ++I;
-            J -= I;
-          }
-          const float* pf = sPf + (I * NB + J) * D;
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            uint32_t a[4], aq[4], b[4];
-            ldsm_x4(a, sKL + (16 * I + (lane & 15)) * LDK + 16 * kk + (lane >> 4) * 8);
-            ldsm_x4(aq, sQL + (16 * I + (lane & 15)) * LDK + 16 * kk + (lane >> 4) * 8);
-            ldsm_x4(b, sKF + (16 * J + (lane & 7) + ((lane >> 4) << 3)) * LDK + 16 * kk + ((lane >> 3) & 1) * 8);
-            const float2 f01 = *reinterpret_cast<const float2*>(pf + 16 * kk + 2 * tq);
-            const float2 f23 = *reinterpret_cast<const float2*>(pf + 16 * kk + 8 + 2 * tq);
-            a[0] = scale_bf16x2(a[0], f01.x, f01.y);
-            a[1] = scale_bf16x2(a[1], f01.x, f01.y);
-            a[2] = scale_bf16x2(a[2], f23.x, f23.y);
-            a[3] = scale_bf16x2(a[3], f23.x, f23.y);
-            aq[0] = scale_bf16x2(aq[0], f01.x, f01.y);
-            aq[1] = scale_bf16x2(aq[1], f01.x, f01.y);
-            aq[2] = scale_bf16x2(aq[2], f23.x, f23.y);
-            aq[3] = scale_bf16x2(aq[3], f23.x, f23.y);
-            mma_bf16(accA[slot][0], a, b[0], b[1]);
-            mma_bf16(accA[slot][1], a, b[2], b[3]);
-            mma_bf16(accQ[slot][0], aq, b[0], b[1]);
-            mma_bf16(accQ[slot][1], aq, b[2], b[3]);
+        for (int e = 0; e < 4; ++e) {
+          o[nt][e] = 0.f;
+          x[nt][e] = 0.f;
+          if (dh == 0) {
+            const int tok = 8 * nt + 2 * tq + (e & 1);
+            const int col = vrow + gq + 8 * (e >> 1);
+            x[nt][e] = __bfloat162float(st.v[tok][col]);
           }
         }
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        uint32_t a[4], an[4], bk[4], bq[4];
+        acc_to_afrag(a, sT[2 * kk], sT[2 * kk + 1]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) an[e] = a[e] ^ 0x80008000u;  // -S^T (exact sign flip)
+        const int row = (lane & 7) + ((lane >> 4) << 3);
+        const int col = k0 + 16 * kk + ((lane >> 3) & 1) * 8;
+        ldsm_x4(bk, &st.kd[row][col]);
+        ldsm_x4(bq, &st.qd[row][col]);
+        mma(x[0], an, bk[0], bk[1]);
+        mma(x[1], an, bk[2], bk[3]);
+        mma(o[0], a, bq[0], bq[1]);
+        mma(o[1], a, bq[2], bq[3]);
       }
-      __syncthreads();
+      // ---- sum X^T over the two key halves (pair exchange)
+      {
+        float4* mine = reinterpret_cast<float4*>(&sh.xbuf[pr][dh][lane][0]);
+        mine[0] = make_float4(x[0][0], x[0][1], x[0][2], x[0][3]);
+        mine[1] = make_float4(x[1][0], x[1][1], x[1][2], x[1][3]);
+        named_bar(2 + pr, 64);
+        const float4* other = reinterpret_cast<const float4*>(&sh.xbuf[pr][dh ^ 1][lane][0]);
+        const float4 u0 = other[0], u1 = other[1];
+        x[0][0] += u0.x; x[0][1] += u0.y; x[0][2] += u0.z; x[0][3] += u0.w;
+        x[1][0] += u1.x; x[1][1] += u1.y; x[1][2] += u1.z; x[1][3] += u1.w;
+      }
+      // ---- Vnew^T = X^T Tb^T
+      float vn[2][4] = {};
+      uint32_t ax[4], av[4];
+      acc_to_afrag(ax, x[0], x[1]);
+      {
+        uint32_t bt[4];
+        ldsm_x4(bt, &st.tb[(lane & 7) + ((lane >> 4) << 3)][((lane >> 3) & 1) * 8]);
+        mma(vn[0], ax, bt[0], bt[1]);
+        mma(vn[1], ax, bt[2], bt[3]);
+      }
+      acc_to_afrag(av, vn[0], vn[1]);
+      // ---- O^T += Vnew^T Aqk^T (once per pair)
+      if (dh == 0) {
+        uint32_t ba[4];
+        ldsm_x4(ba, &st.aqk[(lane & 7) + ((lane >> 4) << 3)][((lane >> 3) & 1) * 8]);
+        mma(o[0], av, ba[0], ba[1]);
+        mma(o[1], av, ba[2], ba[3]);
+      }
+      // ---- S^T <- S^T Diag(gamma) + Vnew^T Kend   (this warp's key half)
 #pragma unroll
-      for (int slot = 0; slot < 2; ++slot) {
-        const int pr = warp + slot * NWARPS;
-        if (pr < kPairs) {
-          int I = 0, J = pr;
-          while (J > I) {
-            ++I;
-            J -= I;
-          }
+      for (int nt = 0; nt < 8; ++nt) {
+        const float2 gm = *reinterpret_cast<const float2*>(&st.gam[k0 + 8 * nt + 2 * tq]);
+        sT[nt][0] *= gm.x;
+        sT[nt][1] *= gm.y;
+        sT[nt][2] *= gm.x;
+        sT[nt][3] *= gm.y;
+      }
 #pragma unroll
-          for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int i = 16 * I + gq + (e >> 1) * 8;
-              const int j = 16 * J + 8 * nt + 2 * tq + (e & 1);
-              sL[i * LDF + j] = (j < i) ? sBeta[i] * accA[slot][nt][e] : 0.f;
-              sAqk[i * LDC + j] = __float2bfloat16_rn((j <= i) ? accQ[slot][nt][e] : 0.f);
-            }
+      for (int np = 0; np < 4; ++np) {
+        uint32_t be[4];
+        ldsm_x4_t(be, &st.ke[(lane & 7) + ((lane >> 3) & 1) * 8][k0 + 16 * np + (lane >> 4) * 8]);
+        mma(sT[2 * np], av, be[0], be[1]);
+        mma(sT[2 * np + 1], av, be[2], be[3]);
+      }
+      // the stage is no longer read by this thread
+      mbar_arrive(&sh.empty[s]);
+      // ---- O: each warp of the pair finishes one 8-token half
+      {
+        const int keep = dh, give = dh ^ 1;
+        *reinterpret_cast<float4*>(&sh.obuf[pr][dh][lane][0]) =
+            make_float4(o[give][0], o[give][1], o[give][2], o[give][3]);
+        named_bar(2 + pr, 64);
+        const float4 u = *reinterpret_cast<const float4*>(&sh.obuf[pr][dh ^ 1][lane][0]);
+        const float o0 = (o[keep][0] + u.x) * p.scale, o1 = (o[keep][1] + u.y) * p.scale;
+        const float o2 = (o[keep][2] + u.z) * p.scale, o3 = (o[keep][3] + u.w) * p.scale;
+        // fragment rows = value columns, cols = tokens -> transpose to token rows
+        const uint32_t r0 = movmatrix_t(pack_bf16(o0, o1));
+        const uint32_t r1 = movmatrix_t(pack_bf16(o2, o3));
+        const int tok = 8 * keep + gq;
+        if (tok < m) {
+          __nv_bfloat16* dst = p.out + (cs + tok) * row_stride + static_cast<size_t>(h) * D + dv0 + vrow + 2 * tq;
+          *reinterpret_cast<uint32_t*>(dst) = r0;
+          *reinterpret_cast<uint32_t*>(dst + 8) = r1;
         }
       }
     }
-    __syncthreads();
-
-    // ================= phase 3: T = (I + L)^{-1}, then Tb = T diag(beta)
-    if (warp < 2) {
-      // diagonal 16 x 16 blocks: one half-warp per block, one lane per column
-      const int I = 2 * warp + (lane >> 4);
-      const int col = lane & 15;
-      const float* Lb = sL + (16 * I) * LDF + 16 * I;
-      float x[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) x[i] = (i == col) ? 1.f : 0.f;
-#pragma unroll
-      for (int mm = 0; mm < 16; ++mm) {
-        const float xm = x[mm];
-#pragma unroll
-        for (int i = mm + 1; i < 16; ++i) x[i] = fmaf(-Lb[i * LDF + mm], xm, x[i]);
-      }
-      float* Tb = sT + (16 * I) * LDF + 16 * I;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) Tb[i * LDF + col] = x[i];
-    }
-    __syncthreads();
-    {
-      // off-diagonal blocks by distance d = I - J:
-      //   T_IJ = -T_II * sum_{K=J}^{I-1} L_IK T_KJ
-      const int r = tid >> 4, cc = tid & 15;
-      for (int d = 1; d < NB; ++d) {
-        for (int J = 0; J + d < NB; ++J) {
-          const int I = J + d;
-          float acc = 0.f;
-          for (int K = J; K < I; ++K) {
-            const float* Lr = sL + (16 * I + r) * LDF + 16 * K;
-            const float* Tc = sT + (16 * K) * LDF + 16 * J + cc;
-#pragma unroll
-            for (int mm = 0; mm < 16; ++mm) acc = fmaf(Lr[mm], Tc[mm * LDF], acc);
-          }
-          sTmp[J * 256 + r * 16 + cc] = acc;
-        }
-        __syncthreads();
-        for (int J = 0; J + d < NB; ++J) {
-          const int I = J + d;
-          const float* Tr = sT + (16 * I + r) * LDF + 16 * I;
-          float acc = 0.f;
-#pragma unroll
-          for (int mm = 0; mm < 16; ++mm) acc = fmaf(Tr[mm], sTmp[J * 256 + mm * 16 + cc], acc);
-          sT[(16 * I + r) * LDF + 16 * J + cc] = -acc;
-        }
-        __syncthreads();
-      }
-      // Tb = T diag(beta) in bf16, lower blocks only (the products below skip J > I)
-      for (int idx = tid; idx < C * C; idx += NTHREADS) {
-        const int i = idx / C, j = idx % C;
-        if ((j >> 4) <= (i >> 4)) sTb[i * LDC + j] = __float2bfloat16_rn(sT[i * LDF + j] * sBeta[j]);
-      }
-    }
-    __syncthreads();
-
-    // ================= phase 4: W = Tb Kd (all 128 channels), U = Tb V (slice)
-    const int I4 = warp >> 1;       // row sub-block of this warp (phases 4 and 5a/5b)
-    float uacc[4][4] = {};          // U tile: rows 16*I4.., columns (warp&1)*32 + 8*nt
-    {
-      const int ch = (warp & 1) * 64;
-      float acc[8][4] = {};
-      for (int J = 0; J <= I4; ++J) {
-        uint32_t a[4];
-        ldsm_x4(a, sTb + (16 * I4 + (lane & 15)) * LDC + 16 * J + (lane >> 4) * 8);
-#pragma unroll
-        for (int np = 0; np < 4; ++np) {
-          uint32_t b[4];
-          ldsm_x4_t(b, sKd + (16 * J + (lane & 7) + ((lane >> 3) & 1) * 8) * LDK + ch + 16 * np + (lane >> 4) * 8);
-          mma_bf16(acc[2 * np], a, b[0], b[1]);
-          mma_bf16(acc[2 * np + 1], a, b[2], b[3]);
-        }
-        const int nh = (warp & 1) * 32;
-#pragma unroll
-        for (int np = 0; np < 2; ++np) {
-          uint32_t b[4];
-          ldsm_x4_t(b, sV + (16 * J + (lane & 7) + ((lane >> 3) & 1) * 8) * LDN + nh + 16 * np + (lane >> 4) * 8);
-          mma_bf16(uacc[2 * np], a, b[0], b[1]);
-          mma_bf16(uacc[2 * np + 1], a, b[2], b[3]);
-        }
-      }
+    if (p.fin) {
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int i = 16 * I4 + gq + 8 * half;
-          const int c = ch + 8 * nt + 2 * tq;
-          *reinterpret_cast<uint32_t*>(sW + i * LDK + c) = pack_bf16(acc[nt][2 * half], acc[nt][2 * half + 1]);
+        for (int e = 0; e < 4; ++e) {
+          const int dv = dv0 + vrow + gq + 8 * (e >> 1);
+          const int dk = k0 + 8 * nt + 2 * tq + (e & 1);
+          p.fin[sbase + static_cast<size_t>(dk) * D + dv] = sT[nt][e];
         }
     }
-    __syncthreads();
+  } else if (warp < NCHAIN + NGATE) {
+    // ============================================================ gate warps
+    const int c = tid - GATE_T0;  // key channel
+    const int gw = warp - NCHAIN;
+    const size_t col_off = static_cast<size_t>(h) * D + c;
+    // raw inputs of the next chunk, prefetched into registers
+    float g_nx[C];
+    uint16_t k_nx[C], q_nx[C];
+    float b_nx = 0.f;
+    auto load_chunk = [&](int n) {
+      const int64_t cs = t0 + static_cast<int64_t>(n) * C;
+#pragma unroll
+      for (int i = 0; i < C; ++i) {
+        const bool ok = (n < nch) && (cs + i < t1);
+        const size_t off = (cs + i) * row_stride + col_off;
+        g_nx[i] = ok ? __ldg(p.g + off) : 0.f;
+        k_nx[i] = ok ? __ldg(reinterpret_cast<const unsigned short*>(p.k) + off) : static_cast<uint16_t>(0);
+        q_nx[i] = ok ? __ldg(reinterpret_cast<const unsigned short*>(p.q) + off) : static_cast<uint16_t>(0);
+      }
+      if (gw == 0 && lane < C) {
+        const bool ok = (n < nch) && (cs + lane < t1);
+        b_nx = ok ? __ldg(p.beta + (cs + lane) * H + h) : 0.f;
+      }
+    };
+    load_chunk(0);
+    for (int n = 0; n < nch; ++n) {
+      const int s = n % NSTAGE;
+      const uint32_t ph = static_cast<uint32_t>(n / NSTAGE) & 1u;
+      float gv[C], kv[C], qv[C];
+#pragma unroll
+      for (int i = 0; i < C; ++i) {
+        gv[i] = g_nx[i];
+        kv[i] = bf16_bits_to_f32(k_nx[i]);
+        qv[i] = bf16_bits_to_f32(q_nx[i]);
+      }
+      const float bv = b_nx;
+      load_chunk(n + 1);
+      Stage& st = sh.st[s];
+      mbar_wait(&sh.empty[s], ph ^ 1u);
 
-    // ================= phase 5a: Vnew = U - W S ; O = Qd S (same B fragments)
-    const int nh = (warp & 1) * 32;
-    float oacc[4][4] = {};
+      // ---- decay factors and operands for key channel c
+      float e[C];
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      uint32_t aw[4], aqd[4];
-      ldsm_x4(aw, sW + (16 * I4 + (lane & 15)) * LDK + 16 * kk + (lane >> 4) * 8);
-      ldsm_x4(aqd, sQd + (16 * I4 + (lane & 15)) * LDK + 16 * kk + (lane >> 4) * 8);
+      for (int i = 0; i < C; ++i) e[i] = __expf(gv[i]);
+      float E = 1.f;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) aw[e] ^= 0x80008000u;  // -W (exact sign flip)
-#pragma unroll
-      for (int np = 0; np < 2; ++np) {
-        uint32_t b[4];
-        ldsm_x4_t(b, sS + (16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8) * LDN + nh + 16 * np + (lane >> 4) * 8);
-        mma_bf16(uacc[2 * np], aw, b[0], b[1]);
-        mma_bf16(uacc[2 * np + 1], aw, b[2], b[3]);
-        mma_bf16(oacc[2 * np], aqd, b[0], b[1]);
-        mma_bf16(oacc[2 * np + 1], aqd, b[2], b[3]);
+      for (int i = 0; i < C; ++i) {
+        E *= e[i];
+        st.kd[i][c] = __float2bfloat16_rn(kv[i] * E);
+        st.qd[i][c] = __float2bfloat16_rn(qv[i] * E);
       }
-    }
+      const float gamma = E;
+      const float rgamma = __frcp_rn(gamma);
+      float F = 1.f;
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int i = 16 * I4 + gq + 8 * half;
-        const int c = nh + 8 * nt + 2 * tq;
-        *reinterpret_cast<uint32_t*>(sVn + i * LDN + c) = pack_bf16(uacc[nt][2 * half], uacc[nt][2 * half + 1]);
+      for (int i = C - 1; i >= 0; --i) {
+        const float kf = kv[i] * F;
+        st.ke[i][c] = __float2bfloat16_rn(kf);
+        st.kr[i][c] = __float2bfloat16_rn(kf * rgamma);
+        F *= e[i];
       }
-    __syncthreads();
+      st.gam[c] = gamma;
+      if (gw == 0 && lane < C) st.beta[lane] = bv;
+      named_bar(1, NGATE * 32);
 
-    // ================= phase 5b: O += Aqk Vnew ; store O
-    for (int J = 0; J <= I4; ++J) {
-      uint32_t a[4];
-      ldsm_x4(a, sAqk + (16 * I4 + (lane & 15)) * LDC + 16 * J + (lane >> 4) * 8);
+      // ---- one 16x8 block of A = Kd KR^T (gate warps 0,1) or Aqk = Qd KR^T (2,3)
+      {
+        const int mat = gw >> 1, nt = gw & 1;
+        const __nv_bfloat16(*src)[LDK] = mat ? st.qd : st.kd;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int np = 0; np < 2; ++np) {
-        uint32_t b[4];
-        ldsm_x4_t(b, sVn + (16 * J + (lane & 7) + ((lane >> 3) & 1) * 8) * LDN + nh + 16 * np + (lane >> 4) * 8);
-        mma_bf16(oacc[2 * np], a, b[0], b[1]);
-        mma_bf16(oacc[2 * np + 1], a, b[2], b[3]);
-      }
-    }
+        for (int kk = 0; kk < D / 16; ++kk) {
+          uint32_t a[4], b[2];
+          ldsm_x4(a, &src[lane & 15][16 * kk + (lane >> 4) * 8]);
+          ldsm_x2(b, &st.kr[8 * nt + (lane & 7)][16 * kk + ((lane >> 3) & 1) * 8]);
+          mma(acc, a, b[0], b[1]);
+        }
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int i = 16 * I4 + gq + 8 * half;
-        if (i < m) {
-          const int c = dv0 + nh + 8 * nt + 2 * tq;
-          *reinterpret_cast<uint32_t*>(p.out + (cs + i) * row_stride + static_cast<size_t>(h) * D + c) =
-              pack_bf16(p.scale * oacc[nt][2 * half], p.scale * oacc[nt][2 * half + 1]);
+        for (int e2 = 0; e2 < 4; ++e2) {
+          const int i = gq + 8 * (e2 >> 1);
+          const int j = 8 * nt + 2 * tq + (e2 & 1);
+          if (mat == 0)
+            st.L[i][j] = (j < i) ? st.beta[i] * acc[e2] : 0.f;
+          else
+            st.aqk[i][j] = __float2bfloat16_rn((j <= i) ? acc[e2] : 0.f);
         }
       }
-
-    // ================= phase 5c: S <- Diag(gamma) S + Kend^T Vnew (rows 16*warp..)
-    {
-      const float g0 = sGam[16 * warp + gq], g1 = sGam[16 * warp + gq + 8];
-#pragma unroll
-      for (int nt = 0; nt < NS / 8; ++nt) {
-        sreg[nt][0] *= g0;
-        sreg[nt][1] *= g0;
-        sreg[nt][2] *= g1;
-        sreg[nt][3] *= g1;
-      }
-#pragma unroll
-      for (int J = 0; J < NB; ++J) {
-        uint32_t a[4];
-        ldsm_x4_t(a, sKe + (16 * J + (lane & 7) + ((lane >> 4) << 3)) * LDK + 16 * warp + ((lane >> 3) & 1) * 8);
-#pragma unroll
-        for (int np = 0; np < NS / 16; ++np) {
-          uint32_t b[4];
-          ldsm_x4_t(b, sVn + (16 * J + (lane & 7) + ((lane >> 3) & 1) * 8) * LDN + 16 * np + (lane >> 4) * 8);
-          mma_bf16(sreg[2 * np], a, b[0], b[1]);
-          mma_bf16(sreg[2 * np + 1], a, b[2], b[3]);
-        }
-      }
-#pragma unroll
-      for (int nt = 0; nt < NS / 8; ++nt)
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int r = 16 * warp + gq + 8 * half;
-          *reinterpret_cast<uint32_t*>(sS + r * LDN + 8 * nt + 2 * tq) = pack_bf16(sreg[nt][2 * half], sreg[nt][2 * half + 1]);
-        }
+      mbar_arrive(&sh.gate_done[s]);
     }
-    __syncthreads();
-  }
-
-  if (p.fin) {
-    const size_t sbase = (static_cast<size_t>(seq) * H + h) * D * D;
+  } else {
+    // =========================================================== solver warp
+    // lanes 0-15: one column of (I + L)^{-1} each; lanes 16-31: value-slice tile
+    const int r = lane - 16;  // value-tile row for lanes 16-31
+    uint4 v_nx[NS / 8];
+    auto load_v = [&](int n) {
+      if (lane >= 16) {
+        const int64_t cs = t0 + static_cast<int64_t>(n) * C;
+        const bool ok = (n < nch) && (cs + r < t1);
 #pragma unroll
-    for (int nt = 0; nt < NS / 8; ++nt)
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int r = 16 * warp + gq + 8 * half;
-        const int c = 8 * nt + 2 * tq;
-        *reinterpret_cast<float2*>(p.fin + sbase + static_cast<size_t>(r) * D + dv0 + c) =
-            make_float2(sreg[nt][2 * half], sreg[nt][2 * half + 1]);
+        for (int j = 0; j < NS / 8; ++j)
+          v_nx[j] = ok ? __ldg(reinterpret_cast<const uint4*>(p.v + (cs + r) * row_stride +
+                                                              static_cast<size_t>(h) * D + dv0) + j)
+                       : make_uint4(0, 0, 0, 0);
       }
+    };
+    load_v(0);
+    for (int n = 0; n < nch; ++n) {
+      const int s = n % NSTAGE;
+      const uint32_t ph = static_cast<uint32_t>(n / NSTAGE) & 1u;
+      Stage& st = sh.st[s];
+      uint4 vcur[NS / 8];
+#pragma unroll
+      for (int j = 0; j < NS / 8; ++j) vcur[j] = v_nx[j];
+      load_v(n + 1);
+      mbar_wait(&sh.gate_done[s], ph);
+      if (lane < 16) {
+        const int col = lane;
+        float xs[C];
+#pragma unroll
+        for (int i = 0; i < C; ++i) xs[i] = (i == col) ? 1.f : 0.f;
+#pragma unroll
+        for (int mm = 0; mm < C; ++mm) {
+          const float xm = xs[mm];
+#pragma unroll
+          for (int i = mm + 1; i < C; ++i) xs[i] = fmaf(-st.L[i][mm], xm, xs[i]);
+        }
+        const float bc = st.beta[col];
+#pragma unroll
+        for (int i = 0; i < C; ++i) st.tb[i][col] = __float2bfloat16_rn(xs[i] * bc);
+      } else {
+#pragma unroll
+        for (int j = 0; j < NS / 8; ++j) *reinterpret_cast<uint4*>(&st.v[r][8 * j]) = vcur[j];
+      }
+      mbar_arrive(&sh.full[s]);
+    }
   }
 }
 
@@ -572,8 +541,8 @@ kda_status_t prepare_device(int dev) {
     g_device_ready[dev] = -1;
     return KDA_ERR_UNSUPPORTED;
   }
-  e = cudaFuncSetAttribute(kda::kda_fwd_chunked_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kda::Smem::kBytes);
+  e = cudaFuncSetAttribute(kda::kda_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(sizeof(kda::Shared)));
   if (e != cudaSuccess) return cuda_fail(e);
   g_device_ready[dev] = 1;
   return KDA_OK;
@@ -615,10 +584,9 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* g
   p.fin = final_state;
   p.T = total_tokens;
   p.H = num_heads;
-  p.nseq = num_seqs;
   p.scale = scale;
   dim3 grid(kda::NSLICE, num_heads, num_seqs);
-  kda::kda_fwd_chunked_kernel<<<grid, kda::NTHREADS, kda::Smem::kBytes, static_cast<cudaStream_t>(stream)>>>(p);
+  kda::kda_fwd_kernel<<<grid, kda::NTHREADS, sizeof(kda::Shared), static_cast<cudaStream_t>(stream)>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return KDA_OK;
