@@ -10,13 +10,16 @@
 //                in mma.sync accumulator registers (fp32) for the whole sequence
 //                and doubles, after a bf16 conversion, as the A operand of the
 //                next chunk's products, so it never touches shared memory.
-//     warps 4-7  "gate":   one key channel per thread. Per chunk they turn the
-//                gates into decay factors and write the chunk operands; then
-//                each warp computes one 16x8 block of A or Aqk.
-//     warp  8    "solver": (I + L)^{-1} by forward substitution, T diag(beta),
-//                and the value-slice tile.
-//   Producers run up to NSTAGE chunks ahead of the chain through a ring of
-//   shared-memory stages guarded by mbarriers.
+//     warps 4-7  "gate":   two key channels x eight tokens per thread. Per
+//                chunk they turn the gates into decay factors and write the
+//                chunk operands; then each warp computes one 16x8 block of A or
+//                Aqk.
+//     warp  8    "solver": (I + L)^{-1} by forward substitution and T diag(beta).
+//     warp  9    "load":   streams the raw rows of q, k, g, beta and the value
+//                slice into a ring of shared-memory stages with 16-byte
+//                asynchronous copies, RSTAGE chunks ahead of the gates.
+//   Producers run up to NSTAGE chunks ahead of the chain through a second ring
+//   of operand stages; every hand-off is an mbarrier.
 //
 // Per chunk of C = 16 tokens, with Gamma_i the inclusive cumulative log-decay
 // inside the chunk (e_i = exp(g_i) per channel):
@@ -56,10 +59,13 @@ constexpr int D = KDA_HEAD_DIM;   // dk = dv = 128
 constexpr int C = 16;             // chunk length (tokens)
 constexpr int NS = 32;            // value columns per CTA
 constexpr int NSLICE = D / NS;    // CTAs per (sequence, head)
-constexpr int NSTAGE = 4;         // producer look-ahead (chunks)
+constexpr int NSTAGE = 3;         // operand stages (gate/solver -> chain)
+constexpr int RSTAGE = 6;         // raw-input stages (load -> gate)
 constexpr int NCHAIN = 4;         // chain warps
-constexpr int NGATE = 4;          // gate warps (one key channel per thread)
-constexpr int NTHREADS = (NCHAIN + NGATE + 1) * 32;
+constexpr int NGATE = 4;          // gate warps
+constexpr int WARP_SOLVER = NCHAIN + NGATE;
+constexpr int WARP_LOAD = WARP_SOLVER + 1;
+constexpr int NTHREADS = (WARP_LOAD + 1) * 32;
 constexpr int GATE_T0 = NCHAIN * 32;  // first gate thread
 
 // Padded row pitches: 272 B, 48 B and 80 B rows keep 8-row ldmatrix reads on
@@ -81,20 +87,35 @@ struct __align__(16) Stage {
   float beta[C];
 };
 
+struct __align__(16) RawStage {
+  __nv_bfloat16 q[C][D];
+  __nv_bfloat16 k[C][D];
+  float g[C][D];
+  __nv_bfloat16 v[C][NS];
+  float beta[C];
+};
+
 struct __align__(16) Shared {
   Stage st[NSTAGE];
+  RawStage raw[RSTAGE];
   float xbuf[2][2][32][8];   // X^T partial sums exchanged inside a chain-warp pair
   float obuf[2][2][32][4];   // O^T partial sums exchanged inside a chain-warp pair
+  float2 gprod[2][64];       // per-half decay products exchanged inside the gate group
   unsigned long long full[NSTAGE];       // solver -> chain
   unsigned long long gate_done[NSTAGE];  // gate -> solver
   unsigned long long empty[NSTAGE];      // chain -> gate
+  unsigned long long raw_full[RSTAGE];   // load -> gate
+  unsigned long long raw_empty[RSTAGE];  // gate -> load
 };
-static_assert(sizeof(Stage) % 16 == 0, "stage alignment");
+static_assert(sizeof(Stage) % 16 == 0 && sizeof(RawStage) % 16 == 0, "stage alignment");
 static_assert(sizeof(Shared) <= 227 * 1024, "shared memory budget");
 
 // Wait budget for every mbarrier wait (cycles). A wait that runs out records
 // a timeout and lets the thread continue, so no barrier is ever left waiting.
 constexpr long long kWaitCycles = 4ll << 30;
+// A waiting thread is suspended in hardware (up to this many ns per try)
+// instead of spinning, so waiting warps leave the issue slots to the others.
+constexpr uint32_t kSuspendHintNs = 20000;
 __device__ unsigned int g_wait_timeouts = 0;
 
 // ---------------------------------------------------------------- primitives
@@ -110,12 +131,19 @@ __device__ __forceinline__ void mbar_arrive(unsigned long long* m) {
   asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(m)) : "memory");
 }
 
+// One arrive per warp: __syncwarp orders every lane's prior shared-memory
+// accesses before lane 0's release-arrive.
+__device__ __forceinline__ void mbar_arrive_warp(unsigned long long* m) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(m);
+}
+
 __device__ __forceinline__ bool mbar_try_wait(unsigned long long* m, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
       : "=r"(ok)
-      : "r"(smem_u32(m)), "r"(parity)
+      : "r"(smem_u32(m)), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }
@@ -123,12 +151,31 @@ __device__ __forceinline__ bool mbar_try_wait(unsigned long long* m, uint32_t pa
 __device__ __forceinline__ void mbar_wait(unsigned long long* m, uint32_t parity) {
   if (mbar_try_wait(m, parity)) return;
   const long long t0 = clock64();
-  while (!mbar_try_wait(m, parity)) {
-    if (clock64() - t0 > kWaitCycles) {
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(m, parity)) return;
+    if ((i & 63u) == 0 && clock64() - t0 > kWaitCycles) {
       atomicAdd(&g_wait_timeouts, 1u);
       return;
     }
   }
+}
+
+// 16-byte asynchronous copy global -> shared; src_bytes = 0 fills zeros
+// without reading global memory.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
+// 4-byte asynchronous copy (zero fill when src_bytes = 0).
+__device__ __forceinline__ void cp_async4(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
+// Arrive on the mbarrier once every cp.async this thread issued has landed.
+__device__ __forceinline__ void cp_async_arrive(unsigned long long* m) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(m)) : "memory");
 }
 
 __device__ __forceinline__ void named_bar(int id, int nthreads) {
@@ -231,9 +278,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) kda_fwd_kernel(const Params p) {
 
   if (tid == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(&sh.full[s], 32);
-      mbar_init(&sh.gate_done[s], NGATE * 32);
-      mbar_init(&sh.empty[s], NCHAIN * 32);
+      mbar_init(&sh.full[s], 1);
+      mbar_init(&sh.gate_done[s], NGATE);
+      mbar_init(&sh.empty[s], NCHAIN);
+    }
+    for (int s = 0; s < RSTAGE; ++s) {
+      mbar_init(&sh.raw_full[s], 32);  // one asynchronous arrive per load lane
+      mbar_init(&sh.raw_empty[s], NGATE);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -341,7 +392,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) kda_fwd_kernel(const Params p) {
         mma(sT[2 * np + 1], av, be[2], be[3]);
       }
       // the stage is no longer read by this thread
-      mbar_arrive(&sh.empty[s]);
+      mbar_arrive_warp(&sh.empty[s]);
       // ---- O: each warp of the pair finishes one 8-token half
       {
         const int keep = dh, give = dh ^ 1;
@@ -374,67 +425,80 @@ __global__ void __launch_bounds__(NTHREADS, 1) kda_fwd_kernel(const Params p) {
     }
   } else if (warp < NCHAIN + NGATE) {
     // ============================================================ gate warps
-    const int c = tid - GATE_T0;  // key channel
+    // Thread layout: channel pair cp (channels 2cp, 2cp+1), token half th
+    // (tokens 8th .. 8th+7). The decay products of the two halves meet through
+    // shared memory.
+    const int gt = tid - GATE_T0;
     const int gw = warp - NCHAIN;
-    const size_t col_off = static_cast<size_t>(h) * D + c;
-    // raw inputs of the next chunk, prefetched into registers
-    float g_nx[C];
-    uint16_t k_nx[C], q_nx[C];
-    float b_nx = 0.f;
-    auto load_chunk = [&](int n) {
-      const int64_t cs = t0 + static_cast<int64_t>(n) * C;
-#pragma unroll
-      for (int i = 0; i < C; ++i) {
-        const bool ok = (n < nch) && (cs + i < t1);
-        const size_t off = (cs + i) * row_stride + col_off;
-        g_nx[i] = ok ? __ldg(p.g + off) : 0.f;
-        k_nx[i] = ok ? __ldg(reinterpret_cast<const unsigned short*>(p.k) + off) : static_cast<uint16_t>(0);
-        q_nx[i] = ok ? __ldg(reinterpret_cast<const unsigned short*>(p.q) + off) : static_cast<uint16_t>(0);
-      }
-      if (gw == 0 && lane < C) {
-        const bool ok = (n < nch) && (cs + lane < t1);
-        b_nx = ok ? __ldg(p.beta + (cs + lane) * H + h) : 0.f;
-      }
-    };
-    load_chunk(0);
+    const int cp = gt & 63;
+    const int th = gt >> 6;
+    const int c0 = 2 * cp;
     for (int n = 0; n < nch; ++n) {
       const int s = n % NSTAGE;
       const uint32_t ph = static_cast<uint32_t>(n / NSTAGE) & 1u;
-      float gv[C], kv[C], qv[C];
-#pragma unroll
-      for (int i = 0; i < C; ++i) {
-        gv[i] = g_nx[i];
-        kv[i] = bf16_bits_to_f32(k_nx[i]);
-        qv[i] = bf16_bits_to_f32(q_nx[i]);
-      }
-      const float bv = b_nx;
-      load_chunk(n + 1);
+      const int rs = n % RSTAGE;
+      const uint32_t rph = static_cast<uint32_t>(n / RSTAGE) & 1u;
+      const int64_t cs = t0 + static_cast<int64_t>(n) * C;
+      const int m = static_cast<int>((t1 - cs) < C ? (t1 - cs) : C);
+      RawStage& rw = sh.raw[rs];
       Stage& st = sh.st[s];
-      mbar_wait(&sh.empty[s], ph ^ 1u);
+      mbar_wait(&sh.raw_full[rs], rph);
 
-      // ---- decay factors and operands for key channel c
-      float e[C];
+      // ---- raw inputs of this thread (rows past the sequence end masked)
+      float2 e[8], kv[8], qv[8];
 #pragma unroll
-      for (int i = 0; i < C; ++i) e[i] = __expf(gv[i]);
-      float E = 1.f;
-#pragma unroll
-      for (int i = 0; i < C; ++i) {
-        E *= e[i];
-        st.kd[i][c] = __float2bfloat16_rn(kv[i] * E);
-        st.qd[i][c] = __float2bfloat16_rn(qv[i] * E);
+      for (int j = 0; j < 8; ++j) {
+        const int i = 8 * th + j;
+        const bool ok = i < m;
+        const float2 gg = *reinterpret_cast<const float2*>(&rw.g[i][c0]);
+        const __nv_bfloat162 kk = *reinterpret_cast<const __nv_bfloat162*>(&rw.k[i][c0]);
+        const __nv_bfloat162 qq = *reinterpret_cast<const __nv_bfloat162*>(&rw.q[i][c0]);
+        e[j] = ok ? make_float2(__expf(gg.x), __expf(gg.y)) : make_float2(1.f, 1.f);
+        kv[j] = ok ? __bfloat1622float2(kk) : make_float2(0.f, 0.f);
+        qv[j] = ok ? __bfloat1622float2(qq) : make_float2(0.f, 0.f);
       }
-      const float gamma = E;
-      const float rgamma = __frcp_rn(gamma);
-      float F = 1.f;
+      uint4 vpiece = make_uint4(0, 0, 0, 0);  // value-slice tile: 16 rows x 64 bytes
+      if (gt < 64 && (gt >> 2) < m) vpiece = *reinterpret_cast<const uint4*>(&rw.v[gt >> 2][8 * (gt & 3)]);
+      float bv = 0.f;
+      if (gt < C) bv = gt < m ? rw.beta[gt] : 0.f;
+      mbar_arrive_warp(&sh.raw_empty[rs]);
+
+      // ---- decay products: this half's total, exchanged with the other half
+      float2 P = make_float2(1.f, 1.f);
 #pragma unroll
-      for (int i = C - 1; i >= 0; --i) {
-        const float kf = kv[i] * F;
-        st.ke[i][c] = __float2bfloat16_rn(kf);
-        st.kr[i][c] = __float2bfloat16_rn(kf * rgamma);
-        F *= e[i];
+      for (int j = 0; j < 8; ++j) {
+        P.x *= e[j].x;
+        P.y *= e[j].y;
       }
-      st.gam[c] = gamma;
-      if (gw == 0 && lane < C) st.beta[lane] = bv;
+      mbar_wait(&sh.empty[s], ph ^ 1u);
+      sh.gprod[th][cp] = P;
+      if (gt < C) st.beta[gt] = bv;
+      if (gt < 64) *reinterpret_cast<uint4*>(&st.v[gt >> 2][8 * (gt & 3)]) = vpiece;
+      named_bar(1, NGATE * 32);
+      const float2 Po = sh.gprod[th ^ 1][cp];
+      // E before this half (1 for the first half), F after it (1 for the second)
+      float2 E = th ? Po : make_float2(1.f, 1.f);
+      float2 F = th ? make_float2(1.f, 1.f) : Po;
+      const float2 gamma = make_float2(P.x * Po.x, P.y * Po.y);
+      const float2 rg = make_float2(__frcp_rn(gamma.x), __frcp_rn(gamma.y));
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = 8 * th + j;
+        E.x *= e[j].x;
+        E.y *= e[j].y;
+        *reinterpret_cast<uint32_t*>(&st.kd[i][c0]) = pack_bf16(kv[j].x * E.x, kv[j].y * E.y);
+        *reinterpret_cast<uint32_t*>(&st.qd[i][c0]) = pack_bf16(qv[j].x * E.x, qv[j].y * E.y);
+      }
+#pragma unroll
+      for (int j = 7; j >= 0; --j) {
+        const int i = 8 * th + j;
+        const float kfx = kv[j].x * F.x, kfy = kv[j].y * F.y;
+        *reinterpret_cast<uint32_t*>(&st.ke[i][c0]) = pack_bf16(kfx, kfy);
+        *reinterpret_cast<uint32_t*>(&st.kr[i][c0]) = pack_bf16(kfx * rg.x, kfy * rg.y);
+        F.x *= e[j].x;
+        F.y *= e[j].y;
+      }
+      if (th == 0) *reinterpret_cast<float2*>(&st.gam[c0]) = gamma;
       named_bar(1, NGATE * 32);
 
       // ---- one 16x8 block of A = Kd KR^T (gate warps 0,1) or Aqk = Qd KR^T (2,3)
@@ -459,35 +523,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) kda_fwd_kernel(const Params p) {
             st.aqk[i][j] = __float2bfloat16_rn((j <= i) ? acc[e2] : 0.f);
         }
       }
-      mbar_arrive(&sh.gate_done[s]);
+      mbar_arrive_warp(&sh.gate_done[s]);
     }
-  } else {
+  } else if (warp == WARP_SOLVER) {
     // =========================================================== solver warp
-    // lanes 0-15: one column of (I + L)^{-1} each; lanes 16-31: value-slice tile
-    const int r = lane - 16;  // value-tile row for lanes 16-31
-    uint4 v_nx[NS / 8];
-    auto load_v = [&](int n) {
-      if (lane >= 16) {
-        const int64_t cs = t0 + static_cast<int64_t>(n) * C;
-        const bool ok = (n < nch) && (cs + r < t1);
-#pragma unroll
-        for (int j = 0; j < NS / 8; ++j)
-          v_nx[j] = ok ? __ldg(reinterpret_cast<const uint4*>(p.v + (cs + r) * row_stride +
-                                                              static_cast<size_t>(h) * D + dv0) + j)
-                       : make_uint4(0, 0, 0, 0);
-      }
-    };
-    load_v(0);
+    // lanes 0-15: one column of (I + L)^{-1} each, scaled by beta of that column
     for (int n = 0; n < nch; ++n) {
       const int s = n % NSTAGE;
       const uint32_t ph = static_cast<uint32_t>(n / NSTAGE) & 1u;
       Stage& st = sh.st[s];
-      uint4 vcur[NS / 8];
-#pragma unroll
-      for (int j = 0; j < NS / 8; ++j) vcur[j] = v_nx[j];
-      load_v(n + 1);
       mbar_wait(&sh.gate_done[s], ph);
-      if (lane < 16) {
+      if (lane < C) {
         const int col = lane;
         float xs[C];
 #pragma unroll
@@ -501,11 +547,46 @@ __global__ void __launch_bounds__(NTHREADS, 1) kda_fwd_kernel(const Params p) {
         const float bc = st.beta[col];
 #pragma unroll
         for (int i = 0; i < C; ++i) st.tb[i][col] = __float2bfloat16_rn(xs[i] * bc);
-      } else {
-#pragma unroll
-        for (int j = 0; j < NS / 8; ++j) *reinterpret_cast<uint4*>(&st.v[r][8 * j]) = vcur[j];
       }
-      mbar_arrive(&sh.full[s]);
+      mbar_arrive_warp(&sh.full[s]);
+    }
+  } else {
+    // ============================================================= load warp
+    // Each lane copies 16-byte pieces of the chunk's rows; rows past the
+    // sequence end are zero-filled without touching global memory.
+    const size_t hoff = static_cast<size_t>(h) * D;
+    constexpr int kQ = C * D * 2 / 16;   // pieces of q (and of k)
+    constexpr int kG = C * D * 4 / 16;   // pieces of g
+    constexpr int kV = C * NS * 2 / 16;  // pieces of the value slice
+    for (int n = 0; n < nch; ++n) {
+      const int rs = n % RSTAGE;
+      const uint32_t rph = static_cast<uint32_t>(n / RSTAGE) & 1u;
+      const int64_t cs = t0 + static_cast<int64_t>(n) * C;
+      const int m = static_cast<int>((t1 - cs) < C ? (t1 - cs) : C);
+      RawStage& rw = sh.raw[rs];
+      mbar_wait(&sh.raw_empty[rs], rph ^ 1u);
+      for (int i = lane; i < kQ; i += 32) {
+        const int r = i / (D / 8), c = (i % (D / 8)) * 8;
+        const bool ok = r < m;
+        const size_t off = ok ? (cs + r) * row_stride + hoff + c : 0;
+        cp_async16(&rw.q[r][c], p.q + off, ok ? 16u : 0u);
+        cp_async16(&rw.k[r][c], p.k + off, ok ? 16u : 0u);
+      }
+      for (int i = lane; i < kG; i += 32) {
+        const int r = i / (D / 4), c = (i % (D / 4)) * 4;
+        const bool ok = r < m;
+        cp_async16(&rw.g[r][c], p.g + (ok ? (cs + r) * row_stride + hoff + c : 0), ok ? 16u : 0u);
+      }
+      for (int i = lane; i < kV; i += 32) {
+        const int r = i / (NS / 8), c = (i % (NS / 8)) * 8;
+        const bool ok = r < m;
+        cp_async16(&rw.v[r][c], p.v + (ok ? (cs + r) * row_stride + hoff + dv0 + c : 0), ok ? 16u : 0u);
+      }
+      if (lane < C) {
+        const bool ok = lane < m;
+        cp_async4(&rw.beta[lane], p.beta + (ok ? (cs + lane) * H + h : 0), ok ? 4u : 0u);
+      }
+      cp_async_arrive(&sh.raw_full[rs]);
     }
   }
 }
