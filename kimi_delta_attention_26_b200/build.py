@@ -9,12 +9,15 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SOURCES = [os.path.join(PKG, "csrc", "kda_fwd.cu")]
-HEADERS = [os.path.join(ROOT, "include", "kda.h")]
+HEADERS = [os.path.join(ROOT, "include", "kda.h"), os.path.abspath(__file__)]
 LIB = os.path.join(PKG, "libkda.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",
+    # Flush fp32 denormals: the gate exponentials run ~2.5x faster, and values
+    # below 1.2e-38 are far under the bf16 resolution of every operand.
+    "-ftz=true",
     "-shared", "-Xcompiler", "-fPIC",
     "-I", os.path.join(ROOT, "include"),
 ]

@@ -12,10 +12,12 @@
 //                next chunk's products, so it never touches shared memory.
 //     warps 4-7  "gate":   two key channels x eight tokens per thread. Per
 //                chunk they turn the gates into decay factors and write the
-//                chunk operands; then each warp computes one 16x8 block of A or
-//                Aqk.
-//     warp  8    "solver": (I + L)^{-1} by forward substitution and T diag(beta).
-//     warp  9    "load":   streams the raw rows of q, k, g, beta and the value
+//                chunk operands.
+//     warp  8    "mma":    A = Kd KR^T and Aqk = Qd KR^T (16 x 16 each), which
+//                share their KR fragments; writes L = diag(beta) tril(A, -1)
+//                and the causal Aqk.
+//     warp  9    "solver": (I + L)^{-1} by forward substitution and T diag(beta).
+//     warps 10-11 "load":  stream the raw rows of q, k, g, beta and the value
 //                slice into a ring of shared-memory stages with 16-byte
 //                asynchronous copies, RSTAGE chunks ahead of the gates.
 //   Producers run up to NSTAGE chunks ahead of the chain through a second ring
@@ -63,9 +65,10 @@ constexpr int NSTAGE = 3;         // operand stages (gate/solver -> chain)
 constexpr int RSTAGE = 6;         // raw-input stages (load -> gate)
 constexpr int NCHAIN = 4;         // chain warps
 constexpr int NGATE = 4;          // gate warps
-constexpr int WARP_SOLVER = NCHAIN + NGATE;
-constexpr int WARP_LOAD = WARP_SOLVER + 1;
-constexpr int NTHREADS = (WARP_LOAD + 1) * 32;
+constexpr int WARP_MMA = NCHAIN + NGATE;
+constexpr int WARP_SOLVER = WARP_MMA + 1;
+constexpr int WARP_LOAD = WARP_SOLVER + 1;  // two load warps
+constexpr int NTHREADS = (WARP_LOAD + 2) * 32;
 constexpr int GATE_T0 = NCHAIN * 32;  // first gate thread
 
 // Padded row pitches: 272 B, 48 B and 80 B rows keep 8-row ldmatrix reads on
@@ -82,7 +85,7 @@ struct __align__(16) Stage {
   __nv_bfloat16 tb[C][LDC];
   __nv_bfloat16 aqk[C][LDC];
   __nv_bfloat16 v[C][LDV];
-  float L[C][C + 1];
+  float L[C][C + 4];   // 80-byte rows: 16-byte aligned for row-broadcast loads
   float gam[D];
   float beta[C];
 };
@@ -100,9 +103,11 @@ struct __align__(16) Shared {
   RawStage raw[RSTAGE];
   float xbuf[2][2][32][8];   // X^T partial sums exchanged inside a chain-warp pair
   float obuf[2][2][32][4];   // O^T partial sums exchanged inside a chain-warp pair
-  float2 gprod[2][64];       // per-half decay products exchanged inside the gate group
+  float2 gprod[2][2][64];    // per-half decay products exchanged inside the gate group,
+                             // double-buffered by chunk parity
   unsigned long long full[NSTAGE];       // solver -> chain
-  unsigned long long gate_done[NSTAGE];  // gate -> solver
+  unsigned long long gate_done[NSTAGE];  // gate -> mma
+  unsigned long long mma_done[NSTAGE];   // mma -> solver
   unsigned long long empty[NSTAGE];      // chain -> gate
   unsigned long long raw_full[RSTAGE];   // load -> gate
   unsigned long long raw_empty[RSTAGE];  // gate -> load
@@ -280,10 +285,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) kda_fwd_kernel(const Params p) {
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(&sh.full[s], 1);
       mbar_init(&sh.gate_done[s], NGATE);
+      mbar_init(&sh.mma_done[s], 1);
       mbar_init(&sh.empty[s], NCHAIN);
     }
     for (int s = 0; s < RSTAGE; ++s) {
-      mbar_init(&sh.raw_full[s], 32);  // one asynchronous arrive per load lane
+      mbar_init(&sh.raw_full[s], 64);  // one asynchronous arrive per load lane
       mbar_init(&sh.raw_empty[s], NGATE);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -471,11 +477,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) kda_fwd_kernel(const Params p) {
         P.y *= e[j].y;
       }
       mbar_wait(&sh.empty[s], ph ^ 1u);
-      sh.gprod[th][cp] = P;
+      sh.gprod[n & 1][th][cp] = P;
       if (gt < C) st.beta[gt] = bv;
       if (gt < 64) *reinterpret_cast<uint4*>(&st.v[gt >> 2][8 * (gt & 3)]) = vpiece;
       named_bar(1, NGATE * 32);
-      const float2 Po = sh.gprod[th ^ 1][cp];
+      const float2 Po = sh.gprod[n & 1][th ^ 1][cp];
       // E before this half (1 for the first half), F after it (1 for the second)
       float2 E = th ? Po : make_float2(1.f, 1.f);
       float2 F = th ? make_float2(1.f, 1.f) : Po;
@@ -499,31 +505,37 @@ __global__ void __launch_bounds__(NTHREADS, 1) kda_fwd_kernel(const Params p) {
         F.y *= e[j].y;
       }
       if (th == 0) *reinterpret_cast<float2*>(&st.gam[c0]) = gamma;
-      named_bar(1, NGATE * 32);
-
-      // ---- one 16x8 block of A = Kd KR^T (gate warps 0,1) or Aqk = Qd KR^T (2,3)
-      {
-        const int mat = gw >> 1, nt = gw & 1;
-        const __nv_bfloat16(*src)[LDK] = mat ? st.qd : st.kd;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      mbar_arrive_warp(&sh.gate_done[s]);
+    }
+  } else if (warp == WARP_MMA) {
+    // ============================================================= mma warp
+    for (int n = 0; n < nch; ++n) {
+      const int s = n % NSTAGE;
+      const uint32_t ph = static_cast<uint32_t>(n / NSTAGE) & 1u;
+      Stage& st = sh.st[s];
+      mbar_wait(&sh.gate_done[s], ph);
+      float accA[2][4] = {}, accQ[2][4] = {};
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          uint32_t a[4], b[2];
-          ldsm_x4(a, &src[lane & 15][16 * kk + (lane >> 4) * 8]);
-          ldsm_x2(b, &st.kr[8 * nt + (lane & 7)][16 * kk + ((lane >> 3) & 1) * 8]);
-          mma(acc, a, b[0], b[1]);
-        }
+      for (int kk = 0; kk < D / 16; ++kk) {
+        uint32_t ak[4], aq[4], b[4];
+        ldsm_x4(ak, &st.kd[lane & 15][16 * kk + (lane >> 4) * 8]);
+        ldsm_x4(aq, &st.qd[lane & 15][16 * kk + (lane >> 4) * 8]);
+        ldsm_x4(b, &st.kr[(lane & 7) + ((lane >> 4) << 3)][16 * kk + ((lane >> 3) & 1) * 8]);
+        mma(accA[0], ak, b[0], b[1]);
+        mma(accA[1], ak, b[2], b[3]);
+        mma(accQ[0], aq, b[0], b[1]);
+        mma(accQ[1], aq, b[2], b[3]);
+      }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e2 = 0; e2 < 4; ++e2) {
           const int i = gq + 8 * (e2 >> 1);
           const int j = 8 * nt + 2 * tq + (e2 & 1);
-          if (mat == 0)
-            st.L[i][j] = (j < i) ? st.beta[i] * acc[e2] : 0.f;
-          else
-            st.aqk[i][j] = __float2bfloat16_rn((j <= i) ? acc[e2] : 0.f);
+          st.L[i][j] = (j < i) ? st.beta[i] * accA[nt][e2] : 0.f;
+          st.aqk[i][j] = __float2bfloat16_rn((j <= i) ? accQ[nt][e2] : 0.f);
         }
-      }
-      mbar_arrive_warp(&sh.gate_done[s]);
+      mbar_arrive_warp(&sh.mma_done[s]);
     }
   } else if (warp == WARP_SOLVER) {
     // =========================================================== solver warp
@@ -532,17 +544,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) kda_fwd_kernel(const Params p) {
       const int s = n % NSTAGE;
       const uint32_t ph = static_cast<uint32_t>(n / NSTAGE) & 1u;
       Stage& st = sh.st[s];
-      mbar_wait(&sh.gate_done[s], ph);
+      mbar_wait(&sh.mma_done[s], ph);
       if (lane < C) {
+        // column `col` of T = (I + L)^{-1}: x_i = [i == col] - sum_{m<i} L[i][m] x_m,
+        // reading each row of L with 16-byte loads that all lanes share
         const int col = lane;
         float xs[C];
 #pragma unroll
-        for (int i = 0; i < C; ++i) xs[i] = (i == col) ? 1.f : 0.f;
+        for (int i = 0; i < C; ++i) {
+          float acc0 = (i == col) ? 1.f : 0.f, acc1 = 0.f;
 #pragma unroll
-        for (int mm = 0; mm < C; ++mm) {
-          const float xm = xs[mm];
-#pragma unroll
-          for (int i = mm + 1; i < C; ++i) xs[i] = fmaf(-st.L[i][mm], xm, xs[i]);
+          for (int m4 = 0; m4 < (i + 3) / 4; ++m4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(&st.L[i][4 * m4]);
+            if (4 * m4 + 0 < i) acc0 = fmaf(-l4.x, xs[4 * m4 + 0], acc0);
+            if (4 * m4 + 1 < i) acc1 = fmaf(-l4.y, xs[4 * m4 + 1], acc1);
+            if (4 * m4 + 2 < i) acc0 = fmaf(-l4.z, xs[4 * m4 + 2], acc0);
+            if (4 * m4 + 3 < i) acc1 = fmaf(-l4.w, xs[4 * m4 + 3], acc1);
+          }
+          xs[i] = acc0 + acc1;
         }
         const float bc = st.beta[col];
 #pragma unroll
@@ -551,13 +570,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) kda_fwd_kernel(const Params p) {
       mbar_arrive_warp(&sh.full[s]);
     }
   } else {
-    // ============================================================= load warp
-    // Each lane copies 16-byte pieces of the chunk's rows; rows past the
-    // sequence end are zero-filled without touching global memory.
+    // ============================================================ load warps
+    // Lane l of load warp lw owns token row r = l & 15 and one quarter of each
+    // of its byte ranges (quarter = 2*lw + (l >> 4)); one base address per
+    // tensor and chunk, constant offsets after that. Rows past the sequence
+    // end are zero-filled without touching global memory.
+    const int lw = warp - WARP_LOAD;
+    const int r = lane & 15;
+    const int qtr = 2 * lw + (lane >> 4);
     const size_t hoff = static_cast<size_t>(h) * D;
-    constexpr int kQ = C * D * 2 / 16;   // pieces of q (and of k)
-    constexpr int kG = C * D * 4 / 16;   // pieces of g
-    constexpr int kV = C * NS * 2 / 16;  // pieces of the value slice
     for (int n = 0; n < nch; ++n) {
       const int rs = n % RSTAGE;
       const uint32_t rph = static_cast<uint32_t>(n / RSTAGE) & 1u;
@@ -565,27 +586,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) kda_fwd_kernel(const Params p) {
       const int m = static_cast<int>((t1 - cs) < C ? (t1 - cs) : C);
       RawStage& rw = sh.raw[rs];
       mbar_wait(&sh.raw_empty[rs], rph ^ 1u);
-      for (int i = lane; i < kQ; i += 32) {
-        const int r = i / (D / 8), c = (i % (D / 8)) * 8;
-        const bool ok = r < m;
-        const size_t off = ok ? (cs + r) * row_stride + hoff + c : 0;
-        cp_async16(&rw.q[r][c], p.q + off, ok ? 16u : 0u);
-        cp_async16(&rw.k[r][c], p.k + off, ok ? 16u : 0u);
+      const bool ok = r < m;
+      const uint32_t sz = ok ? 16u : 0u;
+      const size_t rowoff = ok ? (cs + r) * row_stride + hoff : 0;
+      const __nv_bfloat16* gq_ = p.q + rowoff + 32 * qtr;   // 32 bf16 = 4 pieces per quarter
+      const __nv_bfloat16* gk_ = p.k + rowoff + 32 * qtr;
+      const float* gg_ = p.g + rowoff + 32 * qtr;           // 32 fp32 = 8 pieces per quarter
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        cp_async16(&rw.q[r][32 * qtr + 8 * j], gq_ + 8 * j, sz);
+        cp_async16(&rw.k[r][32 * qtr + 8 * j], gk_ + 8 * j, sz);
       }
-      for (int i = lane; i < kG; i += 32) {
-        const int r = i / (D / 4), c = (i % (D / 4)) * 4;
-        const bool ok = r < m;
-        cp_async16(&rw.g[r][c], p.g + (ok ? (cs + r) * row_stride + hoff + c : 0), ok ? 16u : 0u);
-      }
-      for (int i = lane; i < kV; i += 32) {
-        const int r = i / (NS / 8), c = (i % (NS / 8)) * 8;
-        const bool ok = r < m;
-        cp_async16(&rw.v[r][c], p.v + (ok ? (cs + r) * row_stride + hoff + dv0 + c : 0), ok ? 16u : 0u);
-      }
-      if (lane < C) {
-        const bool ok = lane < m;
-        cp_async4(&rw.beta[lane], p.beta + (ok ? (cs + lane) * H + h : 0), ok ? 4u : 0u);
-      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) cp_async16(&rw.g[r][32 * qtr + 4 * j], gg_ + 4 * j, sz);
+      // value slice: 64 bytes per row = 4 pieces, one per quarter
+      cp_async16(&rw.v[r][8 * qtr], p.v + rowoff + dv0 + 8 * qtr, sz);
+      if (qtr == 0) cp_async4(&rw.beta[r], p.beta + (ok ? (cs + r) * H + h : 0), ok ? 4u : 0u);
       cp_async_arrive(&sh.raw_full[rs]);
     }
   }
