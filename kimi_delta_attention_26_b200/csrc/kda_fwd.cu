@@ -17,9 +17,9 @@
 //                share their KR fragments; writes L = diag(beta) tril(A, -1)
 //                and the causal Aqk.
 //     warp  9    "solver": (I + L)^{-1} by forward substitution and T diag(beta).
-//     warps 10-11 "load":  stream the raw rows of q, k, g, beta and the value
-//                slice into a ring of shared-memory stages with 16-byte
-//                asynchronous copies, RSTAGE chunks ahead of the gates.
+//     warp 10    "load":   one lane issues TMA tensor copies (q, k, g, the value
+//                slice and beta; five requests per chunk) into a ring of
+//                shared-memory stages, RSTAGE chunks ahead of the gates.
 //   Producers run up to NSTAGE chunks ahead of the chain through a second ring
 //   of operand stages; every hand-off is an mbarrier.
 //
@@ -46,8 +46,10 @@
 // plus a ~250-cycle commit/mbarrier round trip; the chain is a serial sequence
 // of such small products, so it stays on the synchronous path.
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <cstdint>
 #include <cstdio>
@@ -67,8 +69,8 @@ constexpr int NCHAIN = 4;         // chain warps
 constexpr int NGATE = 4;          // gate warps
 constexpr int WARP_MMA = NCHAIN + NGATE;
 constexpr int WARP_SOLVER = WARP_MMA + 1;
-constexpr int WARP_LOAD = WARP_SOLVER + 1;  // two load warps
-constexpr int NTHREADS = (WARP_LOAD + 2) * 32;
+constexpr int WARP_LOAD = WARP_SOLVER + 1;
+constexpr int NTHREADS = (WARP_LOAD + 1) * 32;
 constexpr int GATE_T0 = NCHAIN * 32;  // first gate thread
 
 // Padded row pitches: 272 B, 48 B and 80 B rows keep 8-row ldmatrix reads on
@@ -90,17 +92,21 @@ struct __align__(16) Stage {
   float beta[C];
 };
 
-struct __align__(16) RawStage {
+// One chunk of raw inputs, exactly as the TMA boxes land: q, k [16 tokens][128],
+// g [16][128], value slice [16][32]; beta [16] arrives by 4-byte copies.
+struct __align__(128) RawStage {
   __nv_bfloat16 q[C][D];
   __nv_bfloat16 k[C][D];
   float g[C][D];
   __nv_bfloat16 v[C][NS];
   float beta[C];
+  float pad_[32 - C];
 };
+constexpr uint32_t kRawBytes = C * D * 2 * 2 + C * D * 4 + C * NS * 2;  // bytes the TMA boxes bring
 
-struct __align__(16) Shared {
-  Stage st[NSTAGE];
+struct __align__(128) Shared {
   RawStage raw[RSTAGE];
+  Stage st[NSTAGE];
   float xbuf[2][2][32][8];   // X^T partial sums exchanged inside a chain-warp pair
   float obuf[2][2][32][4];   // O^T partial sums exchanged inside a chain-warp pair
   float2 gprod[2][2][64];    // per-half decay products exchanged inside the gate group,
@@ -112,7 +118,7 @@ struct __align__(16) Shared {
   unsigned long long raw_full[RSTAGE];   // load -> gate
   unsigned long long raw_empty[RSTAGE];  // gate -> load
 };
-static_assert(sizeof(Stage) % 16 == 0 && sizeof(RawStage) % 16 == 0, "stage alignment");
+static_assert(sizeof(Stage) % 16 == 0 && sizeof(RawStage) % 128 == 0, "stage alignment");
 static_assert(sizeof(Shared) <= 227 * 1024, "shared memory budget");
 
 // Wait budget for every mbarrier wait (cycles). A wait that runs out records
@@ -165,22 +171,30 @@ __device__ __forceinline__ void mbar_wait(unsigned long long* m, uint32_t parity
   }
 }
 
-// 16-byte asynchronous copy global -> shared; src_bytes = 0 fills zeros
-// without reading global memory.
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-
-// 4-byte asynchronous copy (zero fill when src_bytes = 0).
+// 4-byte asynchronous copy (zero fill when src_bytes = 0) and the arrive that
+// fires once this thread's copies have landed.
 __device__ __forceinline__ void cp_async4(void* dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
                : "memory");
 }
 
-// Arrive on the mbarrier once every cp.async this thread issued has landed.
 __device__ __forceinline__ void cp_async_arrive(unsigned long long* m) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(m)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long* m, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(m)), "r"(bytes)
+               : "memory");
+}
+
+// TMA tiled loads (no multicast). Out-of-range rows of the box are zero-filled.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
+                                            unsigned long long* m) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(m))
+      : "memory");
 }
 
 __device__ __forceinline__ void named_bar(int id, int nthreads) {
@@ -254,7 +268,12 @@ struct Params {
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
 
-__global__ void __launch_bounds__(NTHREADS, 1) kda_fwd_kernel(const Params p) {
+struct TensorMaps {
+  CUtensorMap q, k, g, v;
+};
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    kda_fwd_kernel(const Params p, const __grid_constant__ TensorMaps tm) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   Shared& sh = *reinterpret_cast<Shared*>(smem_raw);
 
@@ -289,7 +308,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) kda_fwd_kernel(const Params p) {
       mbar_init(&sh.empty[s], NCHAIN);
     }
     for (int s = 0; s < RSTAGE; ++s) {
-      mbar_init(&sh.raw_full[s], 64);  // one asynchronous arrive per load lane
+      mbar_init(&sh.raw_full[s], 1 + C);  // expect_tx arrive + one per beta lane
       mbar_init(&sh.raw_empty[s], NGATE);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -399,15 +418,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) kda_fwd_kernel(const Params p) {
       }
       // the stage is no longer read by this thread
       mbar_arrive_warp(&sh.empty[s]);
-      // ---- O: each warp of the pair finishes one 8-token half
+      // ---- O: each warp of the pair finishes one 8-token half (register
+      // selects, not a runtime array index, keep o[][] in registers)
       {
-        const int keep = dh, give = dh ^ 1;
-        *reinterpret_cast<float4*>(&sh.obuf[pr][dh][lane][0]) =
-            make_float4(o[give][0], o[give][1], o[give][2], o[give][3]);
+        const int keep = dh;
+        float mine[4], give[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          mine[e] = dh ? o[1][e] : o[0][e];
+          give[e] = dh ? o[0][e] : o[1][e];
+        }
+        *reinterpret_cast<float4*>(&sh.obuf[pr][dh][lane][0]) = make_float4(give[0], give[1], give[2], give[3]);
         named_bar(2 + pr, 64);
         const float4 u = *reinterpret_cast<const float4*>(&sh.obuf[pr][dh ^ 1][lane][0]);
-        const float o0 = (o[keep][0] + u.x) * p.scale, o1 = (o[keep][1] + u.y) * p.scale;
-        const float o2 = (o[keep][2] + u.z) * p.scale, o3 = (o[keep][3] + u.w) * p.scale;
+        const float o0 = (mine[0] + u.x) * p.scale, o1 = (mine[1] + u.y) * p.scale;
+        const float o2 = (mine[2] + u.z) * p.scale, o3 = (mine[3] + u.w) * p.scale;
         // fragment rows = value columns, cols = tokens -> transpose to token rows
         const uint32_t r0 = movmatrix_t(pack_bf16(o0, o1));
         const uint32_t r1 = movmatrix_t(pack_bf16(o2, o3));
@@ -570,39 +595,27 @@ __global__ void __launch_bounds__(NTHREADS, 1) kda_fwd_kernel(const Params p) {
       mbar_arrive_warp(&sh.full[s]);
     }
   } else {
-    // ============================================================ load warps
-    // Lane l of load warp lw owns token row r = l & 15 and one quarter of each
-    // of its byte ranges (quarter = 2*lw + (l >> 4)); one base address per
-    // tensor and chunk, constant offsets after that. Rows past the sequence
-    // end are zero-filled without touching global memory.
-    const int lw = warp - WARP_LOAD;
-    const int r = lane & 15;
-    const int qtr = 2 * lw + (lane >> 4);
-    const size_t hoff = static_cast<size_t>(h) * D;
+    // ============================================================= load warp
+    // lane 0: TMA boxes of q, k, g and the value slice; lanes 1-16: beta.
     for (int n = 0; n < nch; ++n) {
       const int rs = n % RSTAGE;
       const uint32_t rph = static_cast<uint32_t>(n / RSTAGE) & 1u;
       const int64_t cs = t0 + static_cast<int64_t>(n) * C;
-      const int m = static_cast<int>((t1 - cs) < C ? (t1 - cs) : C);
+      const int tok = static_cast<int>(cs);
       RawStage& rw = sh.raw[rs];
       mbar_wait(&sh.raw_empty[rs], rph ^ 1u);
-      const bool ok = r < m;
-      const uint32_t sz = ok ? 16u : 0u;
-      const size_t rowoff = ok ? (cs + r) * row_stride + hoff : 0;
-      const __nv_bfloat16* gq_ = p.q + rowoff + 32 * qtr;   // 32 bf16 = 4 pieces per quarter
-      const __nv_bfloat16* gk_ = p.k + rowoff + 32 * qtr;
-      const float* gg_ = p.g + rowoff + 32 * qtr;           // 32 fp32 = 8 pieces per quarter
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        cp_async16(&rw.q[r][32 * qtr + 8 * j], gq_ + 8 * j, sz);
-        cp_async16(&rw.k[r][32 * qtr + 8 * j], gk_ + 8 * j, sz);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&sh.raw_full[rs], kRawBytes);
+        tma_load_3d(&rw.q[0][0], &tm.q, 0, h, tok, &sh.raw_full[rs]);
+        tma_load_3d(&rw.k[0][0], &tm.k, 0, h, tok, &sh.raw_full[rs]);
+        tma_load_3d(&rw.g[0][0], &tm.g, 0, h, tok, &sh.raw_full[rs]);
+        tma_load_3d(&rw.v[0][0], &tm.v, dv0, h, tok, &sh.raw_full[rs]);
+      } else if (lane <= C) {
+        const int r = lane - 1;
+        const bool ok = cs + r < t1;
+        cp_async4(&rw.beta[r], p.beta + (ok ? (cs + r) * H + h : 0), ok ? 4u : 0u);
+        cp_async_arrive(&sh.raw_full[rs]);
       }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) cp_async16(&rw.g[r][32 * qtr + 4 * j], gg_ + 4 * j, sz);
-      // value slice: 64 bytes per row = 4 pieces, one per quarter
-      cp_async16(&rw.v[r][8 * qtr], p.v + rowoff + dv0 + 8 * qtr, sz);
-      if (qtr == 0) cp_async4(&rw.beta[r], p.beta + (ok ? (cs + r) * H + h : 0), ok ? 4u : 0u);
-      cp_async_arrive(&sh.raw_full[rs]);
     }
   }
 }
@@ -621,6 +634,41 @@ kda_status_t cuda_fail(cudaError_t e) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+kda_status_t load_encoder() {
+  if (g_encode) return KDA_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (q != cudaDriverEntryPointSuccess || !fn) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled not available");
+    return KDA_ERR_CUDA;
+  }
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return KDA_OK;
+}
+
+// [T, H, inner] row-major tensor; box {box_inner, 1, 16 tokens}.
+kda_status_t encode_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes, int64_t T,
+                       int H, int inner, int box_inner) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(T)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner) * elem_bytes,
+                                 static_cast<cuuint64_t>(H) * inner * elem_bytes};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), 1u, static_cast<cuuint32_t>(kda::C)};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = g_encode(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return KDA_ERR_CUDA;
+  }
+  return KDA_OK;
+}
 
 constexpr int kMaxDevices = 64;
 int g_device_ready[kMaxDevices];  // 0 unknown, 1 ready, -1 unsupported
@@ -659,6 +707,7 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* g
   if (!cu_seqlens && num_seqs != 1) return KDA_ERR_SHAPE;
   if (num_heads > 65535 || num_seqs > 65535) return KDA_ERR_SHAPE;  // grid.y / grid.z limits
   if (total_tokens > (int64_t(1) << 40) / (int64_t(num_heads) * KDA_HEAD_DIM)) return KDA_ERR_SHAPE;
+  if (total_tokens > int64_t(INT32_MAX) - 64) return KDA_ERR_SHAPE;  // TMA coordinates are 32-bit
   const void* ptrs[] = {q, k, v, g, beta, out, initial_state, final_state, cu_seqlens};
   for (const void* ptr : ptrs)
     if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
@@ -682,8 +731,20 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* g
   p.T = total_tokens;
   p.H = num_heads;
   p.scale = scale;
+  kda::TensorMaps tm;
+  std::memset(&tm, 0, sizeof(tm));
+  if (total_tokens > 0) {
+    st = load_encoder();
+    if (st != KDA_OK) return st;
+    const int H = num_heads;
+    if ((st = encode_3d(&tm.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total_tokens, H, kda::D, kda::D)) != KDA_OK ||
+        (st = encode_3d(&tm.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total_tokens, H, kda::D, kda::D)) != KDA_OK ||
+        (st = encode_3d(&tm.g, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total_tokens, H, kda::D, kda::D)) != KDA_OK ||
+        (st = encode_3d(&tm.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total_tokens, H, kda::D, kda::NS)) != KDA_OK)
+      return st;
+  }
   dim3 grid(kda::NSLICE, num_heads, num_seqs);
-  kda::kda_fwd_kernel<<<grid, kda::NTHREADS, sizeof(kda::Shared), static_cast<cudaStream_t>(stream)>>>(p);
+  kda::kda_fwd_kernel<<<grid, kda::NTHREADS, sizeof(kda::Shared), static_cast<cudaStream_t>(stream)>>>(p, tm);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return KDA_OK;
