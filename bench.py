@@ -218,6 +218,22 @@ def aggregate(times_ms, units):
     return sum(units) / (t * 1e-3) / 1e6, t
 
 
+def reduce_over_ranks(ms: float, e2e_ms: float, units: float, device=None):
+    """Max of the per-rank times and sum of the per-rank work units over the
+    default process group (NCCL on GPUs, gloo on CPU). Returns
+    (ms, e2e_ms, total_units); identity without a process group."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return ms, e2e_ms, float(units)
+    tt = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    uu = torch.tensor([float(units)], dtype=torch.float64, device=device)
+    dist.all_reduce(uu)
+    return float(tt[0]), float(tt[1]), float(uu[0])
+
+
 # ---------------------------------------------------------------- reference
 def run_reference(args):
     ws, rank, _ = dist_env()
@@ -350,15 +366,7 @@ def run_kda(args):
 
     # ---- max over ranks
     units = work_units(inp)
-    if ws > 1:
-        tt = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms, e2e_ms = float(tt[0]), float(tt[1])
-        uu = torch.tensor([units], dtype=torch.float64, device=dev)
-        dist.all_reduce(uu)
-        total_units = float(uu[0])
-    else:
-        total_units = float(units)
+    ms, e2e_ms, total_units = reduce_over_ranks(ms, e2e_ms, units, device=dev)
     value = total_units / (ms * 1e-3) / 1e6
     e2e_value = total_units / (e2e_ms * 1e-3) / 1e6
 
