@@ -10,14 +10,14 @@
 //                in mma.sync accumulator registers (fp32) for the whole sequence
 //                and doubles, after a bf16 conversion, as the A operand of the
 //                next chunk's products, so it never touches shared memory.
-//     warps 4-7  "gate":   two key channels x eight tokens per thread. Per
-//                chunk they turn the gates into decay factors and write the
-//                chunk operands.
-//     warp  8    "mma":    A = Kd KR^T and Aqk = Qd KR^T (16 x 16 each), which
+//     warps 4-11 "gate":   two groups of four warps; group j takes chunks
+//                n = j (mod 2). Two key channels x eight tokens per thread; they
+//                turn the gates into decay factors and write the chunk operands.
+//     warp 12    "mma":    A = Kd KR^T and Aqk = Qd KR^T (16 x 16 each), which
 //                share their KR fragments; writes L = diag(beta) tril(A, -1)
 //                and the causal Aqk.
-//     warp  9    "solver": (I + L)^{-1} by forward substitution and T diag(beta).
-//     warp 10    "load":   one lane issues TMA tensor copies (q, k, g, the value
+//     warp 13    "solver": (I + L)^{-1} by forward substitution and T diag(beta).
+//     warp 14    "load":   one lane issues TMA tensor copies (q, k, g, the value
 //                slice and beta; five requests per chunk) into a ring of
 //                shared-memory stages, RSTAGE chunks ahead of the gates.
 //   Producers run up to NSTAGE chunks ahead of the chain through a second ring
@@ -63,11 +63,12 @@ constexpr int D = KDA_HEAD_DIM;   // dk = dv = 128
 constexpr int C = 16;             // chunk length (tokens)
 constexpr int NS = 32;            // value columns per CTA
 constexpr int NSLICE = D / NS;    // CTAs per (sequence, head)
-constexpr int NSTAGE = 3;         // operand stages (gate/solver -> chain)
+constexpr int NSTAGE = 4;         // operand stages (gate/solver -> chain)
 constexpr int RSTAGE = 6;         // raw-input stages (load -> gate)
 constexpr int NCHAIN = 4;         // chain warps
-constexpr int NGATE = 4;          // gate warps
-constexpr int WARP_MMA = NCHAIN + NGATE;
+constexpr int NGATE = 4;          // warps per gate group
+constexpr int NGROUP = 2;         // gate groups; group j takes the chunks n = j (mod 2)
+constexpr int WARP_MMA = NCHAIN + NGROUP * NGATE;
 constexpr int WARP_SOLVER = WARP_MMA + 1;
 constexpr int WARP_LOAD = WARP_SOLVER + 1;
 constexpr int NTHREADS = (WARP_LOAD + 1) * 32;
@@ -109,8 +110,8 @@ struct __align__(128) Shared {
   Stage st[NSTAGE];
   float xbuf[2][2][32][8];   // X^T partial sums exchanged inside a chain-warp pair
   float obuf[2][2][32][4];   // O^T partial sums exchanged inside a chain-warp pair
-  float2 gprod[2][2][64];    // per-half decay products exchanged inside the gate group,
-                             // double-buffered by chunk parity
+  float2 gprod[NGROUP][2][2][64];  // per-half decay products exchanged inside a gate
+                                   // group, double-buffered over the group's chunks
   unsigned long long full[NSTAGE];       // solver -> chain
   unsigned long long gate_done[NSTAGE];  // gate -> mma
   unsigned long long mma_done[NSTAGE];   // mma -> solver
@@ -376,7 +377,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float4* mine = reinterpret_cast<float4*>(&sh.xbuf[pr][dh][lane][0]);
         mine[0] = make_float4(x[0][0], x[0][1], x[0][2], x[0][3]);
         mine[1] = make_float4(x[1][0], x[1][1], x[1][2], x[1][3]);
-        named_bar(2 + pr, 64);
+        named_bar(1 + NGROUP + pr, 64);
         const float4* other = reinterpret_cast<const float4*>(&sh.xbuf[pr][dh ^ 1][lane][0]);
         const float4 u0 = other[0], u1 = other[1];
         x[0][0] += u0.x; x[0][1] += u0.y; x[0][2] += u0.z; x[0][3] += u0.w;
@@ -429,7 +430,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           give[e] = dh ? o[0][e] : o[1][e];
         }
         *reinterpret_cast<float4*>(&sh.obuf[pr][dh][lane][0]) = make_float4(give[0], give[1], give[2], give[3]);
-        named_bar(2 + pr, 64);
+        named_bar(1 + NGROUP + pr, 64);
         const float4 u = *reinterpret_cast<const float4*>(&sh.obuf[pr][dh ^ 1][lane][0]);
         const float o0 = (mine[0] + u.x) * p.scale, o1 = (mine[1] + u.y) * p.scale;
         const float o2 = (mine[2] + u.z) * p.scale, o3 = (mine[3] + u.w) * p.scale;
@@ -454,17 +455,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           p.fin[sbase + static_cast<size_t>(dk) * D + dv] = sT[nt][e];
         }
     }
-  } else if (warp < NCHAIN + NGATE) {
+  } else if (warp < NCHAIN + NGROUP * NGATE) {
     // ============================================================ gate warps
     // Thread layout: channel pair cp (channels 2cp, 2cp+1), token half th
     // (tokens 8th .. 8th+7). The decay products of the two halves meet through
     // shared memory.
-    const int gt = tid - GATE_T0;
-    const int gw = warp - NCHAIN;
+    const int grp = (warp - NCHAIN) / NGATE;
+    const int gt = tid - GATE_T0 - grp * NGATE * 32;
     const int cp = gt & 63;
     const int th = gt >> 6;
     const int c0 = 2 * cp;
-    for (int n = 0; n < nch; ++n) {
+    for (int n = grp; n < nch; n += NGROUP) {
+      const int gb = (n / NGROUP) & 1;  // double-buffer index of the product exchange
       const int s = n % NSTAGE;
       const uint32_t ph = static_cast<uint32_t>(n / NSTAGE) & 1u;
       const int rs = n % RSTAGE;
@@ -502,11 +504,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         P.y *= e[j].y;
       }
       mbar_wait(&sh.empty[s], ph ^ 1u);
-      sh.gprod[n & 1][th][cp] = P;
+      sh.gprod[grp][gb][th][cp] = P;
       if (gt < C) st.beta[gt] = bv;
       if (gt < 64) *reinterpret_cast<uint4*>(&st.v[gt >> 2][8 * (gt & 3)]) = vpiece;
-      named_bar(1, NGATE * 32);
-      const float2 Po = sh.gprod[n & 1][th ^ 1][cp];
+      named_bar(1 + grp, NGATE * 32);
+      const float2 Po = sh.gprod[grp][gb][th ^ 1][cp];
       // E before this half (1 for the first half), F after it (1 for the second)
       float2 E = th ? Po : make_float2(1.f, 1.f);
       float2 F = th ? make_float2(1.f, 1.f) : Po;
