@@ -21,7 +21,9 @@
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers on the current CUDA device.
- *   - The caller owns all memory; kda_fwd allocates nothing.
+ *   - The caller owns all inputs and outputs. kda_fwd takes a small scratch
+ *     ring (num_seqs * H * 8 slots of ~15 KB) from the device's stream-ordered
+ *     memory pool and returns it in stream order after the kernel.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and the call returns without synchronising.
  *   - Argument errors are reported synchronously through the return code and
@@ -91,6 +93,18 @@ const char* kda_status_string(kda_status_t status);
 /* Text of the last CUDA error seen by this thread inside the library
  * (static thread-local storage; "" if none). */
 const char* kda_last_cuda_error(void);
+
+/*
+ * kda_wait_timeouts -- health counter of the current device.
+ *
+ * Every wait inside the kernel (on a pipeline stage, on a peer CTA of the
+ * cluster) is bounded; a wait that runs out of budget increments a device
+ * counter and lets the kernel finish instead of hanging (its results are then
+ * undefined). This reads the counter into *count (synchronising with the
+ * device) and resets it to zero when `reset` is non-zero. A healthy run leaves
+ * it at 0.
+ */
+kda_status_t kda_wait_timeouts(uint32_t* count, int32_t reset);
 
 /* KDA_ABI_VERSION of the loaded library. */
 int32_t kda_abi_version(void);

@@ -14,7 +14,7 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["kda_fwd", "library_path", "KDAError", "HEAD_DIM"]
+__all__ = ["kda_fwd", "library_path", "wait_timeouts", "KDAError", "HEAD_DIM"]
 
 HEAD_DIM = 128
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -23,7 +23,7 @@ _LIB_PATH = os.path.join(_PKG, "libkda.so")
 if not os.path.exists(_LIB_PATH):
     raise ImportError(
         f"{_LIB_PATH} is missing: build the CUDA library first "
-        "(python -m kimi_delta_attention_26_b200.build or __graft_entry__.build())")
+        "(python kimi_delta_attention_26_b200/build.py or __graft_entry__.build())")
 
 _lib = ctypes.CDLL(_LIB_PATH)
 _P = ctypes.c_void_p
@@ -36,6 +36,8 @@ _lib.kda_last_cuda_error.argtypes = []
 _lib.kda_last_cuda_error.restype = ctypes.c_char_p
 _lib.kda_abi_version.argtypes = []
 _lib.kda_abi_version.restype = ctypes.c_int32
+_lib.kda_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32]
+_lib.kda_wait_timeouts.restype = ctypes.c_int
 
 
 class KDAError(RuntimeError):
@@ -48,6 +50,16 @@ class KDAError(RuntimeError):
 
 def library_path() -> str:
     return _LIB_PATH
+
+
+def wait_timeouts(reset: bool = True) -> int:
+    """Bounded in-kernel waits that ran out of budget on the current device
+    since the last reset (0 for a healthy run); synchronises with the device."""
+    n = ctypes.c_uint32(0)
+    rc = _lib.kda_wait_timeouts(ctypes.byref(n), 1 if reset else 0)
+    if rc != 0:
+        raise KDAError(rc)
+    return int(n.value)
 
 
 def _check(t: torch.Tensor, name: str, dtype: torch.dtype, shape: Tuple[int, ...], device) -> None:

@@ -1,44 +1,46 @@
 // kda_fwd.cu -- chunked Kimi Delta Attention forward (prefill) for sm_100a.
 //
 // Work decomposition
-//   One CTA per (sequence, head, 32-column value slice). Columns of the state
-//   evolve independently (the recurrence multiplies S only from the left), so
-//   slices never exchange data. Inside a CTA, warps specialise:
-//     warps 0-3  "chain":  the serial state recurrence. Warp w owns the state
-//                transpose S^T[16 value rows x 64 key columns]: value block
-//                w>>1 (16 of the 32 columns) and key half w&1. The state lives
-//                in mma.sync accumulator registers (fp32) for the whole sequence
-//                and doubles, after a bf16 conversion, as the A operand of the
-//                next chunk's products, so it never touches shared memory.
-//     warps 4-11 "gate":   two groups of four warps; group j takes chunks
-//                n = j (mod 2). Two key channels x eight tokens per thread; they
-//                turn the gates into decay factors and write the chunk operands.
-//     warp 12    "mma":    A = Kd KR^T and Aqk = Qd KR^T (16 x 16 each), which
-//                share their KR fragments; writes L = diag(beta) tril(A, -1)
-//                and the causal Aqk.
-//     warp 13    "solver": (I + L)^{-1} by forward substitution and T diag(beta).
-//     warp 14    "load":   one lane issues TMA tensor copies (q, k, g, the value
-//                slice and beta; five requests per chunk) into a ring of
-//                shared-memory stages, RSTAGE chunks ahead of the gates.
-//   Producers run up to NSTAGE chunks ahead of the chain through a second ring
-//   of operand stages; every hand-off is an mbarrier.
+//   One thread-block cluster per (sequence, head): four CTAs, one per 32-column
+//   value slice. Columns of the state evolve independently (the recurrence
+//   multiplies S only from the left), so the four state chains never exchange
+//   data. What they share is the chunk-local work on keys, queries and gates,
+//   which is identical for every slice: CTA n mod 4 of the cluster produces the
+//   shared operands of chunk n once, stores them to an L2-resident ring in
+//   global memory and signals the four CTAs with remote mbarrier arrivals; every
+//   CTA then pulls the chunk with one bulk copy.
+//
+//   Warp roles inside a CTA:
+//     0-3   chain:  the serial state recurrence of this CTA's value slice. Warp w
+//                   owns S^T[16 value rows x 64 key columns] (value block w>>1, key
+//                   half w&1) in mma.sync accumulator registers for the whole
+//                   sequence; its bf16 conversion is the A operand of the next
+//                   chunk's products, so the state never touches shared memory.
+//     4-7   gate:   (producer) two key channels x eight tokens per thread: decay
+//                   factors and the bf16 operand tiles of the chunks this CTA owns.
+//     8     mma:    (producer) A = Kd KR^T and Aqk = Qd KR^T, 16 x 16 each.
+//     9     solver: (producer) T = (I + L)^{-1} by forward substitution, T diag(beta).
+//     10    store:  (producer) bulk-stores a finished chunk to its ring slot and
+//                   signals the cluster.
+//     11    pload:  (producer) TMA loads of q, k, g (and beta) for owned chunks.
+//     12    cload:  (consumer) bulk-loads every chunk's shared operands from the
+//                   ring and the value slice with TMA, in order, for the chain.
 //
 // Per chunk of C = 16 tokens, with Gamma_i the inclusive cumulative log-decay
 // inside the chunk (e_i = exp(g_i) per channel):
 //   E_i = prod_{s<=i} e_s = exp(Gamma_i),  F_i = prod_{s>i} e_s = exp(Gamma_last - Gamma_i)
-//   Kd = k*E,  Qd = q*E,  KR = k*F/gamma = k*exp(-Gamma),  Kend = k*F,  gamma = E_last
-//   A   = tril(Kd KR^T, -1),  L = diag(beta) A,  Aqk = tril(Qd KR^T)
+//   Kd = -k*E,  Qd = q*E,  KR = k*F/gamma = k*exp(-Gamma),  Kend = k*F,  gamma = E_last
+//   A   = tril(k E (k/E)^T, -1) = -tril(Kd KR^T, -1),  L = diag(beta) A,  Aqk = tril(Qd KR^T)
 //   Tb  = (I + L)^{-1} diag(beta)
-//   X   = V - Kd S,   Vnew = Tb X          (the chunk's delta-rule writes)
+//   X   = V + Kd S  (= V - k*E S),   Vnew = Tb X       (the chunk's delta-rule writes)
 //   O   = scale (Qd S + Aqk Vnew)
 //   S  <- Diag(gamma) S + Kend^T Vnew
-// All factors stay in [e^-80, e^80] because -5 <= g <= 0 and a chunk has 16
-// tokens; this is the bound that lets FlashKDA keep 16-token causal blocks on
-// dense tensor-core products (page "Kimi K3 开源满月…", section
-// "KDA 内核到底难在哪": 16-token chunks, lower_bound = -5). The chain works
-// on S^T so that every product on it takes the register-resident state as
-// its A operand: X^T = V^T - S^T Kd^T, Vnew^T = X^T Tb^T,
-// S^T <- S^T Diag(gamma) + Vnew^T Kend.
+// All factors stay within [e^-80, e^80] because -5 <= g <= 0 and a chunk has 16
+// tokens: the bound that lets FlashKDA keep 16-token causal blocks on dense
+// tensor-core products (page "Kimi K3 开源满月…", section "KDA 内核到底难在哪":
+// 16-token chunks, lower_bound = -5). The chain works on S^T so that every
+// product on it takes the register-resident state as its A operand:
+// X^T = V^T + S^T Kd^T, Vnew^T = X^T Tb^T, S^T <- S^T Diag(gamma) + Vnew^T Kend.
 //
 // Tensor cores: mma.sync m16n8k16 (bf16 in, fp32 accumulate). On this part a
 // dependent m16n8k16 completes in ~21 cycles while a tcgen05.mma of the shapes
@@ -62,69 +64,80 @@ namespace kda {
 constexpr int D = KDA_HEAD_DIM;   // dk = dv = 128
 constexpr int C = 16;             // chunk length (tokens)
 constexpr int NS = 32;            // value columns per CTA
-constexpr int NSLICE = D / NS;    // CTAs per (sequence, head)
-constexpr int NSTAGE = 4;         // operand stages (gate/solver -> chain)
-constexpr int RSTAGE = 6;         // raw-input stages (load -> gate)
-constexpr int NCHAIN = 4;         // chain warps
-constexpr int NGATE = 4;          // warps per gate group
-constexpr int NGROUP = 2;         // gate groups; group j takes the chunks n = j (mod 2)
-constexpr int WARP_MMA = NCHAIN + NGROUP * NGATE;
+constexpr int NSLICE = D / NS;    // CTAs per (sequence, head) = cluster size
+constexpr int RING = 8;           // ring slots per (sequence, head); multiple of NSLICE
+constexpr int PRSTAGE = 2;        // producer raw-input stages
+constexpr int PSTAGE = 2;         // producer operand stages
+constexpr int CSTAGE = 4;         // consumer stages (cload -> chain)
+constexpr int NCHAIN = 4;
+constexpr int NGATE = 4;
+constexpr int WARP_GATE = NCHAIN;
+constexpr int WARP_MMA = WARP_GATE + NGATE;
 constexpr int WARP_SOLVER = WARP_MMA + 1;
-constexpr int WARP_LOAD = WARP_SOLVER + 1;
-constexpr int NTHREADS = (WARP_LOAD + 1) * 32;
-constexpr int GATE_T0 = NCHAIN * 32;  // first gate thread
+constexpr int WARP_STORE = WARP_SOLVER + 1;
+constexpr int WARP_PLOAD = WARP_STORE + 1;
+constexpr int WARP_CLOAD = WARP_PLOAD + 1;
+constexpr int NTHREADS = (WARP_CLOAD + 1) * 32;
+static_assert(RING % NSLICE == 0, "a ring slot must always belong to the same producer CTA");
 
-// Padded row pitches: 272 B, 48 B and 80 B rows keep 8-row ldmatrix reads on
-// distinct banks.
+// Padded row pitches: 272 B and 48 B rows keep 8-row ldmatrix reads on distinct banks.
 constexpr int LDK = D + 8;
 constexpr int LDC = C + 8;
-constexpr int LDV = NS + 8;
 
-struct __align__(16) Stage {
-  __nv_bfloat16 kd[C][LDK];
-  __nv_bfloat16 qd[C][LDK];
-  __nv_bfloat16 kr[C][LDK];
-  __nv_bfloat16 ke[C][LDK];
-  __nv_bfloat16 tb[C][LDC];
-  __nv_bfloat16 aqk[C][LDC];
-  __nv_bfloat16 v[C][LDV];
-  float L[C][C + 4];   // 80-byte rows: 16-byte aligned for row-broadcast loads
-  float gam[D];
-  float beta[C];
-};
-
-// One chunk of raw inputs, exactly as the TMA boxes land: q, k [16 tokens][128],
-// g [16][128], value slice [16][32]; beta [16] arrives by 4-byte copies.
+// Raw inputs of one owned chunk, as the TMA boxes land (beta by 4-byte copies).
 struct __align__(128) RawStage {
   __nv_bfloat16 q[C][D];
   __nv_bfloat16 k[C][D];
   float g[C][D];
-  __nv_bfloat16 v[C][NS];
   float beta[C];
   float pad_[32 - C];
 };
-constexpr uint32_t kRawBytes = C * D * 2 * 2 + C * D * 4 + C * NS * 2;  // bytes the TMA boxes bring
+constexpr uint32_t kRawBytes = C * D * 2 * 2 + C * D * 4;  // bytes the TMA boxes bring
+
+// Shared operands of one chunk; byte-for-byte the layout of a ring slot.
+struct __align__(128) Ops {
+  __nv_bfloat16 kd[C][LDK];   // -k * exp(Gamma)
+  __nv_bfloat16 qd[C][LDK];   //  q * exp(Gamma)
+  __nv_bfloat16 ke[C][LDK];   //  k * exp(Gamma_last - Gamma)
+  __nv_bfloat16 tb[C][LDC];   //  (I + L)^{-1} diag(beta)
+  __nv_bfloat16 aqk[C][LDC];  //  causal Qd KR^T
+  float gam[D];               //  exp(Gamma_last)
+};
+constexpr uint32_t kSlotBytes = sizeof(Ops);
+
+struct __align__(128) ProdStage {
+  Ops ops;
+  __nv_bfloat16 kr[C][LDK];   // k * exp(-Gamma)
+  float L[C][C + 4];          // 80-byte rows: 16-byte aligned for row-broadcast loads
+  float beta[C];
+};
+
+struct __align__(128) ChainStage {
+  Ops ops;
+  __nv_bfloat16 v[C][NS];     // value slice, as its TMA box lands
+};
+constexpr uint32_t kChainBytes = kSlotBytes + C * NS * 2;
 
 struct __align__(128) Shared {
-  RawStage raw[RSTAGE];
-  Stage st[NSTAGE];
+  RawStage raw[PRSTAGE];
+  ProdStage prod[PSTAGE];
+  ChainStage cst[CSTAGE];
   float xbuf[2][2][32][8];   // X^T partial sums exchanged inside a chain-warp pair
   float obuf[2][2][32][4];   // O^T partial sums exchanged inside a chain-warp pair
-  float2 gprod[NGROUP][2][2][64];  // per-half decay products exchanged inside a gate
-                                   // group, double-buffered over the group's chunks
-  unsigned long long full[NSTAGE];       // solver -> chain
-  unsigned long long gate_done[NSTAGE];  // gate -> mma
-  unsigned long long mma_done[NSTAGE];   // mma -> solver
-  unsigned long long empty[NSTAGE];      // chain -> gate
-  unsigned long long raw_full[RSTAGE];   // load -> gate
-  unsigned long long raw_empty[RSTAGE];  // gate -> load
+  float2 gprod[2][2][64];    // per-half decay products exchanged inside the gate group
+  unsigned long long raw_full[PRSTAGE], raw_empty[PRSTAGE];
+  unsigned long long prod_free[PSTAGE], gate_done[PSTAGE], mma_done[PSTAGE], solved[PSTAGE];
+  unsigned long long c_full[CSTAGE], c_empty[CSTAGE];
+  unsigned long long ready[RING];      // arrived (remotely) by the slot's producer
+  unsigned long long slot_free[RING];  // arrived (remotely) by the four consumers
 };
-static_assert(sizeof(Stage) % 16 == 0 && sizeof(RawStage) % 128 == 0, "stage alignment");
+static_assert(sizeof(Ops) % 128 == 0 && sizeof(RawStage) % 128 == 0, "stage alignment");
+static_assert(sizeof(ProdStage) % 128 == 0 && sizeof(ChainStage) % 128 == 0, "stage alignment");
 static_assert(sizeof(Shared) <= 227 * 1024, "shared memory budget");
 
 // Wait budget for every mbarrier wait (cycles). A wait that runs out records
 // a timeout and lets the thread continue, so no barrier is ever left waiting.
-constexpr long long kWaitCycles = 4ll << 30;
+constexpr long long kWaitCycles = 1ll << 28;  // ~0.14 s at 1.9 GHz
 // A waiting thread is suspended in hardware (up to this many ns per try)
 // instead of spinning, so waiting warps leave the issue slots to the others.
 constexpr uint32_t kSuspendHintNs = 20000;
@@ -242,6 +255,67 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return u;
 }
 
+
+// ---- cluster-scope signalling
+__device__ __forceinline__ bool mbar_try_wait_cl(unsigned long long* m, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(smem_u32(m)), "r"(parity), "r"(kSuspendHintNs)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ void mbar_wait_cl(unsigned long long* m, uint32_t parity) {
+  if (mbar_try_wait_cl(m, parity)) return;
+  const long long t0 = clock64();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait_cl(m, parity)) return;
+    if ((i & 63u) == 0 && clock64() - t0 > kWaitCycles) {
+      atomicAdd(&g_wait_timeouts, 1u);
+      return;
+    }
+  }
+}
+
+// Arrive on the mbarrier at the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ void mbar_arrive_remote(unsigned long long* m, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(m)), "r"(rank));
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Generic-proxy shared-memory writes become visible to the bulk-copy engine.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Bulk copy shared -> global; returns once the writes have completed.
+__device__ __forceinline__ void bulk_s2g_sync(void* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(ssrc)),
+               "r"(bytes)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Bulk copy global -> shared, completion counted in bytes on the mbarrier.
+__device__ __forceinline__ void bulk_g2s(void* sdst, const void* gsrc, uint32_t bytes, unsigned long long* m) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(sdst)),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(m))
+      : "memory");
+}
+
 // A fragment (16 rows x 16 k) from two accumulator tiles (16 rows x 8 cols each)
 // holding k columns [0, 8) and [8, 16).
 __device__ __forceinline__ void acc_to_afrag(uint32_t (&a)[4], const float (&lo)[4], const float (&hi)[4]) {
@@ -258,22 +332,21 @@ struct Params {
   const __nv_bfloat16* v;
   const float* g;
   const float* beta;
-  const int32_t* cu;   // may be null: one sequence [0, T)
-  const float* init;   // may be null
+  const int32_t* cu;       // may be null: one sequence [0, T)
+  const float* init;       // may be null
   __nv_bfloat16* out;
-  float* fin;          // may be null
+  float* fin;              // may be null
+  unsigned char* ring;     // [num_seqs * H][RING] slots of kSlotBytes
   int64_t T;
   int32_t H;
   float scale;
 };
 
-__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
-
 struct TensorMaps {
   CUtensorMap q, k, g, v;
 };
 
-__global__ void __launch_bounds__(NTHREADS, 1)
+__global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
     kda_fwd_kernel(const Params p, const __grid_constant__ TensorMaps tm) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   Shared& sh = *reinterpret_cast<Shared*>(smem_raw);
@@ -284,10 +357,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int gq = lane >> 2;  // fragment row group
   const int tq = lane & 3;   // fragment column pair
 
-  const int slice = blockIdx.x;
+  const int rank = blockIdx.x;  // value slice = rank inside the cluster
   const int h = blockIdx.y;
   const int seq = blockIdx.z;
-  const int dv0 = slice * NS;
+  const int dv0 = rank * NS;
   const int H = p.H;
   const int64_t T = p.T;
   const size_t row_stride = static_cast<size_t>(H) * D;  // elements between tokens of q/k/v/g/out
@@ -300,21 +373,32 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     t1 = t1 < t0 ? t0 : (t1 > T ? T : t1);
   }
   const int nch = static_cast<int>((t1 - t0 + C - 1) / C);
+  const int nprod = nch > rank ? (nch - rank + NSLICE - 1) / NSLICE : 0;  // chunks this CTA produces
+  unsigned char* ring = p.ring + (static_cast<size_t>(seq) * H + h) * RING * kSlotBytes;
 
   if (tid == 0) {
-    for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(&sh.full[s], 1);
-      mbar_init(&sh.gate_done[s], NGATE);
-      mbar_init(&sh.mma_done[s], 1);
-      mbar_init(&sh.empty[s], NCHAIN);
-    }
-    for (int s = 0; s < RSTAGE; ++s) {
+    for (int s = 0; s < PRSTAGE; ++s) {
       mbar_init(&sh.raw_full[s], 1 + C);  // expect_tx arrive + one per beta lane
       mbar_init(&sh.raw_empty[s], NGATE);
     }
+    for (int s = 0; s < PSTAGE; ++s) {
+      mbar_init(&sh.prod_free[s], 1);
+      mbar_init(&sh.gate_done[s], NGATE);
+      mbar_init(&sh.mma_done[s], 1);
+      mbar_init(&sh.solved[s], 1);
+    }
+    for (int s = 0; s < CSTAGE; ++s) {
+      mbar_init(&sh.c_full[s], 1);
+      mbar_init(&sh.c_empty[s], NCHAIN);
+    }
+    for (int s = 0; s < RING; ++s) {
+      mbar_init(&sh.ready[s], 1);
+      mbar_init(&sh.slot_free[s], NSLICE);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  __syncthreads();
+  // every CTA's barriers exist before any remote arrive
+  cluster_sync();
 
   if (warp < NCHAIN) {
     // =========================================================== chain warps
@@ -336,14 +420,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
 
     for (int n = 0; n < nch; ++n) {
-      const int s = n % NSTAGE;
-      const uint32_t ph = static_cast<uint32_t>(n / NSTAGE) & 1u;
+      const int s = n % CSTAGE;
+      const uint32_t ph = static_cast<uint32_t>(n / CSTAGE) & 1u;
       const int64_t cs = t0 + static_cast<int64_t>(n) * C;
       const int m = static_cast<int>((t1 - cs) < C ? (t1 - cs) : C);
-      Stage& st = sh.st[s];
-      mbar_wait(&sh.full[s], ph);
+      ChainStage& st = sh.cst[s];
+      mbar_wait(&sh.c_full[s], ph);
+      // the ring slot has been copied here: give it back to its producer
+      if (warp == 0 && lane == 0) mbar_arrive_remote(&sh.slot_free[n % RING], static_cast<uint32_t>(n % NSLICE));
 
-      // ---- X^T = V^T - S^T Kd^T and O^T = S^T Qd^T over this warp's key half
+      // ---- X^T = V^T + S^T Kd^T and O^T = S^T Qd^T over this warp's key half
       float x[2][4], o[2][4];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
@@ -359,16 +445,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        uint32_t a[4], an[4], bk[4], bq[4];
+        uint32_t a[4], bk[4], bq[4];
         acc_to_afrag(a, sT[2 * kk], sT[2 * kk + 1]);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) an[e] = a[e] ^ 0x80008000u;  // -S^T (exact sign flip)
         const int row = (lane & 7) + ((lane >> 4) << 3);
         const int col = k0 + 16 * kk + ((lane >> 3) & 1) * 8;
-        ldsm_x4(bk, &st.kd[row][col]);
-        ldsm_x4(bq, &st.qd[row][col]);
-        mma(x[0], an, bk[0], bk[1]);
-        mma(x[1], an, bk[2], bk[3]);
+        ldsm_x4(bk, &st.ops.kd[row][col]);
+        ldsm_x4(bq, &st.ops.qd[row][col]);
+        mma(x[0], a, bk[0], bk[1]);
+        mma(x[1], a, bk[2], bk[3]);
         mma(o[0], a, bq[0], bq[1]);
         mma(o[1], a, bq[2], bq[3]);
       }
@@ -377,7 +461,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float4* mine = reinterpret_cast<float4*>(&sh.xbuf[pr][dh][lane][0]);
         mine[0] = make_float4(x[0][0], x[0][1], x[0][2], x[0][3]);
         mine[1] = make_float4(x[1][0], x[1][1], x[1][2], x[1][3]);
-        named_bar(1 + NGROUP + pr, 64);
+        named_bar(2 + pr, 64);
         const float4* other = reinterpret_cast<const float4*>(&sh.xbuf[pr][dh ^ 1][lane][0]);
         const float4 u0 = other[0], u1 = other[1];
         x[0][0] += u0.x; x[0][1] += u0.y; x[0][2] += u0.z; x[0][3] += u0.w;
@@ -389,7 +473,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       acc_to_afrag(ax, x[0], x[1]);
       {
         uint32_t bt[4];
-        ldsm_x4(bt, &st.tb[(lane & 7) + ((lane >> 4) << 3)][((lane >> 3) & 1) * 8]);
+        ldsm_x4(bt, &st.ops.tb[(lane & 7) + ((lane >> 4) << 3)][((lane >> 3) & 1) * 8]);
         mma(vn[0], ax, bt[0], bt[1]);
         mma(vn[1], ax, bt[2], bt[3]);
       }
@@ -397,14 +481,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // ---- O^T += Vnew^T Aqk^T (once per pair)
       if (dh == 0) {
         uint32_t ba[4];
-        ldsm_x4(ba, &st.aqk[(lane & 7) + ((lane >> 4) << 3)][((lane >> 3) & 1) * 8]);
+        ldsm_x4(ba, &st.ops.aqk[(lane & 7) + ((lane >> 4) << 3)][((lane >> 3) & 1) * 8]);
         mma(o[0], av, ba[0], ba[1]);
         mma(o[1], av, ba[2], ba[3]);
       }
       // ---- S^T <- S^T Diag(gamma) + Vnew^T Kend   (this warp's key half)
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
-        const float2 gm = *reinterpret_cast<const float2*>(&st.gam[k0 + 8 * nt + 2 * tq]);
+        const float2 gm = *reinterpret_cast<const float2*>(&st.ops.gam[k0 + 8 * nt + 2 * tq]);
         sT[nt][0] *= gm.x;
         sT[nt][1] *= gm.y;
         sT[nt][2] *= gm.x;
@@ -413,16 +497,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
       for (int np = 0; np < 4; ++np) {
         uint32_t be[4];
-        ldsm_x4_t(be, &st.ke[(lane & 7) + ((lane >> 3) & 1) * 8][k0 + 16 * np + (lane >> 4) * 8]);
+        ldsm_x4_t(be, &st.ops.ke[(lane & 7) + ((lane >> 3) & 1) * 8][k0 + 16 * np + (lane >> 4) * 8]);
         mma(sT[2 * np], av, be[0], be[1]);
         mma(sT[2 * np + 1], av, be[2], be[3]);
       }
-      // the stage is no longer read by this thread
-      mbar_arrive_warp(&sh.empty[s]);
+      // the stage is no longer read by this warp
+      mbar_arrive_warp(&sh.c_empty[s]);
       // ---- O: each warp of the pair finishes one 8-token half (register
       // selects, not a runtime array index, keep o[][] in registers)
       {
-        const int keep = dh;
         float mine[4], give[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -430,14 +513,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           give[e] = dh ? o[0][e] : o[1][e];
         }
         *reinterpret_cast<float4*>(&sh.obuf[pr][dh][lane][0]) = make_float4(give[0], give[1], give[2], give[3]);
-        named_bar(1 + NGROUP + pr, 64);
+        named_bar(2 + pr, 64);
         const float4 u = *reinterpret_cast<const float4*>(&sh.obuf[pr][dh ^ 1][lane][0]);
         const float o0 = (mine[0] + u.x) * p.scale, o1 = (mine[1] + u.y) * p.scale;
         const float o2 = (mine[2] + u.z) * p.scale, o3 = (mine[3] + u.w) * p.scale;
         // fragment rows = value columns, cols = tokens -> transpose to token rows
         const uint32_t r0 = movmatrix_t(pack_bf16(o0, o1));
         const uint32_t r1 = movmatrix_t(pack_bf16(o2, o3));
-        const int tok = 8 * keep + gq;
+        const int tok = 8 * dh + gq;
         if (tok < m) {
           __nv_bfloat16* dst = p.out + (cs + tok) * row_stride + static_cast<size_t>(h) * D + dv0 + vrow + 2 * tq;
           *reinterpret_cast<uint32_t*>(dst) = r0;
@@ -455,43 +538,39 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           p.fin[sbase + static_cast<size_t>(dk) * D + dv] = sT[nt][e];
         }
     }
-  } else if (warp < NCHAIN + NGROUP * NGATE) {
+  } else if (warp < WARP_MMA) {
     // ============================================================ gate warps
     // Thread layout: channel pair cp (channels 2cp, 2cp+1), token half th
     // (tokens 8th .. 8th+7). The decay products of the two halves meet through
     // shared memory.
-    const int grp = (warp - NCHAIN) / NGATE;
-    const int gt = tid - GATE_T0 - grp * NGATE * 32;
+    const int gt = tid - WARP_GATE * 32;
     const int cp = gt & 63;
     const int th = gt >> 6;
     const int c0 = 2 * cp;
-    for (int n = grp; n < nch; n += NGROUP) {
-      const int gb = (n / NGROUP) & 1;  // double-buffer index of the product exchange
-      const int s = n % NSTAGE;
-      const uint32_t ph = static_cast<uint32_t>(n / NSTAGE) & 1u;
-      const int rs = n % RSTAGE;
-      const uint32_t rph = static_cast<uint32_t>(n / RSTAGE) & 1u;
+    for (int j = 0; j < nprod; ++j) {
+      const int n = rank + NSLICE * j;
+      const int rs = j % PRSTAGE, ps = j % PSTAGE;
+      const uint32_t rph = static_cast<uint32_t>(j / PRSTAGE) & 1u;
+      const uint32_t pph = static_cast<uint32_t>(j / PSTAGE) & 1u;
       const int64_t cs = t0 + static_cast<int64_t>(n) * C;
       const int m = static_cast<int>((t1 - cs) < C ? (t1 - cs) : C);
       RawStage& rw = sh.raw[rs];
-      Stage& st = sh.st[s];
+      ProdStage& st = sh.prod[ps];
       mbar_wait(&sh.raw_full[rs], rph);
 
       // ---- raw inputs of this thread (rows past the sequence end masked)
       float2 e[8], kv[8], qv[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int i = 8 * th + j;
+      for (int jj = 0; jj < 8; ++jj) {
+        const int i = 8 * th + jj;
         const bool ok = i < m;
         const float2 gg = *reinterpret_cast<const float2*>(&rw.g[i][c0]);
         const __nv_bfloat162 kk = *reinterpret_cast<const __nv_bfloat162*>(&rw.k[i][c0]);
         const __nv_bfloat162 qq = *reinterpret_cast<const __nv_bfloat162*>(&rw.q[i][c0]);
-        e[j] = ok ? make_float2(__expf(gg.x), __expf(gg.y)) : make_float2(1.f, 1.f);
-        kv[j] = ok ? __bfloat1622float2(kk) : make_float2(0.f, 0.f);
-        qv[j] = ok ? __bfloat1622float2(qq) : make_float2(0.f, 0.f);
+        e[jj] = ok ? make_float2(__expf(gg.x), __expf(gg.y)) : make_float2(1.f, 1.f);
+        kv[jj] = ok ? __bfloat1622float2(kk) : make_float2(0.f, 0.f);
+        qv[jj] = ok ? __bfloat1622float2(qq) : make_float2(0.f, 0.f);
       }
-      uint4 vpiece = make_uint4(0, 0, 0, 0);  // value-slice tile: 16 rows x 64 bytes
-      if (gt < 64 && (gt >> 2) < m) vpiece = *reinterpret_cast<const uint4*>(&rw.v[gt >> 2][8 * (gt & 3)]);
       float bv = 0.f;
       if (gt < C) bv = gt < m ? rw.beta[gt] : 0.f;
       mbar_arrive_warp(&sh.raw_empty[rs]);
@@ -499,79 +578,81 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // ---- decay products: this half's total, exchanged with the other half
       float2 P = make_float2(1.f, 1.f);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        P.x *= e[j].x;
-        P.y *= e[j].y;
+      for (int jj = 0; jj < 8; ++jj) {
+        P.x *= e[jj].x;
+        P.y *= e[jj].y;
       }
-      mbar_wait(&sh.empty[s], ph ^ 1u);
-      sh.gprod[grp][gb][th][cp] = P;
+      mbar_wait(&sh.prod_free[ps], pph ^ 1u);
+      sh.gprod[j & 1][th][cp] = P;
       if (gt < C) st.beta[gt] = bv;
-      if (gt < 64) *reinterpret_cast<uint4*>(&st.v[gt >> 2][8 * (gt & 3)]) = vpiece;
-      named_bar(1 + grp, NGATE * 32);
-      const float2 Po = sh.gprod[grp][gb][th ^ 1][cp];
+      named_bar(1, NGATE * 32);
+      const float2 Po = sh.gprod[j & 1][th ^ 1][cp];
       // E before this half (1 for the first half), F after it (1 for the second)
       float2 E = th ? Po : make_float2(1.f, 1.f);
       float2 F = th ? make_float2(1.f, 1.f) : Po;
       const float2 gamma = make_float2(P.x * Po.x, P.y * Po.y);
       const float2 rg = make_float2(__frcp_rn(gamma.x), __frcp_rn(gamma.y));
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int i = 8 * th + j;
-        E.x *= e[j].x;
-        E.y *= e[j].y;
-        *reinterpret_cast<uint32_t*>(&st.kd[i][c0]) = pack_bf16(kv[j].x * E.x, kv[j].y * E.y);
-        *reinterpret_cast<uint32_t*>(&st.qd[i][c0]) = pack_bf16(qv[j].x * E.x, qv[j].y * E.y);
+      for (int jj = 0; jj < 8; ++jj) {
+        const int i = 8 * th + jj;
+        E.x *= e[jj].x;
+        E.y *= e[jj].y;
+        *reinterpret_cast<uint32_t*>(&st.ops.kd[i][c0]) = pack_bf16(-kv[jj].x * E.x, -kv[jj].y * E.y);
+        *reinterpret_cast<uint32_t*>(&st.ops.qd[i][c0]) = pack_bf16(qv[jj].x * E.x, qv[jj].y * E.y);
       }
 #pragma unroll
-      for (int j = 7; j >= 0; --j) {
-        const int i = 8 * th + j;
-        const float kfx = kv[j].x * F.x, kfy = kv[j].y * F.y;
-        *reinterpret_cast<uint32_t*>(&st.ke[i][c0]) = pack_bf16(kfx, kfy);
+      for (int jj = 7; jj >= 0; --jj) {
+        const int i = 8 * th + jj;
+        const float kfx = kv[jj].x * F.x, kfy = kv[jj].y * F.y;
+        *reinterpret_cast<uint32_t*>(&st.ops.ke[i][c0]) = pack_bf16(kfx, kfy);
         *reinterpret_cast<uint32_t*>(&st.kr[i][c0]) = pack_bf16(kfx * rg.x, kfy * rg.y);
-        F.x *= e[j].x;
-        F.y *= e[j].y;
+        F.x *= e[jj].x;
+        F.y *= e[jj].y;
       }
-      if (th == 0) *reinterpret_cast<float2*>(&st.gam[c0]) = gamma;
-      mbar_arrive_warp(&sh.gate_done[s]);
+      if (th == 0) *reinterpret_cast<float2*>(&st.ops.gam[c0]) = gamma;
+      fence_proxy_async_shared();
+      mbar_arrive_warp(&sh.gate_done[ps]);
     }
   } else if (warp == WARP_MMA) {
     // ============================================================= mma warp
-    for (int n = 0; n < nch; ++n) {
-      const int s = n % NSTAGE;
-      const uint32_t ph = static_cast<uint32_t>(n / NSTAGE) & 1u;
-      Stage& st = sh.st[s];
-      mbar_wait(&sh.gate_done[s], ph);
+    for (int j = 0; j < nprod; ++j) {
+      const int ps = j % PSTAGE;
+      const uint32_t pph = static_cast<uint32_t>(j / PSTAGE) & 1u;
+      ProdStage& st = sh.prod[ps];
+      mbar_wait(&sh.gate_done[ps], pph);
       float accA[2][4] = {}, accQ[2][4] = {};
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         uint32_t ak[4], aq[4], b[4];
-        ldsm_x4(ak, &st.kd[lane & 15][16 * kk + (lane >> 4) * 8]);
-        ldsm_x4(aq, &st.qd[lane & 15][16 * kk + (lane >> 4) * 8]);
+        ldsm_x4(ak, &st.ops.kd[lane & 15][16 * kk + (lane >> 4) * 8]);
+        ldsm_x4(aq, &st.ops.qd[lane & 15][16 * kk + (lane >> 4) * 8]);
         ldsm_x4(b, &st.kr[(lane & 7) + ((lane >> 4) << 3)][16 * kk + ((lane >> 3) & 1) * 8]);
         mma(accA[0], ak, b[0], b[1]);
         mma(accA[1], ak, b[2], b[3]);
         mma(accQ[0], aq, b[0], b[1]);
         mma(accQ[1], aq, b[2], b[3]);
       }
+      // accA = -A (Kd carries the sign): L = diag(beta) A = -beta_i accA
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e2 = 0; e2 < 4; ++e2) {
           const int i = gq + 8 * (e2 >> 1);
-          const int j = 8 * nt + 2 * tq + (e2 & 1);
-          st.L[i][j] = (j < i) ? st.beta[i] * accA[nt][e2] : 0.f;
-          st.aqk[i][j] = __float2bfloat16_rn((j <= i) ? accQ[nt][e2] : 0.f);
+          const int jc = 8 * nt + 2 * tq + (e2 & 1);
+          st.L[i][jc] = (jc < i) ? -st.beta[i] * accA[nt][e2] : 0.f;
+          st.ops.aqk[i][jc] = __float2bfloat16_rn((jc <= i) ? accQ[nt][e2] : 0.f);
         }
-      mbar_arrive_warp(&sh.mma_done[s]);
+      fence_proxy_async_shared();
+      mbar_arrive_warp(&sh.mma_done[ps]);
     }
   } else if (warp == WARP_SOLVER) {
     // =========================================================== solver warp
     // lanes 0-15: one column of (I + L)^{-1} each, scaled by beta of that column
-    for (int n = 0; n < nch; ++n) {
-      const int s = n % NSTAGE;
-      const uint32_t ph = static_cast<uint32_t>(n / NSTAGE) & 1u;
-      Stage& st = sh.st[s];
-      mbar_wait(&sh.mma_done[s], ph);
+    for (int j = 0; j < nprod; ++j) {
+      const int ps = j % PSTAGE;
+      const uint32_t pph = static_cast<uint32_t>(j / PSTAGE) & 1u;
+      ProdStage& st = sh.prod[ps];
+      mbar_wait(&sh.mma_done[ps], pph);
       if (lane < C) {
         // column `col` of T = (I + L)^{-1}: x_i = [i == col] - sum_{m<i} L[i][m] x_m,
         // reading each row of L with 16-byte loads that all lanes share
@@ -592,16 +673,36 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         const float bc = st.beta[col];
 #pragma unroll
-        for (int i = 0; i < C; ++i) st.tb[i][col] = __float2bfloat16_rn(xs[i] * bc);
+        for (int i = 0; i < C; ++i) st.ops.tb[i][col] = __float2bfloat16_rn(xs[i] * bc);
       }
-      mbar_arrive_warp(&sh.full[s]);
+      fence_proxy_async_shared();
+      mbar_arrive_warp(&sh.solved[ps]);
     }
-  } else {
-    // ============================================================= load warp
-    // lane 0: TMA boxes of q, k, g and the value slice; lanes 1-16: beta.
-    for (int n = 0; n < nch; ++n) {
-      const int rs = n % RSTAGE;
-      const uint32_t rph = static_cast<uint32_t>(n / RSTAGE) & 1u;
+  } else if (warp == WARP_STORE) {
+    // ============================================================ store warp
+    if (lane == 0) {
+      for (int j = 0; j < nprod; ++j) {
+        const int n = rank + NSLICE * j;
+        const int ps = j % PSTAGE;
+        const uint32_t pph = static_cast<uint32_t>(j / PSTAGE) & 1u;
+        const int slot = n % RING;
+        mbar_wait(&sh.solved[ps], pph);
+        // the slot's previous chunk (n - RING) has been copied by all four CTAs
+        mbar_wait_cl(&sh.slot_free[slot], (static_cast<uint32_t>(n / RING) & 1u) ^ 1u);
+        fence_proxy_async_shared();
+        bulk_s2g_sync(ring + static_cast<size_t>(slot) * kSlotBytes, &sh.prod[ps].ops, kSlotBytes);
+        fence_proxy_async_global();
+        for (int c = 0; c < NSLICE; ++c) mbar_arrive_remote(&sh.ready[slot], static_cast<uint32_t>(c));
+        mbar_arrive(&sh.prod_free[ps]);
+      }
+    }
+  } else if (warp == WARP_PLOAD) {
+    // ====================================================== producer loads
+    // lane 0: TMA boxes of q, k, g; lanes 1-16: beta (zero past the sequence end)
+    for (int j = 0; j < nprod; ++j) {
+      const int n = rank + NSLICE * j;
+      const int rs = j % PRSTAGE;
+      const uint32_t rph = static_cast<uint32_t>(j / PRSTAGE) & 1u;
       const int64_t cs = t0 + static_cast<int64_t>(n) * C;
       const int tok = static_cast<int>(cs);
       RawStage& rw = sh.raw[rs];
@@ -611,7 +712,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tma_load_3d(&rw.q[0][0], &tm.q, 0, h, tok, &sh.raw_full[rs]);
         tma_load_3d(&rw.k[0][0], &tm.k, 0, h, tok, &sh.raw_full[rs]);
         tma_load_3d(&rw.g[0][0], &tm.g, 0, h, tok, &sh.raw_full[rs]);
-        tma_load_3d(&rw.v[0][0], &tm.v, dv0, h, tok, &sh.raw_full[rs]);
       } else if (lane <= C) {
         const int r = lane - 1;
         const bool ok = cs + r < t1;
@@ -619,7 +719,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         cp_async_arrive(&sh.raw_full[rs]);
       }
     }
+  } else {
+    // ====================================================== consumer loads
+    if (lane == 0) {
+      for (int n = 0; n < nch; ++n) {
+        const int s = n % CSTAGE;
+        const uint32_t ph = static_cast<uint32_t>(n / CSTAGE) & 1u;
+        const int slot = n % RING;
+        const int tok = static_cast<int>(t0 + static_cast<int64_t>(n) * C);
+        ChainStage& st = sh.cst[s];
+        mbar_wait(&sh.c_empty[s], ph ^ 1u);
+        mbar_wait_cl(&sh.ready[slot], static_cast<uint32_t>(n / RING) & 1u);
+        fence_proxy_async_global();
+        mbar_arrive_expect_tx(&sh.c_full[s], kChainBytes);
+        bulk_g2s(&st.ops, ring + static_cast<size_t>(slot) * kSlotBytes, kSlotBytes, &sh.c_full[s]);
+        tma_load_3d(&st.v[0][0], &tm.v, dv0, h, tok, &sh.c_full[s]);
+      }
+    }
   }
+  // no CTA leaves while a peer may still arrive on its barriers
+  __syncwarp();
+  cluster_sync();
 }
 
 }  // namespace kda
@@ -733,6 +853,7 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* g
   p.T = total_tokens;
   p.H = num_heads;
   p.scale = scale;
+  p.ring = nullptr;
   kda::TensorMaps tm;
   std::memset(&tm, 0, sizeof(tm));
   if (total_tokens > 0) {
@@ -745,9 +866,24 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* g
         (st = encode_3d(&tm.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total_tokens, H, kda::D, kda::NS)) != KDA_OK)
       return st;
   }
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  // Ring of shared chunk operands, one per (sequence, head): stream-ordered
+  // scratch from the device's memory pool, released in stream order after the
+  // kernel. It stays L2-resident while in use (RING slots per head).
+  void* ring = nullptr;
+  if (total_tokens > 0) {
+    const size_t ring_bytes = static_cast<size_t>(num_seqs) * num_heads * kda::RING * kda::kSlotBytes;
+    e = cudaMallocAsync(&ring, ring_bytes, cs);
+    if (e != cudaSuccess) return cuda_fail(e);
+    p.ring = static_cast<unsigned char*>(ring);
+  }
   dim3 grid(kda::NSLICE, num_heads, num_seqs);
-  kda::kda_fwd_kernel<<<grid, kda::NTHREADS, sizeof(kda::Shared), static_cast<cudaStream_t>(stream)>>>(p, tm);
+  kda::kda_fwd_kernel<<<grid, kda::NTHREADS, sizeof(kda::Shared), cs>>>(p, tm);
   e = cudaGetLastError();
+  if (ring) {
+    const cudaError_t ef = cudaFreeAsync(ring, cs);
+    if (e == cudaSuccess) e = ef;
+  }
   if (e != cudaSuccess) return cuda_fail(e);
   return KDA_OK;
 }
@@ -765,6 +901,18 @@ const char* kda_status_string(kda_status_t s) {
 }
 
 const char* kda_last_cuda_error(void) { return g_last_cuda_error; }
+
+kda_status_t kda_wait_timeouts(uint32_t* count, int32_t reset) {
+  if (!count) return KDA_ERR_NULL;
+  cudaError_t e = cudaMemcpyFromSymbol(count, kda::g_wait_timeouts, sizeof(uint32_t));
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (reset) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbol(kda::g_wait_timeouts, &zero, sizeof(uint32_t));
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return KDA_OK;
+}
 
 int32_t kda_abi_version(void) { return KDA_ABI_VERSION; }
 

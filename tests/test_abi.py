@@ -11,8 +11,13 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def lib():
-    from kimi_delta_attention_26_b200 import build
+    # load the build script by path so a stale library is rebuilt before use
+    import importlib.util
 
+    spec = importlib.util.spec_from_file_location(
+        "kda_build", os.path.join(ROOT, "kimi_delta_attention_26_b200", "build.py"))
+    build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(build)
     build.build()
     return ctypes.CDLL(build.LIB)
 
@@ -71,3 +76,9 @@ def test_rejects_bad_shapes(lib):
 def test_rejects_misaligned_pointers(lib):
     for name in ("q", "k", "v", "g", "beta", "out", "init", "fin", "cu"):
         assert _call(lib, **{name: 0x8008}) == 3, name
+
+
+def test_wait_timeouts_rejects_null(lib):
+    lib.kda_wait_timeouts.argtypes = [ctypes.c_void_p, ctypes.c_int32]
+    lib.kda_wait_timeouts.restype = ctypes.c_int
+    assert lib.kda_wait_timeouts(None, 0) == 1

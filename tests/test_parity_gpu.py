@@ -177,3 +177,11 @@ def test_full_size_workloads_sampled_columns(kda, oracle_mod, cfg):
     cols = slice(40, 56) if cfg != 5 else slice(100, 108)
     mo, ms = _check(oracle_mod, inp, f"config {cfg}", cols=cols)
     print(f"config {cfg}", mo, ms)
+
+
+def test_zz_no_wait_timeouts(kda):
+    """Every bounded in-kernel wait of this module's runs completed in time."""
+    import torch
+
+    torch.cuda.synchronize()
+    assert kda.wait_timeouts(reset=True) == 0
