@@ -21,9 +21,10 @@
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers on the current CUDA device.
- *   - The caller owns all inputs and outputs. kda_fwd takes a small scratch
- *     ring (num_seqs * H * 8 slots of ~15 KB) from the device's stream-ordered
- *     memory pool and returns it in stream order after the kernel.
+ *   - The caller owns all inputs and outputs. kda_fwd takes a scratch ring
+ *     (num_seqs * H * 16 slots of 15104 bytes) from a library-private
+ *     stream-ordered memory pool and returns it in stream order after the
+ *     kernel; the pool keeps its memory for later calls.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and the call returns without synchronising.
  *   - Argument errors are reported synchronously through the return code and

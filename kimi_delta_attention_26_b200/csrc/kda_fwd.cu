@@ -65,10 +65,10 @@ constexpr int D = KDA_HEAD_DIM;   // dk = dv = 128
 constexpr int C = 16;             // chunk length (tokens)
 constexpr int NS = 32;            // value columns per CTA
 constexpr int NSLICE = D / NS;    // CTAs per (sequence, head) = cluster size
-constexpr int RING = 8;           // ring slots per (sequence, head); multiple of NSLICE
+constexpr int RING = 16;          // ring slots per (sequence, head); multiple of NSLICE
 constexpr int PRSTAGE = 2;        // producer raw-input stages
-constexpr int PSTAGE = 2;         // producer operand stages
-constexpr int CSTAGE = 4;         // consumer stages (cload -> chain)
+constexpr int PSTAGE = 3;         // producer operand stages
+constexpr int CSTAGE = 6;         // consumer stages (cload -> chain)
 constexpr int NCHAIN = 4;
 constexpr int NGATE = 4;
 constexpr int WARP_GATE = NCHAIN;
@@ -286,6 +286,14 @@ __device__ __forceinline__ void mbar_arrive_remote(unsigned long long* m, uint32
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
 }
 
+// Relaxed remote arrive: a pure "done reading" signal that publishes no data,
+// so it need not wait for this thread's outstanding global stores.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(unsigned long long* m, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(m)), "r"(rank));
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
+}
+
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
@@ -299,13 +307,19 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// Bulk copy shared -> global; returns once the writes have completed.
-__device__ __forceinline__ void bulk_s2g_sync(void* gdst, const void* ssrc, uint32_t bytes) {
+// Bulk copy shared -> global as one bulk async-group.
+__device__ __forceinline__ void bulk_s2g(void* gdst, const void* ssrc, uint32_t bytes) {
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(ssrc)),
                "r"(bytes)
                : "memory");
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Wait until at most N of this thread's bulk async-groups are still pending
+// (their writes to global memory completed).
+template <int N>
+__device__ __forceinline__ void bulk_wait() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // Bulk copy global -> shared, completion counted in bytes on the mbarrier.
@@ -427,7 +441,8 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
       ChainStage& st = sh.cst[s];
       mbar_wait(&sh.c_full[s], ph);
       // the ring slot has been copied here: give it back to its producer
-      if (warp == 0 && lane == 0) mbar_arrive_remote(&sh.slot_free[n % RING], static_cast<uint32_t>(n % NSLICE));
+      if (warp == 0 && lane == 0)
+        mbar_arrive_remote_relaxed(&sh.slot_free[n % RING], static_cast<uint32_t>(n % NSLICE));
 
       // ---- X^T = V^T + S^T Kd^T and O^T = S^T Qd^T over this warp's key half
       float x[2][4], o[2][4];
@@ -680,7 +695,21 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
     }
   } else if (warp == WARP_STORE) {
     // ============================================================ store warp
+    // Up to two stores in flight: chunk j's slot is announced to the cluster
+    // once store j has completed, which is checked after store j+1 is issued.
     if (lane == 0) {
+      auto announce = [&](int jj) {
+        const int nn = rank + NSLICE * jj;
+        // The slot's bytes were written by the bulk-copy engine and that
+        // write has completed (bulk_wait above); the proxy fence orders it
+        // before the signal. A cluster-scope *release* arrive would also wait
+        // for this SM's unrelated outstanding global stores (~1.5k cycles per
+        // arrive on this part), so the signal itself is relaxed.
+        fence_proxy_async_global();
+        for (int c = 0; c < NSLICE; ++c)
+          mbar_arrive_remote_relaxed(&sh.ready[nn % RING], static_cast<uint32_t>(c));
+        mbar_arrive(&sh.prod_free[jj % PSTAGE]);
+      };
       for (int j = 0; j < nprod; ++j) {
         const int n = rank + NSLICE * j;
         const int ps = j % PSTAGE;
@@ -690,10 +719,15 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
         // the slot's previous chunk (n - RING) has been copied by all four CTAs
         mbar_wait_cl(&sh.slot_free[slot], (static_cast<uint32_t>(n / RING) & 1u) ^ 1u);
         fence_proxy_async_shared();
-        bulk_s2g_sync(ring + static_cast<size_t>(slot) * kSlotBytes, &sh.prod[ps].ops, kSlotBytes);
-        fence_proxy_async_global();
-        for (int c = 0; c < NSLICE; ++c) mbar_arrive_remote(&sh.ready[slot], static_cast<uint32_t>(c));
-        mbar_arrive(&sh.prod_free[ps]);
+        bulk_s2g(ring + static_cast<size_t>(slot) * kSlotBytes, &sh.prod[ps].ops, kSlotBytes);
+        if (j > 0) {
+          bulk_wait<1>();
+          announce(j - 1);
+        }
+      }
+      if (nprod > 0) {
+        bulk_wait<0>();
+        announce(nprod - 1);
       }
     }
   } else if (warp == WARP_PLOAD) {
@@ -794,6 +828,10 @@ kda_status_t encode_3d(CUtensorMap* map, const void* base, CUtensorMapDataType d
 
 constexpr int kMaxDevices = 64;
 int g_device_ready[kMaxDevices];  // 0 unknown, 1 ready, -1 unsupported
+// Library-private stream-ordered pool for the scratch ring. It keeps freed
+// memory (release threshold = max), so steady-state calls never map memory
+// and the process's default pool is left untouched.
+cudaMemPool_t g_pool[kMaxDevices];
 
 kda_status_t prepare_device(int dev) {
   if (dev < 0 || dev >= kMaxDevices) return KDA_ERR_UNSUPPORTED;
@@ -810,6 +848,17 @@ kda_status_t prepare_device(int dev) {
   }
   e = cudaFuncSetAttribute(kda::kda_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(sizeof(kda::Shared)));
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaMemPoolProps props;
+  std::memset(&props, 0, sizeof(props));
+  props.allocType = cudaMemAllocationTypePinned;
+  props.handleTypes = cudaMemHandleTypeNone;
+  props.location.type = cudaMemLocationTypeDevice;
+  props.location.id = dev;
+  e = cudaMemPoolCreate(&g_pool[dev], &props);
+  if (e != cudaSuccess) return cuda_fail(e);
+  uint64_t keep = ~0ull;
+  e = cudaMemPoolSetAttribute(g_pool[dev], cudaMemPoolAttrReleaseThreshold, &keep);
   if (e != cudaSuccess) return cuda_fail(e);
   g_device_ready[dev] = 1;
   return KDA_OK;
@@ -868,12 +917,12 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* g
   }
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   // Ring of shared chunk operands, one per (sequence, head): stream-ordered
-  // scratch from the device's memory pool, released in stream order after the
+  // scratch from the library's pool, released in stream order after the
   // kernel. It stays L2-resident while in use (RING slots per head).
   void* ring = nullptr;
   if (total_tokens > 0) {
     const size_t ring_bytes = static_cast<size_t>(num_seqs) * num_heads * kda::RING * kda::kSlotBytes;
-    e = cudaMallocAsync(&ring, ring_bytes, cs);
+    e = cudaMallocFromPoolAsync(&ring, ring_bytes, g_pool[dev], cs);
     if (e != cudaSuccess) return cuda_fail(e);
     p.ring = static_cast<unsigned char*>(ring);
   }
