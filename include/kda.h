@@ -52,7 +52,9 @@ typedef enum kda_status {
                               cu_seqlens NULL with num_seqs != 1, int overflow) */
   KDA_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned */
   KDA_ERR_UNSUPPORTED = 4, /* the current device is not sm_100 (B200) */
-  KDA_ERR_CUDA = 5         /* a CUDA runtime call or the launch failed */
+  KDA_ERR_CUDA = 5,        /* a CUDA runtime call or the launch failed */
+  KDA_ERR_CAPACITY = 6     /* kda_fwd_noalloc: num_seqs * num_heads exceeds
+                              KDA_NOALLOC_MAX_PAIRS */
 } kda_status_t;
 
 /*
@@ -87,6 +89,39 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* g
                      float scale, const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
                      int32_t num_heads, const float* initial_state, void* out, float* final_state,
                      void* stream);
+
+/*
+ * kda_fwd_noalloc -- kda_fwd without any device-memory allocation.
+ *
+ * The paper has no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory while they run. kda_fwd draws its
+ * scratch ring from a stream-ordered memory pool, which such callers cannot
+ * allow: serving engines that reserve the whole device for their own arena up
+ * front, or deployments where CUDA memory pools are unavailable
+ * (cudaDevAttrMemoryPoolsSupported = 0).
+ *
+ * Arguments, layouts, results and errors are those of kda_fwd, except:
+ *   - The scratch ring lives in a fixed-size array in device memory that the
+ *     library declares at file scope: every GPU that loads the library holds
+ *     it (KDA_NOALLOC_MAX_PAIRS * 16 slots * 15104 bytes = 7.7 MB) until the
+ *     process exits.
+ *   - num_seqs * num_heads must not exceed KDA_NOALLOC_MAX_PAIRS; larger
+ *     problems return KDA_ERR_CAPACITY and nothing is launched.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents (the kernel overwrites every slot before reading it, so nothing
+ *     needs clearing). Calls whose kernels overlap on the GPU -- on different
+ *     streams, or from different threads -- race on it and give wrong results;
+ *     order them on one stream.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define KDA_NOALLOC_MAX_PAIRS 32
+kda_status_t kda_fwd_noalloc(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                             float scale, const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                             int32_t num_heads, const float* initial_state, void* out, float* final_state,
+                             void* stream);
 
 /* Human-readable text of a status code (static storage, never NULL). */
 const char* kda_status_string(kda_status_t status);

@@ -864,6 +864,36 @@ kda_status_t prepare_device(int dev) {
   return KDA_OK;
 }
 
+// ---------------------------------------------------- allocation-free variant
+// Scratch ring of kda_fwd_noalloc: a fixed-size array at file scope in device
+// memory. Host code cannot use the symbol as an address; its device address is
+// looked up once per device (with that device current) and passed to the kernel.
+constexpr size_t kNoAllocRingBytes =
+    static_cast<size_t>(KDA_NOALLOC_MAX_PAIRS) * kda::RING * kda::kSlotBytes;
+static __device__ __align__(256) unsigned char g_noalloc_ring[kNoAllocRingBytes];
+void* g_noalloc_ring_addr[kMaxDevices];
+
+// Capability check, kernel attribute and array address for `dev` (current).
+kda_status_t noalloc_setup(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return KDA_ERR_UNSUPPORTED;
+  if (g_noalloc_ring_addr[dev]) return KDA_OK;
+  int major = 0, minor = 0;
+  cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (major != 10 || minor != 0) return KDA_ERR_UNSUPPORTED;
+  e = cudaFuncSetAttribute(kda::kda_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(sizeof(kda::Shared)));
+  if (e != cudaSuccess) return cuda_fail(e);
+  void* addr = nullptr;
+  e = cudaGetSymbolAddress(&addr, g_noalloc_ring);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (!addr) return KDA_ERR_CUDA;
+  g_noalloc_ring_addr[dev] = addr;
+  return KDA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -937,6 +967,61 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* g
   return KDA_OK;
 }
 
+kda_status_t kda_fwd_noalloc(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                             float scale, const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                             int32_t num_heads, const float* initial_state, void* out, float* final_state,
+                             void* stream) {
+  g_last_cuda_error[0] = '\0';
+  if (total_tokens < 0 || num_heads < 1 || num_seqs < 1) return KDA_ERR_SHAPE;
+  if (total_tokens > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_NULL;
+  if (!cu_seqlens && num_seqs != 1) return KDA_ERR_SHAPE;
+  if (num_heads > 65535 || num_seqs > 65535) return KDA_ERR_SHAPE;
+  if (total_tokens > (int64_t(1) << 40) / (int64_t(num_heads) * KDA_HEAD_DIM)) return KDA_ERR_SHAPE;
+  if (total_tokens > int64_t(INT32_MAX) - 64) return KDA_ERR_SHAPE;
+  if (int64_t(num_seqs) * num_heads > KDA_NOALLOC_MAX_PAIRS) return KDA_ERR_CAPACITY;
+  const void* ptrs[] = {q, k, v, g, beta, out, initial_state, final_state, cu_seqlens};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
+
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  kda_status_t st = noalloc_setup(dev);
+  if (st != KDA_OK) return st;
+
+  kda::Params p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.g = g;
+  p.beta = beta;
+  p.cu = cu_seqlens;
+  p.init = initial_state;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.fin = final_state;
+  p.T = total_tokens;
+  p.H = num_heads;
+  p.scale = scale;
+  p.ring = static_cast<unsigned char*>(g_noalloc_ring_addr[dev]);
+  kda::TensorMaps tm;
+  std::memset(&tm, 0, sizeof(tm));
+  if (total_tokens > 0) {
+    st = load_encoder();
+    if (st != KDA_OK) return st;
+    const int H = num_heads;
+    if ((st = encode_3d(&tm.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total_tokens, H, kda::D, kda::D)) != KDA_OK ||
+        (st = encode_3d(&tm.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total_tokens, H, kda::D, kda::D)) != KDA_OK ||
+        (st = encode_3d(&tm.g, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total_tokens, H, kda::D, kda::D)) != KDA_OK ||
+        (st = encode_3d(&tm.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total_tokens, H, kda::D, kda::NS)) != KDA_OK)
+      return st;
+  }
+  dim3 grid(kda::NSLICE, num_heads, num_seqs);
+  kda::kda_fwd_kernel<<<grid, kda::NTHREADS, sizeof(kda::Shared), static_cast<cudaStream_t>(stream)>>>(p, tm);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return KDA_OK;
+}
+
 const char* kda_status_string(kda_status_t s) {
   switch (s) {
     case KDA_OK: return "ok";
@@ -945,6 +1030,7 @@ const char* kda_status_string(kda_status_t s) {
     case KDA_ERR_ALIGN: return "a tensor pointer is not 16-byte aligned";
     case KDA_ERR_UNSUPPORTED: return "the current device is not sm_100 (B200)";
     case KDA_ERR_CUDA: return "a CUDA call failed (see kda_last_cuda_error)";
+    case KDA_ERR_CAPACITY: return "num_seqs * num_heads exceeds the fixed scratch of kda_fwd_noalloc";
   }
   return "unknown status";
 }
