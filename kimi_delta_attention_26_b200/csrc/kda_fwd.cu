@@ -11,19 +11,19 @@
 //   CTA then pulls the chunk with one bulk copy.
 //
 //   Warp roles inside a CTA:
-//     0-3   chain:  the serial state recurrence of this CTA's value slice. Warp w
-//                   owns S^T[16 value rows x 64 key columns] (value block w>>1, key
-//                   half w&1) in mma.sync accumulator registers for the whole
-//                   sequence; its bf16 conversion is the A operand of the next
-//                   chunk's products, so the state never touches shared memory.
+//     0-1   chain:  the serial state recurrence of this CTA's value slice. Warp w
+//                   owns S[128 keys x 16 value columns] in mma.sync accumulator
+//                   registers for the whole sequence and computes X, Vnew, O and
+//                   the state update of those columns; it shares nothing with
+//                   the other chain warp.
+//     2     mma:    (producer) A = Kd KR^T and Aqk = Qd KR^T, 16 x 16 each, then
+//                   T = (I + L)^{-1} by forward substitution and T diag(beta).
+//     3     store:  (producer) bulk-stores a finished chunk to its ring slot and
+//                   signals the cluster.
 //     4-7   gate:   (producer) two key channels x eight tokens per thread: decay
 //                   factors and the bf16 operand tiles of the chunks this CTA owns.
-//     8     mma:    (producer) A = Kd KR^T and Aqk = Qd KR^T, 16 x 16 each.
-//     9     solver: (producer) T = (I + L)^{-1} by forward substitution, T diag(beta).
-//     10    store:  (producer) bulk-stores a finished chunk to its ring slot and
-//                   signals the cluster.
-//     11    pload:  (producer) TMA loads of q, k, g (and beta) for owned chunks.
-//     12    cload:  (consumer) bulk-loads every chunk's shared operands from the
+//     8     pload:  (producer) TMA loads of q, k, g (and beta) for owned chunks.
+//     9     cload:  (consumer) bulk-loads every chunk's shared operands from the
 //                   ring and the value slice with TMA, in order, for the chain.
 //
 // Per chunk of C = 16 tokens, with Gamma_i the inclusive cumulative log-decay
@@ -38,9 +38,9 @@
 // All factors stay within [e^-80, e^80] because -5 <= g <= 0 and a chunk has 16
 // tokens: the bound that lets FlashKDA keep 16-token causal blocks on dense
 // tensor-core products (page "Kimi K3 开源满月…", section "KDA 内核到底难在哪":
-// 16-token chunks, lower_bound = -5). The chain works on S^T so that every
-// product on it takes the register-resident state as its A operand:
-// X^T = V^T + S^T Kd^T, Vnew^T = X^T Tb^T, S^T <- S^T Diag(gamma) + Vnew^T Kend.
+// 16-token chunks, lower_bound = -5). Every product on the chain takes the
+// register-resident state (or X, Vnew) as its B operand and a shared-memory
+// tile (Kd, Qd, Kend^T, Tb, Aqk) as its A operand.
 //
 // Tensor cores: mma.sync m16n8k16 (bf16 in, fp32 accumulate). On this part a
 // dependent m16n8k16 completes in ~21 cycles while a tcgen05.mma of the shapes
@@ -68,14 +68,13 @@ constexpr int NSLICE = D / NS;    // CTAs per (sequence, head) = cluster size
 constexpr int RING = 16;          // ring slots per (sequence, head); multiple of NSLICE
 constexpr int PRSTAGE = 2;        // producer raw-input stages
 constexpr int PSTAGE = 3;         // producer operand stages
-constexpr int CSTAGE = 6;         // consumer stages (cload -> chain)
-constexpr int NCHAIN = 4;
+constexpr int CSTAGE = 8;         // consumer stages (cload -> chain)
+constexpr int NCHAIN = NS / 16;   // chain warps, 16 value columns each
+constexpr int WARP_MMA = NCHAIN;  // also solves (I + L)^{-1}
+constexpr int WARP_STORE = WARP_MMA + 1;
 constexpr int NGATE = 4;
-constexpr int WARP_GATE = NCHAIN;
-constexpr int WARP_MMA = WARP_GATE + NGATE;
-constexpr int WARP_SOLVER = WARP_MMA + 1;
-constexpr int WARP_STORE = WARP_SOLVER + 1;
-constexpr int WARP_PLOAD = WARP_STORE + 1;
+constexpr int WARP_GATE = WARP_STORE + 1;
+constexpr int WARP_PLOAD = WARP_GATE + NGATE;
 constexpr int WARP_CLOAD = WARP_PLOAD + 1;
 constexpr int NTHREADS = (WARP_CLOAD + 1) * 32;
 static_assert(RING % NSLICE == 0, "a ring slot must always belong to the same producer CTA");
@@ -83,6 +82,11 @@ static_assert(RING % NSLICE == 0, "a ring slot must always belong to the same pr
 // Padded row pitches: 272 B and 48 B rows keep 8-row ldmatrix reads on distinct banks.
 constexpr int LDK = D + 8;
 constexpr int LDC = C + 8;
+
+// Position of key channel c's decay in Ops::gam: the chain lane with group id
+// g = c mod 8 needs channels 16t + g and 16t + g + 8 (t = 0..7), so those
+// sixteen sit in one 80-byte row, read with four 16-byte loads.
+__host__ __device__ constexpr int gamma_index(int c) { return (c & 7) * 20 + 2 * (c >> 4) + ((c >> 3) & 1); }
 
 // Raw inputs of one owned chunk, as the TMA boxes land (beta by 4-byte copies).
 struct __align__(128) RawStage {
@@ -101,7 +105,7 @@ struct __align__(128) Ops {
   __nv_bfloat16 ke[C][LDK];   //  k * exp(Gamma_last - Gamma)
   __nv_bfloat16 tb[C][LDC];   //  (I + L)^{-1} diag(beta)
   __nv_bfloat16 aqk[C][LDC];  //  causal Qd KR^T
-  float gam[D];               //  exp(Gamma_last)
+  float gam[8][20];           //  exp(Gamma_last), permuted for the chain (gamma_index)
 };
 constexpr uint32_t kSlotBytes = sizeof(Ops);
 
@@ -122,11 +126,9 @@ struct __align__(128) Shared {
   RawStage raw[PRSTAGE];
   ProdStage prod[PSTAGE];
   ChainStage cst[CSTAGE];
-  float xbuf[2][2][32][8];   // X^T partial sums exchanged inside a chain-warp pair
-  float obuf[2][2][32][4];   // O^T partial sums exchanged inside a chain-warp pair
   float2 gprod[2][2][64];    // per-half decay products exchanged inside the gate group
   unsigned long long raw_full[PRSTAGE], raw_empty[PRSTAGE];
-  unsigned long long prod_free[PSTAGE], gate_done[PSTAGE], mma_done[PSTAGE], solved[PSTAGE];
+  unsigned long long prod_free[PSTAGE], gate_done[PSTAGE], solved[PSTAGE];
   unsigned long long c_full[CSTAGE], c_empty[CSTAGE];
   unsigned long long ready[RING];      // arrived (remotely) by the slot's producer
   unsigned long long slot_free[RING];  // arrived (remotely) by the four consumers
@@ -172,9 +174,20 @@ __device__ __forceinline__ bool mbar_try_wait(unsigned long long* m, uint32_t pa
       : "memory");
   return ok != 0;
 }
+// Non-blocking probe: cheaper than a suspending try_wait when the phase has
+// long completed, which is the common case for well-fed pipeline stages.
+__device__ __forceinline__ bool mbar_test_wait(unsigned long long* m, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(smem_u32(m)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 
 __device__ __forceinline__ void mbar_wait(unsigned long long* m, uint32_t parity) {
-  if (mbar_try_wait(m, parity)) return;
+  if (mbar_test_wait(m, parity)) return;
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(m, parity)) return;
@@ -398,7 +411,6 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
     for (int s = 0; s < PSTAGE; ++s) {
       mbar_init(&sh.prod_free[s], 1);
       mbar_init(&sh.gate_done[s], NGATE);
-      mbar_init(&sh.mma_done[s], 1);
       mbar_init(&sh.solved[s], 1);
     }
     for (int s = 0; s < CSTAGE; ++s) {
@@ -416,22 +428,29 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
 
   if (warp < NCHAIN) {
     // =========================================================== chain warps
-    const int pr = warp >> 1;          // value block (16 columns) inside the slice
-    const int dh = warp & 1;           // key half
-    const int k0 = 64 * dh;            // first key channel of this warp
-    const int vrow = 16 * pr;          // first value column (slice-local)
-    // S^T fragment: rows = value columns vrow + gq (+8), cols = key channels
-    // k0 + 8*nt + 2*tq (+1), nt = 0..7.
-    float sT[8][4];
+    // Warp w owns S[128 keys x 16 value columns] (columns 16w .. 16w+15 of the
+    // slice) for the whole sequence: s[t][j] is the m16n8 accumulator tile of
+    // keys 16t.. and columns 8j.., so lane (gq, tq) holds keys 16t+gq (+8) x
+    // columns 8j+2tq (+1). Every chunk product takes S (or X, Vnew) as its B
+    // operand; an 8x8 movmatrix transpose turns an accumulator tile into a
+    // B fragment, so nothing of the state leaves the registers and the warp
+    // needs no partner.
+    const int cv = 16 * warp;          // first value column (slice-local)
+    float sacc[8][2][4];
     const size_t sbase = (static_cast<size_t>(seq) * H + h) * D * D;
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
+    for (int t = 0; t < 8; ++t)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int dv = dv0 + vrow + gq + 8 * (e >> 1);
-        const int dk = k0 + 8 * nt + 2 * tq + (e & 1);
-        sT[nt][e] = p.init ? __ldg(p.init + sbase + static_cast<size_t>(dk) * D + dv) : 0.f;
-      }
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int key = 16 * t + gq + 8 * hf;
+          const int col = dv0 + cv + 8 * j + 2 * tq;
+          float2 v2 = make_float2(0.f, 0.f);
+          if (p.init) v2 = __ldg(reinterpret_cast<const float2*>(p.init + sbase + static_cast<size_t>(key) * D + col));
+          sacc[t][j][2 * hf] = v2.x;
+          sacc[t][j][2 * hf + 1] = v2.y;
+        }
 
     for (int n = 0; n < nch; ++n) {
       const int s = n % CSTAGE;
@@ -439,121 +458,138 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
       const int64_t cs = t0 + static_cast<int64_t>(n) * C;
       const int m = static_cast<int>((t1 - cs) < C ? (t1 - cs) : C);
       ChainStage& st = sh.cst[s];
+
+      // S as bf16 B fragments (k = keys 16t.., n = columns 8j..)
+      uint32_t sb[8][2][2];
+#pragma unroll
+      for (int t = 0; t < 8; ++t)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          sb[t][j][0] = movmatrix_t(pack_bf16(sacc[t][j][0], sacc[t][j][1]));
+          sb[t][j][1] = movmatrix_t(pack_bf16(sacc[t][j][2], sacc[t][j][3]));
+        }
+
       mbar_wait(&sh.c_full[s], ph);
       // the ring slot has been copied here: give it back to its producer
       if (warp == 0 && lane == 0)
         mbar_arrive_remote_relaxed(&sh.slot_free[n % RING], static_cast<uint32_t>(n % NSLICE));
 
-      // ---- X^T = V^T + S^T Kd^T and O^T = S^T Qd^T over this warp's key half
-      float x[2][4], o[2][4];
+      // ---- X = V + Kd S   (two accumulator chains per column tile)
+      float xa[2][4], xb[2][4] = {};
+      {
+        uint32_t vv[4];
+        ldsm_x4(vv, &st.v[(lane & 7) + ((lane >> 3) & 1) * 8][cv + (lane >> 4) * 8]);
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+        for (int j = 0; j < 2; ++j)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          o[nt][e] = 0.f;
-          x[nt][e] = 0.f;
-          if (dh == 0) {
-            const int tok = 8 * nt + 2 * tq + (e & 1);
-            const int col = vrow + gq + 8 * (e >> 1);
-            x[nt][e] = __bfloat162float(st.v[tok][col]);
+          for (int hf = 0; hf < 2; ++hf) {
+            const uint32_t w2 = vv[2 * j + hf];
+            xa[j][2 * hf] = __uint_as_float(w2 << 16);
+            xa[j][2 * hf + 1] = __uint_as_float(w2 & 0xffff0000u);
           }
+      }
+      uint32_t ak[8][4];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) ldsm_x4(ak[t], &st.ops.kd[lane & 15][16 * t + (lane >> 4) * 8]);
+#pragma unroll
+      for (int t = 0; t < 8; ++t)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          if (t & 1)
+            mma(xb[j], ak[t], sb[t][j][0], sb[t][j][1]);
+          else
+            mma(xa[j], ak[t], sb[t][j][0], sb[t][j][1]);
+        }
+      uint32_t atb[4], aaq[4];
+      ldsm_x4(atb, &st.ops.tb[lane & 15][(lane >> 4) * 8]);
+      ldsm_x4(aaq, &st.ops.aqk[lane & 15][(lane >> 4) * 8]);
+      // ---- Vnew = Tb X
+      float vn[2][4] = {};
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const uint32_t b0 = movmatrix_t(pack_bf16(xa[j][0] + xb[j][0], xa[j][1] + xb[j][1]));
+        const uint32_t b1 = movmatrix_t(pack_bf16(xa[j][2] + xb[j][2], xa[j][3] + xb[j][3]));
+        mma(vn[j], atb, b0, b1);
+      }
+      // ---- O = Qd S (chunk-start state), issued while Vnew completes
+      float oa[2][4] = {}, ob[2][4] = {};
+#pragma unroll
+      for (int t = 0; t < 8; ++t) ldsm_x4(ak[t], &st.ops.qd[lane & 15][16 * t + (lane >> 4) * 8]);
+#pragma unroll
+      for (int t = 0; t < 8; ++t)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          if (t & 1)
+            mma(ob[j], ak[t], sb[t][j][0], sb[t][j][1]);
+          else
+            mma(oa[j], ak[t], sb[t][j][0], sb[t][j][1]);
+        }
+      uint32_t vb[2][2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        vb[j][0] = movmatrix_t(pack_bf16(vn[j][0], vn[j][1]));
+        vb[j][1] = movmatrix_t(pack_bf16(vn[j][2], vn[j][3]));
+      }
+      // ---- S <- Diag(gamma) S + Kend^T Vnew
+      {
+        const float4* gp = reinterpret_cast<const float4*>(&st.ops.gam[gq][0]);
+        float gmv[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 g4 = gp[i];
+          gmv[4 * i] = g4.x;
+          gmv[4 * i + 1] = g4.y;
+          gmv[4 * i + 2] = g4.z;
+          gmv[4 * i + 3] = g4.w;
         }
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        uint32_t a[4], bk[4], bq[4];
-        acc_to_afrag(a, sT[2 * kk], sT[2 * kk + 1]);
-        const int row = (lane & 7) + ((lane >> 4) << 3);
-        const int col = k0 + 16 * kk + ((lane >> 3) & 1) * 8;
-        ldsm_x4(bk, &st.ops.kd[row][col]);
-        ldsm_x4(bq, &st.ops.qd[row][col]);
-        mma(x[0], a, bk[0], bk[1]);
-        mma(x[1], a, bk[2], bk[3]);
-        mma(o[0], a, bq[0], bq[1]);
-        mma(o[1], a, bq[2], bq[3]);
-      }
-      // ---- sum X^T over the two key halves (pair exchange)
-      {
-        float4* mine = reinterpret_cast<float4*>(&sh.xbuf[pr][dh][lane][0]);
-        mine[0] = make_float4(x[0][0], x[0][1], x[0][2], x[0][3]);
-        mine[1] = make_float4(x[1][0], x[1][1], x[1][2], x[1][3]);
-        named_bar(2 + pr, 64);
-        const float4* other = reinterpret_cast<const float4*>(&sh.xbuf[pr][dh ^ 1][lane][0]);
-        const float4 u0 = other[0], u1 = other[1];
-        x[0][0] += u0.x; x[0][1] += u0.y; x[0][2] += u0.z; x[0][3] += u0.w;
-        x[1][0] += u1.x; x[1][1] += u1.y; x[1][2] += u1.z; x[1][3] += u1.w;
-      }
-      // ---- Vnew^T = X^T Tb^T
-      float vn[2][4] = {};
-      uint32_t ax[4], av[4];
-      acc_to_afrag(ax, x[0], x[1]);
-      {
-        uint32_t bt[4];
-        ldsm_x4(bt, &st.ops.tb[(lane & 7) + ((lane >> 4) << 3)][((lane >> 3) & 1) * 8]);
-        mma(vn[0], ax, bt[0], bt[1]);
-        mma(vn[1], ax, bt[2], bt[3]);
-      }
-      acc_to_afrag(av, vn[0], vn[1]);
-      // ---- O^T += Vnew^T Aqk^T (once per pair)
-      if (dh == 0) {
-        uint32_t ba[4];
-        ldsm_x4(ba, &st.ops.aqk[(lane & 7) + ((lane >> 4) << 3)][((lane >> 3) & 1) * 8]);
-        mma(o[0], av, ba[0], ba[1]);
-        mma(o[1], av, ba[2], ba[3]);
-      }
-      // ---- S^T <- S^T Diag(gamma) + Vnew^T Kend   (this warp's key half)
+        for (int t = 0; t < 8; ++t)
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        const float2 gm = *reinterpret_cast<const float2*>(&st.ops.gam[k0 + 8 * nt + 2 * tq]);
-        sT[nt][0] *= gm.x;
-        sT[nt][1] *= gm.y;
-        sT[nt][2] *= gm.x;
-        sT[nt][3] *= gm.y;
+          for (int j = 0; j < 2; ++j) {
+            sacc[t][j][0] *= gmv[2 * t];
+            sacc[t][j][1] *= gmv[2 * t];
+            sacc[t][j][2] *= gmv[2 * t + 1];
+            sacc[t][j][3] *= gmv[2 * t + 1];
+          }
       }
 #pragma unroll
-      for (int np = 0; np < 4; ++np) {
-        uint32_t be[4];
-        ldsm_x4_t(be, &st.ops.ke[(lane & 7) + ((lane >> 3) & 1) * 8][k0 + 16 * np + (lane >> 4) * 8]);
-        mma(sT[2 * np], av, be[0], be[1]);
-        mma(sT[2 * np + 1], av, be[2], be[3]);
-      }
+      for (int t = 0; t < 8; ++t) ldsm_x4_t(ak[t], &st.ops.ke[(lane & 7) + (lane >> 4) * 8][16 * t + ((lane >> 3) & 1) * 8]);
+#pragma unroll
+      for (int t = 0; t < 8; ++t)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) mma(sacc[t][j], ak[t], vb[j][0], vb[j][1]);
+      // ---- O += Aqk Vnew
+#pragma unroll
+      for (int j = 0; j < 2; ++j) mma(oa[j], aaq, vb[j][0], vb[j][1]);
       // the stage is no longer read by this warp
       mbar_arrive_warp(&sh.c_empty[s]);
-      // ---- O: each warp of the pair finishes one 8-token half (register
-      // selects, not a runtime array index, keep o[][] in registers)
-      {
-        float mine[4], give[4];
+      // ---- store O: lane holds tokens gq (+8) x columns 8j + 2tq (+1)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          mine[e] = dh ? o[1][e] : o[0][e];
-          give[e] = dh ? o[0][e] : o[1][e];
-        }
-        *reinterpret_cast<float4*>(&sh.obuf[pr][dh][lane][0]) = make_float4(give[0], give[1], give[2], give[3]);
-        named_bar(2 + pr, 64);
-        const float4 u = *reinterpret_cast<const float4*>(&sh.obuf[pr][dh ^ 1][lane][0]);
-        const float o0 = (mine[0] + u.x) * p.scale, o1 = (mine[1] + u.y) * p.scale;
-        const float o2 = (mine[2] + u.z) * p.scale, o3 = (mine[3] + u.w) * p.scale;
-        // fragment rows = value columns, cols = tokens -> transpose to token rows
-        const uint32_t r0 = movmatrix_t(pack_bf16(o0, o1));
-        const uint32_t r1 = movmatrix_t(pack_bf16(o2, o3));
-        const int tok = 8 * dh + gq;
+      for (int hf = 0; hf < 2; ++hf) {
+        const int tok = gq + 8 * hf;
         if (tok < m) {
-          __nv_bfloat16* dst = p.out + (cs + tok) * row_stride + static_cast<size_t>(h) * D + dv0 + vrow + 2 * tq;
-          *reinterpret_cast<uint32_t*>(dst) = r0;
-          *reinterpret_cast<uint32_t*>(dst + 8) = r1;
+          __nv_bfloat16* dst = p.out + (cs + tok) * row_stride + static_cast<size_t>(h) * D + dv0 + cv + 2 * tq;
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+            *reinterpret_cast<uint32_t*>(dst + 8 * j) =
+                pack_bf16((oa[j][2 * hf] + ob[j][2 * hf]) * p.scale, (oa[j][2 * hf + 1] + ob[j][2 * hf + 1]) * p.scale);
         }
       }
     }
     if (p.fin) {
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
+      for (int t = 0; t < 8; ++t)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int dv = dv0 + vrow + gq + 8 * (e >> 1);
-          const int dk = k0 + 8 * nt + 2 * tq + (e & 1);
-          p.fin[sbase + static_cast<size_t>(dk) * D + dv] = sT[nt][e];
-        }
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const int key = 16 * t + gq + 8 * hf;
+            const int col = dv0 + cv + 8 * j + 2 * tq;
+            *reinterpret_cast<float2*>(p.fin + sbase + static_cast<size_t>(key) * D + col) =
+                make_float2(sacc[t][j][2 * hf], sacc[t][j][2 * hf + 1]);
+          }
     }
-  } else if (warp < WARP_MMA) {
+  } else if (warp >= WARP_GATE && warp < WARP_GATE + NGATE) {
     // ============================================================ gate warps
     // Thread layout: channel pair cp (channels 2cp, 2cp+1), token half th
     // (tokens 8th .. 8th+7). The decay products of the two halves meet through
@@ -624,7 +660,10 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
         F.x *= e[jj].x;
         F.y *= e[jj].y;
       }
-      if (th == 0) *reinterpret_cast<float2*>(&st.ops.gam[c0]) = gamma;
+      if (th == 0) {
+        (&st.ops.gam[0][0])[gamma_index(c0)] = gamma.x;
+        (&st.ops.gam[0][0])[gamma_index(c0 + 1)] = gamma.y;
+      }
       fence_proxy_async_shared();
       mbar_arrive_warp(&sh.gate_done[ps]);
     }
@@ -657,17 +696,8 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
           st.L[i][jc] = (jc < i) ? -st.beta[i] * accA[nt][e2] : 0.f;
           st.ops.aqk[i][jc] = __float2bfloat16_rn((jc <= i) ? accQ[nt][e2] : 0.f);
         }
-      fence_proxy_async_shared();
-      mbar_arrive_warp(&sh.mma_done[ps]);
-    }
-  } else if (warp == WARP_SOLVER) {
-    // =========================================================== solver warp
-    // lanes 0-15: one column of (I + L)^{-1} each, scaled by beta of that column
-    for (int j = 0; j < nprod; ++j) {
-      const int ps = j % PSTAGE;
-      const uint32_t pph = static_cast<uint32_t>(j / PSTAGE) & 1u;
-      ProdStage& st = sh.prod[ps];
-      mbar_wait(&sh.mma_done[ps], pph);
+      __syncwarp();
+      // (I + L)^{-1} on the same warp: lanes 0-15, one column each
       if (lane < C) {
         // column `col` of T = (I + L)^{-1}: x_i = [i == col] - sum_{m<i} L[i][m] x_m,
         // reading each row of L with 16-byte loads that all lanes share
