@@ -10,21 +10,22 @@
 //   global memory and signals the four CTAs with remote mbarrier arrivals; every
 //   CTA then pulls the chunk with one bulk copy.
 //
-//   Warp roles inside a CTA:
+//   Warp roles inside a CTA (warp w issues on sub-partition w mod 4):
 //     0-1   chain:  the serial state recurrence of this CTA's value slice. Warp w
-//                   owns S[128 keys x 16 value columns] in mma.sync accumulator
+//                   owns S^T[16 value columns x 128 keys] in mma.sync accumulator
 //                   registers for the whole sequence and computes X, Vnew, O and
 //                   the state update of those columns; it shares nothing with
 //                   the other chain warp.
-//     2     mma:    (producer) A = Kd KR^T and Aqk = Qd KR^T, 16 x 16 each, then
-//                   T = (I + L)^{-1} by forward substitution and T diag(beta).
-//     3     store:  (producer) bulk-stores a finished chunk to its ring slot and
-//                   signals the cluster.
-//     4-7   gate:   (producer) two key channels x eight tokens per thread: decay
+//     2,3,6,7 gate: (producer) two key channels x eight tokens per thread: decay
 //                   factors and the bf16 operand tiles of the chunks this CTA owns.
-//     8     pload:  (producer) TMA loads of q, k, g (and beta) for owned chunks.
-//     9     cload:  (consumer) bulk-loads every chunk's shared operands from the
+//     4     pload:  (producer) TMA loads of q, k, g (and beta) for owned chunks.
+//     5     cload:  (consumer) bulk-loads every chunk's shared operands from the
 //                   ring and the value slice with TMA, in order, for the chain.
+//     10    mma:    (producer) A = Kd KR^T and Aqk = Qd KR^T, 16 x 16 each, then
+//                   T = (I + L)^{-1} by forward substitution and T diag(beta).
+//     11    store:  (producer) bulk-stores a finished chunk to its ring slot and
+//                   signals the cluster.
+//     8-9   idle.
 //
 // Per chunk of C = 16 tokens, with Gamma_i the inclusive cumulative log-decay
 // inside the chunk (e_i = exp(g_i) per channel):
@@ -69,24 +70,30 @@ constexpr int RING = 16;          // ring slots per (sequence, head); multiple o
 constexpr int PRSTAGE = 2;        // producer raw-input stages
 constexpr int PSTAGE = 3;         // producer operand stages
 constexpr int CSTAGE = 8;         // consumer stages (cload -> chain)
-constexpr int NCHAIN = NS / 16;   // chain warps, 16 value columns each
-constexpr int WARP_MMA = NCHAIN;  // also solves (I + L)^{-1}
-constexpr int WARP_STORE = WARP_MMA + 1;
-constexpr int NGATE = 4;
-constexpr int WARP_GATE = WARP_STORE + 1;
-constexpr int WARP_PLOAD = WARP_GATE + NGATE;
-constexpr int WARP_CLOAD = WARP_PLOAD + 1;
-constexpr int NTHREADS = (WARP_CLOAD + 1) * 32;
+// Warp w issues on sub-partition w mod 4. The two chain warps get partitions 0
+// and 1 with only the light load warps beside them; the gate, mma and store
+// warps, which burst through ALU and shared-memory work, share partitions 2
+// and 3. Warps 8 and 9 have no role (they fill the numbering).
+constexpr int NCHAIN = NS / 16;   // chain warps (0, 1), 16 value columns each
+constexpr int NGATE = 4;          // gate warps 2, 3, 6, 7
+constexpr int WARP_PLOAD = 4;
+constexpr int WARP_CLOAD = 5;
+constexpr int WARP_MMA = 10;      // also solves (I + L)^{-1}
+constexpr int WARP_STORE = 11;
+constexpr int NTHREADS = 12 * 32;
+__host__ __device__ constexpr bool is_gate_warp(int w) { return (w & 3) >= 2 && w < 8; }
+__host__ __device__ constexpr int gate_warp_index(int w) { return (w & 1) + ((w >> 2) << 1); }
+static_assert(NCHAIN == 2, "warp layout assumes two chain warps");
 static_assert(RING % NSLICE == 0, "a ring slot must always belong to the same producer CTA");
 
 // Padded row pitches: 272 B and 48 B rows keep 8-row ldmatrix reads on distinct banks.
 constexpr int LDK = D + 8;
 constexpr int LDC = C + 8;
 
-// Position of key channel c's decay in Ops::gam: the chain lane with group id
-// g = c mod 8 needs channels 16t + g and 16t + g + 8 (t = 0..7), so those
-// sixteen sit in one 80-byte row, read with four 16-byte loads.
-__host__ __device__ constexpr int gamma_index(int c) { return (c & 7) * 20 + 2 * (c >> 4) + ((c >> 3) & 1); }
+// Position of key channel c's decay in Ops::gam: a chain lane with quad index
+// tq needs channels 8t + 2tq and 8t + 2tq + 1 (t = 0..15), so those 32 sit in
+// one 160-byte row (rows on distinct banks), read with eight 16-byte loads.
+__host__ __device__ constexpr int gamma_index(int c) { return ((c >> 1) & 3) * 40 + 2 * (c >> 3) + (c & 1); }
 
 // Raw inputs of one owned chunk, as the TMA boxes land (beta by 4-byte copies).
 struct __align__(128) RawStage {
@@ -105,7 +112,7 @@ struct __align__(128) Ops {
   __nv_bfloat16 ke[C][LDK];   //  k * exp(Gamma_last - Gamma)
   __nv_bfloat16 tb[C][LDC];   //  (I + L)^{-1} diag(beta)
   __nv_bfloat16 aqk[C][LDC];  //  causal Qd KR^T
-  float gam[8][20];           //  exp(Gamma_last), permuted for the chain (gamma_index)
+  float gam[4][40];           //  exp(Gamma_last), permuted for the chain (gamma_index)
 };
 constexpr uint32_t kSlotBytes = sizeof(Ops);
 
@@ -428,29 +435,24 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
 
   if (warp < NCHAIN) {
     // =========================================================== chain warps
-    // Warp w owns S[128 keys x 16 value columns] (columns 16w .. 16w+15 of the
-    // slice) for the whole sequence: s[t][j] is the m16n8 accumulator tile of
-    // keys 16t.. and columns 8j.., so lane (gq, tq) holds keys 16t+gq (+8) x
-    // columns 8j+2tq (+1). Every chunk product takes S (or X, Vnew) as its B
-    // operand; an 8x8 movmatrix transpose turns an accumulator tile into a
-    // B fragment, so nothing of the state leaves the registers and the warp
-    // needs no partner.
+    // Warp w owns S^T[16 value columns x 128 keys] (columns 16w .. 16w+15 of
+    // the slice) for the whole sequence: tile st[u] holds keys 8u .. 8u+7 as an
+    // m16n8 accumulator, so lane (gq, tq) holds columns gq (+8) x keys 8u+2tq
+    // (+1). Packed to bf16 these registers are, unchanged, the B fragments of
+    // products over the keys (X = Kd S, O = Qd S), and the state update
+    // S^T += Vnew^T Kend takes Vnew^T as its A operand. Nothing of the state
+    // leaves the registers and the warp needs no partner.
     const int cv = 16 * warp;          // first value column (slice-local)
-    float sacc[8][2][4];
+    float sacc[16][4];
     const size_t sbase = (static_cast<size_t>(seq) * H + h) * D * D;
 #pragma unroll
-    for (int t = 0; t < 8; ++t)
+    for (int u = 0; u < 16; ++u)
 #pragma unroll
-      for (int j = 0; j < 2; ++j)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int key = 16 * t + gq + 8 * hf;
-          const int col = dv0 + cv + 8 * j + 2 * tq;
-          float2 v2 = make_float2(0.f, 0.f);
-          if (p.init) v2 = __ldg(reinterpret_cast<const float2*>(p.init + sbase + static_cast<size_t>(key) * D + col));
-          sacc[t][j][2 * hf] = v2.x;
-          sacc[t][j][2 * hf + 1] = v2.y;
-        }
+      for (int e = 0; e < 4; ++e) {
+        const int key = 8 * u + 2 * tq + (e & 1);
+        const int col = dv0 + cv + gq + 8 * (e >> 1);
+        sacc[u][e] = p.init ? __ldg(p.init + sbase + static_cast<size_t>(key) * D + col) : 0.f;
+      }
 
     for (int n = 0; n < nch; ++n) {
       const int s = n % CSTAGE;
@@ -459,22 +461,21 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
       const int m = static_cast<int>((t1 - cs) < C ? (t1 - cs) : C);
       ChainStage& st = sh.cst[s];
 
-      // S as bf16 B fragments (k = keys 16t.., n = columns 8j..)
-      uint32_t sb[8][2][2];
-#pragma unroll
-      for (int t = 0; t < 8; ++t)
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          sb[t][j][0] = movmatrix_t(pack_bf16(sacc[t][j][0], sacc[t][j][1]));
-          sb[t][j][1] = movmatrix_t(pack_bf16(sacc[t][j][2], sacc[t][j][3]));
-        }
-
       mbar_wait(&sh.c_full[s], ph);
       // the ring slot has been copied here: give it back to its producer
       if (warp == 0 && lane == 0)
         mbar_arrive_remote_relaxed(&sh.slot_free[n % RING], static_cast<uint32_t>(n % NSLICE));
 
-      // ---- X = V + Kd S   (two accumulator chains per column tile)
+      // The products are ordered for one in-order warp on one tensor pipe: the
+      // state's own chain (X -> Vnew -> S) goes first at every step and the O
+      // products, which nothing waits for, fill the pipe while a chain result
+      // drains through conversion and transpose.
+      uint32_t ak[8][4];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) ldsm_x4(ak[t], &st.ops.kd[lane & 15][16 * t + (lane >> 4) * 8]);
+      // ---- X = V + Kd S   (two accumulator chains per column tile); each key
+      // tile of S is packed to bf16 (sb, the chunk-start state also used by O)
+      // and then scaled by gamma for the update
       float xa[2][4], xb[2][4] = {};
       {
         uint32_t vv[4];
@@ -488,22 +489,49 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
             xa[j][2 * hf + 1] = __uint_as_float(w2 & 0xffff0000u);
           }
       }
-      uint32_t ak[8][4];
+      uint32_t sb[8][2][2];
+      const float4* gp = reinterpret_cast<const float4*>(&st.ops.gam[tq][0]);
 #pragma unroll
-      for (int t = 0; t < 8; ++t) ldsm_x4(ak[t], &st.ops.kd[lane & 15][16 * t + (lane >> 4) * 8]);
-#pragma unroll
-      for (int t = 0; t < 8; ++t)
+      for (int t = 0; t < 8; ++t) {
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
+          sb[t][j][0] = pack_bf16(sacc[2 * t][2 * j], sacc[2 * t][2 * j + 1]);
+          sb[t][j][1] = pack_bf16(sacc[2 * t + 1][2 * j], sacc[2 * t + 1][2 * j + 1]);
           if (t & 1)
             mma(xb[j], ak[t], sb[t][j][0], sb[t][j][1]);
           else
             mma(xa[j], ak[t], sb[t][j][0], sb[t][j][1]);
         }
-      uint32_t atb[4], aaq[4];
-      ldsm_x4(atb, &st.ops.tb[lane & 15][(lane >> 4) * 8]);
-      ldsm_x4(aaq, &st.ops.aqk[lane & 15][(lane >> 4) * 8]);
+        const float4 g4 = gp[t];
+        sacc[2 * t][0] *= g4.x;
+        sacc[2 * t][1] *= g4.y;
+        sacc[2 * t][2] *= g4.x;
+        sacc[2 * t][3] *= g4.y;
+        sacc[2 * t + 1][0] *= g4.z;
+        sacc[2 * t + 1][1] *= g4.w;
+        sacc[2 * t + 1][2] *= g4.z;
+        sacc[2 * t + 1][3] *= g4.w;
+      }
+      // ---- O = Qd S (chunk-start state) + Aqk Vnew, in three installments
+      float oa[2][4] = {}, ob[2][4] = {};
+      auto o_steps = [&](int t_begin, int t_end) {
+#pragma unroll
+        for (int t = t_begin; t < t_end; ++t) {
+          uint32_t aq[4];
+          ldsm_x4(aq, &st.ops.qd[lane & 15][16 * t + (lane >> 4) * 8]);
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            if (t & 1)
+              mma(ob[j], aq, sb[t][j][0], sb[t][j][1]);
+            else
+              mma(oa[j], aq, sb[t][j][0], sb[t][j][1]);
+          }
+        }
+      };
+      o_steps(0, 3);
       // ---- Vnew = Tb X
+      uint32_t atb[4];
+      ldsm_x4(atb, &st.ops.tb[lane & 15][(lane >> 4) * 8]);
       float vn[2][4] = {};
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
@@ -511,56 +539,34 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
         const uint32_t b1 = movmatrix_t(pack_bf16(xa[j][2] + xb[j][2], xa[j][3] + xb[j][3]));
         mma(vn[j], atb, b0, b1);
       }
-      // ---- O = Qd S (chunk-start state), issued while Vnew completes
-      float oa[2][4] = {}, ob[2][4] = {};
+      // kd fragments are dead: the same registers take Kend^T
 #pragma unroll
-      for (int t = 0; t < 8; ++t) ldsm_x4(ak[t], &st.ops.qd[lane & 15][16 * t + (lane >> 4) * 8]);
-#pragma unroll
-      for (int t = 0; t < 8; ++t)
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          if (t & 1)
-            mma(ob[j], ak[t], sb[t][j][0], sb[t][j][1]);
-          else
-            mma(oa[j], ak[t], sb[t][j][0], sb[t][j][1]);
-        }
+      for (int t = 0; t < 8; ++t) ldsm_x4_t(ak[t], &st.ops.ke[(lane & 7) + ((lane >> 3) & 1) * 8][16 * t + (lane >> 4) * 8]);
+      o_steps(3, 6);
+      // Vnew as B fragments (k = tokens, n = columns 8j..); the same registers
+      // form Vnew^T as an A fragment: {vb[0][0], vb[1][0], vb[0][1], vb[1][1]}
       uint32_t vb[2][2];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         vb[j][0] = movmatrix_t(pack_bf16(vn[j][0], vn[j][1]));
         vb[j][1] = movmatrix_t(pack_bf16(vn[j][2], vn[j][3]));
       }
-      // ---- S <- Diag(gamma) S + Kend^T Vnew
+      // ---- S^T <- S^T Diag(gamma) + Vnew^T Kend  (gamma applied above)
       {
-        const float4* gp = reinterpret_cast<const float4*>(&st.ops.gam[gq][0]);
-        float gmv[16];
+        const uint32_t av[4] = {vb[0][0], vb[1][0], vb[0][1], vb[1][1]};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float4 g4 = gp[i];
-          gmv[4 * i] = g4.x;
-          gmv[4 * i + 1] = g4.y;
-          gmv[4 * i + 2] = g4.z;
-          gmv[4 * i + 3] = g4.w;
+        for (int t = 0; t < 8; ++t) {
+          mma(sacc[2 * t], av, ak[t][0], ak[t][1]);
+          mma(sacc[2 * t + 1], av, ak[t][2], ak[t][3]);
         }
-#pragma unroll
-        for (int t = 0; t < 8; ++t)
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            sacc[t][j][0] *= gmv[2 * t];
-            sacc[t][j][1] *= gmv[2 * t];
-            sacc[t][j][2] *= gmv[2 * t + 1];
-            sacc[t][j][3] *= gmv[2 * t + 1];
-          }
       }
+      o_steps(6, 8);
+      {
+        uint32_t aaq[4];
+        ldsm_x4(aaq, &st.ops.aqk[lane & 15][(lane >> 4) * 8]);
 #pragma unroll
-      for (int t = 0; t < 8; ++t) ldsm_x4_t(ak[t], &st.ops.ke[(lane & 7) + (lane >> 4) * 8][16 * t + ((lane >> 3) & 1) * 8]);
-#pragma unroll
-      for (int t = 0; t < 8; ++t)
-#pragma unroll
-        for (int j = 0; j < 2; ++j) mma(sacc[t][j], ak[t], vb[j][0], vb[j][1]);
-      // ---- O += Aqk Vnew
-#pragma unroll
-      for (int j = 0; j < 2; ++j) mma(oa[j], aaq, vb[j][0], vb[j][1]);
+        for (int j = 0; j < 2; ++j) mma(oa[j], aaq, vb[j][0], vb[j][1]);
+      }
       // the stage is no longer read by this warp
       mbar_arrive_warp(&sh.c_empty[s]);
       // ---- store O: lane holds tokens gq (+8) x columns 8j + 2tq (+1)
@@ -578,23 +584,20 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
     }
     if (p.fin) {
 #pragma unroll
-      for (int t = 0; t < 8; ++t)
+      for (int u = 0; u < 16; ++u)
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            const int key = 16 * t + gq + 8 * hf;
-            const int col = dv0 + cv + 8 * j + 2 * tq;
-            *reinterpret_cast<float2*>(p.fin + sbase + static_cast<size_t>(key) * D + col) =
-                make_float2(sacc[t][j][2 * hf], sacc[t][j][2 * hf + 1]);
-          }
+        for (int e = 0; e < 4; ++e) {
+          const int key = 8 * u + 2 * tq + (e & 1);
+          const int col = dv0 + cv + gq + 8 * (e >> 1);
+          p.fin[sbase + static_cast<size_t>(key) * D + col] = sacc[u][e];
+        }
     }
-  } else if (warp >= WARP_GATE && warp < WARP_GATE + NGATE) {
+  } else if (is_gate_warp(warp)) {
     // ============================================================ gate warps
     // Thread layout: channel pair cp (channels 2cp, 2cp+1), token half th
     // (tokens 8th .. 8th+7). The decay products of the two halves meet through
     // shared memory.
-    const int gt = tid - WARP_GATE * 32;
+    const int gt = gate_warp_index(warp) * 32 + lane;
     const int cp = gt & 63;
     const int th = gt >> 6;
     const int c0 = 2 * cp;
@@ -660,10 +663,7 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
         F.x *= e[jj].x;
         F.y *= e[jj].y;
       }
-      if (th == 0) {
-        (&st.ops.gam[0][0])[gamma_index(c0)] = gamma.x;
-        (&st.ops.gam[0][0])[gamma_index(c0 + 1)] = gamma.y;
-      }
+      if (th == 0) *reinterpret_cast<float2*>(&st.ops.gam[0][0] + gamma_index(c0)) = gamma;
       fence_proxy_async_shared();
       mbar_arrive_warp(&sh.gate_done[ps]);
     }
@@ -783,7 +783,7 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
         cp_async_arrive(&sh.raw_full[rs]);
       }
     }
-  } else {
+  } else if (warp == WARP_CLOAD) {
     // ====================================================== consumer loads
     if (lane == 0) {
       for (int n = 0; n < nch; ++n) {
