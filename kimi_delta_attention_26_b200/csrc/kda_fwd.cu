@@ -25,7 +25,9 @@
 //                   T = (I + L)^{-1} by forward substitution and T diag(beta).
 //     11    store:  (producer) bulk-stores a finished chunk to its ring slot and
 //                   signals the cluster.
-//     8-9   idle.
+//     8     notify: (consumer) relays each landed stage to the chain warps
+//                   through hardware named barriers.
+//     9     idle.
 //
 // Per chunk of C = 16 tokens, with Gamma_i the inclusive cumulative log-decay
 // inside the chunk (e_i = exp(g_i) per channel):
@@ -69,21 +71,27 @@ constexpr int NSLICE = D / NS;    // CTAs per (sequence, head) = cluster size
 constexpr int RING = 16;          // ring slots per (sequence, head); multiple of NSLICE
 constexpr int PRSTAGE = 2;        // producer raw-input stages
 constexpr int PSTAGE = 3;         // producer operand stages
-constexpr int CSTAGE = 8;         // consumer stages (cload -> chain)
+constexpr int CSTAGE = 6;         // consumer stages (cload -> chain)
 // Warp w issues on sub-partition w mod 4. The two chain warps get partitions 0
-// and 1 with only the light load warps beside them; the gate, mma and store
-// warps, which burst through ALU and shared-memory work, share partitions 2
-// and 3. Warps 8 and 9 have no role (they fill the numbering).
+// and 1 with only the light load and notify warps beside them; the gate, mma
+// and store warps, which burst through ALU and shared-memory work, share
+// partitions 2 and 3. Warp 9 has no role (it fills the numbering).
 constexpr int NCHAIN = NS / 16;   // chain warps (0, 1), 16 value columns each
 constexpr int NGATE = 4;          // gate warps 2, 3, 6, 7
 constexpr int WARP_PLOAD = 4;
 constexpr int WARP_CLOAD = 5;
+constexpr int WARP_NOTIFY = 8;    // relays stage completion to the chain warps
 constexpr int WARP_MMA = 10;      // also solves (I + L)^{-1}
 constexpr int WARP_STORE = 11;
 constexpr int NTHREADS = 12 * 32;
 __host__ __device__ constexpr bool is_gate_warp(int w) { return (w & 3) >= 2 && w < 8; }
 __host__ __device__ constexpr int gate_warp_index(int w) { return (w & 1) + ((w >> 2) << 1); }
 static_assert(NCHAIN == 2, "warp layout assumes two chain warps");
+// Hardware named barriers: 0 is the CTA-wide one, 1 the gate group's, and
+// 2 + 2 s + w tells chain warp w that consumer stage s has landed.
+constexpr int BAR_GATE = 1;
+constexpr int BAR_FULL0 = 2;
+static_assert(BAR_FULL0 + 2 * CSTAGE <= 16, "named barrier ids");
 static_assert(RING % NSLICE == 0, "a ring slot must always belong to the same producer CTA");
 
 // Padded row pitches: 272 B and 48 B rows keep 8-row ldmatrix reads on distinct banks.
@@ -231,6 +239,9 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
+__device__ __forceinline__ void named_bar_arrive(int id, int nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 __device__ __forceinline__ void named_bar(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -456,12 +467,12 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
 
     for (int n = 0; n < nch; ++n) {
       const int s = n % CSTAGE;
-      const uint32_t ph = static_cast<uint32_t>(n / CSTAGE) & 1u;
       const int64_t cs = t0 + static_cast<int64_t>(n) * C;
       const int m = static_cast<int>((t1 - cs) < C ? (t1 - cs) : C);
       ChainStage& st = sh.cst[s];
 
-      mbar_wait(&sh.c_full[s], ph);
+      // stage s has landed (the notify warp observed its mbarrier)
+      named_bar(BAR_FULL0 + 2 * s + warp, 64);
       // the ring slot has been copied here: give it back to its producer
       if (warp == 0 && lane == 0)
         mbar_arrive_remote_relaxed(&sh.slot_free[n % RING], static_cast<uint32_t>(n % NSLICE));
@@ -639,7 +650,7 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
       mbar_wait(&sh.prod_free[ps], pph ^ 1u);
       sh.gprod[j & 1][th][cp] = P;
       if (gt < C) st.beta[gt] = bv;
-      named_bar(1, NGATE * 32);
+      named_bar(BAR_GATE, NGATE * 32);
       const float2 Po = sh.gprod[j & 1][th ^ 1][cp];
       // E before this half (1 for the first half), F after it (1 for the second)
       float2 E = th ? Po : make_float2(1.f, 1.f);
@@ -782,6 +793,20 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
         cp_async4(&rw.beta[r], p.beta + (ok ? (cs + r) * H + h : 0), ok ? 4u : 0u);
         cp_async_arrive(&sh.raw_full[rs]);
       }
+    }
+  } else if (warp == WARP_NOTIFY) {
+    // ==================================================== stage notifications
+    // Waiting on a transaction mbarrier costs the waiter ~100 cycles even when
+    // the phase completed long ago; this warp takes that cost off the chain's
+    // critical path and releases each chain warp through a hardware barrier.
+    // The mbarrier acquire makes the landed bytes visible to this warp and the
+    // barrier orders them before the chain warps' reads.
+    for (int n = 0; n < nch; ++n) {
+      const int s = n % CSTAGE;
+      mbar_wait(&sh.c_full[s], static_cast<uint32_t>(n / CSTAGE) & 1u);
+      __syncwarp();
+      named_bar_arrive(BAR_FULL0 + 2 * s, 64);
+      named_bar_arrive(BAR_FULL0 + 2 * s + 1, 64);
     }
   } else if (warp == WARP_CLOAD) {
     // ====================================================== consumer loads
