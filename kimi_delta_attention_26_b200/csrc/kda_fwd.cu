@@ -279,6 +279,16 @@ __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
   return y;
 }
 
+// (x, y) *= (a, b) as one packed fp32 multiply
+__device__ __forceinline__ void mul2(float& x, float& y, float a, float b) {
+  unsigned long long r;
+  asm("mul.rn.f32x2 %0, %1, %2;"
+      : "=l"(r)
+      : "l"((static_cast<unsigned long long>(__float_as_uint(y)) << 32) | __float_as_uint(x)),
+        "l"((static_cast<unsigned long long>(__float_as_uint(b)) << 32) | __float_as_uint(a)));
+  x = __uint_as_float(static_cast<uint32_t>(r));
+  y = __uint_as_float(static_cast<uint32_t>(r >> 32));
+}
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   uint32_t u;
@@ -473,9 +483,6 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
 
       // stage s has landed (the notify warp observed its mbarrier)
       named_bar(BAR_FULL0 + 2 * s + warp, 64);
-      // the ring slot has been copied here: give it back to its producer
-      if (warp == 0 && lane == 0)
-        mbar_arrive_remote_relaxed(&sh.slot_free[n % RING], static_cast<uint32_t>(n % NSLICE));
 
       // The products are ordered for one in-order warp on one tensor pipe: the
       // state's own chain (X -> Vnew -> S) goes first at every step and the O
@@ -514,14 +521,10 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
             mma(xa[j], ak[t], sb[t][j][0], sb[t][j][1]);
         }
         const float4 g4 = gp[t];
-        sacc[2 * t][0] *= g4.x;
-        sacc[2 * t][1] *= g4.y;
-        sacc[2 * t][2] *= g4.x;
-        sacc[2 * t][3] *= g4.y;
-        sacc[2 * t + 1][0] *= g4.z;
-        sacc[2 * t + 1][1] *= g4.w;
-        sacc[2 * t + 1][2] *= g4.z;
-        sacc[2 * t + 1][3] *= g4.w;
+        mul2(sacc[2 * t][0], sacc[2 * t][1], g4.x, g4.y);
+        mul2(sacc[2 * t][2], sacc[2 * t][3], g4.x, g4.y);
+        mul2(sacc[2 * t + 1][0], sacc[2 * t + 1][1], g4.z, g4.w);
+        mul2(sacc[2 * t + 1][2], sacc[2 * t + 1][3], g4.z, g4.w);
       }
       // ---- O = Qd S (chunk-start state) + Aqk Vnew, in three installments
       float oa[2][4] = {}, ob[2][4] = {};
@@ -807,6 +810,8 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
       __syncwarp();
       named_bar_arrive(BAR_FULL0 + 2 * s, 64);
       named_bar_arrive(BAR_FULL0 + 2 * s + 1, 64);
+      // the ring slot has been copied here: give it back to its producer
+      if (lane == 0) mbar_arrive_remote_relaxed(&sh.slot_free[n % RING], static_cast<uint32_t>(n % NSLICE));
     }
   } else if (warp == WARP_CLOAD) {
     // ====================================================== consumer loads
