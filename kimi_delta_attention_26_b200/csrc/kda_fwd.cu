@@ -457,12 +457,11 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
   if (warp < NCHAIN) {
     // =========================================================== chain warps
     // Warp w owns S^T[16 value columns x 128 keys] (columns 16w .. 16w+15 of
-    // the slice) for the whole sequence: tile st[u] holds keys 8u .. 8u+7 as an
-    // m16n8 accumulator, so lane (gq, tq) holds columns gq (+8) x keys 8u+2tq
-    // (+1). Packed to bf16 these registers are, unchanged, the B fragments of
-    // products over the keys (X = Kd S, O = Qd S), and the state update
-    // S^T += Vnew^T Kend takes Vnew^T as its A operand. Nothing of the state
-    // leaves the registers and the warp needs no partner.
+    // the slice) for the whole sequence: tile sacc[u] holds keys 8u .. 8u+7 as
+    // an m16n8 accumulator, so lane (gq, tq) holds columns gq (+8) x keys
+    // 8u+2tq (+1). Packed to bf16 these registers are, unchanged, the A
+    // fragments of products over the keys (X^T = S^T Kd^T, O^T = S^T Qd^T).
+    // Nothing of the state leaves the registers and the warp needs no partner.
     const int cv = 16 * warp;          // first value column (slice-local)
     float sacc[16][4];
     const size_t sbase = (static_cast<size_t>(seq) * H + h) * D * D;
@@ -484,41 +483,46 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
       // stage s has landed (the notify warp observed its mbarrier)
       named_bar(BAR_FULL0 + 2 * s + warp, 64);
 
+      // Every product on the chain takes the register-resident operand as its
+      // A fragment, so nothing on the chain needs a transpose:
+      //   X^T = V^T + S^T Kd^T,  Vnew^T = X^T Tb^T,  S^T <- S^T Diag(gamma) + Vnew^T Kend,
+      //   O^T = S^T Qd^T + Vnew^T Aqk^T.
       // The products are ordered for one in-order warp on one tensor pipe: the
       // state's own chain (X -> Vnew -> S) goes first at every step and the O
       // products, which nothing waits for, fill the pipe while a chain result
-      // drains through conversion and transpose.
-      uint32_t ak[8][4];
+      // drains through conversion.
+      uint32_t bk[8][4];
 #pragma unroll
-      for (int t = 0; t < 8; ++t) ldsm_x4(ak[t], &st.ops.kd[lane & 15][16 * t + (lane >> 4) * 8]);
-      // ---- X = V + Kd S   (two accumulator chains per column tile); each key
-      // tile of S is packed to bf16 (sb, the chunk-start state also used by O)
-      // and then scaled by gamma for the update
+      for (int t = 0; t < 8; ++t) ldsm_x4(bk[t], &st.ops.kd[(lane & 7) + ((lane >> 4) << 3)][16 * t + ((lane >> 3) & 1) * 8]);
+      // ---- X^T (two accumulator chains per 8-token tile); each key tile of S
+      // is packed to bf16 (sa: the chunk-start state, also used by O) and then
+      // scaled by gamma for the update. Lane (gq, tq) of tile nt holds columns
+      // gq (+8) x tokens 8nt + 2tq (+1).
       float xa[2][4], xb[2][4] = {};
       {
-        uint32_t vv[4];
-        ldsm_x4(vv, &st.v[(lane & 7) + ((lane >> 3) & 1) * 8][cv + (lane >> 4) * 8]);
+        uint32_t vt[4];
+        ldsm_x4_t(vt, &st.v[(lane & 7) + ((lane >> 3) & 1) * 8][cv + (lane >> 4) * 8]);
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            const uint32_t w2 = vv[2 * j + hf];
-            xa[j][2 * hf] = __uint_as_float(w2 << 16);
-            xa[j][2 * hf + 1] = __uint_as_float(w2 & 0xffff0000u);
-          }
+        for (int j = 0; j < 4; ++j) {
+          const int nt = j & 1, e0 = 2 * (j >> 1);
+          xa[nt][e0] = __uint_as_float(vt[j] << 16);
+          xa[nt][e0 + 1] = __uint_as_float(vt[j] & 0xffff0000u);
+        }
       }
-      uint32_t sb[8][2][2];
+      uint32_t sa[8][4];
       const float4* gp = reinterpret_cast<const float4*>(&st.ops.gam[tq][0]);
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
+        sa[t][0] = pack_bf16(sacc[2 * t][0], sacc[2 * t][1]);
+        sa[t][1] = pack_bf16(sacc[2 * t][2], sacc[2 * t][3]);
+        sa[t][2] = pack_bf16(sacc[2 * t + 1][0], sacc[2 * t + 1][1]);
+        sa[t][3] = pack_bf16(sacc[2 * t + 1][2], sacc[2 * t + 1][3]);
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          sb[t][j][0] = pack_bf16(sacc[2 * t][2 * j], sacc[2 * t][2 * j + 1]);
-          sb[t][j][1] = pack_bf16(sacc[2 * t + 1][2 * j], sacc[2 * t + 1][2 * j + 1]);
+        for (int nt = 0; nt < 2; ++nt) {
           if (t & 1)
-            mma(xb[j], ak[t], sb[t][j][0], sb[t][j][1]);
+            mma(xb[nt], sa[t], bk[t][2 * nt], bk[t][2 * nt + 1]);
           else
-            mma(xa[j], ak[t], sb[t][j][0], sb[t][j][1]);
+            mma(xa[nt], sa[t], bk[t][2 * nt], bk[t][2 * nt + 1]);
         }
         const float4 g4 = gp[t];
         mul2(sacc[2 * t][0], sacc[2 * t][1], g4.x, g4.y);
@@ -526,73 +530,78 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
         mul2(sacc[2 * t + 1][0], sacc[2 * t + 1][1], g4.z, g4.w);
         mul2(sacc[2 * t + 1][2], sacc[2 * t + 1][3], g4.z, g4.w);
       }
-      // ---- O = Qd S (chunk-start state) + Aqk Vnew, in three installments
+      // ---- O^T = S^T Qd^T (chunk-start state) + Vnew^T Aqk^T, in three installments
       float oa[2][4] = {}, ob[2][4] = {};
       auto o_steps = [&](int t_begin, int t_end) {
 #pragma unroll
         for (int t = t_begin; t < t_end; ++t) {
-          uint32_t aq[4];
-          ldsm_x4(aq, &st.ops.qd[lane & 15][16 * t + (lane >> 4) * 8]);
+          uint32_t bq[4];
+          ldsm_x4(bq, &st.ops.qd[(lane & 7) + ((lane >> 4) << 3)][16 * t + ((lane >> 3) & 1) * 8]);
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
+          for (int nt = 0; nt < 2; ++nt) {
             if (t & 1)
-              mma(ob[j], aq, sb[t][j][0], sb[t][j][1]);
+              mma(ob[nt], sa[t], bq[2 * nt], bq[2 * nt + 1]);
             else
-              mma(oa[j], aq, sb[t][j][0], sb[t][j][1]);
+              mma(oa[nt], sa[t], bq[2 * nt], bq[2 * nt + 1]);
           }
         }
       };
       o_steps(0, 3);
-      // ---- Vnew = Tb X
-      uint32_t atb[4];
-      ldsm_x4(atb, &st.ops.tb[lane & 15][(lane >> 4) * 8]);
+      // ---- Vnew^T = X^T Tb^T
+      uint32_t bt[4];
+      ldsm_x4(bt, &st.ops.tb[(lane & 7) + ((lane >> 4) << 3)][((lane >> 3) & 1) * 8]);
       float vn[2][4] = {};
+      {
+        uint32_t ax[4];
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const uint32_t b0 = movmatrix_t(pack_bf16(xa[j][0] + xb[j][0], xa[j][1] + xb[j][1]));
-        const uint32_t b1 = movmatrix_t(pack_bf16(xa[j][2] + xb[j][2], xa[j][3] + xb[j][3]));
-        mma(vn[j], atb, b0, b1);
+        for (int nt = 0; nt < 2; ++nt) {
+          ax[2 * nt] = pack_bf16(xa[nt][0] + xb[nt][0], xa[nt][1] + xb[nt][1]);
+          ax[2 * nt + 1] = pack_bf16(xa[nt][2] + xb[nt][2], xa[nt][3] + xb[nt][3]);
+        }
+        mma(vn[0], ax, bt[0], bt[1]);
+        mma(vn[1], ax, bt[2], bt[3]);
       }
-      // kd fragments are dead: the same registers take Kend^T
+      // kd fragments are dead: the same registers take Kend
 #pragma unroll
-      for (int t = 0; t < 8; ++t) ldsm_x4_t(ak[t], &st.ops.ke[(lane & 7) + ((lane >> 3) & 1) * 8][16 * t + (lane >> 4) * 8]);
+      for (int t = 0; t < 8; ++t) ldsm_x4_t(bk[t], &st.ops.ke[(lane & 7) + ((lane >> 3) & 1) * 8][16 * t + (lane >> 4) * 8]);
       o_steps(3, 6);
-      // Vnew as B fragments (k = tokens, n = columns 8j..); the same registers
-      // form Vnew^T as an A fragment: {vb[0][0], vb[1][0], vb[0][1], vb[1][1]}
-      uint32_t vb[2][2];
+      // Vnew^T as an A fragment (rows = columns, k = tokens)
+      uint32_t av[4];
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        vb[j][0] = movmatrix_t(pack_bf16(vn[j][0], vn[j][1]));
-        vb[j][1] = movmatrix_t(pack_bf16(vn[j][2], vn[j][3]));
+      for (int nt = 0; nt < 2; ++nt) {
+        av[2 * nt] = pack_bf16(vn[nt][0], vn[nt][1]);
+        av[2 * nt + 1] = pack_bf16(vn[nt][2], vn[nt][3]);
       }
       // ---- S^T <- S^T Diag(gamma) + Vnew^T Kend  (gamma applied above)
-      {
-        const uint32_t av[4] = {vb[0][0], vb[1][0], vb[0][1], vb[1][1]};
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          mma(sacc[2 * t], av, ak[t][0], ak[t][1]);
-          mma(sacc[2 * t + 1], av, ak[t][2], ak[t][3]);
-        }
+      for (int t = 0; t < 8; ++t) {
+        mma(sacc[2 * t], av, bk[t][0], bk[t][1]);
+        mma(sacc[2 * t + 1], av, bk[t][2], bk[t][3]);
       }
       o_steps(6, 8);
       {
-        uint32_t aaq[4];
-        ldsm_x4(aaq, &st.ops.aqk[lane & 15][(lane >> 4) * 8]);
-#pragma unroll
-        for (int j = 0; j < 2; ++j) mma(oa[j], aaq, vb[j][0], vb[j][1]);
+        uint32_t ba[4];
+        ldsm_x4(ba, &st.ops.aqk[(lane & 7) + ((lane >> 4) << 3)][((lane >> 3) & 1) * 8]);
+        mma(oa[0], av, ba[0], ba[1]);
+        mma(oa[1], av, ba[2], ba[3]);
       }
       // the stage is no longer read by this warp
       mbar_arrive_warp(&sh.c_empty[s]);
-      // ---- store O: lane holds tokens gq (+8) x columns 8j + 2tq (+1)
+      // ---- store O: an 8x8 transpose per tile turns (column, token pair) into
+      // (token, column pair)
+      uint32_t r[2][2];
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const int tok = gq + 8 * hf;
+      for (int nt = 0; nt < 2; ++nt) {
+        r[nt][0] = movmatrix_t(pack_bf16((oa[nt][0] + ob[nt][0]) * p.scale, (oa[nt][1] + ob[nt][1]) * p.scale));
+        r[nt][1] = movmatrix_t(pack_bf16((oa[nt][2] + ob[nt][2]) * p.scale, (oa[nt][3] + ob[nt][3]) * p.scale));
+      }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int tok = 8 * nt + gq;
         if (tok < m) {
           __nv_bfloat16* dst = p.out + (cs + tok) * row_stride + static_cast<size_t>(h) * D + dv0 + cv + 2 * tq;
-#pragma unroll
-          for (int j = 0; j < 2; ++j)
-            *reinterpret_cast<uint32_t*>(dst + 8 * j) =
-                pack_bf16((oa[j][2 * hf] + ob[j][2 * hf]) * p.scale, (oa[j][2 * hf + 1] + ob[j][2 * hf + 1]) * p.scale);
+          *reinterpret_cast<uint32_t*>(dst) = r[nt][0];
+          *reinterpret_cast<uint32_t*>(dst + 8) = r[nt][1];
         }
       }
     }
