@@ -43,7 +43,7 @@ extern "C" {
 #endif
 
 #define KDA_HEAD_DIM 128
-#define KDA_ABI_VERSION 1
+#define KDA_ABI_VERSION 2
 
 typedef enum kda_status {
   KDA_OK = 0,
@@ -93,7 +93,7 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* g
 /*
  * kda_fwd_noalloc -- kda_fwd without any device-memory allocation.
  *
- * The paper has no counterpart to this entry point; it exists for callers
+ * The method's sources have no counterpart to this entry point; it exists for callers
  * that cannot allocate device memory while they run. kda_fwd draws its
  * scratch ring from a stream-ordered memory pool, which such callers cannot
  * allow: serving engines that reserve the whole device for their own arena up
@@ -103,7 +103,7 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* g
  * Arguments, layouts, results and errors are those of kda_fwd, except:
  *   - The scratch ring lives in a fixed-size array in device memory that the
  *     library declares at file scope: every GPU that loads the library holds
- *     it (KDA_NOALLOC_MAX_PAIRS * 16 slots * 15104 bytes = 7.7 MB) until the
+ *     it (KDA_NOALLOC_MAX_PAIRS * 16 slots * 15232 bytes = 7.8 MB) until the
  *     process exits.
  *   - num_seqs * num_heads must not exceed KDA_NOALLOC_MAX_PAIRS; larger
  *     problems return KDA_ERR_CAPACITY and nothing is launched.
@@ -122,6 +122,21 @@ kda_status_t kda_fwd_noalloc(const void* q, const void* k, const void* v, const 
                              float scale, const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
                              int32_t num_heads, const float* initial_state, void* out, float* final_state,
                              void* stream);
+
+/*
+ * kda_set_slice_columns -- value columns per CTA for later calls (tuning).
+ *
+ * Each (sequence, head) runs as one thread-block cluster whose CTAs split the
+ * 128 value columns. columns = 32 uses 4 CTAs per (sequence, head); 16 uses
+ * 8, which doubles the SMs working on the same serial chains when there are
+ * few sequences and heads. columns = 0 (the default) chooses per call: 16
+ * when num_seqs * num_heads * 4 is at most half the device's SM count, else
+ * 32. Each column's arithmetic is the same either way, so the results are
+ * bitwise identical. Process-wide; affects kda_fwd and
+ * kda_fwd_noalloc. Returns KDA_ERR_SHAPE for any other value (the setting is
+ * then unchanged).
+ */
+kda_status_t kda_set_slice_columns(int32_t columns);
 
 /* Human-readable text of a status code (static storage, never NULL). */
 const char* kda_status_string(kda_status_t status);

@@ -14,7 +14,7 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["kda_fwd", "library_path", "wait_timeouts", "KDAError", "HEAD_DIM"]
+__all__ = ["kda_fwd", "library_path", "wait_timeouts", "set_slice_columns", "KDAError", "HEAD_DIM"]
 
 HEAD_DIM = 128
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -38,6 +38,8 @@ _lib.kda_abi_version.argtypes = []
 _lib.kda_abi_version.restype = ctypes.c_int32
 _lib.kda_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32]
 _lib.kda_wait_timeouts.restype = ctypes.c_int
+_lib.kda_set_slice_columns.argtypes = [ctypes.c_int32]
+_lib.kda_set_slice_columns.restype = ctypes.c_int
 
 
 class KDAError(RuntimeError):
@@ -60,6 +62,14 @@ def wait_timeouts(reset: bool = True) -> int:
     if rc != 0:
         raise KDAError(rc)
     return int(n.value)
+
+
+def set_slice_columns(columns: int) -> None:
+    """Value columns per CTA for later calls: 0 chooses per call (default), 16
+    or 32 forces that kernel variant. Process-wide."""
+    rc = _lib.kda_set_slice_columns(int(columns))
+    if rc != 0:
+        raise KDAError(rc)
 
 
 def _check(t: torch.Tensor, name: str, dtype: torch.dtype, shape: Tuple[int, ...], device) -> None:

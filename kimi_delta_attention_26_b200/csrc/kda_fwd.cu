@@ -56,6 +56,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -66,9 +67,10 @@ namespace kda {
 
 constexpr int D = KDA_HEAD_DIM;   // dk = dv = 128
 constexpr int C = 16;             // chunk length (tokens)
-constexpr int NS = 32;            // value columns per CTA
-constexpr int NSLICE = D / NS;    // CTAs per (sequence, head) = cluster size
-constexpr int RING = 16;          // ring slots per (sequence, head); multiple of NSLICE
+// Value columns per CTA (NS) is a template parameter of the kernel: 32 (four
+// CTAs per (sequence, head), two chain warps each) or, when that grid would
+// leave most SMs idle, 16 (eight CTAs, one chain warp each).
+constexpr int RING = 16;          // ring slots per (sequence, head); multiple of the cluster size
 constexpr int PRSTAGE = 2;        // producer raw-input stages
 constexpr int PSTAGE = 3;         // producer operand stages
 constexpr int CSTAGE = 6;         // consumer stages (cload -> chain)
@@ -76,7 +78,7 @@ constexpr int CSTAGE = 6;         // consumer stages (cload -> chain)
 // and 1 with only the light load and notify warps beside them; the gate, mma
 // and store warps, which burst through ALU and shared-memory work, share
 // partitions 2 and 3. Warp 9 has no role (it fills the numbering).
-constexpr int NCHAIN = NS / 16;   // chain warps (0, 1), 16 value columns each
+constexpr int MAX_CHAIN = 2;      // chain warps 0 (and 1), 16 value columns each
 constexpr int NGATE = 4;          // gate warps 2, 3, 6, 7
 constexpr int WARP_PLOAD = 4;
 constexpr int WARP_CLOAD = 5;
@@ -86,13 +88,13 @@ constexpr int WARP_STORE = 11;
 constexpr int NTHREADS = 12 * 32;
 __host__ __device__ constexpr bool is_gate_warp(int w) { return (w & 3) >= 2 && w < 8; }
 __host__ __device__ constexpr int gate_warp_index(int w) { return (w & 1) + ((w >> 2) << 1); }
-static_assert(NCHAIN == 2, "warp layout assumes two chain warps");
+
 // Hardware named barriers: 0 is the CTA-wide one, 1 the gate group's, and
 // 2 + 2 s + w tells chain warp w that consumer stage s has landed.
 constexpr int BAR_GATE = 1;
 constexpr int BAR_FULL0 = 2;
 static_assert(BAR_FULL0 + 2 * CSTAGE <= 16, "named barrier ids");
-static_assert(RING % NSLICE == 0, "a ring slot must always belong to the same producer CTA");
+static_assert(RING % (D / 16) == 0, "a ring slot must always belong to the same producer CTA");
 
 // Padded row pitches: 272 B and 48 B rows keep 8-row ldmatrix reads on distinct banks.
 constexpr int LDK = D + 8;
@@ -131,16 +133,19 @@ struct __align__(128) ProdStage {
   float beta[C];
 };
 
+template <int NS>
 struct __align__(128) ChainStage {
   Ops ops;
   __nv_bfloat16 v[C][NS];     // value slice, as its TMA box lands
 };
-constexpr uint32_t kChainBytes = kSlotBytes + C * NS * 2;
+template <int NS>
+__host__ __device__ constexpr uint32_t chain_bytes() { return kSlotBytes + C * NS * 2; }
 
+template <int NS>
 struct __align__(128) Shared {
   RawStage raw[PRSTAGE];
   ProdStage prod[PSTAGE];
-  ChainStage cst[CSTAGE];
+  ChainStage<NS> cst[CSTAGE];
   float2 gprod[2][2][64];    // per-half decay products exchanged inside the gate group
   unsigned long long raw_full[PRSTAGE], raw_empty[PRSTAGE];
   unsigned long long prod_free[PSTAGE], gate_done[PSTAGE], solved[PSTAGE];
@@ -149,8 +154,9 @@ struct __align__(128) Shared {
   unsigned long long slot_free[RING];  // arrived (remotely) by the four consumers
 };
 static_assert(sizeof(Ops) % 128 == 0 && sizeof(RawStage) % 128 == 0, "stage alignment");
-static_assert(sizeof(ProdStage) % 128 == 0 && sizeof(ChainStage) % 128 == 0, "stage alignment");
-static_assert(sizeof(Shared) <= 227 * 1024, "shared memory budget");
+static_assert(sizeof(ProdStage) % 128 == 0 && sizeof(ChainStage<16>) % 128 == 0 && sizeof(ChainStage<32>) % 128 == 0,
+              "stage alignment");
+static_assert(sizeof(Shared<32>) <= 227 * 1024 && sizeof(Shared<16>) <= 227 * 1024, "shared memory budget");
 
 // Wait budget for every mbarrier wait (cycles). A wait that runs out records
 // a timeout and lets the thread continue, so no barrier is ever left waiting.
@@ -401,10 +407,15 @@ struct TensorMaps {
   CUtensorMap q, k, g, v;
 };
 
-__global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
+template <int NS>
+__global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
     kda_fwd_kernel(const Params p, const __grid_constant__ TensorMaps tm) {
+  constexpr int NSLICE = D / NS;   // CTAs per (sequence, head) = cluster size
+  constexpr int NCHAIN = NS / 16;  // chain warps
+  static_assert(NS == 16 || NS == 32, "value slice of 16 or 32 columns");
+  static_assert(NCHAIN <= MAX_CHAIN, "warp layout");
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  Shared& sh = *reinterpret_cast<Shared*>(smem_raw);
+  Shared<NS>& sh = *reinterpret_cast<Shared<NS>*>(smem_raw);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -478,7 +489,7 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
       const int s = n % CSTAGE;
       const int64_t cs = t0 + static_cast<int64_t>(n) * C;
       const int m = static_cast<int>((t1 - cs) < C ? (t1 - cs) : C);
-      ChainStage& st = sh.cst[s];
+      ChainStage<NS>& st = sh.cst[s];
 
       // stage s has landed (the notify warp observed its mbarrier)
       named_bar(BAR_FULL0 + 2 * s + warp, 64);
@@ -817,8 +828,8 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
       const int s = n % CSTAGE;
       mbar_wait(&sh.c_full[s], static_cast<uint32_t>(n / CSTAGE) & 1u);
       __syncwarp();
-      named_bar_arrive(BAR_FULL0 + 2 * s, 64);
-      named_bar_arrive(BAR_FULL0 + 2 * s + 1, 64);
+#pragma unroll
+      for (int w = 0; w < NCHAIN; ++w) named_bar_arrive(BAR_FULL0 + 2 * s + w, 64);
       // the ring slot has been copied here: give it back to its producer
       if (lane == 0) mbar_arrive_remote_relaxed(&sh.slot_free[n % RING], static_cast<uint32_t>(n % NSLICE));
     }
@@ -830,11 +841,11 @@ __global__ void __cluster_dims__(NSLICE, 1, 1) __launch_bounds__(NTHREADS, 1)
         const uint32_t ph = static_cast<uint32_t>(n / CSTAGE) & 1u;
         const int slot = n % RING;
         const int tok = static_cast<int>(t0 + static_cast<int64_t>(n) * C);
-        ChainStage& st = sh.cst[s];
+        ChainStage<NS>& st = sh.cst[s];
         mbar_wait(&sh.c_empty[s], ph ^ 1u);
         mbar_wait_cl(&sh.ready[slot], static_cast<uint32_t>(n / RING) & 1u);
         fence_proxy_async_global();
-        mbar_arrive_expect_tx(&sh.c_full[s], kChainBytes);
+        mbar_arrive_expect_tx(&sh.c_full[s], chain_bytes<NS>());
         bulk_g2s(&st.ops, ring + static_cast<size_t>(slot) * kSlotBytes, kSlotBytes, &sh.c_full[s]);
         tma_load_3d(&st.v[0][0], &tm.v, dv0, h, tok, &sh.c_full[s]);
       }
@@ -897,16 +908,26 @@ kda_status_t encode_3d(CUtensorMap* map, const void* base, CUtensorMapDataType d
 
 constexpr int kMaxDevices = 64;
 int g_device_ready[kMaxDevices];  // 0 unknown, 1 ready, -1 unsupported
+int g_num_sms[kMaxDevices];
 // Library-private stream-ordered pool for the scratch ring. It keeps freed
 // memory (release threshold = max), so steady-state calls never map memory
 // and the process's default pool is left untouched.
 cudaMemPool_t g_pool[kMaxDevices];
+// Value columns per CTA: 0 chooses per call, 16 or 32 forces that variant.
+std::atomic<int> g_slice_columns{0};
 
-kda_status_t prepare_device(int dev) {
+template <int NS>
+cudaError_t set_smem_attribute() {
+  return cudaFuncSetAttribute(kda::kda_fwd_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(sizeof(kda::Shared<NS>)));
+}
+
+// Capability check, kernel attributes and SM count for `dev` (current).
+kda_status_t check_device(int dev) {
   if (dev < 0 || dev >= kMaxDevices) return KDA_ERR_UNSUPPORTED;
   if (g_device_ready[dev] == 1) return KDA_OK;
   if (g_device_ready[dev] == -1) return KDA_ERR_UNSUPPORTED;
-  int major = 0, minor = 0;
+  int major = 0, minor = 0, sms = 0;
   cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
   if (e != cudaSuccess) return cuda_fail(e);
   e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
@@ -915,22 +936,42 @@ kda_status_t prepare_device(int dev) {
     g_device_ready[dev] = -1;
     return KDA_ERR_UNSUPPORTED;
   }
-  e = cudaFuncSetAttribute(kda::kda_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(sizeof(kda::Shared)));
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return cuda_fail(e);
+  if ((e = set_smem_attribute<32>()) != cudaSuccess) return cuda_fail(e);
+  if ((e = set_smem_attribute<16>()) != cudaSuccess) return cuda_fail(e);
+  g_num_sms[dev] = sms;
+  g_device_ready[dev] = 1;
+  return KDA_OK;
+}
+
+// The pool of kda_fwd's scratch rings, created once per device.
+kda_status_t prepare_pool(int dev) {
+  if (g_pool[dev]) return KDA_OK;
   cudaMemPoolProps props;
   std::memset(&props, 0, sizeof(props));
   props.allocType = cudaMemAllocationTypePinned;
   props.handleTypes = cudaMemHandleTypeNone;
   props.location.type = cudaMemLocationTypeDevice;
   props.location.id = dev;
-  e = cudaMemPoolCreate(&g_pool[dev], &props);
+  cudaMemPool_t pool = nullptr;
+  cudaError_t e = cudaMemPoolCreate(&pool, &props);
   if (e != cudaSuccess) return cuda_fail(e);
   uint64_t keep = ~0ull;
-  e = cudaMemPoolSetAttribute(g_pool[dev], cudaMemPoolAttrReleaseThreshold, &keep);
+  e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
   if (e != cudaSuccess) return cuda_fail(e);
-  g_device_ready[dev] = 1;
+  g_pool[dev] = pool;
   return KDA_OK;
+}
+
+// 32-column slices unless that grid would fill at most half of the SMs (few
+// heads and sequences); then 16-column slices double the CTAs working on
+// the same serial chains.
+int slice_columns(int dev, int32_t num_seqs, int32_t num_heads) {
+  const int forced = g_slice_columns.load();
+  if (forced == 16 || forced == 32) return forced;
+  const int64_t ctas32 = int64_t(num_seqs) * num_heads * (KDA_HEAD_DIM / 32);
+  return 2 * ctas32 <= g_num_sms[dev] ? 16 : 32;
 }
 
 // ---------------------------------------------------- allocation-free variant
@@ -942,24 +983,74 @@ constexpr size_t kNoAllocRingBytes =
 static __device__ __align__(256) unsigned char g_noalloc_ring[kNoAllocRingBytes];
 void* g_noalloc_ring_addr[kMaxDevices];
 
-// Capability check, kernel attribute and array address for `dev` (current).
 kda_status_t noalloc_setup(int dev) {
-  if (dev < 0 || dev >= kMaxDevices) return KDA_ERR_UNSUPPORTED;
   if (g_noalloc_ring_addr[dev]) return KDA_OK;
-  int major = 0, minor = 0;
-  cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-  if (e != cudaSuccess) return cuda_fail(e);
-  e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
-  if (e != cudaSuccess) return cuda_fail(e);
-  if (major != 10 || minor != 0) return KDA_ERR_UNSUPPORTED;
-  e = cudaFuncSetAttribute(kda::kda_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(sizeof(kda::Shared)));
-  if (e != cudaSuccess) return cuda_fail(e);
   void* addr = nullptr;
-  e = cudaGetSymbolAddress(&addr, g_noalloc_ring);
+  cudaError_t e = cudaGetSymbolAddress(&addr, g_noalloc_ring);
   if (e != cudaSuccess) return cuda_fail(e);
   if (!addr) return KDA_ERR_CUDA;
   g_noalloc_ring_addr[dev] = addr;
+  return KDA_OK;
+}
+
+// Host-side checks shared by both entry points (synchronous, no device work).
+kda_status_t check_args(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                        const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens, int32_t num_heads,
+                        const float* initial_state, const void* out, const float* final_state) {
+  if (total_tokens < 0 || num_heads < 1 || num_seqs < 1) return KDA_ERR_SHAPE;
+  if (total_tokens > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_NULL;
+  if (!cu_seqlens && num_seqs != 1) return KDA_ERR_SHAPE;
+  if (num_heads > 65535 || num_seqs > 65535) return KDA_ERR_SHAPE;  // grid.y / grid.z limits
+  if (total_tokens > (int64_t(1) << 40) / (int64_t(num_heads) * KDA_HEAD_DIM)) return KDA_ERR_SHAPE;
+  if (total_tokens > int64_t(INT32_MAX) - 64) return KDA_ERR_SHAPE;  // TMA coordinates are 32-bit
+  const void* ptrs[] = {q, k, v, g, beta, out, initial_state, final_state, cu_seqlens};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
+  return KDA_OK;
+}
+
+// Tensor maps, variant choice and launch; `ring` holds RING slots per
+// (sequence, head).
+kda_status_t launch(const void* q, const void* k, const void* v, const float* g, const float* beta, float scale,
+                    const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens, int32_t num_heads,
+                    const float* initial_state, void* out, float* final_state, unsigned char* ring, int dev,
+                    cudaStream_t stream) {
+  kda::Params p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.g = g;
+  p.beta = beta;
+  p.cu = cu_seqlens;
+  p.init = initial_state;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.fin = final_state;
+  p.T = total_tokens;
+  p.H = num_heads;
+  p.scale = scale;
+  p.ring = ring;
+  const int ns = slice_columns(dev, num_seqs, num_heads);
+  kda::TensorMaps tm;
+  std::memset(&tm, 0, sizeof(tm));
+  if (total_tokens > 0) {
+    kda_status_t st = load_encoder();
+    if (st != KDA_OK) return st;
+    const int H = num_heads;
+    if ((st = encode_3d(&tm.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total_tokens, H, kda::D, kda::D)) != KDA_OK ||
+        (st = encode_3d(&tm.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total_tokens, H, kda::D, kda::D)) != KDA_OK ||
+        (st = encode_3d(&tm.g, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total_tokens, H, kda::D, kda::D)) != KDA_OK ||
+        (st = encode_3d(&tm.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total_tokens, H, kda::D, ns)) != KDA_OK)
+      return st;
+  }
+  if (ns == 16) {
+    kda::kda_fwd_kernel<16><<<dim3(kda::D / 16, num_heads, num_seqs), kda::NTHREADS, sizeof(kda::Shared<16>),
+                              stream>>>(p, tm);
+  } else {
+    kda::kda_fwd_kernel<32><<<dim3(kda::D / 32, num_heads, num_seqs), kda::NTHREADS, sizeof(kda::Shared<32>),
+                              stream>>>(p, tm);
+  }
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
   return KDA_OK;
 }
 
@@ -972,48 +1063,14 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* g
                      int32_t num_heads, const float* initial_state, void* out, float* final_state,
                      void* stream) {
   g_last_cuda_error[0] = '\0';
-  if (total_tokens < 0 || num_heads < 1 || num_seqs < 1) return KDA_ERR_SHAPE;
-  if (total_tokens > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_NULL;
-  if (!cu_seqlens && num_seqs != 1) return KDA_ERR_SHAPE;
-  if (num_heads > 65535 || num_seqs > 65535) return KDA_ERR_SHAPE;  // grid.y / grid.z limits
-  if (total_tokens > (int64_t(1) << 40) / (int64_t(num_heads) * KDA_HEAD_DIM)) return KDA_ERR_SHAPE;
-  if (total_tokens > int64_t(INT32_MAX) - 64) return KDA_ERR_SHAPE;  // TMA coordinates are 32-bit
-  const void* ptrs[] = {q, k, v, g, beta, out, initial_state, final_state, cu_seqlens};
-  for (const void* ptr : ptrs)
-    if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
-
+  kda_status_t st = check_args(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens, num_heads, initial_state, out,
+                               final_state);
+  if (st != KDA_OK) return st;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
-  kda_status_t st = prepare_device(dev);
-  if (st != KDA_OK) return st;
-
-  kda::Params p;
-  p.q = static_cast<const __nv_bfloat16*>(q);
-  p.k = static_cast<const __nv_bfloat16*>(k);
-  p.v = static_cast<const __nv_bfloat16*>(v);
-  p.g = g;
-  p.beta = beta;
-  p.cu = cu_seqlens;
-  p.init = initial_state;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.fin = final_state;
-  p.T = total_tokens;
-  p.H = num_heads;
-  p.scale = scale;
-  p.ring = nullptr;
-  kda::TensorMaps tm;
-  std::memset(&tm, 0, sizeof(tm));
-  if (total_tokens > 0) {
-    st = load_encoder();
-    if (st != KDA_OK) return st;
-    const int H = num_heads;
-    if ((st = encode_3d(&tm.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total_tokens, H, kda::D, kda::D)) != KDA_OK ||
-        (st = encode_3d(&tm.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total_tokens, H, kda::D, kda::D)) != KDA_OK ||
-        (st = encode_3d(&tm.g, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total_tokens, H, kda::D, kda::D)) != KDA_OK ||
-        (st = encode_3d(&tm.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total_tokens, H, kda::D, kda::NS)) != KDA_OK)
-      return st;
-  }
+  if ((st = check_device(dev)) != KDA_OK) return st;
+  if ((st = prepare_pool(dev)) != KDA_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   // Ring of shared chunk operands, one per (sequence, head): stream-ordered
   // scratch from the library's pool, released in stream order after the
@@ -1023,17 +1080,14 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* g
     const size_t ring_bytes = static_cast<size_t>(num_seqs) * num_heads * kda::RING * kda::kSlotBytes;
     e = cudaMallocFromPoolAsync(&ring, ring_bytes, g_pool[dev], cs);
     if (e != cudaSuccess) return cuda_fail(e);
-    p.ring = static_cast<unsigned char*>(ring);
   }
-  dim3 grid(kda::NSLICE, num_heads, num_seqs);
-  kda::kda_fwd_kernel<<<grid, kda::NTHREADS, sizeof(kda::Shared), cs>>>(p, tm);
-  e = cudaGetLastError();
+  st = launch(q, k, v, g, beta, scale, cu_seqlens, num_seqs, total_tokens, num_heads, initial_state, out, final_state,
+              static_cast<unsigned char*>(ring), dev, cs);
   if (ring) {
     const cudaError_t ef = cudaFreeAsync(ring, cs);
-    if (e == cudaSuccess) e = ef;
+    if (st == KDA_OK && ef != cudaSuccess) return cuda_fail(ef);
   }
-  if (e != cudaSuccess) return cuda_fail(e);
-  return KDA_OK;
+  return st;
 }
 
 kda_status_t kda_fwd_noalloc(const void* q, const void* k, const void* v, const float* g, const float* beta,
@@ -1041,53 +1095,23 @@ kda_status_t kda_fwd_noalloc(const void* q, const void* k, const void* v, const 
                              int32_t num_heads, const float* initial_state, void* out, float* final_state,
                              void* stream) {
   g_last_cuda_error[0] = '\0';
-  if (total_tokens < 0 || num_heads < 1 || num_seqs < 1) return KDA_ERR_SHAPE;
-  if (total_tokens > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_NULL;
-  if (!cu_seqlens && num_seqs != 1) return KDA_ERR_SHAPE;
-  if (num_heads > 65535 || num_seqs > 65535) return KDA_ERR_SHAPE;
-  if (total_tokens > (int64_t(1) << 40) / (int64_t(num_heads) * KDA_HEAD_DIM)) return KDA_ERR_SHAPE;
-  if (total_tokens > int64_t(INT32_MAX) - 64) return KDA_ERR_SHAPE;
+  kda_status_t st = check_args(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens, num_heads, initial_state, out,
+                               final_state);
+  if (st != KDA_OK) return st;
   if (int64_t(num_seqs) * num_heads > KDA_NOALLOC_MAX_PAIRS) return KDA_ERR_CAPACITY;
-  const void* ptrs[] = {q, k, v, g, beta, out, initial_state, final_state, cu_seqlens};
-  for (const void* ptr : ptrs)
-    if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
-
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
-  kda_status_t st = noalloc_setup(dev);
-  if (st != KDA_OK) return st;
+  if ((st = check_device(dev)) != KDA_OK) return st;
+  if ((st = noalloc_setup(dev)) != KDA_OK) return st;
+  return launch(q, k, v, g, beta, scale, cu_seqlens, num_seqs, total_tokens, num_heads, initial_state, out,
+                final_state, static_cast<unsigned char*>(g_noalloc_ring_addr[dev]), dev,
+                static_cast<cudaStream_t>(stream));
+}
 
-  kda::Params p;
-  p.q = static_cast<const __nv_bfloat16*>(q);
-  p.k = static_cast<const __nv_bfloat16*>(k);
-  p.v = static_cast<const __nv_bfloat16*>(v);
-  p.g = g;
-  p.beta = beta;
-  p.cu = cu_seqlens;
-  p.init = initial_state;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.fin = final_state;
-  p.T = total_tokens;
-  p.H = num_heads;
-  p.scale = scale;
-  p.ring = static_cast<unsigned char*>(g_noalloc_ring_addr[dev]);
-  kda::TensorMaps tm;
-  std::memset(&tm, 0, sizeof(tm));
-  if (total_tokens > 0) {
-    st = load_encoder();
-    if (st != KDA_OK) return st;
-    const int H = num_heads;
-    if ((st = encode_3d(&tm.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total_tokens, H, kda::D, kda::D)) != KDA_OK ||
-        (st = encode_3d(&tm.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total_tokens, H, kda::D, kda::D)) != KDA_OK ||
-        (st = encode_3d(&tm.g, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total_tokens, H, kda::D, kda::D)) != KDA_OK ||
-        (st = encode_3d(&tm.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total_tokens, H, kda::D, kda::NS)) != KDA_OK)
-      return st;
-  }
-  dim3 grid(kda::NSLICE, num_heads, num_seqs);
-  kda::kda_fwd_kernel<<<grid, kda::NTHREADS, sizeof(kda::Shared), static_cast<cudaStream_t>(stream)>>>(p, tm);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e);
+kda_status_t kda_set_slice_columns(int32_t columns) {
+  if (columns != 0 && columns != 16 && columns != 32) return KDA_ERR_SHAPE;
+  g_slice_columns.store(columns);
   return KDA_OK;
 }
 

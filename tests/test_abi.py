@@ -37,7 +37,7 @@ def test_exports_every_declared_symbol(lib):
 
 def test_abi_version_and_status_strings(lib):
     lib.kda_abi_version.restype = ctypes.c_int32
-    assert lib.kda_abi_version() == 1
+    assert lib.kda_abi_version() == 2
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_status_string.argtypes = [ctypes.c_int]
     for code in range(6):
@@ -52,6 +52,15 @@ def _call(lib, q=0x1000, k=0x2000, v=0x3000, g=0x4000, beta=0x5000, scale=1.0, c
                             P, P, P, P]
     lib.kda_fwd.restype = ctypes.c_int
     return lib.kda_fwd(q, k, v, g, beta, scale, cu, nseq, T, H, init, out, fin, None)
+
+
+def test_slice_columns_setting_validated(lib):
+    lib.kda_set_slice_columns.argtypes = [ctypes.c_int32]
+    lib.kda_set_slice_columns.restype = ctypes.c_int
+    for bad in (-1, 1, 8, 24, 64, 128):
+        assert lib.kda_set_slice_columns(bad) == 2  # KDA_ERR_SHAPE
+    for good in (16, 32, 0):
+        assert lib.kda_set_slice_columns(good) == 0
 
 
 # These calls fail validation before any CUDA call, so the fake addresses are

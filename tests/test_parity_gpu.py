@@ -24,6 +24,15 @@ def kda():
     return m
 
 
+@pytest.fixture(params=[16, 32], ids=["slice16", "slice32"])
+def slice_cols(request, kda):
+    """Both kernel variants (16- and 32-column value slices per CTA); the
+    automatic choice is restored afterwards."""
+    kda.set_slice_columns(request.param)
+    yield request.param
+    kda.set_slice_columns(0)
+
+
 def _check(oracle_mod, inp, label, cols=None, **kw):
     out, fin = H.run_gpu(inp, **kw)
     if cols is None:
@@ -33,14 +42,14 @@ def _check(oracle_mod, inp, label, cols=None, **kw):
     return H.assert_parity(out, fin, o_ref, f_ref, cols=cols, label=label)
 
 
-def test_tiny_config(kda, oracle_mod):
+def test_tiny_config(kda, oracle_mod, slice_cols):
     inp = kda_inputs.workload(1).make()
     mo, ms = _check(oracle_mod, inp, "tiny T=256 H=2")
     print("tiny", mo, ms)
 
 
 @pytest.mark.parametrize("seed", [0, 1])
-def test_ragged_varlen_small(kda, oracle_mod, seed):
+def test_ragged_varlen_small(kda, oracle_mod, seed, slice_cols):
     # lengths around the 16-token anchor blocks and 64-token chunks, an empty
     # sequence, several chunks, random initial states
     lens = [1, 15, 16, 17, 63, 64, 65, 200, 0, 129, 300]
@@ -58,7 +67,7 @@ def test_zero_initial_state_null_equals_zeros(kda):
     assert torch.equal(out_a, out_b) and torch.equal(fin_a, fin_b)
 
 
-def test_gate_extremes(kda, oracle_mod):
+def test_gate_extremes(kda, oracle_mod, slice_cols):
     # g at the lower bound everywhere (fastest decay) and g = 0 (no decay)
     for fill in (-5.0, 0.0):
         inp = kda_inputs.make_inputs([150, 70], 2, seed=8, random_initial_state=True)
@@ -66,7 +75,7 @@ def test_gate_extremes(kda, oracle_mod):
         _check(oracle_mod, inp, f"g={fill}")
 
 
-def test_single_token_and_all_empty(kda, oracle_mod):
+def test_single_token_and_all_empty(kda, oracle_mod, slice_cols):
     import torch
 
     inp = kda_inputs.make_inputs([1], 4, seed=9, random_initial_state=True)
@@ -77,7 +86,7 @@ def test_single_token_and_all_empty(kda, oracle_mod):
     assert torch.equal(fin.cpu(), torch.from_numpy(inp.initial_state))
 
 
-def test_segments_bit_exact(kda):
+def test_segments_bit_exact(kda, slice_cols):
     """A packed batch restricted to one sequence equals that sequence run alone, bitwise."""
     import torch
 
@@ -107,7 +116,7 @@ def test_no_cu_seqlens_equals_single_sequence(kda):
 
 
 @pytest.mark.parametrize("t1", [64, 100])
-def test_resume_from_final_state(kda, oracle_mod, t1):
+def test_resume_from_final_state(kda, oracle_mod, t1, slice_cols):
     import torch
 
     inp = kda_inputs.make_inputs([257], 2, seed=13, random_initial_state=True)
@@ -126,7 +135,7 @@ def test_resume_from_final_state(kda, oracle_mod, t1):
         assert torch.equal(b_f, full_f)
 
 
-def test_in_place_state_update(kda):
+def test_in_place_state_update(kda, slice_cols):
     import torch
 
     inp = kda_inputs.make_inputs([90, 10], 2, seed=14, random_initial_state=True)
@@ -148,7 +157,7 @@ def test_deterministic(kda):
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
-def test_no_writes_outside_outputs(kda):
+def test_no_writes_outside_outputs(kda, slice_cols):
     """Guard regions around out and final_state keep their sentinel values."""
     import torch
 
@@ -173,10 +182,27 @@ def test_no_writes_outside_outputs(kda):
 # independently, so a column subset is exact) for every token and head.
 @pytest.mark.parametrize("cfg", [2, 3, 4, 5])
 def test_full_size_workloads_sampled_columns(kda, oracle_mod, cfg):
+    # the automatic variant choice: 32-column slices for configs 2-4, 16 for 5
     inp = kda_inputs.workload(cfg).make()
     cols = slice(40, 56) if cfg != 5 else slice(100, 108)
     mo, ms = _check(oracle_mod, inp, f"config {cfg}", cols=cols)
     print(f"config {cfg}", mo, ms)
+
+
+def test_slice_variants_bitwise_equal(kda):
+    """Each column's arithmetic does not depend on how many columns a CTA
+    holds, so the two variants give the same bits."""
+    import torch
+
+    inp = kda_inputs.make_inputs([700, 129, 64], 3, seed=17, random_initial_state=True)
+    res = {}
+    for cols in (16, 32):
+        kda.set_slice_columns(cols)
+        res[cols] = H.run_gpu(inp)
+    kda.set_slice_columns(0)
+    o16, f16 = res[16]
+    o32, f32 = res[32]
+    assert torch.equal(o16, o32) and torch.equal(f16, f32)
 
 
 def test_zz_no_wait_timeouts(kda):
