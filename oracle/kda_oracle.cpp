@@ -20,7 +20,7 @@
 // FlashAttention cu_seqlens convention (same FlashKDA page, section
 // "تكامل مباشر مع flash-linear-attention").
 //
-// Readings taken where the pages are silent (all listed in the design doc):
+// Readings taken where the pages are silent:
 //   * g_t scales the KEY rows of S (Diag multiplies S from the left).
 //   * decay first, then erase, then write -- exactly the order of the formula.
 //   * o_t reads S_t, i.e. after token t's own decay and write.
