@@ -75,6 +75,21 @@ def test_gate_extremes(kda, oracle_mod, slice_cols):
         _check(oracle_mod, inp, f"g={fill}")
 
 
+def test_beta_zero_reads_only_the_decayed_initial_state(kda, oracle_mod, slice_cols):
+    # beta = 0: no token writes, so o_t = scale (q_t * exp G_t)^T S_0 and the
+    # final state is Diag(exp G_T) S_0 (checked against the oracle's scan)
+    inp = kda_inputs.make_inputs([90, 33], 2, seed=19, random_initial_state=True)
+    inp.beta[:] = 0.0
+    _check(oracle_mod, inp, "beta=0")
+
+
+def test_chunk_boundary_lengths_with_empty_sequences(kda, oracle_mod, slice_cols):
+    # every length around 16-token chunk boundaries, empty sequences between
+    lens = [15, 0, 16, 17, 0, 0, 31, 32, 33, 47, 48, 49, 0]
+    inp = kda_inputs.make_inputs(lens, 2, seed=21, random_initial_state=True)
+    _check(oracle_mod, inp, "chunk-boundary lengths")
+
+
 def test_single_token_and_all_empty(kda, oracle_mod, slice_cols):
     import torch
 
