@@ -48,11 +48,37 @@ def log(*a):
     print(*a, file=sys.stderr, flush=True)
 
 
+def _code_only(src: str) -> str:
+    """C/C++/CUDA source with comments removed and whitespace collapsed, so
+    that editing a comment does not count as changing the kernel."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        if src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        elif src[i] in "\"'":
+            q, j = src[i], i + 1
+            while j < n and src[j] != q:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        else:
+            out.append(src[i])
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_sha() -> str:
+    """Hash of the kernel's code (comments and layout excluded): a profile's
+    DRAM traffic applies while this matches the hash recorded with it."""
     h = hashlib.sha256()
     for p in KERNEL_SOURCES:
-        with open(p, "rb") as f:
-            h.update(f.read())
+        with open(p, encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()
 
 

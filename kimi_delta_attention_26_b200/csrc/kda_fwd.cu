@@ -1,17 +1,20 @@
 // kda_fwd.cu -- chunked Kimi Delta Attention forward (prefill) for sm_100a.
 //
 // Work decomposition
-//   One thread-block cluster per (sequence, head): four CTAs, one per 32-column
-//   value slice. Columns of the state evolve independently (the recurrence
-//   multiplies S only from the left), so the four state chains never exchange
-//   data. What they share is the chunk-local work on keys, queries and gates,
-//   which is identical for every slice: CTA n mod 4 of the cluster produces the
-//   shared operands of chunk n once, stores them to an L2-resident ring in
-//   global memory and signals the four CTAs with remote mbarrier arrivals; every
-//   CTA then pulls the chunk with one bulk copy.
+//   One thread-block cluster per (sequence, head): one CTA per value slice of
+//   NS columns (NS = 32: four CTAs; NS = 16, for few sequences and heads:
+//   eight). Columns of the state evolve independently (the recurrence
+//   multiplies S only from the left), so the slices' state chains never
+//   exchange data. What they share is the chunk-local work on keys, queries
+//   and gates, which is identical for every slice: CTA n mod (cluster size)
+//   produces the shared operands of chunk n once, stores them to an
+//   L2-resident ring in global memory and signals every CTA of the cluster
+//   with remote mbarrier arrivals; every CTA then pulls the chunk with one
+//   bulk copy.
 //
 //   Warp roles inside a CTA (warp w issues on sub-partition w mod 4):
-//     0-1   chain:  the serial state recurrence of this CTA's value slice. Warp w
+//     0-1   chain:  the serial state recurrence of this CTA's value slice (warp 0
+//                   only when NS = 16). Warp w
 //                   owns S^T[16 value columns x 128 keys] in mma.sync accumulator
 //                   registers for the whole sequence and computes X, Vnew, O and
 //                   the state update of those columns; it shares nothing with
@@ -26,7 +29,8 @@
 //     11    store:  (producer) bulk-stores a finished chunk to its ring slot and
 //                   signals the cluster.
 //     8     notify: (consumer) relays each landed stage to the chain warps
-//                   through hardware named barriers.
+//                   through hardware named barriers and returns the ring slot
+//                   to its producer.
 //     9     idle.
 //
 // Per chunk of C = 16 tokens, with Gamma_i the inclusive cumulative log-decay
@@ -41,9 +45,11 @@
 // All factors stay within [e^-80, e^80] because -5 <= g <= 0 and a chunk has 16
 // tokens: the bound that lets FlashKDA keep 16-token causal blocks on dense
 // tensor-core products (page "Kimi K3 开源满月…", section "KDA 内核到底难在哪":
-// 16-token chunks, lower_bound = -5). Every product on the chain takes the
-// register-resident state (or X, Vnew) as its B operand and a shared-memory
-// tile (Kd, Qd, Kend^T, Tb, Aqk) as its A operand.
+// 16-token chunks, lower_bound = -5). The chain works on transposes,
+//   X^T = V^T + S^T Kd^T,  Vnew^T = X^T Tb^T,  S^T <- S^T Diag(gamma) + Vnew^T Kend,
+//   O^T = scale (S^T Qd^T + Vnew^T Aqk^T),
+// so that every product takes the register-resident state (or X, Vnew) as its
+// A operand and a shared-memory tile as its B operand.
 //
 // Tensor cores: mma.sync m16n8k16 (bf16 in, fp32 accumulate). On this part a
 // dependent m16n8k16 completes in ~21 cycles while a tcgen05.mma of the shapes
@@ -151,7 +157,7 @@ struct __align__(128) Shared {
   unsigned long long prod_free[PSTAGE], gate_done[PSTAGE], solved[PSTAGE];
   unsigned long long c_full[CSTAGE], c_empty[CSTAGE];
   unsigned long long ready[RING];      // arrived (remotely) by the slot's producer
-  unsigned long long slot_free[RING];  // arrived (remotely) by the four consumers
+  unsigned long long slot_free[RING];  // arrived (remotely) by every CTA of the cluster
 };
 static_assert(sizeof(Ops) % 128 == 0 && sizeof(RawStage) % 128 == 0, "stage alignment");
 static_assert(sizeof(ProdStage) % 128 == 0 && sizeof(ChainStage<16>) % 128 == 0 && sizeof(ChainStage<32>) % 128 == 0,
@@ -258,12 +264,6 @@ __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
                : "r"(smem_u32(p)));
 }
 
-__device__ __forceinline__ void ldsm_x2(uint32_t (&r)[2], const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
-               : "=r"(r[0]), "=r"(r[1])
-               : "r"(smem_u32(p)));
-}
-
 __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -326,15 +326,10 @@ __device__ __forceinline__ void mbar_wait_cl(unsigned long long* m, uint32_t par
   }
 }
 
-// Arrive on the mbarrier at the same shared-memory offset in CTA `rank` of the cluster.
-__device__ __forceinline__ void mbar_arrive_remote(unsigned long long* m, uint32_t rank) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(m)), "r"(rank));
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
-}
-
-// Relaxed remote arrive: a pure "done reading" signal that publishes no data,
-// so it need not wait for this thread's outstanding global stores.
+// Arrive on the mbarrier at the same shared-memory offset in CTA `rank` of the
+// cluster. Relaxed: a "done" signal whose data (if any) was already made
+// complete and visible by its sender, so it need not wait for this thread's
+// outstanding global stores.
 __device__ __forceinline__ void mbar_arrive_remote_relaxed(unsigned long long* m, uint32_t rank) {
   uint32_t remote;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(m)), "r"(rank));
@@ -375,15 +370,6 @@ __device__ __forceinline__ void bulk_g2s(void* sdst, const void* gsrc, uint32_t 
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(sdst)),
       "l"(gsrc), "r"(bytes), "r"(smem_u32(m))
       : "memory");
-}
-
-// A fragment (16 rows x 16 k) from two accumulator tiles (16 rows x 8 cols each)
-// holding k columns [0, 8) and [8, 16).
-__device__ __forceinline__ void acc_to_afrag(uint32_t (&a)[4], const float (&lo)[4], const float (&hi)[4]) {
-  a[0] = pack_bf16(lo[0], lo[1]);
-  a[1] = pack_bf16(lo[2], lo[3]);
-  a[2] = pack_bf16(hi[0], hi[1]);
-  a[3] = pack_bf16(hi[2], hi[3]);
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -497,7 +483,7 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
       // Every product on the chain takes the register-resident operand as its
       // A fragment, so nothing on the chain needs a transpose:
       //   X^T = V^T + S^T Kd^T,  Vnew^T = X^T Tb^T,  S^T <- S^T Diag(gamma) + Vnew^T Kend,
-      //   O^T = S^T Qd^T + Vnew^T Aqk^T.
+      //   O^T = S^T Qd^T + Vnew^T Aqk^T  (times scale at the store).
       // The products are ordered for one in-order warp on one tensor pipe: the
       // state's own chain (X -> Vnew -> S) goes first at every step and the O
       // products, which nothing waits for, fill the pipe while a chain result
@@ -780,7 +766,7 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
         const uint32_t pph = static_cast<uint32_t>(j / PSTAGE) & 1u;
         const int slot = n % RING;
         mbar_wait(&sh.solved[ps], pph);
-        // the slot's previous chunk (n - RING) has been copied by all four CTAs
+        // the slot's previous chunk (n - RING) has been copied by every CTA of the cluster
         mbar_wait_cl(&sh.slot_free[slot], (static_cast<uint32_t>(n / RING) & 1u) ^ 1u);
         fence_proxy_async_shared();
         bulk_s2g(ring + static_cast<size_t>(slot) * kSlotBytes, &sh.prod[ps].ops, kSlotBytes);
