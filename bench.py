@@ -261,6 +261,28 @@ def reduce_over_ranks(ms: float, e2e_ms: float, units: float, device=None):
 
 
 # ---------------------------------------------------------------- reference
+def input_bytes(inp) -> int:
+    """Bytes of the inputs the kernel reads (q, k, v, g, beta, cu_seqlens and
+    the initial state when there is one)."""
+    arrs = [inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens]
+    if inp.initial_state is not None:
+        arrs.append(inp.initial_state)
+    return int(sum(a.nbytes for a in arrs))
+
+
+def workload_config(wl, inp, ws: int) -> dict:
+    """The `config` object of both arms' JSON lines for this workload."""
+    in_bytes = input_bytes(inp)
+    T, H, N = inp.total_tokens, inp.num_heads, inp.num_seqs
+    return {"workload": wl.name, "seq_lens": list(wl.seqlens) if len(wl.seqlens) <= 16 else None,
+            "total_tokens": T, "num_heads": H, "head_dim": D, "num_seqs": N,
+            "initial_state": "random" if inp.initial_state is not None else "zero", "final_state": True,
+            "global_batch": N * ws, "seq_len": T,
+            "l2": "flushed between launches" if in_bytes < 2 * L2_BYTES
+                  else f"inputs larger than L2 ({in_bytes / 2**20:.0f} MiB)",
+            "parallelism": f"dp{ws} (independent batch per GPU)", "seed": wl.seed}
+
+
 def run_reference(args):
     ws, rank, _ = dist_env()
     if rank != 0:
@@ -282,8 +304,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "seq_lens": list(wl.seqlens), "num_heads": wl.num_heads, "head_dim": D,
-                   "sample_tokens": ntok},
+        "config": workload_config(wl, inp, ws),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle",
                          "sample": f"fp64 token scan on the first {ntok} of {inp.total_tokens} tokens, "
                                    f"all {inp.num_heads} heads, per step"},
@@ -331,6 +352,7 @@ def run_kda(args):
     h_fin = torch.empty((N, H, D, D), dtype=torch.float32).pin_memory()
 
     in_bytes = sum(t.numel() * t.element_size() for t in d.values())
+    assert in_bytes == input_bytes(inp)
     flush = None
     if in_bytes < 2 * L2_BYTES:
         flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
@@ -418,13 +440,7 @@ def run_kda(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": wl.name, "seq_lens": list(wl.seqlens) if len(wl.seqlens) <= 16 else None,
-                       "total_tokens": T, "num_heads": H, "head_dim": D, "num_seqs": N,
-                       "initial_state": "random" if with_init else "zero", "final_state": True,
-                       "global_batch": N * ws, "seq_len": T,
-                       "l2": "flushed between launches" if flush is not None
-                             else f"inputs larger than L2 ({in_bytes / 2**20:.0f} MiB)",
-                       "parallelism": f"dp{ws} (independent batch per GPU)", "seed": wl.seed},
+            "config": workload_config(wl, inp, ws),
             "roofline": roof,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms},
