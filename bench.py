@@ -41,7 +41,8 @@ STATE_BYTES = D * D * 4                                    # one (sequence, head
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-KERNEL_SOURCES = [os.path.join(ROOT, "kimi_delta_attention_26_b200", "csrc", "kda_fwd.cu")]
+KERNEL_SOURCES = [os.path.join(ROOT, "kimi_delta_attention_26_b200", "csrc", f)
+                  for f in ("kda_prims.cuh", "kda_fwd16.cuh", "kda_fwd64.cuh", "kda_api.cu")]
 
 
 def log(*a):
@@ -330,6 +331,7 @@ def run_kda(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     import kimi_delta_attention_26_b200 as kda
 
+    kda.set_path(args.path)
     wl = kda_inputs.workload(args.config)
     inp = wl.make(seed=wl.seed + rank)  # an independent batch per rank
     with_init = inp.initial_state is not None
@@ -466,6 +468,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", type=int, default=0, choices=[0, 16, 64],
+                    help="kernel: 0 = library default (64-token chunks on tcgen05), 16 = 16-token chunks on mma.sync")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         log("note: raising --warmup to 3 (minimum)")

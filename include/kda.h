@@ -20,11 +20,13 @@
  * section "تكامل مباشر مع flash-linear-attention").
  *
  * Conventions shared by every entry point
- *   - All tensor pointers are DEVICE pointers on the current CUDA device.
+ *   - Tensors are described by kda_tensor_t: a DEVICE pointer on the current
+ *     CUDA device, a dtype, a shape and element strides (any order of the
+ *     outer dimensions; see kda_fwd for what each tensor must satisfy).
  *   - The caller owns all inputs and outputs. kda_fwd takes a scratch ring
- *     (num_seqs * H * 16 slots of 15104 bytes) from a library-private
- *     stream-ordered memory pool and returns it in stream order after the
- *     kernel; the pool keeps its memory for later calls.
+ *     (num_seqs * H slots of KDA_RING_BYTES_PER_PAIR bytes) from a
+ *     library-private stream-ordered memory pool and returns it in stream
+ *     order after the kernel; the pool keeps its memory for later calls.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and the call returns without synchronising.
  *   - Argument errors are reported synchronously through the return code and
@@ -32,6 +34,9 @@
  *   - Results are deterministic: no atomics, no split reductions, and each
  *     (sequence, head) is computed independently of the rest of the batch, so
  *     a sequence gives bit-identical results alone or inside any batch.
+ *   - First-call setup per device (capability check, kernel attributes, the
+ *     memory pool) is guarded by a lock: concurrent first calls from several
+ *     host threads are safe.
  */
 #ifndef KDA_H_
 #define KDA_H_
@@ -43,24 +48,45 @@ extern "C" {
 #endif
 
 #define KDA_HEAD_DIM 128
-#define KDA_ABI_VERSION 2
+#define KDA_ABI_VERSION 3
 
 typedef enum kda_status {
   KDA_OK = 0,
-  KDA_ERR_NULL = 1,        /* a required pointer is NULL */
-  KDA_ERR_SHAPE = 2,       /* invalid sizes (negative T, H < 1, num_seqs < 1,
-                              cu_seqlens NULL with num_seqs != 1, int overflow) */
-  KDA_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned */
+  KDA_ERR_NULL = 1,        /* a required tensor or pointer is NULL */
+  KDA_ERR_SHAPE = 2,       /* wrong ndim or shape, or inconsistent sizes
+                              (T, H, num_seqs), or an int overflow */
+  KDA_ERR_ALIGN = 3,       /* a data pointer is not 16-byte aligned */
   KDA_ERR_UNSUPPORTED = 4, /* the current device is not sm_100 (B200) */
   KDA_ERR_CUDA = 5,        /* a CUDA runtime call or the launch failed */
-  KDA_ERR_CAPACITY = 6     /* kda_fwd_noalloc: num_seqs * num_heads exceeds
+  KDA_ERR_CAPACITY = 6,    /* kda_fwd_noalloc: num_seqs * num_heads exceeds
                               KDA_NOALLOC_MAX_PAIRS */
+  KDA_ERR_DTYPE = 7,       /* a tensor has the wrong dtype */
+  KDA_ERR_STRIDE = 8,      /* a tensor's strides are not supported (see kda_fwd) */
+  KDA_ERR_DEVICE = 9       /* kda_device_status: the device recorded a fault */
 } kda_status_t;
+
+typedef enum kda_dtype { KDA_BF16 = 1, KDA_F32 = 2, KDA_I32 = 3 } kda_dtype_t;
+
+/*
+ * A strided tensor in device memory. shape[0..ndim) and stride[0..ndim) are
+ * in elements; entries at or beyond ndim are ignored. The caller keeps
+ * ownership of `data`.
+ */
+typedef struct kda_tensor {
+  void* data;
+  int32_t ndim;
+  kda_dtype_t dtype;
+  int64_t shape[4];
+  int64_t stride[4];
+} kda_tensor_t;
+
+/* Scratch bytes per (sequence, head) that kda_fwd takes from its pool. */
+#define KDA_RING_BYTES_PER_PAIR (6 * 66560)
 
 /*
  * kda_fwd -- chunked KDA forward (prefill) for a packed batch.
  *
- * Layouts (row-major, contiguous, T = total_tokens, H = num_heads, N = num_seqs):
+ * Tensors (T = total tokens, H = heads, N = num_seqs):
  *   q, k, v, out   bf16  [T, H, 128]
  *   g              fp32  [T, H, 128]   natural-log decay per key channel.
  *                  Precondition: -5 <= g <= 0 (the gate lower bound of
@@ -68,27 +94,39 @@ typedef enum kda_status {
  *                  "KDA 内核到底难在哪"); outside it results are undefined
  *                  (may be inf/NaN), never an out-of-bounds access.
  *   beta           fp32  [T, H]
- *   initial_state  fp32  [N, H, 128 (key), 128 (value)] or NULL (zero state)
- *   final_state    fp32  [N, H, 128, 128] or NULL (not written); may alias
- *                  initial_state (each (sequence, head) reads its slice before
- *                  writing it).
+ *   initial_state  fp32  [N, H, 128 (key), 128 (value)], contiguous, or NULL
+ *                  (zero state)
+ *   final_state    fp32  [N, H, 128, 128], contiguous, or NULL (not
+ *                  written); may alias initial_state (each (sequence, head)
+ *                  reads its slice before writing it).
  *   cu_seqlens     int32 [N + 1] on the device, cu[0] = 0, non-decreasing,
- *                  cu[N] = T; or NULL, meaning one sequence of T tokens
- *                  (then num_seqs must be 1). Its contents are not checked on
- *                  the host (that would need a synchronisation); the kernel
- *                  clamps every boundary into [0, T], so bad contents give
- *                  wrong results, never an out-of-bounds access.
+ *                  cu[N] = T; or NULL, meaning one sequence of T tokens (then
+ *                  num_seqs must be 1). Its contents are not read on the host
+ *                  (that would need a synchronisation): the kernel clamps every
+ *                  boundary into [0, T], so bad contents give wrong results but
+ *                  never an out-of-bounds access, and it records them in the
+ *                  device status word (kda_device_status).
  *   scale          the output scale (usually 1/sqrt(128)).
- * Alignment: every tensor pointer must be 16-byte aligned.
+ * Strides: the last dimension of q, k, v, g and out must have stride 1; their
+ *   token and head strides must be positive multiples of 16 bytes (8 bf16 or
+ *   4 fp32 elements), so that views of a fused projection output (for
+ *   example q, k, v as slices of one [T, H, 3 * 128] tensor) work without a
+ *   copy. out must not overlap itself (token and head strides nest). beta may
+ *   have any positive strides. States must be contiguous.
+ * Alignment: every data pointer must be 16-byte aligned.
  * Zero-length sequences are allowed: their final state equals their initial
- * state (or zeros). T = 0 is allowed; then q, k, v, g, beta and out may be
- * NULL (they are never read or written).
+ * state (or zeros). T = 0 is allowed; then the token tensors' data pointers
+ * may be NULL (they are never read or written).
+ * Errors: KDA_ERR_NULL (a required descriptor or pointer missing),
+ * KDA_ERR_DTYPE, KDA_ERR_SHAPE, KDA_ERR_STRIDE, KDA_ERR_ALIGN,
+ * KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA; nothing is enqueued on any error.
  * Returns KDA_OK once the work is enqueued.
  */
-kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                     float scale, const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
-                     int32_t num_heads, const float* initial_state, void* out, float* final_state,
-                     void* stream);
+kda_status_t kda_fwd(const kda_tensor_t* q, const kda_tensor_t* k, const kda_tensor_t* v,
+                     const kda_tensor_t* g, const kda_tensor_t* beta, float scale,
+                     const int32_t* cu_seqlens, int32_t num_seqs,
+                     const kda_tensor_t* initial_state, const kda_tensor_t* out,
+                     const kda_tensor_t* final_state, void* stream);
 
 /*
  * kda_fwd_noalloc -- kda_fwd without any device-memory allocation.
@@ -103,13 +141,15 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* g
  * Arguments, layouts, results and errors are those of kda_fwd, except:
  *   - The scratch ring lives in a fixed-size array in device memory that the
  *     library declares at file scope: every GPU that loads the library holds
- *     it (KDA_NOALLOC_MAX_PAIRS * 16 slots * 15232 bytes = 7.8 MB) until the
+ *     it (KDA_NOALLOC_MAX_PAIRS * KDA_RING_BYTES_PER_PAIR = 12.8 MB) until the
  *     process exits.
  *   - num_seqs * num_heads must not exceed KDA_NOALLOC_MAX_PAIRS; larger
  *     problems return KDA_ERR_CAPACITY and nothing is launched.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *   - The first call on a device loads the library's device code there (CUDA
+ *     loads modules lazily), which allocates the array, and then looks up its
+ *     device address (cudaGetSymbolAddress) with that device current. Make that
+ *     first call before reserving the device's memory for an arena, and before
+ *     any stream capture.
  *   - All calls on a device share the one array and it keeps the last call's
  *     contents (the kernel overwrites every slot before reading it, so nothing
  *     needs clearing). Calls whose kernels overlap on the GPU -- on different
@@ -118,23 +158,38 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* g
  *   - It calls no cudaMalloc, cudaFree or other allocating routine.
  */
 #define KDA_NOALLOC_MAX_PAIRS 32
-kda_status_t kda_fwd_noalloc(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                             float scale, const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
-                             int32_t num_heads, const float* initial_state, void* out, float* final_state,
-                             void* stream);
+kda_status_t kda_fwd_noalloc(const kda_tensor_t* q, const kda_tensor_t* k, const kda_tensor_t* v,
+                             const kda_tensor_t* g, const kda_tensor_t* beta, float scale,
+                             const int32_t* cu_seqlens, int32_t num_seqs,
+                             const kda_tensor_t* initial_state, const kda_tensor_t* out,
+                             const kda_tensor_t* final_state, void* stream);
 
 /*
- * kda_set_slice_columns -- value columns per CTA for later calls (tuning).
+ * kda_set_path -- which kernel later calls use (tuning and testing).
  *
- * Each (sequence, head) runs as one thread-block cluster whose CTAs split the
- * 128 value columns. columns = 32 uses 4 CTAs per (sequence, head); 16 uses
- * 8, which doubles the SMs working on the same serial chains when there are
- * few sequences and heads. columns = 0 (the default) chooses per call: 16
- * when num_seqs * num_heads * 4 is at most half the device's SM count, else
- * 32. Each column's arithmetic is the same either way, so the results are
- * bitwise identical. Process-wide; affects kda_fwd and
- * kda_fwd_noalloc. Returns KDA_ERR_SHAPE for any other value (the setting is
- * then unchanged).
+ *   64: 64-token chunks on tcgen05 tensor cores, one 4-CTA cluster per
+ *       (sequence, head): the whole state in tensor memory on one SM, three
+ *       SMs preparing the chunks' operands.
+ *   16: 16-token chunks on mma.sync, the value columns split over a cluster
+ *       of 4 (or 8) CTAs with the state in registers.
+ *    0: the default: the path that measured faster on B200 for the workloads
+ *       tried so far, currently 16.
+ * The two paths round differently (their results agree within the library's
+ * accuracy bounds, not bitwise). Process-wide. Returns KDA_ERR_SHAPE for any
+ * other value (the setting is then unchanged).
+ */
+kda_status_t kda_set_path(int32_t path);
+
+/*
+ * kda_set_slice_columns -- value columns per CTA of the 16-token path.
+ *
+ * columns = 32 uses 4 CTAs per (sequence, head); 16 uses 8, which doubles the
+ * SMs working on the same serial chains when there are few sequences and
+ * heads. columns = 0 (the default) chooses per call: 16 when
+ * num_seqs * num_heads * 4 is at most half the device's SM count, else 32.
+ * Each column's arithmetic is the same either way, so the results are bitwise
+ * identical. Process-wide. Returns KDA_ERR_SHAPE for any other value (the
+ * setting is then unchanged).
  */
 kda_status_t kda_set_slice_columns(int32_t columns);
 
@@ -146,14 +201,28 @@ const char* kda_status_string(kda_status_t status);
 const char* kda_last_cuda_error(void);
 
 /*
- * kda_wait_timeouts -- health counter of the current device.
+ * kda_device_status -- the current device's status word.
  *
- * Every wait inside the kernel (on a pipeline stage, on a peer CTA of the
- * cluster) is bounded; a wait that runs out of budget increments a device
- * counter and lets the kernel finish instead of hanging (its results are then
- * undefined). This reads the counter into *count (synchronising with the
- * device) and resets it to zero when `reset` is non-zero. A healthy run leaves
- * it at 0.
+ * Bits (OR-ed over every kernel since the last reset):
+ *   KDA_DEVICE_BAD_CU_SEQLENS  some cu_seqlens was not a non-decreasing
+ *                              partition of [0, T) (those results are wrong)
+ *   KDA_DEVICE_WAIT_TIMEOUT    a bounded in-kernel wait ran out of budget (the
+ *                              kernel stopped early; its results are undefined)
+ * Writes the bits to *flags (synchronising with the device), clears them when
+ * `reset` is non-zero, and returns KDA_ERR_DEVICE if any bit is set, else
+ * KDA_OK (or KDA_ERR_NULL / KDA_ERR_CUDA).
+ */
+#define KDA_DEVICE_BAD_CU_SEQLENS 1u
+#define KDA_DEVICE_WAIT_TIMEOUT 2u
+kda_status_t kda_device_status(uint32_t* flags, int32_t reset);
+
+/*
+ * kda_wait_timeouts -- how many bounded in-kernel waits ran out of budget on
+ * the current device since the last reset (0 for a healthy run). Every wait
+ * inside the kernels (on a pipeline stage, on a peer CTA of the cluster) is
+ * bounded; a wait that runs out increments this counter and makes its CTA
+ * stop issuing work, so the GPU is never left hanging. Synchronises with the
+ * device; resets the counter when `reset` is non-zero.
  */
 kda_status_t kda_wait_timeouts(uint32_t* count, int32_t reset);
 

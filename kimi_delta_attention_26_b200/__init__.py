@@ -14,7 +14,8 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["kda_fwd", "library_path", "wait_timeouts", "set_slice_columns", "KDAError", "HEAD_DIM"]
+__all__ = ["kda_fwd", "library_path", "wait_timeouts", "device_status", "set_slice_columns", "set_path",
+           "describe", "KDAError", "HEAD_DIM"]
 
 HEAD_DIM = 128
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -26,10 +27,40 @@ if not os.path.exists(_LIB_PATH):
         "(python kimi_delta_attention_26_b200/build.py or __graft_entry__.build())")
 
 _lib = ctypes.CDLL(_LIB_PATH)
+
+KDA_BF16, KDA_F32, KDA_I32 = 1, 2, 3
+_DTYPE = {torch.bfloat16: KDA_BF16, torch.float32: KDA_F32, torch.int32: KDA_I32}
+
+
+class TensorDesc(ctypes.Structure):
+    """``kda_tensor_t``: data pointer, ndim, dtype, shape[4], stride[4] (elements)."""
+    _fields_ = [("data", ctypes.c_void_p), ("ndim", ctypes.c_int32), ("dtype", ctypes.c_int),
+                ("shape", ctypes.c_int64 * 4), ("stride", ctypes.c_int64 * 4)]
+
+
+def describe(t: Optional[torch.Tensor]):
+    """A ``kda_tensor_t`` for a torch tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if t.dim() > 4:
+        raise ValueError("at most 4 dimensions")
+    d = TensorDesc()
+    d.data = t.data_ptr() if t.numel() else None
+    d.ndim = t.dim()
+    d.dtype = _DTYPE.get(t.dtype, 0)
+    for i, (n, st) in enumerate(zip(t.shape, t.stride())):
+        d.shape[i] = n
+        d.stride[i] = st
+    return ctypes.byref(d), d  # keep d alive with the reference
+
+
 _P = ctypes.c_void_p
-_lib.kda_fwd.argtypes = [_P, _P, _P, _P, _P, ctypes.c_float, _P, ctypes.c_int32, ctypes.c_int64,
-                         ctypes.c_int32, _P, _P, _P, _P]
+_T = ctypes.POINTER(TensorDesc)
+_FWD_ARGS = [_T, _T, _T, _T, _T, ctypes.c_float, _P, ctypes.c_int32, _T, _T, _T, _P]
+_lib.kda_fwd.argtypes = _FWD_ARGS
 _lib.kda_fwd.restype = ctypes.c_int
+_lib.kda_fwd_noalloc.argtypes = _FWD_ARGS
+_lib.kda_fwd_noalloc.restype = ctypes.c_int
 _lib.kda_status_string.argtypes = [ctypes.c_int]
 _lib.kda_status_string.restype = ctypes.c_char_p
 _lib.kda_last_cuda_error.argtypes = []
@@ -38,8 +69,12 @@ _lib.kda_abi_version.argtypes = []
 _lib.kda_abi_version.restype = ctypes.c_int32
 _lib.kda_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32]
 _lib.kda_wait_timeouts.restype = ctypes.c_int
+_lib.kda_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32]
+_lib.kda_device_status.restype = ctypes.c_int
 _lib.kda_set_slice_columns.argtypes = [ctypes.c_int32]
 _lib.kda_set_slice_columns.restype = ctypes.c_int
+_lib.kda_set_path.argtypes = [ctypes.c_int32]
+_lib.kda_set_path.restype = ctypes.c_int
 
 
 class KDAError(RuntimeError):
@@ -65,14 +100,33 @@ def wait_timeouts(reset: bool = True) -> int:
 
 
 def set_slice_columns(columns: int) -> None:
-    """Value columns per CTA for later calls: 0 chooses per call (default), 16
-    or 32 forces that kernel variant. Process-wide."""
+    """Value columns per CTA of the 16-token path for later calls: 0 chooses per
+    call (default), 16 or 32 forces that variant. Process-wide."""
     rc = _lib.kda_set_slice_columns(int(columns))
     if rc != 0:
         raise KDAError(rc)
 
 
-def _check(t: torch.Tensor, name: str, dtype: torch.dtype, shape: Tuple[int, ...], device) -> None:
+def set_path(path: int) -> None:
+    """Kernel for later calls: 16 (16-token chunks on mma.sync), 64 (64-token
+    chunks on tcgen05) or 0 (the library's default). Process-wide."""
+    rc = _lib.kda_set_path(int(path))
+    if rc != 0:
+        raise KDAError(rc)
+
+
+def device_status(reset: bool = True) -> int:
+    """The device status word (bit 0: a bad cu_seqlens was seen, bit 1: a
+    bounded in-kernel wait ran out); synchronises with the device."""
+    n = ctypes.c_uint32(0)
+    rc = _lib.kda_device_status(ctypes.byref(n), 1 if reset else 0)
+    if rc not in (0, 9):
+        raise KDAError(rc)
+    return int(n.value)
+
+
+def _check(t: torch.Tensor, name: str, dtype: torch.dtype, shape: Tuple[int, ...], device,
+           contiguous: bool = False) -> None:
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if t.dtype != dtype:
@@ -81,7 +135,7 @@ def _check(t: torch.Tensor, name: str, dtype: torch.dtype, shape: Tuple[int, ...
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
     if t.device != device:
         raise ValueError(f"{name} is on {t.device}, expected {device}")
-    if not t.is_contiguous():
+    if contiguous and not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
 
 
@@ -93,7 +147,7 @@ def kda_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, 
             scale: Optional[float] = None, cu_seqlens: Optional[torch.Tensor] = None,
             initial_state: Optional[torch.Tensor] = None, output_final_state: bool = True,
             out: Optional[torch.Tensor] = None, final_state: Optional[torch.Tensor] = None,
-            stream: Optional[torch.cuda.Stream] = None):
+            stream: Optional[torch.cuda.Stream] = None, noalloc: bool = False):
     """Chunked KDA forward on packed sequences (see ``include/kda.h``).
 
     q, k, v: bf16 [T, H, 128]; g: fp32 [T, H, 128] (log decay, in [-5, 0]);
@@ -116,24 +170,26 @@ def kda_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, 
     _check(g, "g", torch.float32, (T, H, d), dev)
     _check(beta, "beta", torch.float32, (T, H), dev)
     if cu_seqlens is not None:
-        _check(cu_seqlens, "cu_seqlens", torch.int32, (N + 1,), dev)
+        _check(cu_seqlens, "cu_seqlens", torch.int32, (N + 1,), dev, contiguous=True)
     if initial_state is not None:
-        _check(initial_state, "initial_state", torch.float32, (N, H, d, d), dev)
+        _check(initial_state, "initial_state", torch.float32, (N, H, d, d), dev, contiguous=True)
     if out is None:
         out = torch.empty((T, H, d), dtype=torch.bfloat16, device=dev)
     _check(out, "out", torch.bfloat16, (T, H, d), dev)
     if final_state is None and output_final_state:
         final_state = torch.empty((N, H, d, d), dtype=torch.float32, device=dev)
     if final_state is not None:
-        _check(final_state, "final_state", torch.float32, (N, H, d, d), dev)
+        _check(final_state, "final_state", torch.float32, (N, H, d, d), dev, contiguous=True)
     if scale is None:
         scale = d ** -0.5
     if stream is None:
         stream = torch.cuda.current_stream(dev)
+    descs = [describe(t) for t in (q, k, v, g, beta, initial_state, out, final_state)]
+    ref = [None if d is None else d[0] for d in descs]
+    fn = _lib.kda_fwd_noalloc if noalloc else _lib.kda_fwd
     with torch.cuda.device(dev):
-        rc = _lib.kda_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), ctypes.c_float(scale),
-                          _ptr(cu_seqlens), N, T, H, _ptr(initial_state), _ptr(out), _ptr(final_state),
-                          ctypes.c_void_p(stream.cuda_stream))
+        rc = fn(ref[0], ref[1], ref[2], ref[3], ref[4], ctypes.c_float(scale), _ptr(cu_seqlens), N,
+                ref[5], ref[6], ref[7], ctypes.c_void_p(stream.cuda_stream))
     if rc != 0:
         raise KDAError(rc)
     return out, final_state

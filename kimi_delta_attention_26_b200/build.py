@@ -8,8 +8,9 @@ import sys
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
-SOURCES = [os.path.join(PKG, "csrc", "kda_fwd.cu")]
-HEADERS = [os.path.join(ROOT, "include", "kda.h"), os.path.abspath(__file__)]
+SOURCES = [os.path.join(PKG, "csrc", "kda_api.cu")]
+HEADERS = [os.path.join(ROOT, "include", "kda.h"), os.path.abspath(__file__)] + [
+    os.path.join(PKG, "csrc", f) for f in ("kda_prims.cuh", "kda_fwd16.cuh", "kda_fwd64.cuh")]
 LIB = os.path.join(PKG, "libkda.so")
 
 NVCC_FLAGS = [

@@ -1,0 +1,479 @@
+// kda_api.cu -- the C ABI of libkda.so (declared in include/kda.h): argument
+// checks on kda_tensor_t descriptors, per-device setup, scratch rings, tensor
+// maps, and the launch of one of the two prefill kernels:
+//   kda_fwd16.cuh  16-token chunks on mma.sync (the default path)
+//   kda_fwd64.cuh  64-token chunks on tcgen05
+// This file is the library's only translation unit.
+
+#include "kda_prims.cuh"
+#include "kda_fwd16.cuh"
+#include "kda_fwd64.cuh"
+
+#include <atomic>
+#include <cstdio>
+#include <mutex>
+
+namespace {
+
+thread_local char g_last_cuda_error[256] = "";
+
+kda_status_t cuda_fail(cudaError_t e) {
+  std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(e),
+                cudaGetErrorString(e));
+  return KDA_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------ argument checks
+// A token tensor [T, H, inner] (inner = 128) or [T, H] (inner = 0) after
+// validation: base pointer and element strides over tokens and heads.
+struct TokView {
+  void* data;
+  int64_t st, sh;
+};
+
+int elem_bytes(kda_dtype_t dt) { return dt == KDA_BF16 ? 2 : 4; }
+
+// T and H are taken from q; every other tensor must match them.
+kda_status_t view_tokens(const kda_tensor_t* t, kda_dtype_t dt, int64_t T, int64_t H, bool inner, bool is_out,
+                         TokView* res) {
+  if (!t) return KDA_ERR_NULL;
+  if (t->dtype != dt) return KDA_ERR_DTYPE;
+  if (t->ndim != (inner ? 3 : 2)) return KDA_ERR_SHAPE;
+  if (t->shape[0] != T || t->shape[1] != H || (inner && t->shape[2] != KDA_HEAD_DIM)) return KDA_ERR_SHAPE;
+  const int64_t st = t->stride[0], sh = t->stride[1];
+  if (st <= 0 || sh <= 0) return KDA_ERR_STRIDE;
+  if (inner) {
+    const int64_t unit = 16 / elem_bytes(dt);  // 16-byte multiples (tensor-map strides, vector stores)
+    if (t->stride[2] != 1 || st % unit != 0 || sh % unit != 0) return KDA_ERR_STRIDE;
+    if (st * elem_bytes(dt) >= (int64_t(1) << 40) || sh * elem_bytes(dt) >= (int64_t(1) << 40)) return KDA_ERR_STRIDE;
+    if (is_out) {
+      // rows of 128 elements must not overlap: one of the two outer strides nests the other
+      const bool nest_h = sh >= KDA_HEAD_DIM && (T <= 1 || st >= H * sh);
+      const bool nest_t = st >= KDA_HEAD_DIM && (H <= 1 || sh >= T * st);
+      if (!nest_h && !nest_t) return KDA_ERR_STRIDE;
+    }
+  }
+  if (T > 0) {
+    if (!t->data) return KDA_ERR_NULL;
+    if (!aligned16(t->data)) return KDA_ERR_ALIGN;
+  }
+  res->data = t->data;
+  res->st = st;
+  res->sh = sh;
+  return KDA_OK;
+}
+
+kda_status_t check_state(const kda_tensor_t* t, int64_t N, int64_t H) {
+  if (!t) return KDA_OK;
+  if (t->dtype != KDA_F32) return KDA_ERR_DTYPE;
+  if (t->ndim != 4 || t->shape[0] != N || t->shape[1] != H || t->shape[2] != KDA_HEAD_DIM ||
+      t->shape[3] != KDA_HEAD_DIM)
+    return KDA_ERR_SHAPE;
+  const int64_t d = KDA_HEAD_DIM;
+  if (t->stride[3] != 1 || t->stride[2] != d || (H > 1 && t->stride[1] != d * d) || (N > 1 && t->stride[0] != H * d * d))
+    return KDA_ERR_STRIDE;
+  if (!t->data) return KDA_ERR_NULL;
+  if (!aligned16(t->data)) return KDA_ERR_ALIGN;
+  return KDA_OK;
+}
+
+struct Problem {
+  TokView q, k, v, g, beta, out;
+  const float* init;
+  float* fin;
+  const int32_t* cu;
+  int32_t num_seqs, num_heads;
+  int64_t T;
+  float scale;
+};
+
+kda_status_t check_args(const kda_tensor_t* q, const kda_tensor_t* k, const kda_tensor_t* v, const kda_tensor_t* g,
+                        const kda_tensor_t* beta, float scale, const int32_t* cu_seqlens, int32_t num_seqs,
+                        const kda_tensor_t* initial_state, const kda_tensor_t* out, const kda_tensor_t* final_state,
+                        Problem* P) {
+  if (!q || !k || !v || !g || !beta || !out) return KDA_ERR_NULL;
+  if (q->ndim != 3) return KDA_ERR_SHAPE;
+  const int64_t T = q->shape[0], H = q->shape[1];
+  if (T < 0 || H < 1 || num_seqs < 1) return KDA_ERR_SHAPE;
+  if (!cu_seqlens && num_seqs != 1) return KDA_ERR_SHAPE;
+  if (H > 65535 || num_seqs > 65535) return KDA_ERR_SHAPE;            // grid.y / grid.z limits
+  if (T > int64_t(INT32_MAX) - 256) return KDA_ERR_SHAPE;             // tensor-map coordinates are 32-bit
+  if (T > (int64_t(1) << 40) / (H * KDA_HEAD_DIM)) return KDA_ERR_SHAPE;
+  kda_status_t st;
+  if ((st = view_tokens(q, KDA_BF16, T, H, true, false, &P->q)) != KDA_OK) return st;
+  if ((st = view_tokens(k, KDA_BF16, T, H, true, false, &P->k)) != KDA_OK) return st;
+  if ((st = view_tokens(v, KDA_BF16, T, H, true, false, &P->v)) != KDA_OK) return st;
+  if ((st = view_tokens(g, KDA_F32, T, H, true, false, &P->g)) != KDA_OK) return st;
+  if ((st = view_tokens(beta, KDA_F32, T, H, false, false, &P->beta)) != KDA_OK) return st;
+  if ((st = view_tokens(out, KDA_BF16, T, H, true, true, &P->out)) != KDA_OK) return st;
+  if ((st = check_state(initial_state, num_seqs, H)) != KDA_OK) return st;
+  if ((st = check_state(final_state, num_seqs, H)) != KDA_OK) return st;
+  if (cu_seqlens && !aligned16(cu_seqlens)) return KDA_ERR_ALIGN;
+  P->init = initial_state ? static_cast<const float*>(initial_state->data) : nullptr;
+  P->fin = final_state ? static_cast<float*>(final_state->data) : nullptr;
+  P->cu = cu_seqlens;
+  P->num_seqs = num_seqs;
+  P->num_heads = static_cast<int32_t>(H);
+  P->T = T;
+  P->scale = scale;
+  return KDA_OK;
+}
+
+// ------------------------------------------------------------- tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+kda_status_t load_encoder() {
+  if (g_encode) return KDA_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult qr = cudaDriverEntryPointSymbolNotFound;
+  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (qr != cudaDriverEntryPointSuccess || !fn) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled not available");
+    return KDA_ERR_CUDA;
+  }
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return KDA_OK;
+}
+
+// [T, H, 128] view with element strides (st, sh); box {box_inner, 1, box_tok}
+// starting at column 0 / box_inner.
+kda_status_t encode_3d(CUtensorMap* map, const TokView& t, CUtensorMapDataType dt, int eb, int64_t T, int H,
+                       int box_inner, int box_tok, CUtensorMapSwizzle swz) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kda::D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(t.sh) * eb, static_cast<cuuint64_t>(t.st) * eb};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), 1u, static_cast<cuuint32_t>(box_tok)};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = g_encode(map, dt, 3, t.data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed (%d)",
+                  static_cast<int>(r));
+    return KDA_ERR_CUDA;
+  }
+  return KDA_OK;
+}
+
+// ------------------------------------------------------------ device setup
+constexpr int kMaxDevices = 64;
+std::mutex g_setup_mutex;                      // guards first-call setup of every device
+std::atomic<int> g_device_ready[kMaxDevices];  // 0 unknown, 1 ready, -1 unsupported
+int g_num_sms[kMaxDevices];
+// Library-private stream-ordered pool for the scratch rings. It keeps freed
+// memory (release threshold = max), so steady-state calls never map memory
+// and the process's default pool is left untouched.
+std::atomic<cudaMemPool_t> g_pool[kMaxDevices];
+std::atomic<void*> g_noalloc_ring_addr[kMaxDevices];
+std::atomic<int> g_slice_columns{0};  // 16-token path: 0 chooses per call, 16 or 32 forces
+std::atomic<int> g_path{0};           // 0 (the default path), 16 or 64
+
+template <int NS>
+cudaError_t set_smem16() {
+  return cudaFuncSetAttribute(kda::kda_fwd_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(sizeof(kda::Shared<NS>)));
+}
+
+// Capability check and kernel attributes for `dev` (current), once.
+kda_status_t check_device(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return KDA_ERR_UNSUPPORTED;
+  const int state = g_device_ready[dev].load(std::memory_order_acquire);
+  if (state == 1) return KDA_OK;
+  if (state == -1) return KDA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  if (g_device_ready[dev].load() == 1) return KDA_OK;
+  int major = 0, minor = 0, sms = 0;
+  cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (major != 10 || minor != 0) {
+    g_device_ready[dev].store(-1);
+    return KDA_ERR_UNSUPPORTED;
+  }
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if ((e = set_smem16<32>()) != cudaSuccess) return cuda_fail(e);
+  if ((e = set_smem16<16>()) != cudaSuccess) return cuda_fail(e);
+  if ((e = cudaFuncSetAttribute(kda::c64::kda_fwd64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(kda::c64::SMEM_BYTES))) != cudaSuccess)
+    return cuda_fail(e);
+  g_num_sms[dev] = sms;
+  g_device_ready[dev].store(1, std::memory_order_release);
+  return KDA_OK;
+}
+
+// The pool of kda_fwd's scratch rings, created once per device.
+kda_status_t prepare_pool(int dev) {
+  if (g_pool[dev].load(std::memory_order_acquire)) return KDA_OK;
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  if (g_pool[dev].load()) return KDA_OK;
+  cudaMemPoolProps props;
+  std::memset(&props, 0, sizeof(props));
+  props.allocType = cudaMemAllocationTypePinned;
+  props.handleTypes = cudaMemHandleTypeNone;
+  props.location.type = cudaMemLocationTypeDevice;
+  props.location.id = dev;
+  cudaMemPool_t pool = nullptr;
+  cudaError_t e = cudaMemPoolCreate(&pool, &props);
+  if (e != cudaSuccess) return cuda_fail(e);
+  uint64_t keep = ~0ull;
+  e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+  if (e != cudaSuccess) {
+    cudaMemPoolDestroy(pool);
+    return cuda_fail(e);
+  }
+  g_pool[dev].store(pool, std::memory_order_release);
+  return KDA_OK;
+}
+
+// 0 picks the path that measured faster on B200 for every workload so far:
+// the 16-token one.
+int use_path() {
+  const int p = g_path.load();
+  return p == 64 ? 64 : 16;
+}
+
+// 16-token path: 32-column slices unless that grid would fill at most half of
+// the SMs (few heads and sequences); then 16-column slices.
+int slice_columns(int dev, int32_t num_seqs, int32_t num_heads) {
+  const int forced = g_slice_columns.load();
+  if (forced == 16 || forced == 32) return forced;
+  const int64_t ctas32 = int64_t(num_seqs) * num_heads * (KDA_HEAD_DIM / 32);
+  return 2 * ctas32 <= g_num_sms[dev] ? 16 : 32;
+}
+
+size_t ring_bytes(int path, const Problem& P) {
+  const size_t pairs = static_cast<size_t>(P.num_seqs) * P.num_heads;
+  return path == 16 ? pairs * kda::RING * kda::kSlotBytes : pairs * kda::c64::RING * kda::c64::SLOT_BYTES;
+}
+
+// ---------------------------------------------------- allocation-free variant
+// Scratch ring of kda_fwd_noalloc: a fixed-size array at file scope in device
+// memory, sized for either path at KDA_NOALLOC_MAX_PAIRS pairs. Host code
+// cannot use the symbol as an address; its device address is looked up once
+// per device (with that device current) and passed to the kernel.
+constexpr size_t kNoAllocBytes16 = static_cast<size_t>(KDA_NOALLOC_MAX_PAIRS) * kda::RING * kda::kSlotBytes;
+constexpr size_t kNoAllocBytes64 = static_cast<size_t>(KDA_NOALLOC_MAX_PAIRS) * kda::c64::RING * kda::c64::SLOT_BYTES;
+constexpr size_t kNoAllocRingBytes = kNoAllocBytes16 > kNoAllocBytes64 ? kNoAllocBytes16 : kNoAllocBytes64;
+static_assert(kda::c64::RING * kda::c64::SLOT_BYTES == KDA_RING_BYTES_PER_PAIR, "header constant");
+static __device__ __align__(256) unsigned char g_noalloc_ring[kNoAllocRingBytes];
+
+kda_status_t noalloc_setup(int dev) {
+  if (g_noalloc_ring_addr[dev].load(std::memory_order_acquire)) return KDA_OK;
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  if (g_noalloc_ring_addr[dev].load()) return KDA_OK;
+  void* addr = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&addr, g_noalloc_ring);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (!addr) return KDA_ERR_CUDA;
+  g_noalloc_ring_addr[dev].store(addr, std::memory_order_release);
+  return KDA_OK;
+}
+
+// --------------------------------------------------------------- launches
+kda_status_t launch16(const Problem& P, unsigned char* ring, int dev, cudaStream_t stream) {
+  kda::Params p;
+  p.q = static_cast<const __nv_bfloat16*>(P.q.data);
+  p.k = static_cast<const __nv_bfloat16*>(P.k.data);
+  p.v = static_cast<const __nv_bfloat16*>(P.v.data);
+  p.g = static_cast<const float*>(P.g.data);
+  p.beta = static_cast<const float*>(P.beta.data);
+  p.cu = P.cu;
+  p.init = P.init;
+  p.out = static_cast<__nv_bfloat16*>(P.out.data);
+  p.fin = P.fin;
+  p.ring = ring;
+  p.T = P.T;
+  p.beta_st = P.beta.st;
+  p.beta_sh = P.beta.sh;
+  p.out_st = P.out.st;
+  p.out_sh = P.out.sh;
+  p.H = P.num_heads;
+  p.scale = P.scale;
+  const int ns = slice_columns(dev, P.num_seqs, P.num_heads);
+  kda::TensorMaps tm;
+  std::memset(&tm, 0, sizeof(tm));
+  if (P.T > 0) {
+    kda_status_t st = load_encoder();
+    if (st != KDA_OK) return st;
+    const int H = P.num_heads;
+    constexpr auto NONE = CU_TENSOR_MAP_SWIZZLE_NONE;
+    if ((st = encode_3d(&tm.q, P.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.T, H, kda::D, kda::C, NONE)) != KDA_OK ||
+        (st = encode_3d(&tm.k, P.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.T, H, kda::D, kda::C, NONE)) != KDA_OK ||
+        (st = encode_3d(&tm.g, P.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, P.T, H, kda::D, kda::C, NONE)) != KDA_OK ||
+        (st = encode_3d(&tm.v, P.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.T, H, ns, kda::C, NONE)) != KDA_OK)
+      return st;
+  }
+  if (ns == 16) {
+    kda::kda_fwd_kernel<16><<<dim3(kda::D / 16, P.num_heads, P.num_seqs), kda::NTHREADS, sizeof(kda::Shared<16>),
+                              stream>>>(p, tm);
+  } else {
+    kda::kda_fwd_kernel<32><<<dim3(kda::D / 32, P.num_heads, P.num_seqs), kda::NTHREADS, sizeof(kda::Shared<32>),
+                              stream>>>(p, tm);
+  }
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return KDA_OK;
+}
+
+kda_status_t launch64(const Problem& P, unsigned char* ring, cudaStream_t stream) {
+  namespace c = kda::c64;
+  c::Params p;
+  p.beta = static_cast<const float*>(P.beta.data);
+  p.cu = P.cu;
+  p.init = P.init;
+  p.out = static_cast<__nv_bfloat16*>(P.out.data);
+  p.fin = P.fin;
+  p.ring = ring;
+  p.T = P.T;
+  p.beta_st = P.beta.st;
+  p.beta_sh = P.beta.sh;
+  p.out_st = P.out.st;
+  p.out_sh = P.out.sh;
+  p.H = P.num_heads;
+  p.scale = P.scale;
+  c::Maps tm;
+  std::memset(&tm, 0, sizeof(tm));
+  if (P.T > 0) {
+    kda_status_t st = load_encoder();
+    if (st != KDA_OK) return st;
+    const int H = P.num_heads;
+    constexpr auto NONE = CU_TENSOR_MAP_SWIZZLE_NONE;
+    if ((st = encode_3d(&tm.q, P.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.T, H, kda::D, c::CH, NONE)) != KDA_OK ||
+        (st = encode_3d(&tm.k, P.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.T, H, kda::D, c::CH, NONE)) != KDA_OK ||
+        (st = encode_3d(&tm.g, P.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, P.T, H, kda::D, c::CH, NONE)) != KDA_OK ||
+        (st = encode_3d(&tm.v, P.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.T, H, 64, c::CH,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != KDA_OK)
+      return st;
+  }
+  c::kda_fwd64_kernel<<<dim3(c::CLUSTER, P.num_heads, P.num_seqs), c::NTHREADS, c::SMEM_BYTES, stream>>>(p, tm);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return KDA_OK;
+}
+
+kda_status_t launch(const Problem& P, unsigned char* ring, int path, int dev, cudaStream_t stream) {
+  return path == 16 ? launch16(P, ring, dev, stream) : launch64(P, ring, stream);
+}
+
+kda_status_t prologue(int* dev) {
+  g_last_cuda_error[0] = '\0';
+  cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return check_device(*dev);
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status_t kda_fwd(const kda_tensor_t* q, const kda_tensor_t* k, const kda_tensor_t* v, const kda_tensor_t* g,
+                     const kda_tensor_t* beta, float scale, const int32_t* cu_seqlens, int32_t num_seqs,
+                     const kda_tensor_t* initial_state, const kda_tensor_t* out, const kda_tensor_t* final_state,
+                     void* stream) {
+  g_last_cuda_error[0] = '\0';
+  Problem P;
+  kda_status_t st = check_args(q, k, v, g, beta, scale, cu_seqlens, num_seqs, initial_state, out, final_state, &P);
+  if (st != KDA_OK) return st;
+  int dev = 0;
+  if ((st = prologue(&dev)) != KDA_OK) return st;
+  if ((st = prepare_pool(dev)) != KDA_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const int path = use_path();
+  // Ring of chunk operands, one per (sequence, head): stream-ordered scratch
+  // from the library's pool, released in stream order after the kernel.
+  void* ring = nullptr;
+  if (P.T > 0) {
+    const cudaError_t e = cudaMallocFromPoolAsync(&ring, ring_bytes(path, P), g_pool[dev].load(), cs);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  st = launch(P, static_cast<unsigned char*>(ring), path, dev, cs);
+  if (ring) {
+    const cudaError_t ef = cudaFreeAsync(ring, cs);
+    if (st == KDA_OK && ef != cudaSuccess) return cuda_fail(ef);
+  }
+  return st;
+}
+
+kda_status_t kda_fwd_noalloc(const kda_tensor_t* q, const kda_tensor_t* k, const kda_tensor_t* v,
+                             const kda_tensor_t* g, const kda_tensor_t* beta, float scale,
+                             const int32_t* cu_seqlens, int32_t num_seqs, const kda_tensor_t* initial_state,
+                             const kda_tensor_t* out, const kda_tensor_t* final_state, void* stream) {
+  g_last_cuda_error[0] = '\0';
+  Problem P;
+  kda_status_t st = check_args(q, k, v, g, beta, scale, cu_seqlens, num_seqs, initial_state, out, final_state, &P);
+  if (st != KDA_OK) return st;
+  if (int64_t(P.num_seqs) * P.num_heads > KDA_NOALLOC_MAX_PAIRS) return KDA_ERR_CAPACITY;
+  int dev = 0;
+  if ((st = prologue(&dev)) != KDA_OK) return st;
+  if ((st = noalloc_setup(dev)) != KDA_OK) return st;
+  return launch(P, static_cast<unsigned char*>(g_noalloc_ring_addr[dev].load()), use_path(), dev,
+                static_cast<cudaStream_t>(stream));
+}
+
+kda_status_t kda_set_path(int32_t path) {
+  if (path != 0 && path != 16 && path != 64) return KDA_ERR_SHAPE;
+  g_path.store(path);
+  return KDA_OK;
+}
+
+kda_status_t kda_set_slice_columns(int32_t columns) {
+  if (columns != 0 && columns != 16 && columns != 32) return KDA_ERR_SHAPE;
+  g_slice_columns.store(columns);
+  return KDA_OK;
+}
+
+const char* kda_status_string(kda_status_t s) {
+  switch (s) {
+    case KDA_OK: return "ok";
+    case KDA_ERR_NULL: return "a required tensor or pointer is NULL";
+    case KDA_ERR_SHAPE: return "invalid shape or sizes";
+    case KDA_ERR_ALIGN: return "a data pointer is not 16-byte aligned";
+    case KDA_ERR_UNSUPPORTED: return "the current device is not sm_100 (B200)";
+    case KDA_ERR_CUDA: return "a CUDA call failed (see kda_last_cuda_error)";
+    case KDA_ERR_CAPACITY: return "num_seqs * num_heads exceeds the fixed scratch of kda_fwd_noalloc";
+    case KDA_ERR_DTYPE: return "a tensor has the wrong dtype";
+    case KDA_ERR_STRIDE: return "a tensor's strides are not supported";
+    case KDA_ERR_DEVICE: return "the device recorded a fault (see kda_device_status)";
+  }
+  return "unknown status";
+}
+
+const char* kda_last_cuda_error(void) { return g_last_cuda_error; }
+
+kda_status_t kda_device_status(uint32_t* flags, int32_t reset) {
+  if (!flags) return KDA_ERR_NULL;
+  g_last_cuda_error[0] = '\0';
+  uint32_t bits = 0, waits = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&bits, kda::g_device_flags, sizeof(uint32_t));
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaMemcpyFromSymbol(&waits, kda::g_wait_timeouts, sizeof(uint32_t));
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (waits) bits |= KDA_DEVICE_WAIT_TIMEOUT;
+  *flags = bits;
+  if (reset) {
+    const uint32_t zero = 0;
+    if ((e = cudaMemcpyToSymbol(kda::g_device_flags, &zero, sizeof(uint32_t))) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaMemcpyToSymbol(kda::g_wait_timeouts, &zero, sizeof(uint32_t))) != cudaSuccess) return cuda_fail(e);
+  }
+  return bits ? KDA_ERR_DEVICE : KDA_OK;
+}
+
+kda_status_t kda_wait_timeouts(uint32_t* count, int32_t reset) {
+  if (!count) return KDA_ERR_NULL;
+  g_last_cuda_error[0] = '\0';
+  cudaError_t e = cudaMemcpyFromSymbol(count, kda::g_wait_timeouts, sizeof(uint32_t));
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (reset) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbol(kda::g_wait_timeouts, &zero, sizeof(uint32_t));
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return KDA_OK;
+}
+
+int32_t kda_abi_version(void) { return KDA_ABI_VERSION; }
+
+}  // extern "C"

@@ -1,4 +1,4 @@
-// kda_fwd.cu -- chunked Kimi Delta Attention forward (prefill) for sm_100a.
+// kda_fwd16.cuh -- chunk-16 Kimi Delta Attention forward (prefill) on mma.sync.
 //
 // Work decomposition
 //   One thread-block cluster per (sequence, head): one CTA per value slice of
@@ -57,21 +57,12 @@
 // plus a ~250-cycle commit/mbarrier round trip; the chain is a serial sequence
 // of such small products, so it stays on the synchronous path.
 
-#include <cuda.h>
-#include <cuda_bf16.h>
-#include <cuda_runtime.h>
-#include <cudaTypedefs.h>
+#pragma once
 
-#include <atomic>
-#include <cstdint>
-#include <cstdio>
-#include <cstring>
-
-#include "../../include/kda.h"
+#include "kda_prims.cuh"
 
 namespace kda {
 
-constexpr int D = KDA_HEAD_DIM;   // dk = dv = 128
 constexpr int C = 16;             // chunk length (tokens)
 // Value columns per CTA (NS) is a template parameter of the kernel: 32 (four
 // CTAs per (sequence, head), two chain warps each) or, when that grid would
@@ -164,214 +155,6 @@ static_assert(sizeof(ProdStage) % 128 == 0 && sizeof(ChainStage<16>) % 128 == 0 
               "stage alignment");
 static_assert(sizeof(Shared<32>) <= 227 * 1024 && sizeof(Shared<16>) <= 227 * 1024, "shared memory budget");
 
-// Wait budget for every mbarrier wait (cycles). A wait that runs out records
-// a timeout and lets the thread continue, so no barrier is ever left waiting.
-constexpr long long kWaitCycles = 1ll << 28;  // ~0.14 s at 1.9 GHz
-// A waiting thread is suspended in hardware (up to this many ns per try)
-// instead of spinning, so waiting warps leave the issue slots to the others.
-constexpr uint32_t kSuspendHintNs = 20000;
-__device__ unsigned int g_wait_timeouts = 0;
-
-// ---------------------------------------------------------------- primitives
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(unsigned long long* m, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(m)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(unsigned long long* m) {
-  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(m)) : "memory");
-}
-
-// One arrive per warp: __syncwarp orders every lane's prior shared-memory
-// accesses before lane 0's release-arrive.
-__device__ __forceinline__ void mbar_arrive_warp(unsigned long long* m) {
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(m);
-}
-
-__device__ __forceinline__ bool mbar_try_wait(unsigned long long* m, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
-      : "=r"(ok)
-      : "r"(smem_u32(m)), "r"(parity), "r"(kSuspendHintNs)
-      : "memory");
-  return ok != 0;
-}
-// Non-blocking probe: cheaper than a suspending try_wait when the phase has
-// long completed, which is the common case for well-fed pipeline stages.
-__device__ __forceinline__ bool mbar_test_wait(unsigned long long* m, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{ .reg .pred p; mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-      : "=r"(ok)
-      : "r"(smem_u32(m)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-__device__ __forceinline__ void mbar_wait(unsigned long long* m, uint32_t parity) {
-  if (mbar_test_wait(m, parity)) return;
-  const long long t0 = clock64();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(m, parity)) return;
-    if ((i & 63u) == 0 && clock64() - t0 > kWaitCycles) {
-      atomicAdd(&g_wait_timeouts, 1u);
-      return;
-    }
-  }
-}
-
-// 4-byte asynchronous copy (zero fill when src_bytes = 0) and the arrive that
-// fires once this thread's copies have landed.
-__device__ __forceinline__ void cp_async4(void* dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void cp_async_arrive(unsigned long long* m) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(m)) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long* m, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(m)), "r"(bytes)
-               : "memory");
-}
-
-// TMA tiled loads (no multicast). Out-of-range rows of the box are zero-filled.
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
-                                            unsigned long long* m) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
-      "[%5];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(m))
-      : "memory");
-}
-
-__device__ __forceinline__ void named_bar_arrive(int id, int nthreads) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-__device__ __forceinline__ void named_bar(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(smem_u32(p)));
-}
-
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(smem_u32(p)));
-}
-
-// D += A(16x16 row-major fragment) * B(16x8 column fragment); bf16 in, fp32 acc.
-__device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
-  uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
-
-// (x, y) *= (a, b) as one packed fp32 multiply
-__device__ __forceinline__ void mul2(float& x, float& y, float a, float b) {
-  unsigned long long r;
-  asm("mul.rn.f32x2 %0, %1, %2;"
-      : "=l"(r)
-      : "l"((static_cast<unsigned long long>(__float_as_uint(y)) << 32) | __float_as_uint(x)),
-        "l"((static_cast<unsigned long long>(__float_as_uint(b)) << 32) | __float_as_uint(a)));
-  x = __uint_as_float(static_cast<uint32_t>(r));
-  y = __uint_as_float(static_cast<uint32_t>(r >> 32));
-}
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  uint32_t u;
-  memcpy(&u, &h, 4);
-  return u;
-}
-
-
-// ---- cluster-scope signalling
-__device__ __forceinline__ bool mbar_try_wait_cl(unsigned long long* m, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
-      : "=r"(ok)
-      : "r"(smem_u32(m)), "r"(parity), "r"(kSuspendHintNs)
-      : "memory");
-  return ok != 0;
-}
-
-__device__ __forceinline__ void mbar_wait_cl(unsigned long long* m, uint32_t parity) {
-  if (mbar_try_wait_cl(m, parity)) return;
-  const long long t0 = clock64();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait_cl(m, parity)) return;
-    if ((i & 63u) == 0 && clock64() - t0 > kWaitCycles) {
-      atomicAdd(&g_wait_timeouts, 1u);
-      return;
-    }
-  }
-}
-
-// Arrive on the mbarrier at the same shared-memory offset in CTA `rank` of the
-// cluster. Relaxed: a "done" signal whose data (if any) was already made
-// complete and visible by its sender, so it need not wait for this thread's
-// outstanding global stores.
-__device__ __forceinline__ void mbar_arrive_remote_relaxed(unsigned long long* m, uint32_t rank) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(m)), "r"(rank));
-  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
-}
-
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Generic-proxy shared-memory writes become visible to the bulk-copy engine.
-__device__ __forceinline__ void fence_proxy_async_shared() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-// Bulk copy shared -> global as one bulk async-group.
-__device__ __forceinline__ void bulk_s2g(void* gdst, const void* ssrc, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(ssrc)),
-               "r"(bytes)
-               : "memory");
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-// Wait until at most N of this thread's bulk async-groups are still pending
-// (their writes to global memory completed).
-template <int N>
-__device__ __forceinline__ void bulk_wait() {
-  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
-}
-
-// Bulk copy global -> shared, completion counted in bytes on the mbarrier.
-__device__ __forceinline__ void bulk_g2s(void* sdst, const void* gsrc, uint32_t bytes, unsigned long long* m) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(sdst)),
-      "l"(gsrc), "r"(bytes), "r"(smem_u32(m))
-      : "memory");
-}
-
 // ---------------------------------------------------------------- the kernel
 struct Params {
   const __nv_bfloat16* q;
@@ -385,6 +168,8 @@ struct Params {
   float* fin;              // may be null
   unsigned char* ring;     // [num_seqs * H][RING] slots of kSlotBytes
   int64_t T;
+  int64_t beta_st, beta_sh;  // element strides of beta over tokens and heads
+  int64_t out_st, out_sh;    // element strides of out over tokens and heads
   int32_t H;
   float scale;
 };
@@ -415,10 +200,10 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
   const int dv0 = rank * NS;
   const int H = p.H;
   const int64_t T = p.T;
-  const size_t row_stride = static_cast<size_t>(H) * D;  // elements between tokens of q/k/v/g/out
 
   int64_t t0 = 0, t1 = T;
   if (p.cu) {
+    if (tid == 0 && rank == 0 && h == 0) check_bounds(p.cu, seq, static_cast<int>(gridDim.z), T);
     t0 = p.cu[seq];
     t1 = p.cu[seq + 1];
     t0 = t0 < 0 ? 0 : (t0 > T ? T : t0);
@@ -596,7 +381,7 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
       for (int nt = 0; nt < 2; ++nt) {
         const int tok = 8 * nt + gq;
         if (tok < m) {
-          __nv_bfloat16* dst = p.out + (cs + tok) * row_stride + static_cast<size_t>(h) * D + dv0 + cv + 2 * tq;
+          __nv_bfloat16* dst = p.out + (cs + tok) * p.out_st + static_cast<int64_t>(h) * p.out_sh + dv0 + cv + 2 * tq;
           *reinterpret_cast<uint32_t*>(dst) = r[nt][0];
           *reinterpret_cast<uint32_t*>(dst + 8) = r[nt][1];
         }
@@ -799,7 +584,7 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
       } else if (lane <= C) {
         const int r = lane - 1;
         const bool ok = cs + r < t1;
-        cp_async4(&rw.beta[r], p.beta + (ok ? (cs + r) * H + h : 0), ok ? 4u : 0u);
+        cp_async4(&rw.beta[r], p.beta + (ok ? (cs + r) * p.beta_st + h * p.beta_sh : 0), ok ? 4u : 0u);
         cp_async_arrive(&sh.raw_full[rs]);
       }
     }
@@ -843,291 +628,3 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
 }
 
 }  // namespace kda
-
-// =================================================================== C ABI
-namespace {
-
-thread_local char g_last_cuda_error[256] = "";
-
-kda_status_t cuda_fail(cudaError_t e) {
-  std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(e),
-                cudaGetErrorString(e));
-  return KDA_ERR_CUDA;
-}
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-
-kda_status_t load_encoder() {
-  if (g_encode) return KDA_OK;
-  void* fn = nullptr;
-  cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
-  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
-  if (e != cudaSuccess) return cuda_fail(e);
-  if (q != cudaDriverEntryPointSuccess || !fn) {
-    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled not available");
-    return KDA_ERR_CUDA;
-  }
-  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  return KDA_OK;
-}
-
-// [T, H, inner] row-major tensor; box {box_inner, 1, 16 tokens}.
-kda_status_t encode_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes, int64_t T,
-                       int H, int inner, int box_inner) {
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(H),
-                              static_cast<cuuint64_t>(T)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner) * elem_bytes,
-                                 static_cast<cuuint64_t>(H) * inner * elem_bytes};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), 1u, static_cast<cuuint32_t>(kda::C)};
-  const cuuint32_t estr[3] = {1u, 1u, 1u};
-  CUresult r = g_encode(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) {
-    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
-    return KDA_ERR_CUDA;
-  }
-  return KDA_OK;
-}
-
-constexpr int kMaxDevices = 64;
-int g_device_ready[kMaxDevices];  // 0 unknown, 1 ready, -1 unsupported
-int g_num_sms[kMaxDevices];
-// Library-private stream-ordered pool for the scratch ring. It keeps freed
-// memory (release threshold = max), so steady-state calls never map memory
-// and the process's default pool is left untouched.
-cudaMemPool_t g_pool[kMaxDevices];
-// Value columns per CTA: 0 chooses per call, 16 or 32 forces that variant.
-std::atomic<int> g_slice_columns{0};
-
-template <int NS>
-cudaError_t set_smem_attribute() {
-  return cudaFuncSetAttribute(kda::kda_fwd_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(sizeof(kda::Shared<NS>)));
-}
-
-// Capability check, kernel attributes and SM count for `dev` (current).
-kda_status_t check_device(int dev) {
-  if (dev < 0 || dev >= kMaxDevices) return KDA_ERR_UNSUPPORTED;
-  if (g_device_ready[dev] == 1) return KDA_OK;
-  if (g_device_ready[dev] == -1) return KDA_ERR_UNSUPPORTED;
-  int major = 0, minor = 0, sms = 0;
-  cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-  if (e != cudaSuccess) return cuda_fail(e);
-  e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
-  if (e != cudaSuccess) return cuda_fail(e);
-  if (major != 10 || minor != 0) {
-    g_device_ready[dev] = -1;
-    return KDA_ERR_UNSUPPORTED;
-  }
-  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return cuda_fail(e);
-  if ((e = set_smem_attribute<32>()) != cudaSuccess) return cuda_fail(e);
-  if ((e = set_smem_attribute<16>()) != cudaSuccess) return cuda_fail(e);
-  g_num_sms[dev] = sms;
-  g_device_ready[dev] = 1;
-  return KDA_OK;
-}
-
-// The pool of kda_fwd's scratch rings, created once per device.
-kda_status_t prepare_pool(int dev) {
-  if (g_pool[dev]) return KDA_OK;
-  cudaMemPoolProps props;
-  std::memset(&props, 0, sizeof(props));
-  props.allocType = cudaMemAllocationTypePinned;
-  props.handleTypes = cudaMemHandleTypeNone;
-  props.location.type = cudaMemLocationTypeDevice;
-  props.location.id = dev;
-  cudaMemPool_t pool = nullptr;
-  cudaError_t e = cudaMemPoolCreate(&pool, &props);
-  if (e != cudaSuccess) return cuda_fail(e);
-  uint64_t keep = ~0ull;
-  e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
-  if (e != cudaSuccess) return cuda_fail(e);
-  g_pool[dev] = pool;
-  return KDA_OK;
-}
-
-// 32-column slices unless that grid would fill at most half of the SMs (few
-// heads and sequences); then 16-column slices double the CTAs working on
-// the same serial chains.
-int slice_columns(int dev, int32_t num_seqs, int32_t num_heads) {
-  const int forced = g_slice_columns.load();
-  if (forced == 16 || forced == 32) return forced;
-  const int64_t ctas32 = int64_t(num_seqs) * num_heads * (KDA_HEAD_DIM / 32);
-  return 2 * ctas32 <= g_num_sms[dev] ? 16 : 32;
-}
-
-// ---------------------------------------------------- allocation-free variant
-// Scratch ring of kda_fwd_noalloc: a fixed-size array at file scope in device
-// memory. Host code cannot use the symbol as an address; its device address is
-// looked up once per device (with that device current) and passed to the kernel.
-constexpr size_t kNoAllocRingBytes =
-    static_cast<size_t>(KDA_NOALLOC_MAX_PAIRS) * kda::RING * kda::kSlotBytes;
-static __device__ __align__(256) unsigned char g_noalloc_ring[kNoAllocRingBytes];
-void* g_noalloc_ring_addr[kMaxDevices];
-
-kda_status_t noalloc_setup(int dev) {
-  if (g_noalloc_ring_addr[dev]) return KDA_OK;
-  void* addr = nullptr;
-  cudaError_t e = cudaGetSymbolAddress(&addr, g_noalloc_ring);
-  if (e != cudaSuccess) return cuda_fail(e);
-  if (!addr) return KDA_ERR_CUDA;
-  g_noalloc_ring_addr[dev] = addr;
-  return KDA_OK;
-}
-
-// Host-side checks shared by both entry points (synchronous, no device work).
-kda_status_t check_args(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                        const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens, int32_t num_heads,
-                        const float* initial_state, const void* out, const float* final_state) {
-  if (total_tokens < 0 || num_heads < 1 || num_seqs < 1) return KDA_ERR_SHAPE;
-  if (total_tokens > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_NULL;
-  if (!cu_seqlens && num_seqs != 1) return KDA_ERR_SHAPE;
-  if (num_heads > 65535 || num_seqs > 65535) return KDA_ERR_SHAPE;  // grid.y / grid.z limits
-  if (total_tokens > (int64_t(1) << 40) / (int64_t(num_heads) * KDA_HEAD_DIM)) return KDA_ERR_SHAPE;
-  if (total_tokens > int64_t(INT32_MAX) - 64) return KDA_ERR_SHAPE;  // TMA coordinates are 32-bit
-  const void* ptrs[] = {q, k, v, g, beta, out, initial_state, final_state, cu_seqlens};
-  for (const void* ptr : ptrs)
-    if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
-  return KDA_OK;
-}
-
-// Tensor maps, variant choice and launch; `ring` holds RING slots per
-// (sequence, head).
-kda_status_t launch(const void* q, const void* k, const void* v, const float* g, const float* beta, float scale,
-                    const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens, int32_t num_heads,
-                    const float* initial_state, void* out, float* final_state, unsigned char* ring, int dev,
-                    cudaStream_t stream) {
-  kda::Params p;
-  p.q = static_cast<const __nv_bfloat16*>(q);
-  p.k = static_cast<const __nv_bfloat16*>(k);
-  p.v = static_cast<const __nv_bfloat16*>(v);
-  p.g = g;
-  p.beta = beta;
-  p.cu = cu_seqlens;
-  p.init = initial_state;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.fin = final_state;
-  p.T = total_tokens;
-  p.H = num_heads;
-  p.scale = scale;
-  p.ring = ring;
-  const int ns = slice_columns(dev, num_seqs, num_heads);
-  kda::TensorMaps tm;
-  std::memset(&tm, 0, sizeof(tm));
-  if (total_tokens > 0) {
-    kda_status_t st = load_encoder();
-    if (st != KDA_OK) return st;
-    const int H = num_heads;
-    if ((st = encode_3d(&tm.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total_tokens, H, kda::D, kda::D)) != KDA_OK ||
-        (st = encode_3d(&tm.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total_tokens, H, kda::D, kda::D)) != KDA_OK ||
-        (st = encode_3d(&tm.g, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total_tokens, H, kda::D, kda::D)) != KDA_OK ||
-        (st = encode_3d(&tm.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total_tokens, H, kda::D, ns)) != KDA_OK)
-      return st;
-  }
-  if (ns == 16) {
-    kda::kda_fwd_kernel<16><<<dim3(kda::D / 16, num_heads, num_seqs), kda::NTHREADS, sizeof(kda::Shared<16>),
-                              stream>>>(p, tm);
-  } else {
-    kda::kda_fwd_kernel<32><<<dim3(kda::D / 32, num_heads, num_seqs), kda::NTHREADS, sizeof(kda::Shared<32>),
-                              stream>>>(p, tm);
-  }
-  const cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e);
-  return KDA_OK;
-}
-
-}  // namespace
-
-extern "C" {
-
-kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                     float scale, const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
-                     int32_t num_heads, const float* initial_state, void* out, float* final_state,
-                     void* stream) {
-  g_last_cuda_error[0] = '\0';
-  kda_status_t st = check_args(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens, num_heads, initial_state, out,
-                               final_state);
-  if (st != KDA_OK) return st;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e);
-  if ((st = check_device(dev)) != KDA_OK) return st;
-  if ((st = prepare_pool(dev)) != KDA_OK) return st;
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  // Ring of shared chunk operands, one per (sequence, head): stream-ordered
-  // scratch from the library's pool, released in stream order after the
-  // kernel. It stays L2-resident while in use (RING slots per head).
-  void* ring = nullptr;
-  if (total_tokens > 0) {
-    const size_t ring_bytes = static_cast<size_t>(num_seqs) * num_heads * kda::RING * kda::kSlotBytes;
-    e = cudaMallocFromPoolAsync(&ring, ring_bytes, g_pool[dev], cs);
-    if (e != cudaSuccess) return cuda_fail(e);
-  }
-  st = launch(q, k, v, g, beta, scale, cu_seqlens, num_seqs, total_tokens, num_heads, initial_state, out, final_state,
-              static_cast<unsigned char*>(ring), dev, cs);
-  if (ring) {
-    const cudaError_t ef = cudaFreeAsync(ring, cs);
-    if (st == KDA_OK && ef != cudaSuccess) return cuda_fail(ef);
-  }
-  return st;
-}
-
-kda_status_t kda_fwd_noalloc(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                             float scale, const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
-                             int32_t num_heads, const float* initial_state, void* out, float* final_state,
-                             void* stream) {
-  g_last_cuda_error[0] = '\0';
-  kda_status_t st = check_args(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens, num_heads, initial_state, out,
-                               final_state);
-  if (st != KDA_OK) return st;
-  if (int64_t(num_seqs) * num_heads > KDA_NOALLOC_MAX_PAIRS) return KDA_ERR_CAPACITY;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e);
-  if ((st = check_device(dev)) != KDA_OK) return st;
-  if ((st = noalloc_setup(dev)) != KDA_OK) return st;
-  return launch(q, k, v, g, beta, scale, cu_seqlens, num_seqs, total_tokens, num_heads, initial_state, out,
-                final_state, static_cast<unsigned char*>(g_noalloc_ring_addr[dev]), dev,
-                static_cast<cudaStream_t>(stream));
-}
-
-kda_status_t kda_set_slice_columns(int32_t columns) {
-  if (columns != 0 && columns != 16 && columns != 32) return KDA_ERR_SHAPE;
-  g_slice_columns.store(columns);
-  return KDA_OK;
-}
-
-const char* kda_status_string(kda_status_t s) {
-  switch (s) {
-    case KDA_OK: return "ok";
-    case KDA_ERR_NULL: return "a required pointer is NULL";
-    case KDA_ERR_SHAPE: return "invalid sizes";
-    case KDA_ERR_ALIGN: return "a tensor pointer is not 16-byte aligned";
-    case KDA_ERR_UNSUPPORTED: return "the current device is not sm_100 (B200)";
-    case KDA_ERR_CUDA: return "a CUDA call failed (see kda_last_cuda_error)";
-    case KDA_ERR_CAPACITY: return "num_seqs * num_heads exceeds the fixed scratch of kda_fwd_noalloc";
-  }
-  return "unknown status";
-}
-
-const char* kda_last_cuda_error(void) { return g_last_cuda_error; }
-
-kda_status_t kda_wait_timeouts(uint32_t* count, int32_t reset) {
-  if (!count) return KDA_ERR_NULL;
-  cudaError_t e = cudaMemcpyFromSymbol(count, kda::g_wait_timeouts, sizeof(uint32_t));
-  if (e != cudaSuccess) return cuda_fail(e);
-  if (reset) {
-    const uint32_t zero = 0;
-    e = cudaMemcpyToSymbol(kda::g_wait_timeouts, &zero, sizeof(uint32_t));
-    if (e != cudaSuccess) return cuda_fail(e);
-  }
-  return KDA_OK;
-}
-
-int32_t kda_abi_version(void) { return KDA_ABI_VERSION; }
-
-}  // extern "C"

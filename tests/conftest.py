@@ -18,3 +18,10 @@ def oracle_mod():
 
     oracle.build()
     return oracle
+
+
+def pytest_sessionfinish(session, exitstatus):
+    # per-case parity errors of the GPU tests, as a table (JSON) when asked for
+    from tests import helpers
+
+    helpers.write_report()

@@ -1,5 +1,11 @@
 """The C-ABI library loads, exports every declared symbol, and rejects bad
-arguments on the host before touching the GPU (CPU only)."""
+arguments on the host before touching the GPU (CPU only).
+
+Every call here fails validation before any CUDA call, so the fake device
+addresses are never dereferenced or handed to the driver. The one test that
+lets a call pass validation runs only where no GPU is present (the call then
+stops at the CUDA device query).
+"""
 import ctypes
 import os
 import re
@@ -7,6 +13,33 @@ import re
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+KDA_OK, KDA_ERR_NULL, KDA_ERR_SHAPE, KDA_ERR_ALIGN = 0, 1, 2, 3
+KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_CAPACITY = 4, 5, 6
+KDA_ERR_DTYPE, KDA_ERR_STRIDE, KDA_ERR_DEVICE = 7, 8, 9
+BF16, F32, I32 = 1, 2, 3
+
+
+class Desc(ctypes.Structure):
+    """Mirror of kda_tensor_t (include/kda.h)."""
+    _fields_ = [("data", ctypes.c_void_p), ("ndim", ctypes.c_int32), ("dtype", ctypes.c_int),
+                ("shape", ctypes.c_int64 * 4), ("stride", ctypes.c_int64 * 4)]
+
+
+def desc(addr, dtype, shape, stride=None):
+    d = Desc()
+    d.data = addr
+    d.ndim = len(shape)
+    d.dtype = dtype
+    if stride is None:  # contiguous
+        stride, acc = [], 1
+        for n in reversed(shape):
+            stride.insert(0, acc)
+            acc *= n
+    for i, (n, s) in enumerate(zip(shape, stride)):
+        d.shape[i] = n
+        d.stride[i] = s
+    return d
 
 
 @pytest.fixture(scope="module")
@@ -19,7 +52,13 @@ def lib():
     build = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(build)
     build.build()
-    return ctypes.CDLL(build.LIB)
+    lib = ctypes.CDLL(build.LIB)
+    P = ctypes.POINTER(Desc)
+    for name in ("kda_fwd", "kda_fwd_noalloc"):
+        fn = getattr(lib, name)
+        fn.argtypes = [P, P, P, P, P, ctypes.c_float, ctypes.c_void_p, ctypes.c_int32, P, P, P, ctypes.c_void_p]
+        fn.restype = ctypes.c_int
+    return lib
 
 
 def _declared_functions():
@@ -30,64 +69,175 @@ def _declared_functions():
 
 def test_exports_every_declared_symbol(lib):
     names = _declared_functions()
-    assert "kda_fwd" in names and len(names) >= 4
+    assert "kda_fwd" in names and "kda_fwd_noalloc" in names and len(names) >= 8
     for n in names:
         assert hasattr(lib, n), f"libkda.so does not export {n}"
 
 
 def test_abi_version_and_status_strings(lib):
     lib.kda_abi_version.restype = ctypes.c_int32
-    assert lib.kda_abi_version() == 2
+    assert lib.kda_abi_version() == 3
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_status_string.argtypes = [ctypes.c_int]
-    for code in range(6):
-        assert len(lib.kda_status_string(code)) > 0
+    texts = {lib.kda_status_string(code) for code in range(10)}
+    assert len(texts) == 10 and b"unknown status" not in texts
     assert lib.kda_status_string(99) == b"unknown status"
 
 
-def _call(lib, q=0x1000, k=0x2000, v=0x3000, g=0x4000, beta=0x5000, scale=1.0, cu=0x6000, nseq=1,
-          T=4, H=1, init=None, out=0x7000, fin=None):
-    P = ctypes.c_void_p
-    lib.kda_fwd.argtypes = [P, P, P, P, P, ctypes.c_float, P, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32,
-                            P, P, P, P]
-    lib.kda_fwd.restype = ctypes.c_int
-    return lib.kda_fwd(q, k, v, g, beta, scale, cu, nseq, T, H, init, out, fin, None)
+class Call:
+    """A valid-looking problem (T tokens, H heads, N sequences) on fake
+    16-byte-aligned addresses; tests override one tensor at a time."""
+
+    def __init__(self, T=64, H=2, N=1):
+        self.T, self.H, self.N = T, H, N
+        self.t = {
+            "q": desc(0x10000, BF16, [T, H, 128]),
+            "k": desc(0x20000, BF16, [T, H, 128]),
+            "v": desc(0x30000, BF16, [T, H, 128]),
+            "g": desc(0x40000, F32, [T, H, 128]),
+            "beta": desc(0x50000, F32, [T, H]),
+            "init": None,
+            "out": desc(0x60000, BF16, [T, H, 128]),
+            "fin": None,
+        }
+        self.cu = 0x70000
+        self.scale = 1.0
+
+    def run(self, lib, fn="kda_fwd", num_seqs=None, **over):
+        t = dict(self.t)
+        t.update({k: v for k, v in over.items() if k in t})
+        cu = over.get("cu", self.cu)
+        ref = {k: (None if d is None else ctypes.byref(d)) for k, d in t.items()}
+        return getattr(lib, fn)(ref["q"], ref["k"], ref["v"], ref["g"], ref["beta"], self.scale, cu,
+                                self.N if num_seqs is None else num_seqs, ref["init"], ref["out"], ref["fin"], None)
 
 
-def test_slice_columns_setting_validated(lib):
+def test_path_and_slice_settings_validated(lib):
     lib.kda_set_slice_columns.argtypes = [ctypes.c_int32]
     lib.kda_set_slice_columns.restype = ctypes.c_int
+    lib.kda_set_path.argtypes = [ctypes.c_int32]
+    lib.kda_set_path.restype = ctypes.c_int
     for bad in (-1, 1, 8, 24, 64, 128):
-        assert lib.kda_set_slice_columns(bad) == 2  # KDA_ERR_SHAPE
+        assert lib.kda_set_slice_columns(bad) == KDA_ERR_SHAPE
     for good in (16, 32, 0):
-        assert lib.kda_set_slice_columns(good) == 0
+        assert lib.kda_set_slice_columns(good) == KDA_OK
+    for bad in (-1, 1, 32, 128):
+        assert lib.kda_set_path(bad) == KDA_ERR_SHAPE
+    for good in (16, 64, 0):
+        assert lib.kda_set_path(good) == KDA_OK
 
 
-# These calls fail validation before any CUDA call, so the fake addresses are
-# never dereferenced or handed to the driver.
-def test_rejects_null_pointers(lib):
+@pytest.mark.parametrize("fn", ["kda_fwd", "kda_fwd_noalloc"])
+def test_rejects_missing_tensors(lib, fn):
+    c = Call()
     for name in ("q", "k", "v", "g", "beta", "out"):
-        assert _call(lib, **{name: None}) == 1, name
-        # with T = 0 the token tensors are never touched, so NULL is fine; the
-        # call then goes on to a misaligned init pointer and stops there
-        assert _call(lib, T=0, init=0x8008, **{name: None}) == 3, name
+        assert c.run(lib, fn, **{name: None}) == KDA_ERR_NULL, name
+    # a descriptor whose data pointer is NULL while T > 0
+    assert c.run(lib, fn, q=desc(None, BF16, [64, 2, 128])) == KDA_ERR_NULL
+    assert c.run(lib, fn, init=desc(None, F32, [1, 2, 128, 128])) == KDA_ERR_NULL
 
 
-def test_rejects_bad_shapes(lib):
-    assert _call(lib, T=-1) == 2
-    assert _call(lib, H=0) == 2
-    assert _call(lib, nseq=0) == 2
-    assert _call(lib, cu=None, nseq=2) == 2
-    assert _call(lib, H=70000) == 2
-    assert _call(lib, T=1 << 40, H=32) == 2
+@pytest.mark.parametrize("fn", ["kda_fwd", "kda_fwd_noalloc"])
+def test_rejects_wrong_dtypes(lib, fn):
+    c = Call()
+    assert c.run(lib, fn, q=desc(0x10000, F32, [64, 2, 128])) == KDA_ERR_DTYPE
+    assert c.run(lib, fn, v=desc(0x30000, I32, [64, 2, 128])) == KDA_ERR_DTYPE
+    assert c.run(lib, fn, g=desc(0x40000, BF16, [64, 2, 128])) == KDA_ERR_DTYPE
+    assert c.run(lib, fn, beta=desc(0x50000, BF16, [64, 2])) == KDA_ERR_DTYPE
+    assert c.run(lib, fn, out=desc(0x60000, F32, [64, 2, 128])) == KDA_ERR_DTYPE
+    assert c.run(lib, fn, init=desc(0x80000, BF16, [1, 2, 128, 128])) == KDA_ERR_DTYPE
+    assert c.run(lib, fn, fin=desc(0x90000, I32, [1, 2, 128, 128])) == KDA_ERR_DTYPE
 
 
-def test_rejects_misaligned_pointers(lib):
-    for name in ("q", "k", "v", "g", "beta", "out", "init", "fin", "cu"):
-        assert _call(lib, **{name: 0x8008}) == 3, name
+@pytest.mark.parametrize("fn", ["kda_fwd", "kda_fwd_noalloc"])
+def test_rejects_bad_shapes(lib, fn):
+    c = Call()
+    assert c.run(lib, fn, k=desc(0x20000, BF16, [63, 2, 128])) == KDA_ERR_SHAPE      # T mismatch
+    assert c.run(lib, fn, v=desc(0x30000, BF16, [64, 3, 128])) == KDA_ERR_SHAPE      # H mismatch
+    assert c.run(lib, fn, g=desc(0x40000, F32, [64, 2, 64])) == KDA_ERR_SHAPE        # head dim
+    assert c.run(lib, fn, beta=desc(0x50000, F32, [64, 2, 1])) == KDA_ERR_SHAPE      # ndim
+    assert c.run(lib, fn, q=desc(0x10000, BF16, [64, 0, 128]), k=desc(0x20000, BF16, [64, 0, 128])) == KDA_ERR_SHAPE
+    assert c.run(lib, fn, init=desc(0x80000, F32, [2, 2, 128, 128])) == KDA_ERR_SHAPE  # N mismatch
+    assert c.run(lib, fn, cu=None, num_seqs=2) == KDA_ERR_SHAPE
+    assert c.run(lib, fn, num_seqs=0) == KDA_ERR_SHAPE
+    big = Call(T=1 << 31, H=1)
+    assert big.run(lib, fn) == KDA_ERR_SHAPE
 
 
-def test_wait_timeouts_rejects_null(lib):
+@pytest.mark.parametrize("fn", ["kda_fwd", "kda_fwd_noalloc"])
+def test_rejects_bad_strides(lib, fn):
+    c = Call()
+    T, H = 64, 2
+    # innermost dimension not contiguous
+    assert c.run(lib, fn, q=desc(0x10000, BF16, [T, H, 128], [H * 256, 256, 2])) == KDA_ERR_STRIDE
+    # token stride not a multiple of 16 bytes
+    assert c.run(lib, fn, k=desc(0x20000, BF16, [T, H, 128], [H * 128 + 4, 128, 1])) == KDA_ERR_STRIDE
+    assert c.run(lib, fn, g=desc(0x40000, F32, [T, H, 128], [H * 128 + 2, 128, 1])) == KDA_ERR_STRIDE
+    # zero or negative outer strides
+    assert c.run(lib, fn, v=desc(0x30000, BF16, [T, H, 128], [0, 128, 1])) == KDA_ERR_STRIDE
+    assert c.run(lib, fn, beta=desc(0x50000, F32, [T, H], [-H, 1])) == KDA_ERR_STRIDE
+    # out rows overlapping each other
+    assert c.run(lib, fn, out=desc(0x60000, BF16, [T, H, 128], [128, 64, 1])) == KDA_ERR_STRIDE
+    # non-contiguous states
+    assert c.run(lib, fn, init=desc(0x80000, F32, [1, H, 128, 128], [H * 128 * 128, 128 * 128, 1, 128])) == KDA_ERR_STRIDE
+    assert c.run(lib, fn, fin=desc(0x90000, F32, [1, H, 128, 128], [H * 128 * 256, 128 * 256, 256, 1])) == KDA_ERR_STRIDE
+
+
+@pytest.mark.parametrize("fn", ["kda_fwd", "kda_fwd_noalloc"])
+def test_rejects_misaligned_pointers(lib, fn):
+    c = Call()
+    for name, dt, shape in (("q", BF16, [64, 2, 128]), ("k", BF16, [64, 2, 128]), ("v", BF16, [64, 2, 128]),
+                            ("g", F32, [64, 2, 128]), ("beta", F32, [64, 2]), ("out", BF16, [64, 2, 128]),
+                            ("init", F32, [1, 2, 128, 128]), ("fin", F32, [1, 2, 128, 128])):
+        assert c.run(lib, fn, **{name: desc(0xA0008, dt, shape)}) == KDA_ERR_ALIGN, name
+    assert c.run(lib, fn, cu=0xB0008) == KDA_ERR_ALIGN
+
+
+def test_empty_batch_may_have_null_token_pointers(lib):
+    # T = 0: the token tensors are never read or written, so NULL data is fine;
+    # the call then stops at the misaligned initial state
+    c = Call(T=0)
+    z = {n: desc(None, c.t[n].dtype, [0] + list(c.t[n].shape[1:c.t[n].ndim])) for n in ("q", "k", "v", "g", "beta", "out")}
+    assert c.run(lib, init=desc(0xA0008, F32, [1, 2, 128, 128]), **z) == KDA_ERR_ALIGN
+
+
+def test_noalloc_capacity_rejected_before_any_gpu_work(lib):
+    H = 32 // 2 + 1  # two sequences: 34 (sequence, head) pairs > 32
+    c = Call(T=64, H=H, N=2)
+    assert c.run(lib, "kda_fwd_noalloc") == KDA_ERR_CAPACITY
+
+
+def test_strided_views_pass_validation():
+    """q, k, v as slices of one fused [T, H, 3 * 128] projection and beta as a
+    column of a wider matrix are accepted (checked on a host without a GPU,
+    where the call stops at the device query after validation)."""
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("validation-only check; needs a host without a GPU")
+    import importlib.util
+
+    spec = importlib.util.spec_from_file_location(
+        "kda_build", os.path.join(ROOT, "kimi_delta_attention_26_b200", "build.py"))
+    build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(build)
+    lib = ctypes.CDLL(build.build())
+    P = ctypes.POINTER(Desc)
+    lib.kda_fwd.argtypes = [P, P, P, P, P, ctypes.c_float, ctypes.c_void_p, ctypes.c_int32, P, P, P, ctypes.c_void_p]
+    lib.kda_fwd.restype = ctypes.c_int
+    T, H = 64, 2
+    c = Call(T, H)
+    fused = [H * 384, 384, 1]
+    rc = c.run(lib, q=desc(0x100000, BF16, [T, H, 128], fused), k=desc(0x100100, BF16, [T, H, 128], fused),
+               v=desc(0x100200, BF16, [T, H, 128], fused), beta=desc(0x50000, F32, [T, H], [4 * H, 4]),
+               out=desc(0x60000, BF16, [T, H, 128], [128, T * 128, 1]))   # head-major output
+    assert rc == KDA_ERR_CUDA  # validation passed; no device to run on
+
+
+def test_device_status_and_wait_counter_reject_null(lib):
     lib.kda_wait_timeouts.argtypes = [ctypes.c_void_p, ctypes.c_int32]
     lib.kda_wait_timeouts.restype = ctypes.c_int
-    assert lib.kda_wait_timeouts(None, 0) == 1
+    lib.kda_device_status.argtypes = [ctypes.c_void_p, ctypes.c_int32]
+    lib.kda_device_status.restype = ctypes.c_int
+    assert lib.kda_wait_timeouts(None, 0) == KDA_ERR_NULL
+    assert lib.kda_device_status(None, 0) == KDA_ERR_NULL

@@ -1,8 +1,11 @@
-"""GPU parity: the CUDA path against the fp64 oracle on the same seeded inputs.
+"""GPU parity: the CUDA paths against the fp64 oracle on the same seeded inputs.
 
 All calls go through the C ABI (``libkda.so``) via the thin Python binding.
 Bars: o max-abs <= 3e-2 and rel-RMS <= 5e-3; final state rel-RMS <= 5e-3;
 segment handling bit-exact (a sequence gives the same bits alone or packed).
+
+Every behaviour test runs on each kernel variant: the 16-token path with 32-
+and 16-column value slices per CTA, and the 64-token tcgen05 path.
 """
 import numpy as np
 import pytest
@@ -11,6 +14,8 @@ import kda_inputs
 from tests import helpers as H
 
 pytestmark = pytest.mark.gpu
+
+VARIANTS = {"p16s32": (16, 32), "p16s16": (16, 16), "p64": (64, 0)}
 
 
 @pytest.fixture(scope="module")
@@ -24,40 +29,51 @@ def kda():
     return m
 
 
-@pytest.fixture(params=[16, 32], ids=["slice16", "slice32"])
-def slice_cols(request, kda):
-    """Both kernel variants (16- and 32-column value slices per CTA); the
-    automatic choice is restored afterwards."""
-    kda.set_slice_columns(request.param)
+@pytest.fixture(params=list(VARIANTS), ids=list(VARIANTS))
+def variant(request, kda):
+    """One kernel variant for the test; the library defaults are restored after."""
+    path, cols = VARIANTS[request.param]
+    kda.set_path(path)
+    kda.set_slice_columns(cols)
     yield request.param
+    kda.set_path(0)
     kda.set_slice_columns(0)
 
 
-def _check(oracle_mod, inp, label, cols=None, **kw):
+@pytest.fixture(params=[16, 64], ids=["p16", "p64"])
+def path(request, kda):
+    kda.set_path(request.param)
+    yield request.param
+    kda.set_path(0)
+
+
+def _check(oracle_mod, inp, label, col_ranges=None, **kw):
     out, fin = H.run_gpu(inp, **kw)
-    if cols is None:
+    if col_ranges is None:
         o_ref, f_ref = oracle_mod.scan_inputs(inp)
         return H.assert_parity(out, fin, o_ref, f_ref, label=label)
-    o_ref, f_ref = oracle_mod.scan_inputs(inp, col_begin=cols.start, col_end=cols.stop)
-    return H.assert_parity(out, fin, o_ref, f_ref, cols=cols, label=label)
+    res = None
+    for a, b in col_ranges:
+        o_ref, f_ref = oracle_mod.scan_inputs(inp, col_begin=a, col_end=b)
+        res = H.assert_parity(out, fin, o_ref, f_ref, cols=slice(a, b), label=f"{label} cols {a}-{b}")
+    return res
 
 
-def test_tiny_config(kda, oracle_mod, slice_cols):
+def test_tiny_config(kda, oracle_mod, variant):
     inp = kda_inputs.workload(1).make()
-    mo, ms = _check(oracle_mod, inp, "tiny T=256 H=2")
-    print("tiny", mo, ms)
+    _check(oracle_mod, inp, f"tiny T=256 H=2 [{variant}]")
 
 
 @pytest.mark.parametrize("seed", [0, 1])
-def test_ragged_varlen_small(kda, oracle_mod, seed, slice_cols):
-    # lengths around the 16-token anchor blocks and 64-token chunks, an empty
-    # sequence, several chunks, random initial states
+def test_ragged_varlen_small(kda, oracle_mod, seed, variant):
+    # lengths around the 16- and 64-token chunks, an empty sequence, several
+    # chunks, random initial states
     lens = [1, 15, 16, 17, 63, 64, 65, 200, 0, 129, 300]
     inp = kda_inputs.make_inputs(lens, 3, seed=50 + seed, random_initial_state=True)
-    _check(oracle_mod, inp, f"ragged seed={seed}")
+    _check(oracle_mod, inp, f"ragged seed={seed} [{variant}]")
 
 
-def test_zero_initial_state_null_equals_zeros(kda):
+def test_zero_initial_state_null_equals_zeros(kda, path):
     import torch
 
     inp = kda_inputs.make_inputs([100, 37], 2, seed=3)
@@ -67,41 +83,41 @@ def test_zero_initial_state_null_equals_zeros(kda):
     assert torch.equal(out_a, out_b) and torch.equal(fin_a, fin_b)
 
 
-def test_gate_extremes(kda, oracle_mod, slice_cols):
+def test_gate_extremes(kda, oracle_mod, variant):
     # g at the lower bound everywhere (fastest decay) and g = 0 (no decay)
     for fill in (-5.0, 0.0):
         inp = kda_inputs.make_inputs([150, 70], 2, seed=8, random_initial_state=True)
         inp.g[:] = fill
-        _check(oracle_mod, inp, f"g={fill}")
+        _check(oracle_mod, inp, f"g={fill} [{variant}]")
 
 
-def test_beta_zero_reads_only_the_decayed_initial_state(kda, oracle_mod, slice_cols):
+def test_beta_zero_reads_only_the_decayed_initial_state(kda, oracle_mod, variant):
     # beta = 0: no token writes, so o_t = scale (q_t * exp G_t)^T S_0 and the
     # final state is Diag(exp G_T) S_0 (checked against the oracle's scan)
     inp = kda_inputs.make_inputs([90, 33], 2, seed=19, random_initial_state=True)
     inp.beta[:] = 0.0
-    _check(oracle_mod, inp, "beta=0")
+    _check(oracle_mod, inp, f"beta=0 [{variant}]")
 
 
-def test_chunk_boundary_lengths_with_empty_sequences(kda, oracle_mod, slice_cols):
-    # every length around 16-token chunk boundaries, empty sequences between
-    lens = [15, 0, 16, 17, 0, 0, 31, 32, 33, 47, 48, 49, 0]
+def test_chunk_boundary_lengths_with_empty_sequences(kda, oracle_mod, variant):
+    # every length around 16- and 64-token chunk boundaries, empty sequences between
+    lens = [15, 0, 16, 17, 0, 0, 31, 32, 33, 47, 48, 49, 63, 64, 65, 127, 128, 129, 0]
     inp = kda_inputs.make_inputs(lens, 2, seed=21, random_initial_state=True)
-    _check(oracle_mod, inp, "chunk-boundary lengths")
+    _check(oracle_mod, inp, f"chunk-boundary lengths [{variant}]")
 
 
-def test_single_token_and_all_empty(kda, oracle_mod, slice_cols):
+def test_single_token_and_all_empty(kda, oracle_mod, variant):
     import torch
 
     inp = kda_inputs.make_inputs([1], 4, seed=9, random_initial_state=True)
-    _check(oracle_mod, inp, "T=1")
+    _check(oracle_mod, inp, f"T=1 [{variant}]")
     inp = kda_inputs.make_inputs([0, 0, 0], 2, seed=10, random_initial_state=True)
     out, fin = H.run_gpu(inp)
     assert out.numel() == 0
     assert torch.equal(fin.cpu(), torch.from_numpy(inp.initial_state))
 
 
-def test_segments_bit_exact(kda, slice_cols):
+def test_segments_bit_exact(kda, variant):
     """A packed batch restricted to one sequence equals that sequence run alone, bitwise."""
     import torch
 
@@ -120,7 +136,7 @@ def test_segments_bit_exact(kda, slice_cols):
         assert torch.equal(fin[i], f_i[0]), f"segment {i}: state bits differ"
 
 
-def test_no_cu_seqlens_equals_single_sequence(kda):
+def test_no_cu_seqlens_equals_single_sequence(kda, path):
     import torch
 
     inp = kda_inputs.make_inputs([333], 2, seed=12, random_initial_state=True)
@@ -131,7 +147,7 @@ def test_no_cu_seqlens_equals_single_sequence(kda):
 
 
 @pytest.mark.parametrize("t1", [64, 100])
-def test_resume_from_final_state(kda, oracle_mod, t1, slice_cols):
+def test_resume_from_final_state(kda, oracle_mod, t1, variant):
     import torch
 
     inp = kda_inputs.make_inputs([257], 2, seed=13, random_initial_state=True)
@@ -143,14 +159,14 @@ def test_resume_from_final_state(kda, oracle_mod, t1, slice_cols):
                            d["g"][t1:].contiguous(), d["beta"][t1:].contiguous(), inp.scale, None, a_f)
     torch.cuda.synchronize()
     o_ref, f_ref = oracle_mod.scan_inputs(inp)
-    H.assert_parity(torch.cat([a_o, b_o]), b_f, o_ref, f_ref, label=f"resume t1={t1}")
+    H.assert_parity(torch.cat([a_o, b_o]), b_f, o_ref, f_ref, label=f"resume t1={t1} [{variant}]")
     if t1 % 64 == 0:
         # splitting on a chunk boundary changes nothing but the state's fp32 round trip
         assert torch.equal(torch.cat([a_o, b_o]), full_o)
         assert torch.equal(b_f, full_f)
 
 
-def test_in_place_state_update(kda, slice_cols):
+def test_in_place_state_update(kda, variant):
     import torch
 
     inp = kda_inputs.make_inputs([90, 10], 2, seed=14, random_initial_state=True)
@@ -163,7 +179,7 @@ def test_in_place_state_update(kda, slice_cols):
     assert torch.equal(o1, o2) and torch.equal(f1, st)
 
 
-def test_deterministic(kda):
+def test_deterministic(kda, path):
     import torch
 
     inp = kda_inputs.make_inputs([500, 3, 260], 4, seed=15, random_initial_state=True)
@@ -172,7 +188,7 @@ def test_deterministic(kda):
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
-def test_no_writes_outside_outputs(kda, slice_cols):
+def test_no_writes_outside_outputs(kda, variant):
     """Guard regions around out and final_state keep their sentinel values."""
     import torch
 
@@ -191,30 +207,88 @@ def test_no_writes_outside_outputs(kda, slice_cols):
         assert bool((buf[:guard] == 7.0).all()) and bool((buf[-guard:] == 7.0).all())
 
 
+def test_strided_views_bitwise_equal_contiguous(kda, path):
+    """q, k, v as slices of one fused [T, H, 384] projection, beta as a column
+    of a wider matrix and a head-major output give the same bits as
+    contiguous tensors."""
+    import torch
+
+    inp = kda_inputs.make_inputs([200, 65], 3, seed=23, random_initial_state=True)
+    d = H.to_device(inp)
+    ref_o, ref_f = kda.kda_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], inp.scale, d["cu_seqlens"],
+                               d["initial_state"])
+    T, nh = inp.total_tokens, inp.num_heads
+    fused = torch.cat([d["q"], d["k"], d["v"]], dim=2)               # [T, H, 384]
+    bwide = torch.zeros((T, nh, 4), dtype=torch.float32, device="cuda")
+    bwide[:, :, 2] = d["beta"]
+    out_hm = torch.empty((nh, T, 128), dtype=torch.bfloat16, device="cuda").transpose(0, 1)  # head-major
+    o, f = kda.kda_fwd(fused[:, :, :128], fused[:, :, 128:256], fused[:, :, 256:], d["g"], bwide[:, :, 2],
+                       inp.scale, d["cu_seqlens"], d["initial_state"], out=out_hm)
+    torch.cuda.synchronize()
+    assert torch.equal(o, ref_o) and torch.equal(f, ref_f)
+
+
+def test_paths_agree(kda):
+    """The two kernels round differently but agree within the parity bar."""
+    inp = kda_inputs.make_inputs([700, 129, 64, 3], 3, seed=24, random_initial_state=True)
+    res = {}
+    for p in (16, 64):
+        kda.set_path(p)
+        res[p] = H.run_gpu(inp)
+    kda.set_path(0)
+    o16, f16 = (x.float().cpu().numpy().astype(np.float64) for x in res[16])
+    o64, f64 = (x.float().cpu().numpy().astype(np.float64) for x in res[64])
+    mo, ms = H.metrics(o64, o16), H.metrics(f64, f16)
+    assert mo["max_abs"] <= H.O_MAX_ABS and mo["rel_rms"] <= 2 * H.O_REL_RMS, mo
+    assert ms["rel_rms"] <= 2 * H.S_REL_RMS, ms
+
+
+def test_bad_cu_seqlens_is_recorded(kda, path):
+    """A cu_seqlens that is not a non-decreasing partition of [0, T) is
+    clamped by the kernel (no access outside the tensors) and recorded in the
+    device status word."""
+    import torch
+
+    kda.device_status(reset=True)
+    inp = kda_inputs.make_inputs([40, 60], 2, seed=25, random_initial_state=True)
+    d = H.to_device(inp)
+    for bad in ([0, 60, 40], [0, 40, 90], [8, 40, 100]):  # decreasing; past T; not starting at 0
+        cu = torch.tensor(bad, dtype=torch.int32, device="cuda")
+        kda.kda_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], inp.scale, cu, d["initial_state"])
+        torch.cuda.synchronize()
+        assert kda.device_status(reset=True) & 1, bad
+    kda.kda_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], inp.scale, d["cu_seqlens"], d["initial_state"])
+    assert kda.device_status(reset=True) == 0
+
+
 # --------------------------------------------------------------- full sizes
 # The five workloads at their full sizes, in the launch configuration the
 # bench times; the oracle computes a sample of value columns (columns evolve
-# independently, so a column subset is exact) for every token and head.
+# independently, so a column subset is exact) for every token and head. The
+# sample has 8 columns in each 32-column slice, so every CTA of a cluster
+# (16-token path) is checked.
+FULL_COLS = [(8, 16), (40, 48), (72, 80), (104, 112)]
+
+
 @pytest.mark.parametrize("cfg", [2, 3, 4, 5])
-def test_full_size_workloads_sampled_columns(kda, oracle_mod, cfg):
-    # the automatic variant choice: 32-column slices for configs 2-4, 16 for 5
+def test_full_size_workloads_sampled_columns(kda, oracle_mod, cfg, path):
     inp = kda_inputs.workload(cfg).make()
-    cols = slice(40, 56) if cfg != 5 else slice(100, 108)
-    mo, ms = _check(oracle_mod, inp, f"config {cfg}", cols=cols)
-    print(f"config {cfg}", mo, ms)
+    _check(oracle_mod, inp, f"config {cfg} [p{path}]", col_ranges=FULL_COLS)
 
 
 def test_slice_variants_bitwise_equal(kda):
     """Each column's arithmetic does not depend on how many columns a CTA
-    holds, so the two variants give the same bits."""
+    holds, so the two 16-token variants give the same bits."""
     import torch
 
     inp = kda_inputs.make_inputs([700, 129, 64], 3, seed=17, random_initial_state=True)
     res = {}
+    kda.set_path(16)
     for cols in (16, 32):
         kda.set_slice_columns(cols)
         res[cols] = H.run_gpu(inp)
     kda.set_slice_columns(0)
+    kda.set_path(0)
     o16, f16 = res[16]
     o32, f32 = res[32]
     assert torch.equal(o16, o32) and torch.equal(f16, f32)
