@@ -113,10 +113,11 @@ typedef struct kda_tensor {
  *   example q, k, v as slices of one [T, H, 3 * 128] tensor) work without a
  *   copy. out must not overlap itself (token and head strides nest). beta may
  *   have any positive strides. States must be contiguous.
- * Alignment: every data pointer must be 16-byte aligned.
+ * Alignment: every data pointer must be 16-byte aligned, except beta's (4 bytes).
  * Zero-length sequences are allowed: their final state equals their initial
  * state (or zeros). T = 0 is allowed; then the token tensors' data pointers
- * may be NULL (they are never read or written).
+ * may be NULL and their strides are not checked (they are never read or
+ * written).
  * Errors: KDA_ERR_NULL (a required descriptor or pointer missing),
  * KDA_ERR_DTYPE, KDA_ERR_SHAPE, KDA_ERR_STRIDE, KDA_ERR_ALIGN,
  * KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA; nothing is enqueued on any error.

@@ -43,6 +43,10 @@ kda_status_t view_tokens(const kda_tensor_t* t, kda_dtype_t dt, int64_t T, int64
   if (t->ndim != (inner ? 3 : 2)) return KDA_ERR_SHAPE;
   if (t->shape[0] != T || t->shape[1] != H || (inner && t->shape[2] != KDA_HEAD_DIM)) return KDA_ERR_SHAPE;
   const int64_t st = t->stride[0], sh = t->stride[1];
+  res->data = t->data;
+  res->st = st;
+  res->sh = sh;
+  if (T == 0) return KDA_OK;  // no element is ever read or written: layout is irrelevant
   if (st <= 0 || sh <= 0) return KDA_ERR_STRIDE;
   if (inner) {
     const int64_t unit = 16 / elem_bytes(dt);  // 16-byte multiples (tensor-map strides, vector stores)
@@ -55,13 +59,9 @@ kda_status_t view_tokens(const kda_tensor_t* t, kda_dtype_t dt, int64_t T, int64
       if (!nest_h && !nest_t) return KDA_ERR_STRIDE;
     }
   }
-  if (T > 0) {
-    if (!t->data) return KDA_ERR_NULL;
-    if (!aligned16(t->data)) return KDA_ERR_ALIGN;
-  }
-  res->data = t->data;
-  res->st = st;
-  res->sh = sh;
+  if (!t->data) return KDA_ERR_NULL;
+  // tensor-map bases and vector accesses need 16 bytes; beta is read 4 bytes at a time
+  if (inner ? !aligned16(t->data) : (reinterpret_cast<uintptr_t>(t->data) & 3u) != 0) return KDA_ERR_ALIGN;
   return KDA_OK;
 }
 

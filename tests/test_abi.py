@@ -187,9 +187,11 @@ def test_rejects_bad_strides(lib, fn):
 def test_rejects_misaligned_pointers(lib, fn):
     c = Call()
     for name, dt, shape in (("q", BF16, [64, 2, 128]), ("k", BF16, [64, 2, 128]), ("v", BF16, [64, 2, 128]),
-                            ("g", F32, [64, 2, 128]), ("beta", F32, [64, 2]), ("out", BF16, [64, 2, 128]),
+                            ("g", F32, [64, 2, 128]), ("out", BF16, [64, 2, 128]),
                             ("init", F32, [1, 2, 128, 128]), ("fin", F32, [1, 2, 128, 128])):
         assert c.run(lib, fn, **{name: desc(0xA0008, dt, shape)}) == KDA_ERR_ALIGN, name
+    # beta is read 4 bytes at a time: 4-byte alignment suffices
+    assert c.run(lib, fn, beta=desc(0xA0002, F32, [64, 2])) == KDA_ERR_ALIGN
     assert c.run(lib, fn, cu=0xB0008) == KDA_ERR_ALIGN
 
 
