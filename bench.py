@@ -315,6 +315,96 @@ def run_reference(args):
     return 0
 
 
+
+def hide_host_latency(stream, cycles: int = 400_000):
+    """Keep the device busy (~0.2 ms) while the host prepares the next launch,
+    so that the start event and the kernel run back to back on the device:
+    the timed interval then holds device time only, not the binding's host
+    work between the two enqueues."""
+    import torch
+
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(cycles)
+
+
+def roofline_fields(inp, ms: float, with_init: bool, wl_name: str):
+    """Throughput and roofline figures of one launch of `ms` milliseconds."""
+    hbm_peak, tc_peak, peak_kind = measured_peaks()
+    units = work_units(inp)
+    bytes_launch = algorithmic_bytes(inp, with_init, True)
+    flops_launch = units * FLOPS_PER_TOKHEAD
+    gbs = bytes_launch / (ms * 1e-3) / 1e9
+    tflops = flops_launch / (ms * 1e-3) / 1e12
+    t_hbm = bytes_launch / (hbm_peak * 1e9)
+    t_tc = flops_launch / (tc_peak * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    roof = {"bound": bound,
+            "achieved": gbs if bound == "hbm" else tflops,
+            "peak": hbm_peak if bound == "hbm" else tc_peak,
+            "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+            "peak_source": f"{peak_kind} ({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'recipe fallback'})",
+            "traffic": recorded_traffic(wl_name),
+            "algorithmic_bytes_per_launch": bytes_launch,
+            "tflops_counted": tflops}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    return roof
+
+
+def time_launches(launch, steps: int, warmup: int, stream, flush, dev):
+    """Per-launch device times (ms) of `steps` launches on `stream`, after
+    `warmup` untimed ones, with an L2 flush before each timed launch."""
+    import torch
+
+    for _ in range(warmup):
+        launch()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        if flush is not None:
+            flush.add_(1.0)
+        hide_host_latency(stream)
+        ev[i][0].record(stream)
+        launch()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def per_config_table(kda, dev, stream, steps: int, paths):
+    """Every workload, each kernel path: device time per launch (inputs
+    resident, L2 flushed between launches) and the roofline figures."""
+    import torch
+
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    table = {}
+    for cfg in sorted(kda_inputs.WORKLOADS):
+        wl = kda_inputs.workload(cfg)
+        inp = wl.make()
+        t = lambda a: torch.from_numpy(a).to(dev)
+        q, k, v = (t(x).view(torch.bfloat16) for x in (inp.q, inp.k, inp.v))
+        g, beta, cu = t(inp.g), t(inp.beta), t(inp.cu_seqlens)
+        init = None if inp.initial_state is None else t(inp.initial_state)
+        out = torch.empty_like(q)
+        fin = torch.empty((inp.num_seqs, inp.num_heads, D, D), dtype=torch.float32, device=dev)
+        row = {"workload": wl.name, "config": cfg, "tokens": inp.total_tokens, "heads": inp.num_heads}
+        for path in paths:
+            kda.set_path(path)
+            launch = lambda: kda.kda_fwd(q, k, v, g, beta, inp.scale, cu, init, out=out, final_state=fin,
+                                         stream=stream)
+            ms_l = time_launches(launch, steps, 3, stream, flush, dev)
+            ms = sum(ms_l) / len(ms_l)
+            roof = roofline_fields(inp, ms, init is not None, wl.name if path == 0 else f"{wl.name}_p{path}")
+            row[f"path{path}" if path else "default"] = {
+                "ms": ms, "value": work_units(inp) / (ms * 1e-3) / 1e6, "unit": UNIT,
+                "roofline_frac": roof["frac"], "gbs": roof["achieved"] if roof["bound"] == "hbm" else None,
+                "tflops_counted": roof["tflops_counted"], "traffic": roof["traffic"],
+                "algorithmic_bytes_per_launch": roof["algorithmic_bytes_per_launch"]}
+        kda.set_path(0)
+        table[wl.name] = row
+        del q, k, v, g, beta, cu, init, out, fin
+    return table
+
+
 # ---------------------------------------------------------------------- kda
 def run_kda(args):
     import torch
@@ -379,6 +469,7 @@ def run_kda(args):
     for i in range(args.steps):
         if flush is not None:
             flush.add_(1.0)  # evict the previous launch's working set from L2
+        hide_host_latency(stream)
         ev[i][0].record(stream)
         step()
         ev[i][1].record(stream)
@@ -421,23 +512,7 @@ def run_kda(args):
     e2e_value = total_units / (e2e_ms * 1e-3) / 1e6
 
     if rank == 0:
-        hbm_peak, tc_peak, peak_kind = measured_peaks()
-        bytes_launch = algorithmic_bytes(inp, with_init, True)
-        flops_launch = units * FLOPS_PER_TOKHEAD
-        gbs = bytes_launch / (ms * 1e-3) / 1e9
-        tflops = flops_launch / (ms * 1e-3) / 1e12
-        t_hbm = bytes_launch / (hbm_peak * 1e9)
-        t_tc = flops_launch / (tc_peak * 1e12)
-        bound = "hbm" if t_hbm >= t_tc else "tensor"
-        roof = {"bound": bound,
-                "achieved": gbs if bound == "hbm" else tflops,
-                "peak": hbm_peak if bound == "hbm" else tc_peak,
-                "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
-                "peak_source": f"{peak_kind} ({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'recipe fallback'})",
-                "traffic": recorded_traffic(wl.name),
-                "algorithmic_bytes_per_launch": bytes_launch,
-                "tflops_counted": tflops}
-        roof["frac"] = roof["achieved"] / roof["peak"]
+        roof = roofline_fields(inp, ms, with_init, wl.name)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -452,6 +527,8 @@ def run_kda(args):
         }
         if ws == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(inp, args.cpu_seconds)
+        if ws == 1 and not args.no_per_config:
+            line["per_config"] = per_config_table(kda, dev, stream, min(args.steps, 20), (0, 64))
         print(json.dumps(line), flush=True)
     if ws > 1:
         dist.barrier()
@@ -468,6 +545,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per-workload table (every workload, both kernel paths)")
     ap.add_argument("--path", type=int, default=0, choices=[0, 16, 64],
                     help="kernel: 0 = library default (64-token chunks on tcgen05), 16 = 16-token chunks on mma.sync")
     args = ap.parse_args(argv)

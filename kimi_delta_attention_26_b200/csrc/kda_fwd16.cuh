@@ -31,7 +31,8 @@
 //     8     notify: (consumer) relays each landed stage to the chain warps
 //                   through hardware named barriers and returns the ring slot
 //                   to its producer.
-//     9     idle.
+//     9     bounds: records a cu_seqlens that is not a partition of [0, T)
+//                   in the device status word (rank 0 of head 0's clusters).
 //
 // Per chunk of C = 16 tokens, with Gamma_i the inclusive cumulative log-decay
 // inside the chunk (e_i = exp(g_i) per channel):
@@ -74,7 +75,7 @@ constexpr int CSTAGE = 6;         // consumer stages (cload -> chain)
 // Warp w issues on sub-partition w mod 4. The two chain warps get partitions 0
 // and 1 with only the light load and notify warps beside them; the gate, mma
 // and store warps, which burst through ALU and shared-memory work, share
-// partitions 2 and 3. Warp 9 has no role (it fills the numbering).
+// partitions 2 and 3. Warp 9 only checks the sequence bounds once.
 constexpr int MAX_CHAIN = 2;      // chain warps 0 (and 1), 16 value columns each
 constexpr int NGATE = 4;          // gate warps 2, 3, 6, 7
 constexpr int WARP_PLOAD = 4;
@@ -203,7 +204,6 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
 
   int64_t t0 = 0, t1 = T;
   if (p.cu) {
-    if (tid == 0 && rank == 0 && h == 0) check_bounds(p.cu, seq, static_cast<int>(gridDim.z), T);
     t0 = p.cu[seq];
     t1 = p.cu[seq + 1];
     t0 = t0 < 0 ? 0 : (t0 > T ? T : t0);
@@ -247,6 +247,9 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
     const int cv = 16 * warp;          // first value column (slice-local)
     float sacc[16][4];
     const size_t sbase = (static_cast<size_t>(seq) * H + h) * D * D;
+    // this lane's output columns of head h; rows step by the token stride
+    __nv_bfloat16* const out_base = p.out + static_cast<int64_t>(h) * p.out_sh + dv0 + cv + 2 * tq;
+    const int64_t out_st = p.out_st;
 #pragma unroll
     for (int u = 0; u < 16; ++u)
 #pragma unroll
@@ -381,7 +384,7 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
       for (int nt = 0; nt < 2; ++nt) {
         const int tok = 8 * nt + gq;
         if (tok < m) {
-          __nv_bfloat16* dst = p.out + (cs + tok) * p.out_st + static_cast<int64_t>(h) * p.out_sh + dv0 + cv + 2 * tq;
+          __nv_bfloat16* dst = out_base + (cs + tok) * out_st;
           *reinterpret_cast<uint32_t*>(dst) = r[nt][0];
           *reinterpret_cast<uint32_t*>(dst + 8) = r[nt][1];
         }
@@ -536,11 +539,13 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
       auto announce = [&](int jj) {
         const int nn = rank + NSLICE * jj;
         // The slot's bytes were written by the bulk-copy engine and that
-        // write has completed (bulk_wait above); the proxy fence orders it
-        // before the signal. A cluster-scope *release* arrive would also wait
-        // for this SM's unrelated outstanding global stores (~1.5k cycles per
-        // arrive on this part), so the signal itself is relaxed.
+        // write has completed (bulk_wait above). The proxy fence makes them
+        // visible to this thread's generic proxy and one cluster-scope
+        // release fence orders them before every signal that follows, so the
+        // relaxed arrivals below carry them to the consumers' acquire waits
+        // (one fence per chunk rather than a release per arrival).
         fence_proxy_async_global();
+        asm volatile("fence.acq_rel.cluster;" ::: "memory");
         for (int c = 0; c < NSLICE; ++c)
           mbar_arrive_remote_relaxed(&sh.ready[nn % RING], static_cast<uint32_t>(c));
         mbar_arrive(&sh.prod_free[jj % PSTAGE]);
@@ -604,6 +609,8 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
       // the ring slot has been copied here: give it back to its producer
       if (lane == 0) mbar_arrive_remote_relaxed(&sh.slot_free[n % RING], static_cast<uint32_t>(n % NSLICE));
     }
+  } else if (warp == 9) {
+    if (lane == 0 && p.cu && rank == 0 && h == 0) check_bounds(p.cu, seq, static_cast<int>(gridDim.z), T);
   } else if (warp == WARP_CLOAD) {
     // ====================================================== consumer loads
     if (lane == 0) {
