@@ -41,8 +41,10 @@ STATE_BYTES = D * D * 4                                    # one (sequence, head
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-KERNEL_SOURCES = [os.path.join(ROOT, "kimi_delta_attention_26_b200", "csrc", f)
-                  for f in ("kda_prims.cuh", "kda_fwd16.cuh", "kda_fwd64.cuh", "kda_api.cu")]
+CSRC = os.path.join(ROOT, "kimi_delta_attention_26_b200", "csrc")
+KERNEL_SOURCES = [os.path.join(CSRC, f)
+                  for f in ("kda_prims.cuh", "kda_fwd16.cuh", "kda_fwd64.cuh", "kda_split.cuh", "kda_decode.cuh",
+                            "kda_api.cu")]
 
 
 def log(*a):
@@ -73,11 +75,13 @@ def _code_only(src: str) -> str:
     return " ".join("".join(out).split())
 
 
-def kernel_source_sha() -> str:
-    """Hash of the kernel's code (comments and layout excluded): a profile's
-    DRAM traffic applies while this matches the hash recorded with it."""
+def kernel_source_sha(names=None) -> str:
+    """Hash of the kernels' code (comments and layout excluded) over the named
+    csrc files (default: all): a profile's DRAM traffic applies while this
+    matches the hash recorded with it."""
+    paths = KERNEL_SOURCES if not names else [os.path.join(CSRC, n) for n in names]
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in paths:
         with open(p, encoding="utf-8") as f:
             h.update(_code_only(f.read()).encode())
     return h.hexdigest()
@@ -101,7 +105,9 @@ def recorded_traffic(workload_name: str):
     txt = open(p).read()
     m_b = re.search(r"traffic_bytes_per_launch\s*=\s*([0-9.eE+]+)", txt)
     m_s = re.search(r"kernel_source_sha256\s*=\s*([0-9a-f]{64})", txt)
-    if not m_b or not m_s or m_s.group(1) != kernel_source_sha():
+    m_n = re.search(r"kernel_sources\s*=\s*([\w. ]+)", txt)
+    names = m_n.group(1).split() if m_n else None
+    if not m_b or not m_s or m_s.group(1) != kernel_source_sha(names):
         return None
     return float(m_b.group(1))
 
@@ -405,6 +411,34 @@ def per_config_table(kda, dev, stream, steps: int, paths):
     return table
 
 
+def decode_entry(kda, dev, stream, steps: int):
+    """The decode step (one token for each of 256 requests, H=32, states
+    resident and updated in place): device time per launch and its HBM
+    roofline (the step reads and writes every state once)."""
+    import torch
+
+    wl = kda_inputs.DECODE
+    inp = wl.make()
+    t = lambda a: torch.from_numpy(a).to(dev)
+    q, k, v = (t(x).view(torch.bfloat16) for x in (inp.q, inp.k, inp.v))
+    g, beta, state = t(inp.g), t(inp.beta), t(inp.initial_state)
+    out = torch.empty_like(q)
+    launch = lambda: kda.kda_decode(q, k, v, g, beta, state, scale=inp.scale, out=out, stream=stream)
+    # the states (512 MiB) exceed L2, so launches need no flush between them
+    ms_l = time_launches(launch, steps, 3, stream, None, dev)
+    ms = sum(ms_l) / len(ms_l)
+    hbm_peak, _, peak_kind = measured_peaks()
+    units = work_units(inp)
+    bytes_launch = units * (BYTES_PER_TOKHEAD + 2 * STATE_BYTES)
+    gbs = bytes_launch / (ms * 1e-3) / 1e9
+    return {"workload": wl.name, "requests": inp.num_seqs, "heads": inp.num_heads, "ms": ms,
+            "value": units / (ms * 1e-3) / 1e6, "unit": UNIT,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                         "peak_source": peak_kind, "algorithmic_bytes_per_launch": bytes_launch,
+                         "traffic": recorded_traffic(wl.name)},
+            "l2": "states (512 MiB) larger than L2"}
+
+
 # ---------------------------------------------------------------------- kda
 def run_kda(args):
     import torch
@@ -529,6 +563,7 @@ def run_kda(args):
             line["cpu_baseline"] = cpu_baseline(inp, args.cpu_seconds)
         if ws == 1 and not args.no_per_config:
             line["per_config"] = per_config_table(kda, dev, stream, min(args.steps, 20), (0, 64))
+            line["decode"] = decode_entry(kda, dev, stream, min(args.steps, 20))
         print(json.dumps(line), flush=True)
     if ws > 1:
         dist.barrier()

@@ -2,7 +2,8 @@
  * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention prefill library.
  *
  * The library computes the chunked forward (prefill) of Kimi Delta Attention
- * (KDA) for head dimension dk = dv = 128 on one GPU. Per sequence and head:
+ * (KDA) for head dimension dk = dv = 128 on one GPU, and the one-token decode
+ * step against resident states. Per sequence and head:
  *
  *   S_t = (I - beta_t k_t k_t^T) Diag(exp g_t) S_{t-1} + beta_t k_t v_t^T
  *   o_t = scale * S_t^T q_t
@@ -194,6 +195,61 @@ kda_status_t kda_set_path(int32_t path);
  */
 kda_status_t kda_set_slice_columns(int32_t columns);
 
+/*
+ * kda_set_time_split -- the time-split prefill of kda_fwd (16-token path).
+ *
+ * A batch of ONE sequence (num_seqs = 1) with few heads leaves most SMs idle:
+ * each head is one serial chain. The time split runs the sequence's two
+ * halves at once: the first from the initial state, the second twice in
+ * parallel -- from the zero state, and with v = 0 from the identity, which
+ * gives the map from its (not yet known) start state to its outputs and end
+ * state -- and then combines them (o_t += S_a^T o_M(t), S_T = M S_a + B; the
+ * recurrence is linear in its initial state). It takes extra scratch from the
+ * pool (about T/2 x H x 768 bytes plus three rings and three states) and two
+ * helper streams (created once per device; the call stays ordered on
+ * `stream`). Results agree with the unsplit path within the library's
+ * accuracy bounds, not bitwise.
+ *   mode 0 (default): split when num_seqs = 1, T >= 8192 and the device holds
+ *                     all 3 * H clusters of the three launches at once;
+ *   mode 1: never;   mode 2: whenever num_seqs = 1 and T >= 32 (testing).
+ * kda_fwd_noalloc never splits. Process-wide. Returns KDA_ERR_SHAPE for any
+ * other mode (the setting is then unchanged).
+ */
+kda_status_t kda_set_time_split(int32_t mode);
+
+/*
+ * kda_decode -- one decode step for a batch of B requests: each request's
+ * per-head state advances by one token (the recurrence above with T = 1) in
+ * place, and the token's output is written.
+ *
+ * The sources describe a fixed-size state per head as what makes long-context
+ * decoding cheap (FlashKDA page, section "سياق Kimi Linear"); this is that
+ * step for states kept resident in device memory between calls (for example a
+ * serving engine's pool of request states).
+ *
+ * Tensors (B = requests, H = heads, P = state slots):
+ *   q, k, v, out   bf16  [B, H, 128]     one token per request
+ *   g              fp32  [B, H, 128]     precondition -5 <= g <= 0, as for kda_fwd
+ *   beta           fp32  [B, H]
+ *   state          fp32  [P, H, 128 (key), 128 (value)], contiguous; read and
+ *                  written in place
+ *   state_indices  int32 [B] on the device: the state slot of each request;
+ *                  or NULL, meaning slot b for request b (then P >= B).
+ *                  Slots of one call must be distinct (requests sharing a
+ *                  slot race). A slot outside [0, P) skips its request (its
+ *                  out row is not written) and sets KDA_DEVICE_BAD_STATE_INDEX
+ *                  in the device status word.
+ * Strides and alignment of the token tensors: as for kda_fwd (B in place of
+ * T). state_indices must be 4-byte aligned. B = 0 is allowed (nothing runs).
+ * Errors: KDA_ERR_NULL, KDA_ERR_DTYPE, KDA_ERR_SHAPE, KDA_ERR_STRIDE,
+ * KDA_ERR_ALIGN, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA; nothing is enqueued on any
+ * error. Allocates nothing. Returns KDA_OK once the work is enqueued.
+ */
+kda_status_t kda_decode(const kda_tensor_t* q, const kda_tensor_t* k, const kda_tensor_t* v,
+                        const kda_tensor_t* g, const kda_tensor_t* beta, float scale,
+                        const kda_tensor_t* state, const int32_t* state_indices,
+                        const kda_tensor_t* out, void* stream);
+
 /* Human-readable text of a status code (static storage, never NULL). */
 const char* kda_status_string(kda_status_t status);
 
@@ -209,12 +265,15 @@ const char* kda_last_cuda_error(void);
  *                              partition of [0, T) (those results are wrong)
  *   KDA_DEVICE_WAIT_TIMEOUT    a bounded in-kernel wait ran out of budget (the
  *                              kernel stopped early; its results are undefined)
+ *   KDA_DEVICE_BAD_STATE_INDEX kda_decode met a state index outside [0, P)
+ *                              (that request was skipped)
  * Writes the bits to *flags (synchronising with the device), clears them when
  * `reset` is non-zero, and returns KDA_ERR_DEVICE if any bit is set, else
  * KDA_OK (or KDA_ERR_NULL / KDA_ERR_CUDA).
  */
 #define KDA_DEVICE_BAD_CU_SEQLENS 1u
 #define KDA_DEVICE_WAIT_TIMEOUT 2u
+#define KDA_DEVICE_BAD_STATE_INDEX 4u
 kda_status_t kda_device_status(uint32_t* flags, int32_t reset);
 
 /*

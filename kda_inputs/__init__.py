@@ -201,5 +201,12 @@ WORKLOADS = {
 }
 
 
+# One decode step of a serving batch: 256 requests with one token each against
+# resident per-request states (random, like the prefill workloads' initial
+# states), H=32 (the Kimi-Linear-shaped head count of the prefill workloads).
+DECODE = Workload("decode_B256_H32", (1,) * 256, 32, True, seed=1006,
+                  description="decode step: 256 requests x 1 token, H=32, resident random states")
+
+
 def workload(n: int) -> Workload:
     return WORKLOADS[int(n)]

@@ -14,8 +14,8 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["kda_fwd", "library_path", "wait_timeouts", "device_status", "set_slice_columns", "set_path",
-           "describe", "KDAError", "HEAD_DIM"]
+__all__ = ["kda_fwd", "kda_decode", "library_path", "wait_timeouts", "device_status", "set_slice_columns", "set_path",
+           "set_time_split", "describe", "KDAError", "HEAD_DIM"]
 
 HEAD_DIM = 128
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -75,13 +75,17 @@ _lib.kda_set_slice_columns.argtypes = [ctypes.c_int32]
 _lib.kda_set_slice_columns.restype = ctypes.c_int
 _lib.kda_set_path.argtypes = [ctypes.c_int32]
 _lib.kda_set_path.restype = ctypes.c_int
+_lib.kda_set_time_split.argtypes = [ctypes.c_int32]
+_lib.kda_set_time_split.restype = ctypes.c_int
+_lib.kda_decode.argtypes = [_T, _T, _T, _T, _T, ctypes.c_float, _T, _P, _T, _P]
+_lib.kda_decode.restype = ctypes.c_int
 
 
 class KDAError(RuntimeError):
     def __init__(self, code: int):
         msg = _lib.kda_status_string(code).decode()
         cuda = _lib.kda_last_cuda_error().decode()
-        super().__init__(f"kda_fwd failed ({code}): {msg}" + (f" [{cuda}]" if cuda else ""))
+        super().__init__(f"KDA call failed ({code}): {msg}" + (f" [{cuda}]" if cuda else ""))
         self.code = code
 
 
@@ -115,9 +119,18 @@ def set_path(path: int) -> None:
         raise KDAError(rc)
 
 
+def set_time_split(mode: int) -> None:
+    """Time-split prefill of one long sequence (16-token path): 0 automatic
+    (default), 1 never, 2 whenever possible. Process-wide."""
+    rc = _lib.kda_set_time_split(int(mode))
+    if rc != 0:
+        raise KDAError(rc)
+
+
 def device_status(reset: bool = True) -> int:
     """The device status word (bit 0: a bad cu_seqlens was seen, bit 1: a
-    bounded in-kernel wait ran out); synchronises with the device."""
+    bounded in-kernel wait ran out, bit 2: kda_decode met a state index out of
+    range); synchronises with the device."""
     n = ctypes.c_uint32(0)
     rc = _lib.kda_device_status(ctypes.byref(n), 1 if reset else 0)
     if rc not in (0, 9):
@@ -193,3 +206,48 @@ def kda_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, 
     if rc != 0:
         raise KDAError(rc)
     return out, final_state
+
+
+def kda_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, beta: torch.Tensor,
+               state: torch.Tensor, scale: Optional[float] = None, state_indices: Optional[torch.Tensor] = None,
+               out: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """One decode step for B requests (see ``include/kda.h``): advances each
+    request's state by its token, in place, and returns the outputs.
+
+    q, k, v: bf16 [B, H, 128]; g: fp32 [B, H, 128] (log decay, in [-5, 0]);
+    beta: fp32 [B, H]; state: fp32 [P, H, 128, 128], updated in place;
+    state_indices: int32 [B] on the device (distinct slots), or None for slot b.
+    """
+    if q.dim() != 3:
+        raise ValueError("q must be [B, H, 128]")
+    B, H, d = q.shape
+    if d != HEAD_DIM:
+        raise ValueError(f"head dimension must be {HEAD_DIM}")
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("kda_decode runs on CUDA tensors only")
+    _check(q, "q", torch.bfloat16, (B, H, d), dev)
+    _check(k, "k", torch.bfloat16, (B, H, d), dev)
+    _check(v, "v", torch.bfloat16, (B, H, d), dev)
+    _check(g, "g", torch.float32, (B, H, d), dev)
+    _check(beta, "beta", torch.float32, (B, H), dev)
+    if state.dim() != 4:
+        raise ValueError("state must be [P, H, 128, 128]")
+    _check(state, "state", torch.float32, (state.shape[0], H, d, d), dev, contiguous=True)
+    if state_indices is not None:
+        _check(state_indices, "state_indices", torch.int32, (B,), dev, contiguous=True)
+    if out is None:
+        out = torch.empty((B, H, d), dtype=torch.bfloat16, device=dev)
+    _check(out, "out", torch.bfloat16, (B, H, d), dev)
+    if scale is None:
+        scale = d ** -0.5
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    descs = [describe(t) for t in (q, k, v, g, beta, state, out)]
+    ref = [x[0] for x in descs]
+    with torch.cuda.device(dev):
+        rc = _lib.kda_decode(ref[0], ref[1], ref[2], ref[3], ref[4], ctypes.c_float(scale), ref[5],
+                             _ptr(state_indices), ref[6], ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise KDAError(rc)
+    return out

@@ -3,12 +3,17 @@
 // maps, and the launch of one of the two prefill kernels:
 //   kda_fwd16.cuh  16-token chunks on mma.sync (the default path)
 //   kda_fwd64.cuh  64-token chunks on tcgen05
+// and, for one long sequence with few heads, the time-split prefill (the
+// 16-token kernel on both halves at once, combined by kda_split.cuh).
 // This file is the library's only translation unit.
 
 #include "kda_prims.cuh"
 #include "kda_fwd16.cuh"
 #include "kda_fwd64.cuh"
+#include "kda_split.cuh"
+#include "kda_decode.cuh"
 
+#include <algorithm>
 #include <atomic>
 #include <cstdio>
 #include <mutex>
@@ -161,6 +166,7 @@ constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;                      // guards first-call setup of every device
 std::atomic<int> g_device_ready[kMaxDevices];  // 0 unknown, 1 ready, -1 unsupported
 int g_num_sms[kMaxDevices];
+int g_max_clusters32[kMaxDevices];  // co-resident 4-CTA clusters of the 32-column kernel
 // Library-private stream-ordered pool for the scratch rings. It keeps freed
 // memory (release threshold = max), so steady-state calls never map memory
 // and the process's default pool is left untouched.
@@ -196,9 +202,23 @@ kda_status_t check_device(int dev) {
   if (e != cudaSuccess) return cuda_fail(e);
   if ((e = set_smem16<32>()) != cudaSuccess) return cuda_fail(e);
   if ((e = set_smem16<16>()) != cudaSuccess) return cuda_fail(e);
+  if ((e = cudaFuncSetAttribute(kda::split::split_correct_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(kda::split::SMEM_BYTES))) != cudaSuccess)
+    return cuda_fail(e);
   if ((e = cudaFuncSetAttribute(kda::c64::kda_fwd64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(kda::c64::SMEM_BYTES))) != cudaSuccess)
     return cuda_fail(e);
+  // How many clusters of the 32-column kernel the GPU holds at once: clusters
+  // are placed whole inside one GPC, so this can be below SMs / 4.
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(kda::D / 32, 1, 1);
+  cfg.blockDim = dim3(kda::NTHREADS, 1, 1);
+  cfg.dynamicSmemBytes = sizeof(kda::Shared<32>);
+  int clusters = 0;
+  if ((e = cudaOccupancyMaxActiveClusters(&clusters, kda::kda_fwd_kernel<32>, &cfg)) != cudaSuccess)
+    return cuda_fail(e);
+  g_max_clusters32[dev] = clusters;
   g_num_sms[dev] = sms;
   g_device_ready[dev].store(1, std::memory_order_release);
   return KDA_OK;
@@ -258,6 +278,8 @@ constexpr size_t kNoAllocBytes16 = static_cast<size_t>(KDA_NOALLOC_MAX_PAIRS) * 
 constexpr size_t kNoAllocBytes64 = static_cast<size_t>(KDA_NOALLOC_MAX_PAIRS) * kda::c64::RING * kda::c64::SLOT_BYTES;
 constexpr size_t kNoAllocRingBytes = kNoAllocBytes16 > kNoAllocBytes64 ? kNoAllocBytes16 : kNoAllocBytes64;
 static_assert(kda::c64::RING * kda::c64::SLOT_BYTES == KDA_RING_BYTES_PER_PAIR, "header constant");
+static_assert(kda::dec::kFlagBadIndex == KDA_DEVICE_BAD_STATE_INDEX, "header constant");
+static_assert(kda::kFlagBadCuSeqlens == KDA_DEVICE_BAD_CU_SEQLENS, "header constant");
 static __device__ __align__(256) unsigned char g_noalloc_ring[kNoAllocRingBytes];
 
 kda_status_t noalloc_setup(int dev) {
@@ -273,7 +295,8 @@ kda_status_t noalloc_setup(int dev) {
 }
 
 // --------------------------------------------------------------- launches
-kda_status_t launch16(const Problem& P, unsigned char* ring, int dev, cudaStream_t stream) {
+kda_status_t launch16(const Problem& P, unsigned char* ring, int dev, cudaStream_t stream, uint32_t mode = 0,
+                      float* outf = nullptr, int ns_forced = 0) {
   kda::Params p;
   p.q = static_cast<const __nv_bfloat16*>(P.q.data);
   p.k = static_cast<const __nv_bfloat16*>(P.k.data);
@@ -292,7 +315,10 @@ kda_status_t launch16(const Problem& P, unsigned char* ring, int dev, cudaStream
   p.out_sh = P.out.sh;
   p.H = P.num_heads;
   p.scale = P.scale;
-  const int ns = slice_columns(dev, P.num_seqs, P.num_heads);
+  p.mode = mode;
+  p.outf = outf;
+  p.outf_st = static_cast<int64_t>(P.num_heads) * kda::D;
+  const int ns = ns_forced ? ns_forced : slice_columns(dev, P.num_seqs, P.num_heads);
   kda::TensorMaps tm;
   std::memset(&tm, 0, sizeof(tm));
   if (P.T > 0) {
@@ -354,6 +380,130 @@ kda_status_t launch64(const Problem& P, unsigned char* ring, cudaStream_t stream
   return KDA_OK;
 }
 
+// ---------------------------------------------------------- time-split prefill
+std::atomic<int> g_split{0};                 // 0 automatic, 1 never, 2 whenever possible
+std::atomic<cudaStream_t> g_side[kMaxDevices][2];  // helper streams of the time split, per device
+
+// One long sequence whose (head) chains would leave most SMs idle: its two
+// halves run at once (three 16-token launches of one 4-CTA cluster per head
+// each). Automatic only where all 3 H clusters are resident together (else
+// the third launch waits for a whole wave and the split loses) and the
+// sequence is long enough to repay the combine step (measured on B200: from
+// T = 8192 the split wins for every H with 3 H resident clusters).
+bool split_applies(const Problem& P, int dev) {
+  const int mode = g_split.load();
+  if (mode == 1 || P.num_seqs != 1 || P.T < 32) return false;
+  if (mode == 2) return true;
+  return P.T >= 8192 && 3 * static_cast<int64_t>(P.num_heads) <= g_max_clusters32[dev];
+}
+
+// Tokens [t0, t0 + len) of P's single sequence.
+Problem token_range(const Problem& P, int64_t t0, int64_t len) {
+  Problem S = P;
+  auto shift = [&](TokView& t, int eb) {
+    if (t.data) t.data = static_cast<unsigned char*>(t.data) + t0 * t.st * eb;
+  };
+  shift(S.q, 2);
+  shift(S.k, 2);
+  shift(S.v, 2);
+  shift(S.g, 4);
+  shift(S.beta, 4);
+  shift(S.out, 2);
+  S.T = len;
+  S.cu = nullptr;
+  S.num_seqs = 1;
+  return S;
+}
+
+kda_status_t side_streams(int dev, cudaStream_t (&s)[2]) {
+  if (!g_side[dev][1].load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    for (int i = 0; i < 2; ++i) {
+      if (g_side[dev][i].load()) continue;
+      cudaStream_t st = nullptr;
+      const cudaError_t e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking);
+      if (e != cudaSuccess) return cuda_fail(e);
+      g_side[dev][i].store(st, std::memory_order_release);
+    }
+  }
+  s[0] = g_side[dev][0].load();
+  s[1] = g_side[dev][1].load();
+  return KDA_OK;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// First half from the initial state on `stream`; second half from zero (o_loc,
+// end state B) and, with v = 0, from the identity (o_M, end state M) on two
+// helper streams; then o = o_loc + S_a^T o_M and S_T = M S_a + B.
+kda_status_t launch16_split(const Problem& P, int dev, cudaStream_t stream) {
+  namespace sp = kda::split;
+  // The zero-start run writes fp32 outputs and runs ~6 % slower per token than
+  // the first half, so the first half takes ~51.6 % of the tokens (measured).
+  const int64_t T = P.T, Ta = (T * 33 / 64) & ~static_cast<int64_t>(kda::C - 1), T1 = T - Ta;
+  const int H = P.num_heads;
+  const size_t st_bytes = round256(static_cast<size_t>(H) * kda::D * kda::D * 4);
+  const size_t o_bytes = round256(static_cast<size_t>(T1) * H * kda::D * 4);     // o_loc, fp32
+  const size_t om_bytes = round256(static_cast<size_t>(T1) * H * kda::D * 2);    // o_M, bf16
+  const size_t ring_b = round256(static_cast<size_t>(H) * kda::RING * kda::kSlotBytes);
+  cudaStream_t side[2];
+  kda_status_t st = side_streams(dev, side);
+  if (st != KDA_OK) return st;
+  void* scratch = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(&scratch, 3 * st_bytes + o_bytes + om_bytes + 3 * ring_b,
+                                          g_pool[dev].load(), stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  unsigned char* b = static_cast<unsigned char*>(scratch);
+  float* sa = reinterpret_cast<float*>(b);
+  float* bm = reinterpret_cast<float*>(b + st_bytes);
+  float* mm = reinterpret_cast<float*>(b + 2 * st_bytes);
+  float* oloc = reinterpret_cast<float*>(b + 3 * st_bytes);
+  __nv_bfloat16* om = reinterpret_cast<__nv_bfloat16*>(b + 3 * st_bytes + o_bytes);
+  unsigned char* rings = b + 3 * st_bytes + o_bytes + om_bytes;
+  cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};
+  for (int i = 0; i < 3 && st == KDA_OK; ++i)
+    if ((e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming)) != cudaSuccess) st = cuda_fail(e);
+  if (st == KDA_OK) {
+    Problem A = token_range(P, 0, Ta);
+    A.fin = sa;
+    Problem L = token_range(P, Ta, T1);
+    L.init = nullptr;
+    L.fin = bm;
+    L.out.data = nullptr;
+    Problem M = L;
+    M.fin = mm;
+    M.out.data = om;  // bf16 [T1, H, 128], packed
+    M.out.st = static_cast<int64_t>(H) * kda::D;
+    M.out.sh = kda::D;
+    // the helper streams start once the scratch exists, not after the first half
+    if ((e = cudaEventRecord(ev[0], stream)) != cudaSuccess) st = cuda_fail(e);
+    for (int i = 0; i < 2 && st == KDA_OK; ++i)
+      if ((e = cudaStreamWaitEvent(side[i], ev[0], 0)) != cudaSuccess) st = cuda_fail(e);
+    if (st == KDA_OK) st = launch16(A, rings, dev, stream, 0, nullptr, 32);
+    if (st == KDA_OK) st = launch16(L, rings + ring_b, dev, side[0], kda::kModeOutF32, oloc, 32);
+    if (st == KDA_OK)
+      st = launch16(M, rings + 2 * ring_b, dev, side[1], kda::kModeZeroV | kda::kModeIdentityInit, nullptr, 32);
+    for (int i = 0; i < 2 && st == KDA_OK; ++i) {
+      if ((e = cudaEventRecord(ev[1 + i], side[i])) != cudaSuccess) st = cuda_fail(e);
+      else if ((e = cudaStreamWaitEvent(stream, ev[1 + i], 0)) != cudaSuccess) st = cuda_fail(e);
+    }
+    if (st == KDA_OK) {
+      // persistent: about two CTAs per SM in all, each staging its head's S_a once
+      const int64_t tiles = (T1 + sp::TOK - 1) / sp::TOK;
+      const int64_t per_head = std::max<int64_t>(1, std::min<int64_t>(tiles, 2 * g_num_sms[dev] / H));
+      sp::split_correct_kernel<<<dim3(static_cast<unsigned>(per_head), H), sp::NTHREADS, sp::SMEM_BYTES, stream>>>(
+          oloc, om, sa, static_cast<__nv_bfloat16*>(P.out.data) + Ta * P.out.st, P.out.st, P.out.sh, T1, H);
+      if (P.fin) sp::split_state_kernel<<<dim3(kda::D / 16, H), 128, 0, stream>>>(mm, sa, bm, P.fin);
+      if ((e = cudaGetLastError()) != cudaSuccess) st = cuda_fail(e);
+    }
+  }
+  for (int i = 0; i < 3; ++i)
+    if (ev[i]) cudaEventDestroy(ev[i]);  // released once the work that records or waits on it is done
+  const cudaError_t ef = cudaFreeAsync(scratch, stream);
+  if (st == KDA_OK && ef != cudaSuccess) return cuda_fail(ef);
+  return st;
+}
+
 kda_status_t launch(const Problem& P, unsigned char* ring, int path, int dev, cudaStream_t stream) {
   return path == 16 ? launch16(P, ring, dev, stream) : launch64(P, ring, stream);
 }
@@ -382,6 +532,7 @@ kda_status_t kda_fwd(const kda_tensor_t* q, const kda_tensor_t* k, const kda_ten
   if ((st = prepare_pool(dev)) != KDA_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const int path = use_path();
+  if (path == 16 && split_applies(P, dev)) return launch16_split(P, dev, cs);
   // Ring of chunk operands, one per (sequence, head): stream-ordered scratch
   // from the library's pool, released in stream order after the kernel.
   void* ring = nullptr;
@@ -413,9 +564,64 @@ kda_status_t kda_fwd_noalloc(const kda_tensor_t* q, const kda_tensor_t* k, const
                 static_cast<cudaStream_t>(stream));
 }
 
+kda_status_t kda_decode(const kda_tensor_t* q, const kda_tensor_t* k, const kda_tensor_t* v, const kda_tensor_t* g,
+                        const kda_tensor_t* beta, float scale, const kda_tensor_t* state,
+                        const int32_t* state_indices, const kda_tensor_t* out, void* stream) {
+  g_last_cuda_error[0] = '\0';
+  if (!q || !k || !v || !g || !beta || !state || !out) return KDA_ERR_NULL;
+  if (q->ndim != 3 || state->ndim != 4) return KDA_ERR_SHAPE;
+  const int64_t B = q->shape[0], H = q->shape[1], pool = state->shape[0];
+  if (B < 0 || H < 1 || pool < 1 || H > 65535) return KDA_ERR_SHAPE;
+  if (!state_indices && pool < B) return KDA_ERR_SHAPE;
+  if (B * H > int64_t(INT32_MAX)) return KDA_ERR_SHAPE;  // one CTA per (request, head) in grid.x
+  if (pool > (int64_t(1) << 40) / (H * KDA_HEAD_DIM * KDA_HEAD_DIM)) return KDA_ERR_SHAPE;
+  TokView tq, tk, tv, tg, tb, to;
+  kda_status_t st;
+  if ((st = view_tokens(q, KDA_BF16, B, H, true, false, &tq)) != KDA_OK) return st;
+  if ((st = view_tokens(k, KDA_BF16, B, H, true, false, &tk)) != KDA_OK) return st;
+  if ((st = view_tokens(v, KDA_BF16, B, H, true, false, &tv)) != KDA_OK) return st;
+  if ((st = view_tokens(g, KDA_F32, B, H, true, false, &tg)) != KDA_OK) return st;
+  if ((st = view_tokens(beta, KDA_F32, B, H, false, false, &tb)) != KDA_OK) return st;
+  if ((st = view_tokens(out, KDA_BF16, B, H, true, true, &to)) != KDA_OK) return st;
+  if ((st = check_state(state, pool, H)) != KDA_OK) return st;
+  if (state_indices && (reinterpret_cast<uintptr_t>(state_indices) & 3u) != 0) return KDA_ERR_ALIGN;
+  int dev = 0;
+  if ((st = prologue(&dev)) != KDA_OK) return st;
+  if (B == 0) return KDA_OK;
+  kda::dec::Params p;
+  p.q = static_cast<const __nv_bfloat16*>(tq.data);
+  p.k = static_cast<const __nv_bfloat16*>(tk.data);
+  p.v = static_cast<const __nv_bfloat16*>(tv.data);
+  p.g = static_cast<const float*>(tg.data);
+  p.beta = static_cast<const float*>(tb.data);
+  p.state = static_cast<float*>(state->data);
+  p.idx = state_indices;
+  p.out = static_cast<__nv_bfloat16*>(to.data);
+  p.q_st = tq.st; p.q_sh = tq.sh;
+  p.k_st = tk.st; p.k_sh = tk.sh;
+  p.v_st = tv.st; p.v_sh = tv.sh;
+  p.g_st = tg.st; p.g_sh = tg.sh;
+  p.b_st = tb.st; p.b_sh = tb.sh;
+  p.o_st = to.st; p.o_sh = to.sh;
+  p.pool = pool;
+  p.H = static_cast<int>(H);
+  p.scale = scale;
+  kda::dec::kda_decode_kernel<<<static_cast<unsigned>(B * H), kda::dec::NTHREADS, 0,
+                                static_cast<cudaStream_t>(stream)>>>(p);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return KDA_OK;
+}
+
 kda_status_t kda_set_path(int32_t path) {
   if (path != 0 && path != 16 && path != 64) return KDA_ERR_SHAPE;
   g_path.store(path);
+  return KDA_OK;
+}
+
+kda_status_t kda_set_time_split(int32_t mode) {
+  if (mode < 0 || mode > 2) return KDA_ERR_SHAPE;
+  g_split.store(mode);
   return KDA_OK;
 }
 

@@ -173,7 +173,18 @@ struct Params {
   int64_t out_st, out_sh;    // element strides of out over tokens and heads
   int32_t H;
   float scale;
+  // Launch modes of the time-split prefill (0 for a plain call):
+  //   kModeZeroV        the value tensor reads as zero (v is not loaded);
+  //   kModeIdentityInit every (sequence, head) starts from the 128 x 128
+  //                     identity (value column c = key c), which turns the
+  //                     final state into the segment's transition map;
+  //   kModeOutF32       o is written in fp32 to outf [T, H, 128] (token
+  //                     stride outf_st) instead of bf16 to out.
+  uint32_t mode;
+  float* outf;
+  int64_t outf_st;
 };
+constexpr uint32_t kModeZeroV = 1u, kModeIdentityInit = 2u, kModeOutF32 = 4u;
 
 struct TensorMaps {
   CUtensorMap q, k, g, v;
@@ -256,7 +267,8 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
       for (int e = 0; e < 4; ++e) {
         const int key = 8 * u + 2 * tq + (e & 1);
         const int col = dv0 + cv + gq + 8 * (e >> 1);
-        sacc[u][e] = p.init ? __ldg(p.init + sbase + static_cast<size_t>(key) * D + col) : 0.f;
+        sacc[u][e] = (p.mode & kModeIdentityInit) ? (key == col ? 1.f : 0.f)
+                     : p.init ? __ldg(p.init + sbase + static_cast<size_t>(key) * D + col) : 0.f;
       }
 
     for (int n = 0; n < nch; ++n) {
@@ -286,7 +298,11 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
       float xa[2][4], xb[2][4] = {};
       {
         uint32_t vt[4];
-        ldsm_x4_t(vt, &st.v[(lane & 7) + ((lane >> 3) & 1) * 8][cv + (lane >> 4) * 8]);
+        if (p.mode & kModeZeroV) {
+          vt[0] = vt[1] = vt[2] = vt[3] = 0u;
+        } else {
+          ldsm_x4_t(vt, &st.v[(lane & 7) + ((lane >> 3) & 1) * 8][cv + (lane >> 4) * 8]);
+        }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int nt = j & 1, e0 = 2 * (j >> 1);
@@ -372,6 +388,19 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
       }
       // the stage is no longer read by this warp
       mbar_arrive_warp(&sh.c_empty[s]);
+      if (p.mode & kModeOutF32) {
+        // fp32 O: lane (gq, tq) of tile nt holds columns gq (+8) x tokens
+        // 8nt + 2tq (+1)
+        float* fbase = p.outf + static_cast<int64_t>(h) * D + dv0 + cv + gq;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int tok = 8 * nt + 2 * tq + (e & 1);
+            if (tok < m) fbase[(cs + tok) * p.outf_st + 8 * (e >> 1)] = (oa[nt][e] + ob[nt][e]) * p.scale;
+          }
+        continue;
+      }
       // ---- store O: an 8x8 transpose per tile turns (column, token pair) into
       // (token, column pair)
       uint32_t r[2][2];
@@ -623,9 +652,9 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
         mbar_wait(&sh.c_empty[s], ph ^ 1u);
         mbar_wait_cl(&sh.ready[slot], static_cast<uint32_t>(n / RING) & 1u);
         fence_proxy_async_global();
-        mbar_arrive_expect_tx(&sh.c_full[s], chain_bytes<NS>());
+        mbar_arrive_expect_tx(&sh.c_full[s], (p.mode & kModeZeroV) ? kSlotBytes : chain_bytes<NS>());
         bulk_g2s(&st.ops, ring + static_cast<size_t>(slot) * kSlotBytes, kSlotBytes, &sh.c_full[s]);
-        tma_load_3d(&st.v[0][0], &tm.v, dv0, h, tok, &sh.c_full[s]);
+        if (!(p.mode & kModeZeroV)) tma_load_3d(&st.v[0][0], &tm.v, dv0, h, tok, &sh.c_full[s]);
       }
     }
   }

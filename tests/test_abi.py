@@ -125,6 +125,12 @@ def test_path_and_slice_settings_validated(lib):
         assert lib.kda_set_path(bad) == KDA_ERR_SHAPE
     for good in (16, 64, 0):
         assert lib.kda_set_path(good) == KDA_OK
+    lib.kda_set_time_split.argtypes = [ctypes.c_int32]
+    lib.kda_set_time_split.restype = ctypes.c_int
+    for bad in (-1, 3, 16):
+        assert lib.kda_set_time_split(bad) == KDA_ERR_SHAPE
+    for good in (1, 2, 0):
+        assert lib.kda_set_time_split(good) == KDA_OK
 
 
 @pytest.mark.parametrize("fn", ["kda_fwd", "kda_fwd_noalloc"])
@@ -243,3 +249,71 @@ def test_device_status_and_wait_counter_reject_null(lib):
     lib.kda_device_status.restype = ctypes.c_int
     assert lib.kda_wait_timeouts(None, 0) == KDA_ERR_NULL
     assert lib.kda_device_status(None, 0) == KDA_ERR_NULL
+
+
+# ------------------------------------------------------------------ decode
+class DecodeCall:
+    """A valid-looking decode step (B requests, H heads, P state slots) on fake
+    16-byte-aligned addresses; tests override one argument at a time."""
+
+    def __init__(self, B=4, H=2, P=4):
+        self.B, self.H, self.P = B, H, P
+        self.t = {
+            "q": desc(0x10000, BF16, [B, H, 128]),
+            "k": desc(0x20000, BF16, [B, H, 128]),
+            "v": desc(0x30000, BF16, [B, H, 128]),
+            "g": desc(0x40000, F32, [B, H, 128]),
+            "beta": desc(0x50000, F32, [B, H]),
+            "state": desc(0x100000, F32, [P, H, 128, 128]),
+            "out": desc(0x60000, BF16, [B, H, 128]),
+        }
+        self.idx = None
+
+    def run(self, lib, **over):
+        P = ctypes.POINTER(Desc)
+        lib.kda_decode.argtypes = [P, P, P, P, P, ctypes.c_float, P, ctypes.c_void_p, P, ctypes.c_void_p]
+        lib.kda_decode.restype = ctypes.c_int
+        t = dict(self.t)
+        t.update({k: v for k, v in over.items() if k in t})
+        idx = over.get("idx", self.idx)
+        ref = {k: (None if d is None else ctypes.byref(d)) for k, d in t.items()}
+        return lib.kda_decode(ref["q"], ref["k"], ref["v"], ref["g"], ref["beta"], 1.0, ref["state"], idx,
+                              ref["out"], None)
+
+
+def test_decode_rejects_bad_arguments(lib):
+    c = DecodeCall()
+    for name in c.t:
+        assert c.run(lib, **{name: None}) == KDA_ERR_NULL, name
+    # dtypes
+    assert c.run(lib, q=desc(0x10000, F32, [4, 2, 128])) == KDA_ERR_DTYPE
+    assert c.run(lib, g=desc(0x40000, BF16, [4, 2, 128])) == KDA_ERR_DTYPE
+    assert c.run(lib, state=desc(0x100000, BF16, [4, 2, 128, 128])) == KDA_ERR_DTYPE
+    assert c.run(lib, out=desc(0x60000, F32, [4, 2, 128])) == KDA_ERR_DTYPE
+    # shapes: batch or heads disagree, head dim, state dims, too few slots without indices
+    assert c.run(lib, k=desc(0x20000, BF16, [3, 2, 128])) == KDA_ERR_SHAPE
+    assert c.run(lib, beta=desc(0x50000, F32, [4, 3])) == KDA_ERR_SHAPE
+    assert c.run(lib, v=desc(0x30000, BF16, [4, 2, 64])) == KDA_ERR_SHAPE
+    assert c.run(lib, state=desc(0x100000, F32, [4, 2, 128, 64])) == KDA_ERR_SHAPE
+    assert c.run(lib, state=desc(0x100000, F32, [4, 3, 128, 128])) == KDA_ERR_SHAPE
+    assert c.run(lib, state=desc(0x100000, F32, [3, 2, 128, 128])) == KDA_ERR_SHAPE
+    # strides: non-unit inner stride, a non-contiguous state
+    assert c.run(lib, q=desc(0x10000, BF16, [4, 2, 128], [512, 256, 2])) == KDA_ERR_STRIDE
+    assert c.run(lib, state=desc(0x100000, F32, [4, 2, 128, 128], [2 * 128 * 256, 128 * 256, 256, 1])) \
+        == KDA_ERR_STRIDE
+    # alignment: token tensors, state, indices
+    assert c.run(lib, k=desc(0x20008, BF16, [4, 2, 128])) == KDA_ERR_ALIGN
+    assert c.run(lib, state=desc(0x100004, F32, [4, 2, 128, 128])) == KDA_ERR_ALIGN
+    assert c.run(lib, idx=0x70002) == KDA_ERR_ALIGN
+
+
+def test_decode_accepts_a_small_pool_with_indices(lib):
+    """With state_indices, the pool may hold fewer slots than requests; the
+    call then passes validation (and stops at the device query without a GPU)."""
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("would launch on the fake addresses")
+    c = DecodeCall(B=4, H=2, P=2)
+    assert c.run(lib, idx=0x70000) in (KDA_ERR_CUDA, KDA_ERR_UNSUPPORTED)
+    assert c.run(lib) == KDA_ERR_SHAPE

@@ -300,3 +300,54 @@ def test_zz_no_wait_timeouts(kda):
 
     torch.cuda.synchronize()
     assert kda.wait_timeouts(reset=True) == 0
+
+
+# --------------------------------------------------------------- time split
+@pytest.fixture
+def split_on(kda):
+    """The time-split prefill forced on for one sequence (16-token path)."""
+    kda.set_path(16)
+    kda.set_time_split(2)
+    yield
+    kda.set_time_split(0)
+    kda.set_path(0)
+
+
+@pytest.mark.parametrize("T,rinit", [(64, True), (300, True), (1000, False), (4097, True)])
+def test_time_split_matches_oracle(kda, oracle_mod, split_on, T, rinit):
+    inp = kda_inputs.make_inputs([T], 3, seed=30 + T, random_initial_state=rinit)
+    _check(oracle_mod, inp, f"time split T={T} init={rinit}")
+
+
+def test_time_split_in_place_state_and_guards(kda, split_on):
+    """The split writes only out and final_state (which may alias the initial state)."""
+    import torch
+
+    inp = kda_inputs.make_inputs([777], 2, seed=31, random_initial_state=True)
+    d = H.to_device(inp)
+    ref_o, ref_f = kda.kda_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], inp.scale, None, d["initial_state"])
+    guard = 4096
+    T = inp.total_tokens
+    ob = torch.full((T * 2 * 128 + 2 * guard,), 7.0, dtype=torch.bfloat16, device="cuda")
+    out = ob[guard:guard + T * 2 * 128].view(T, 2, 128)
+    st = d["initial_state"].clone()
+    o, f = kda.kda_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], inp.scale, None, st, out=out, final_state=st)
+    torch.cuda.synchronize()
+    assert torch.equal(o, ref_o) and torch.equal(st, ref_f)
+    assert bool((ob[:guard] == 7.0).all()) and bool((ob[-guard:] == 7.0).all())
+
+
+def test_time_split_agrees_with_unsplit(kda):
+    inp = kda_inputs.make_inputs([3000], 4, seed=32, random_initial_state=True)
+    kda.set_path(16)
+    res = {}
+    for mode in (1, 2):
+        kda.set_time_split(mode)
+        res[mode] = H.run_gpu(inp)
+    kda.set_time_split(0)
+    kda.set_path(0)
+    o1, f1 = (x.float().cpu().numpy().astype(np.float64) for x in res[1])
+    o2, f2 = (x.float().cpu().numpy().astype(np.float64) for x in res[2])
+    mo, ms = H.metrics(o2, o1), H.metrics(f2, f1)
+    assert mo["max_abs"] <= H.O_MAX_ABS and mo["rel_rms"] <= 2 * H.O_REL_RMS, mo
+    assert ms["rel_rms"] <= 2 * H.S_REL_RMS, ms
