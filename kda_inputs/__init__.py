@@ -79,6 +79,13 @@ class KDAInputs:
     initial_state: Optional[np.ndarray]  # float32 [N, H, dk, dv] or None
     scale: float
     seed: int
+    # The raw draws behind q, k, g and beta (make_inputs(..., raw=True)), for
+    # the fused-preprocessing entry point: q, k before normalisation (bf16
+    # bits), the gate logits x and the beta logits (float32).
+    q_raw: Optional[np.ndarray] = None
+    k_raw: Optional[np.ndarray] = None
+    g_logit: Optional[np.ndarray] = None
+    beta_logit: Optional[np.ndarray] = None
 
     @property
     def total_tokens(self) -> int:
@@ -116,12 +123,14 @@ def _logsigmoid_f64(x: np.ndarray) -> np.ndarray:
 def make_inputs(seqlens: Sequence[int], num_heads: int, seed: int, *, dk: int = 128,
                 dv: int = 128, gate_mean: float = 3.0, gate_std: float = 1.5,
                 random_initial_state: bool = False, init_std: float = 0.1,
-                scale: Optional[float] = None, row_block: int = 1 << 20) -> KDAInputs:
+                scale: Optional[float] = None, row_block: int = 1 << 20, raw: bool = False) -> KDAInputs:
     """Draw one packed (varlen) batch.
 
     ``row_block`` bounds the float32 temporaries (tokens drawn per step); the
     values do not depend on it because each tensor's Philox stream is consumed
-    in row order.
+    in row order. ``raw`` also keeps the draws before normalisation and
+    activation (``q_raw``, ``k_raw`` rounded to bf16; ``g_logit`` and
+    ``beta_logit`` in float32); the other tensors are the same either way.
     """
     seqlens = [int(s) for s in seqlens]
     if any(s < 0 for s in seqlens):
@@ -138,21 +147,35 @@ def make_inputs(seqlens: Sequence[int], num_heads: int, seed: int, *, dk: int = 
     v = np.empty((T, H, dv), dtype=np.uint16)
     g = np.empty((T, H, dk), dtype=np.float32)
     rq, rk, rv, rg = (_rng(seed, n) for n in ("q", "k", "v", "g"))
+    if raw:
+        q_raw = np.empty((T, H, dk), dtype=np.uint16)
+        k_raw = np.empty((T, H, dk), dtype=np.uint16)
+        g_logit = np.empty((T, H, dk), dtype=np.float32)
     for t0 in range(0, T, row_block):
         t1 = min(T, t0 + row_block)
         n = t1 - t0
-        q[t0:t1] = f32_to_bf16_bits(_l2_normalise_f32(rq.standard_normal((n, H, dk), dtype=np.float32)))
-        k[t0:t1] = f32_to_bf16_bits(_l2_normalise_f32(rk.standard_normal((n, H, dk), dtype=np.float32)))
+        dq = rq.standard_normal((n, H, dk), dtype=np.float32)
+        dkk = rk.standard_normal((n, H, dk), dtype=np.float32)
+        q[t0:t1] = f32_to_bf16_bits(_l2_normalise_f32(dq))
+        k[t0:t1] = f32_to_bf16_bits(_l2_normalise_f32(dkk))
         v[t0:t1] = f32_to_bf16_bits(rv.standard_normal((n, H, dv), dtype=np.float32))
         x = rg.standard_normal((n, H, dk), dtype=np.float32).astype(np.float64) * gate_std + gate_mean
         g[t0:t1] = np.clip(_logsigmoid_f64(x), GATE_LOWER_BOUND, 0.0).astype(np.float32)
+        if raw:
+            q_raw[t0:t1] = f32_to_bf16_bits(dq)
+            k_raw[t0:t1] = f32_to_bf16_bits(dkk)
+            g_logit[t0:t1] = x.astype(np.float32)
     xb = _normal(seed, "beta", (T, H)).astype(np.float64)
     beta = (1.0 / (1.0 + np.exp(-xb))).astype(np.float32)
     init = None
     if random_initial_state:
         init = (_normal(seed, "init", (len(seqlens), H, dk, dv)) * np.float32(init_std)).astype(np.float32)
-    return KDAInputs(q=q, k=k, v=v, g=g, beta=beta, cu_seqlens=cu, initial_state=init,
-                     scale=float(scale), seed=int(seed))
+    out = KDAInputs(q=q, k=k, v=v, g=g, beta=beta, cu_seqlens=cu, initial_state=init,
+                    scale=float(scale), seed=int(seed))
+    if raw:
+        out.q_raw, out.k_raw, out.g_logit = q_raw, k_raw, g_logit
+        out.beta_logit = xb.astype(np.float32)
+    return out
 
 
 # ---------------------------------------------------------------------------

@@ -55,6 +55,8 @@ def _load():
             lib.kda_oracle_chunked_f64.restype = ctypes.c_int
             lib.kda_oracle_unit_lower_inverse.argtypes = [P, i32, P, i32]
             lib.kda_oracle_unit_lower_inverse.restype = ctypes.c_int
+            lib.kda_oracle_preprocess.argtypes = [P, P, P, P, i64, i32, i32, f64, f64, P, P, P, P]
+            lib.kda_oracle_preprocess.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -143,3 +145,31 @@ def unit_lower_inverse(L: np.ndarray, method: str = "substitution") -> np.ndarra
 def scan_inputs(inp, **kw):
     """Run the scan on a ``kda_inputs.KDAInputs`` batch."""
     return scan(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens, inp.scale, inp.initial_state, **kw)
+
+
+def preprocess(q_raw, k_raw, g_logit, beta_logit, lower_bound=-5.0, eps=1e-6):
+    """fp64 gate preprocessing (see ``kda_oracle_preprocess``): returns
+    ``(q_hat, k_hat, g, beta)`` as float64 arrays from bf16-bit q/k and fp32
+    logits."""
+    lib = _load()
+    q_raw, k_raw = _c(q_raw, np.uint16), _c(k_raw, np.uint16)
+    g_logit, beta_logit = _c(g_logit, np.float32), _c(beta_logit, np.float32)
+    T, H, dk = q_raw.shape
+    qo, ko, go = (np.empty((T, H, dk), np.float64) for _ in range(3))
+    bo = np.empty((T, H), np.float64)
+    rc = lib.kda_oracle_preprocess(_ptr(q_raw), _ptr(k_raw), _ptr(g_logit), _ptr(beta_logit), T, H, dk,
+                                   float(lower_bound), float(eps), _ptr(qo), _ptr(ko), _ptr(go), _ptr(bo))
+    if rc != 0:
+        raise ValueError(f"oracle preprocess rejected its arguments (code {rc})")
+    return qo, ko, go, bo
+
+
+def scan_raw_inputs(inp, lower_bound=-5.0, **kw):
+    """Preprocess a batch's raw tensors (``kda_inputs.make_inputs(..., raw=True)``)
+    and run the fp64 scan on the result."""
+    from kda_inputs import bf16_bits_to_f32  # input-format widening only
+
+    qh, kh, g, beta = preprocess(inp.q_raw, inp.k_raw, inp.g_logit, inp.beta_logit, lower_bound)
+    v = bf16_bits_to_f32(inp.v).astype(np.float64)
+    init = None if inp.initial_state is None else inp.initial_state.astype(np.float64)
+    return scan(qh, kh, v, g, beta, inp.cu_seqlens, inp.scale, init, **kw)

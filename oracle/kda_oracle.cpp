@@ -40,11 +40,19 @@
 //                             forward substitution or by the Neumann/doubling
 //                             product (page "Kimi K3 开源满月…", section
 //                             "KDA 内核到底难在哪": L^16 = 0 for 16x16 L).
+//   kda_oracle_preprocess  -- the gate preprocessing that precedes the
+//                             recurrence in a layer: q, k L2-normalised per
+//                             (token, head); g = max(log sigmoid(x), lower_bound)
+//                             from gate logits x (the lower bound that keeps
+//                             the decay range bounded, page "Kimi K3 开源满月…",
+//                             section "KDA 内核到底难在哪"); beta = sigmoid(b)
+//                             from logits b.
 //
 // Parity status: the scan is pinned by closed forms and invariants in
 // tests/test_oracle_pins.py; the chunked rewrite is pinned by agreement with
 // the scan. No function here is "parity unpinned".
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -403,6 +411,39 @@ int kda_oracle_unit_lower_inverse(const double* L, int32_t n, double* X, int32_t
   else
     return 2;
   std::memcpy(X, Xm.data(), sizeof(double) * n * n);
+  return 0;
+}
+
+// Gate preprocessing, fp64, elementwise except for the per-(token, head)
+// norms:
+//   q_hat = q / max(||q||_2, eps), k_hat likewise   (q, k: bf16 bit patterns [T, H, dk])
+//   g     = max(log(sigmoid(x)), lower_bound)      (x: fp32 gate logits [T, H, dk])
+//   beta  = sigmoid(b)                             (b: fp32 logits [T, H])
+// log(sigmoid(x)) is evaluated as -log1p(exp(-x)) for x >= 0 and
+// x - log1p(exp(x)) for x < 0 (no overflow for any x).
+int kda_oracle_preprocess(const uint16_t* q, const uint16_t* k, const float* x, const float* b, int64_t T,
+                          int32_t H, int32_t dk, double lower_bound, double eps, double* q_out, double* k_out,
+                          double* g_out, double* beta_out) {
+  if (!q || !k || !x || !b || !q_out || !k_out || !g_out || !beta_out || T < 0 || H < 1 || dk < 1) return 1;
+  for (int64_t t = 0; t < T; ++t)
+    for (int32_t h = 0; h < H; ++h) {
+      const size_t row = (static_cast<size_t>(t) * H + h) * dk;
+      double nq = 0.0, nk = 0.0;
+      for (int32_t c = 0; c < dk; ++c) {
+        nq += widen(q[row + c]) * widen(q[row + c]);
+        nk += widen(k[row + c]) * widen(k[row + c]);
+      }
+      const double dq = std::max(std::sqrt(nq), eps), dkn = std::max(std::sqrt(nk), eps);
+      for (int32_t c = 0; c < dk; ++c) {
+        q_out[row + c] = widen(q[row + c]) / dq;
+        k_out[row + c] = widen(k[row + c]) / dkn;
+        const double xv = widen(x[row + c]);
+        const double ls = xv >= 0.0 ? -std::log1p(std::exp(-xv)) : xv - std::log1p(std::exp(xv));
+        g_out[row + c] = std::max(ls, lower_bound);
+      }
+      const double bv = widen(b[static_cast<size_t>(t) * H + h]);
+      beta_out[static_cast<size_t>(t) * H + h] = 1.0 / (1.0 + std::exp(-bv));
+    }
   return 0;
 }
 

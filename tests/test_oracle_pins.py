@@ -23,6 +23,14 @@ P7  a packed batch equals its sequences run one by one (incl. empty and
 P8  resume: run(T1) then run(T2) from the final state equals run(T1 + T2).
 P9  the naive chunked WY rewrite equals the scan (chunk sizes 1..64, ragged
     tails); the doubling inverse equals forward substitution.
+P10 gate preprocessing (preprocess): unit norms per (token, head) over the
+    channel axis and agreement with the input generator's own float32
+    normalisation -> normalisation axis, missing square root; the exact
+    identities log sigmoid(x) - log sigmoid(-x) = x and
+    sigmoid(x) + sigmoid(-x) = 1, log sigmoid(0) = -log 2 -> sign errors,
+    wrong branch of the stable form; the lower bound clamps exactly where
+    log sigmoid falls below it; agreement with the generator's gates and
+    betas computed from the same draws.
 """
 import json
 import os
@@ -310,3 +318,72 @@ def test_inputs_generator_is_deterministic_and_shaped():
     # round-to-nearest-even on exactly representable halfway cases
     x = np.array([1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8], dtype=np.float32)
     assert list(kda_inputs.bf16_bits_to_f32(kda_inputs.f32_to_bf16_bits(x))) == [1.0, 1.0 + 2 ** -6]
+
+
+# ----------------------------------------------------------------------------- P10
+def _raw_batch(seed=40):
+    import kda_inputs
+
+    return kda_inputs.make_inputs([33, 0, 70], 3, seed=seed, raw=True, random_initial_state=True)
+
+
+def test_p10_normalisation_unit_norm_and_generator_agreement(oracle_mod):
+    import kda_inputs
+
+    inp = _raw_batch()
+    qh, kh, _, _ = oracle_mod.preprocess(inp.q_raw, inp.k_raw, inp.g_logit, inp.beta_logit)
+    for x in (qh, kh):
+        assert np.allclose(np.linalg.norm(x, axis=-1), 1.0, rtol=0, atol=1e-14)
+    # the generator normalised the unrounded float32 draws, then rounded to
+    # bf16; the oracle normalises the bf16-rounded draws in fp64. Per element
+    # the two differ by at most three bf16 roundings (the draw's, its effect on
+    # the norm, the generator's output), each at most 2^-8 relative
+    for x, ref in ((qh, inp.q), (kh, inp.k)):
+        r = kda_inputs.bf16_bits_to_f32(ref).astype(np.float64)
+        assert np.all(np.abs(x - r) <= 3 * 2.0 ** -8 * np.abs(r) + 1e-7)
+    # a zero row stays zero (the norm is floored at eps), a scaled row gives the same direction
+    qz = inp.q_raw.copy()
+    qz[0, 0, :] = 0
+    qz[1, 1, :] = kda_inputs.f32_to_bf16_bits(4.0 * kda_inputs.bf16_bits_to_f32(inp.q_raw[1, 1]))
+    qh2, _, _, _ = oracle_mod.preprocess(qz, inp.k_raw, inp.g_logit, inp.beta_logit)
+    assert np.all(qh2[0, 0] == 0.0)
+    assert np.allclose(qh2[1, 1], qh[1, 1], rtol=0, atol=1e-15)
+
+
+def test_p10_gate_identities_and_lower_bound(oracle_mod):
+    x = np.array([[[-100.0, -30.0, -5.5, -1.0, -1e-3, 0.0, 1e-3, 0.7, 3.0, 25.0, 90.0, 200.0]]], np.float32)
+    T, H, dk = x.shape
+    q = np.full((T, H, dk), 0x3F80, np.uint16)  # bf16 1.0
+    b = np.array([[-3.0]], np.float32)
+    _, _, g_pos, beta_pos = oracle_mod.preprocess(q, q, x, b, lower_bound=-1e300)
+    _, _, g_neg, beta_neg = oracle_mod.preprocess(q, q, -x, -b, lower_bound=-1e300)
+    xd = x.astype(np.float64)
+    assert np.allclose(g_pos - g_neg, xd, rtol=1e-15, atol=1e-13)          # ls(x) - ls(-x) = x
+    assert np.allclose(np.exp(g_pos) + np.exp(g_neg), 1.0, rtol=0, atol=1e-15)
+    assert g_pos[0, 0, 5] == -np.log(2.0)
+    assert np.all(g_pos <= 0.0)
+    assert abs(beta_pos[0, 0] + beta_neg[0, 0] - 1.0) < 1e-15 and beta_pos[0, 0] < 0.5
+    # the lower bound replaces exactly the values below it
+    _, _, g5, _ = oracle_mod.preprocess(q, q, x, b, lower_bound=-5.0)
+    below = g_pos < -5.0
+    assert np.all(g5[below] == -5.0) and np.all(g5[~below] == g_pos[~below])
+    assert below.sum() == 3  # x = -100, -30, -5.5
+
+
+def test_p10_gates_and_betas_agree_with_generator(oracle_mod):
+    inp = _raw_batch(41)
+    _, _, g, beta = oracle_mod.preprocess(inp.q_raw, inp.k_raw, inp.g_logit, inp.beta_logit)
+    # the generator computed from the unrounded float64 logits and rounded
+    # its results to float32; the logits here are their float32 roundings
+    assert np.max(np.abs(g - inp.g.astype(np.float64))) <= 1e-5
+    assert np.max(np.abs(beta - inp.beta.astype(np.float64))) <= 1e-6
+
+
+def test_p10_preprocessed_scan_matches_generator_scan(oracle_mod):
+    """The scan on preprocessed raw draws and the scan on the generator's
+    inputs differ only by the generator's bf16 rounding of q and k."""
+    inp = _raw_batch(42)
+    o1, f1 = oracle_mod.scan_raw_inputs(inp)
+    o2, f2 = oracle_mod.scan_inputs(inp)
+    assert np.linalg.norm(o1 - o2) / np.linalg.norm(o2) < 1e-2
+    assert np.linalg.norm(f1 - f2) / np.linalg.norm(f2) < 1e-2
