@@ -96,10 +96,11 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def recorded_traffic(workload_name: str):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source (else None)."""
-    p = os.path.join(ROOT, "profiles", f"kda_fwd_{workload_name}.md")
+def recorded_traffic(profile: str):
+    """DRAM bytes per launch from the committed ncu summary
+    profiles/<profile>.md, if it was taken on the current source of the
+    kernels it names (else None)."""
+    p = os.path.join(ROOT, "profiles", f"{profile}.md")
     if not os.path.exists(p):
         return None
     txt = open(p).read()
@@ -349,7 +350,7 @@ def roofline_fields(inp, ms: float, with_init: bool, wl_name: str):
             "peak": hbm_peak if bound == "hbm" else tc_peak,
             "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
             "peak_source": f"{peak_kind} ({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'recipe fallback'})",
-            "traffic": recorded_traffic(wl_name),
+            "traffic": recorded_traffic(f"kda_fwd_{wl_name}"),
             "algorithmic_bytes_per_launch": bytes_launch,
             "tflops_counted": tflops}
     roof["frac"] = roof["achieved"] / roof["peak"]
@@ -435,8 +436,33 @@ def decode_entry(kda, dev, stream, steps: int):
             "value": units / (ms * 1e-3) / 1e6, "unit": UNIT,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
                          "peak_source": peak_kind, "algorithmic_bytes_per_launch": bytes_launch,
-                         "traffic": recorded_traffic(wl.name)},
+                         "traffic": recorded_traffic(f"kda_decode_{wl.name}")},
             "l2": "states (512 MiB) larger than L2"}
+
+
+def fused_entry(kda, dev, stream, steps: int):
+    """kda_fwd_fused on the Kimi-Linear-shaped workload (T=8192, H=32) from
+    the raw draws (q, k unnormalised, gate and beta logits): device time per
+    launch, L2 flushed between launches, and its HBM roofline (the same
+    bytes per token and head as kda_fwd)."""
+    import torch
+
+    wl = kda_inputs.workload(2)
+    inp = wl.make(raw=True)
+    t = lambda a: torch.from_numpy(a).to(dev)
+    q, k, v = (t(x).view(torch.bfloat16) for x in (inp.q_raw, inp.k_raw, inp.v))
+    g, beta = t(inp.g_logit), t(inp.beta_logit)
+    out = torch.empty_like(q)
+    fin = torch.empty((inp.num_seqs, inp.num_heads, D, D), dtype=torch.float32, device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    launch = lambda: kda.kda_fwd_fused(q, k, v, g, beta, inp.scale, -5.0, out=out, final_state=fin, stream=stream)
+    ms_l = time_launches(launch, steps, 3, stream, flush, dev)
+    ms = sum(ms_l) / len(ms_l)
+    roof = roofline_fields(inp, ms, False, f"{wl.name}_fused")
+    return {"workload": wl.name + " (raw q/k, gate and beta logits)", "ms": ms,
+            "value": work_units(inp) / (ms * 1e-3) / 1e6, "unit": UNIT, "roofline_frac": roof["frac"],
+            "gbs": roof["achieved"], "traffic": roof["traffic"],
+            "algorithmic_bytes_per_launch": roof["algorithmic_bytes_per_launch"]}
 
 
 # ---------------------------------------------------------------------- kda
@@ -456,6 +482,13 @@ def run_kda(args):
     import kimi_delta_attention_26_b200 as kda
 
     kda.set_path(args.path)
+    if args.only_decode:
+        if rank == 0:
+            print(json.dumps(decode_entry(kda, dev, torch.cuda.current_stream(dev), args.steps)), flush=True)
+        if ws > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
     wl = kda_inputs.workload(args.config)
     inp = wl.make(seed=wl.seed + rank)  # an independent batch per rank
     with_init = inp.initial_state is not None
@@ -564,6 +597,7 @@ def run_kda(args):
         if ws == 1 and not args.no_per_config:
             line["per_config"] = per_config_table(kda, dev, stream, min(args.steps, 20), (0, 64))
             line["decode"] = decode_entry(kda, dev, stream, min(args.steps, 20))
+            line["fused_gate"] = fused_entry(kda, dev, stream, min(args.steps, 20))
         print(json.dumps(line), flush=True)
     if ws > 1:
         dist.barrier()
@@ -582,8 +616,11 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip the per-workload table (every workload, both kernel paths)")
+    ap.add_argument("--only-decode", action="store_true",
+                    help="time only the decode step (256 requests, H=32) and print its JSON object")
     ap.add_argument("--path", type=int, default=0, choices=[0, 16, 64],
-                    help="kernel: 0 = library default (64-token chunks on tcgen05), 16 = 16-token chunks on mma.sync")
+                    help="kernel: 0 = library default (16-token chunks on mma.sync, time split where it wins), "
+                         "16 = 16-token chunks, 64 = 64-token chunks on tcgen05")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         log("note: raising --warmup to 3 (minimum)")

@@ -49,7 +49,7 @@ extern "C" {
 #endif
 
 #define KDA_HEAD_DIM 128
-#define KDA_ABI_VERSION 3
+#define KDA_ABI_VERSION 4
 
 typedef enum kda_status {
   KDA_OK = 0,
@@ -63,7 +63,8 @@ typedef enum kda_status {
                               KDA_NOALLOC_MAX_PAIRS */
   KDA_ERR_DTYPE = 7,       /* a tensor has the wrong dtype */
   KDA_ERR_STRIDE = 8,      /* a tensor's strides are not supported (see kda_fwd) */
-  KDA_ERR_DEVICE = 9       /* kda_device_status: the device recorded a fault */
+  KDA_ERR_DEVICE = 9,      /* kda_device_status: the device recorded a fault */
+  KDA_ERR_VALUE = 10       /* a scalar argument is outside its range */
 } kda_status_t;
 
 typedef enum kda_dtype { KDA_BF16 = 1, KDA_F32 = 2, KDA_I32 = 3 } kda_dtype_t;
@@ -129,6 +130,32 @@ kda_status_t kda_fwd(const kda_tensor_t* q, const kda_tensor_t* k, const kda_ten
                      const int32_t* cu_seqlens, int32_t num_seqs,
                      const kda_tensor_t* initial_state, const kda_tensor_t* out,
                      const kda_tensor_t* final_state, void* stream);
+
+/*
+ * kda_fwd_fused -- kda_fwd with the gate preprocessing of a KDA layer fused
+ * into the kernel: it takes the raw tensors that precede the recurrence.
+ *
+ *   q, k   bf16 [T, H, 128]  raw projections; the kernel L2-normalises each
+ *                            (token, head) row: q / max(||q||_2, 1e-6)
+ *   g      fp32 [T, H, 128]  gate logits x; the decay is
+ *                            g = max(log sigmoid(x), lower_bound)
+ *   beta   fp32 [T, H]       logits b; the write strength is sigmoid(b)
+ *   lower_bound              in [-5, 0): the gate lower bound that keeps every
+ *                            decay factor of a chunk in range (page "Kimi K3
+ *                            开源满月…", section "KDA 内核到底难在哪", uses -5);
+ *                            else KDA_ERR_VALUE
+ * Everything else (v, states, cu_seqlens, out, layouts, strides, scratch,
+ * errors) is as for kda_fwd. The preprocessed q, k, g and beta exist only
+ * inside the kernel (fp32, then the bf16 operands of the tensor-core
+ * products); they are never written to memory. Always runs the 16-token path
+ * (kda_set_path does not apply), with the time split where kda_fwd would
+ * take it.
+ */
+kda_status_t kda_fwd_fused(const kda_tensor_t* q, const kda_tensor_t* k, const kda_tensor_t* v,
+                           const kda_tensor_t* g, const kda_tensor_t* beta, float scale, float lower_bound,
+                           const int32_t* cu_seqlens, int32_t num_seqs,
+                           const kda_tensor_t* initial_state, const kda_tensor_t* out,
+                           const kda_tensor_t* final_state, void* stream);
 
 /*
  * kda_fwd_noalloc -- kda_fwd without any device-memory allocation.

@@ -14,7 +14,7 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["kda_fwd", "kda_decode", "library_path", "wait_timeouts", "device_status", "set_slice_columns", "set_path",
+__all__ = ["kda_fwd", "kda_fwd_fused", "kda_decode", "library_path", "wait_timeouts", "device_status", "set_slice_columns", "set_path",
            "set_time_split", "describe", "KDAError", "HEAD_DIM"]
 
 HEAD_DIM = 128
@@ -77,6 +77,8 @@ _lib.kda_set_path.argtypes = [ctypes.c_int32]
 _lib.kda_set_path.restype = ctypes.c_int
 _lib.kda_set_time_split.argtypes = [ctypes.c_int32]
 _lib.kda_set_time_split.restype = ctypes.c_int
+_lib.kda_fwd_fused.argtypes = [_T, _T, _T, _T, _T, ctypes.c_float, ctypes.c_float, _P, ctypes.c_int32, _T, _T, _T, _P]
+_lib.kda_fwd_fused.restype = ctypes.c_int
 _lib.kda_decode.argtypes = [_T, _T, _T, _T, _T, ctypes.c_float, _T, _P, _T, _P]
 _lib.kda_decode.restype = ctypes.c_int
 
@@ -160,13 +162,16 @@ def kda_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, 
             scale: Optional[float] = None, cu_seqlens: Optional[torch.Tensor] = None,
             initial_state: Optional[torch.Tensor] = None, output_final_state: bool = True,
             out: Optional[torch.Tensor] = None, final_state: Optional[torch.Tensor] = None,
-            stream: Optional[torch.cuda.Stream] = None, noalloc: bool = False):
+            stream: Optional[torch.cuda.Stream] = None, noalloc: bool = False,
+            fused_lower_bound: Optional[float] = None):
     """Chunked KDA forward on packed sequences (see ``include/kda.h``).
 
     q, k, v: bf16 [T, H, 128]; g: fp32 [T, H, 128] (log decay, in [-5, 0]);
     beta: fp32 [T, H]; cu_seqlens: int32 [N + 1] on the device (None: one
     sequence); initial_state: fp32 [N, H, 128, 128] or None.
     Returns ``(out, final_state)``; ``final_state`` is None unless requested.
+    With ``fused_lower_bound`` set, calls ``kda_fwd_fused``: q and k are raw
+    projections, g and beta are logits (see ``kda_fwd_fused``).
     """
     if q.dim() != 3:
         raise ValueError("q must be [T, H, 128]")
@@ -199,13 +204,29 @@ def kda_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, 
         stream = torch.cuda.current_stream(dev)
     descs = [describe(t) for t in (q, k, v, g, beta, initial_state, out, final_state)]
     ref = [None if d is None else d[0] for d in descs]
-    fn = _lib.kda_fwd_noalloc if noalloc else _lib.kda_fwd
     with torch.cuda.device(dev):
-        rc = fn(ref[0], ref[1], ref[2], ref[3], ref[4], ctypes.c_float(scale), _ptr(cu_seqlens), N,
-                ref[5], ref[6], ref[7], ctypes.c_void_p(stream.cuda_stream))
+        if fused_lower_bound is not None:
+            if noalloc:
+                raise ValueError("the fused preprocessing has no allocation-free entry point")
+            rc = _lib.kda_fwd_fused(ref[0], ref[1], ref[2], ref[3], ref[4], ctypes.c_float(scale),
+                                    ctypes.c_float(fused_lower_bound), _ptr(cu_seqlens), N, ref[5], ref[6], ref[7],
+                                    ctypes.c_void_p(stream.cuda_stream))
+        else:
+            fn = _lib.kda_fwd_noalloc if noalloc else _lib.kda_fwd
+            rc = fn(ref[0], ref[1], ref[2], ref[3], ref[4], ctypes.c_float(scale), _ptr(cu_seqlens), N,
+                    ref[5], ref[6], ref[7], ctypes.c_void_p(stream.cuda_stream))
     if rc != 0:
         raise KDAError(rc)
     return out, final_state
+
+
+def kda_fwd_fused(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g_logit: torch.Tensor,
+                  beta_logit: torch.Tensor, scale: Optional[float] = None, lower_bound: float = -5.0, **kw):
+    """``kda_fwd`` with the gate preprocessing fused (see ``include/kda.h``):
+    q, k raw bf16 projections (L2-normalised in the kernel), g_logit fp32
+    gate logits (decay max(log sigmoid(x), lower_bound)), beta_logit fp32
+    (write strength sigmoid(b)). Other arguments as for ``kda_fwd``."""
+    return kda_fwd(q, k, v, g_logit, beta_logit, scale, fused_lower_bound=float(lower_bound), **kw)
 
 
 def kda_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, beta: torch.Tensor,

@@ -15,6 +15,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cmath>
 #include <cstdio>
 #include <mutex>
 
@@ -92,6 +93,8 @@ struct Problem {
   int32_t num_seqs, num_heads;
   int64_t T;
   float scale;
+  bool fused = false;    // kda_fwd_fused: raw q/k, gate and beta logits
+  float exp_lb = 0.f;    // exp(lower_bound) of the fused gate
 };
 
 kda_status_t check_args(const kda_tensor_t* q, const kda_tensor_t* k, const kda_tensor_t* v, const kda_tensor_t* g,
@@ -177,7 +180,10 @@ std::atomic<int> g_path{0};           // 0 (the default path), 16 or 64
 
 template <int NS>
 cudaError_t set_smem16() {
-  return cudaFuncSetAttribute(kda::kda_fwd_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(kda::kda_fwd_kernel<NS, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(sizeof(kda::Shared<NS>)));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(kda::kda_fwd_kernel<NS, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(sizeof(kda::Shared<NS>)));
 }
 
@@ -216,7 +222,7 @@ kda_status_t check_device(int dev) {
   cfg.blockDim = dim3(kda::NTHREADS, 1, 1);
   cfg.dynamicSmemBytes = sizeof(kda::Shared<32>);
   int clusters = 0;
-  if ((e = cudaOccupancyMaxActiveClusters(&clusters, kda::kda_fwd_kernel<32>, &cfg)) != cudaSuccess)
+  if ((e = cudaOccupancyMaxActiveClusters(&clusters, kda::kda_fwd_kernel<32, false>, &cfg)) != cudaSuccess)
     return cuda_fail(e);
   g_max_clusters32[dev] = clusters;
   g_num_sms[dev] = sms;
@@ -315,7 +321,8 @@ kda_status_t launch16(const Problem& P, unsigned char* ring, int dev, cudaStream
   p.out_sh = P.out.sh;
   p.H = P.num_heads;
   p.scale = P.scale;
-  p.mode = mode;
+  p.mode = mode | (P.fused ? kda::kModeFusedGate : 0u);
+  p.exp_lb = P.exp_lb;
   p.outf = outf;
   p.outf_st = static_cast<int64_t>(P.num_heads) * kda::D;
   const int ns = ns_forced ? ns_forced : slice_columns(dev, P.num_seqs, P.num_heads);
@@ -332,12 +339,15 @@ kda_status_t launch16(const Problem& P, unsigned char* ring, int dev, cudaStream
         (st = encode_3d(&tm.v, P.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.T, H, ns, kda::C, NONE)) != KDA_OK)
       return st;
   }
-  if (ns == 16) {
-    kda::kda_fwd_kernel<16><<<dim3(kda::D / 16, P.num_heads, P.num_seqs), kda::NTHREADS, sizeof(kda::Shared<16>),
-                              stream>>>(p, tm);
+  const dim3 grid16(kda::D / 16, P.num_heads, P.num_seqs), grid32(kda::D / 32, P.num_heads, P.num_seqs);
+  if (ns == 16 && P.fused) {
+    kda::kda_fwd_kernel<16, true><<<grid16, kda::NTHREADS, sizeof(kda::Shared<16>), stream>>>(p, tm);
+  } else if (ns == 16) {
+    kda::kda_fwd_kernel<16, false><<<grid16, kda::NTHREADS, sizeof(kda::Shared<16>), stream>>>(p, tm);
+  } else if (P.fused) {
+    kda::kda_fwd_kernel<32, true><<<grid32, kda::NTHREADS, sizeof(kda::Shared<32>), stream>>>(p, tm);
   } else {
-    kda::kda_fwd_kernel<32><<<dim3(kda::D / 32, P.num_heads, P.num_seqs), kda::NTHREADS, sizeof(kda::Shared<32>),
-                              stream>>>(p, tm);
+    kda::kda_fwd_kernel<32, false><<<grid32, kda::NTHREADS, sizeof(kda::Shared<32>), stream>>>(p, tm);
   }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
@@ -515,23 +525,15 @@ kda_status_t prologue(int* dev) {
   return check_device(*dev);
 }
 
-}  // namespace
-
-extern "C" {
-
-kda_status_t kda_fwd(const kda_tensor_t* q, const kda_tensor_t* k, const kda_tensor_t* v, const kda_tensor_t* g,
-                     const kda_tensor_t* beta, float scale, const int32_t* cu_seqlens, int32_t num_seqs,
-                     const kda_tensor_t* initial_state, const kda_tensor_t* out, const kda_tensor_t* final_state,
-                     void* stream) {
-  g_last_cuda_error[0] = '\0';
-  Problem P;
-  kda_status_t st = check_args(q, k, v, g, beta, scale, cu_seqlens, num_seqs, initial_state, out, final_state, &P);
-  if (st != KDA_OK) return st;
+// kda_fwd and kda_fwd_fused after validation: the time split where it
+// applies, else one launch on a ring from the pool.
+kda_status_t fwd_pooled(const Problem& P, void* stream) {
+  kda_status_t st;
   int dev = 0;
   if ((st = prologue(&dev)) != KDA_OK) return st;
   if ((st = prepare_pool(dev)) != KDA_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  const int path = use_path();
+  const int path = P.fused ? 16 : use_path();
   if (path == 16 && split_applies(P, dev)) return launch16_split(P, dev, cs);
   // Ring of chunk operands, one per (sequence, head): stream-ordered scratch
   // from the library's pool, released in stream order after the kernel.
@@ -546,6 +548,36 @@ kda_status_t kda_fwd(const kda_tensor_t* q, const kda_tensor_t* k, const kda_ten
     if (st == KDA_OK && ef != cudaSuccess) return cuda_fail(ef);
   }
   return st;
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status_t kda_fwd(const kda_tensor_t* q, const kda_tensor_t* k, const kda_tensor_t* v, const kda_tensor_t* g,
+                     const kda_tensor_t* beta, float scale, const int32_t* cu_seqlens, int32_t num_seqs,
+                     const kda_tensor_t* initial_state, const kda_tensor_t* out, const kda_tensor_t* final_state,
+                     void* stream) {
+  g_last_cuda_error[0] = '\0';
+  Problem P;
+  kda_status_t st = check_args(q, k, v, g, beta, scale, cu_seqlens, num_seqs, initial_state, out, final_state, &P);
+  if (st != KDA_OK) return st;
+  return fwd_pooled(P, stream);
+}
+
+kda_status_t kda_fwd_fused(const kda_tensor_t* q, const kda_tensor_t* k, const kda_tensor_t* v,
+                           const kda_tensor_t* g, const kda_tensor_t* beta, float scale, float lower_bound,
+                           const int32_t* cu_seqlens, int32_t num_seqs, const kda_tensor_t* initial_state,
+                           const kda_tensor_t* out, const kda_tensor_t* final_state, void* stream) {
+  g_last_cuda_error[0] = '\0';
+  // the 16-token chunks keep every decay factor within e^(16 lower_bound) >= e^-80
+  if (!(lower_bound >= -5.f && lower_bound < 0.f)) return KDA_ERR_VALUE;
+  Problem P;
+  kda_status_t st = check_args(q, k, v, g, beta, scale, cu_seqlens, num_seqs, initial_state, out, final_state, &P);
+  if (st != KDA_OK) return st;
+  P.fused = true;
+  P.exp_lb = std::exp(lower_bound);
+  return fwd_pooled(P, stream);
 }
 
 kda_status_t kda_fwd_noalloc(const kda_tensor_t* q, const kda_tensor_t* k, const kda_tensor_t* v,
@@ -643,6 +675,7 @@ const char* kda_status_string(kda_status_t s) {
     case KDA_ERR_DTYPE: return "a tensor has the wrong dtype";
     case KDA_ERR_STRIDE: return "a tensor's strides are not supported";
     case KDA_ERR_DEVICE: return "the device recorded a fault (see kda_device_status)";
+    case KDA_ERR_VALUE: return "a scalar argument is out of its range";
   }
   return "unknown status";
 }

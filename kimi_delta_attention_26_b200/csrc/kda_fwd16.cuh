@@ -145,6 +145,7 @@ struct __align__(128) Shared {
   ProdStage prod[PSTAGE];
   ChainStage<NS> cst[CSTAGE];
   float2 gprod[2][2][64];    // per-half decay products exchanged inside the gate group
+  float gnorm[2][4][16];     // fused preprocessing: per-gate-warp partial squared norms (8 q, 8 k)
   unsigned long long raw_full[PRSTAGE], raw_empty[PRSTAGE];
   unsigned long long prod_free[PSTAGE], gate_done[PSTAGE], solved[PSTAGE];
   unsigned long long c_full[CSTAGE], c_empty[CSTAGE];
@@ -180,17 +181,28 @@ struct Params {
   //                     final state into the segment's transition map;
   //   kModeOutF32       o is written in fp32 to outf [T, H, 128] (token
   //                     stride outf_st) instead of bf16 to out.
+  // Input mode of the fused preprocessing (any call; set together with the
+  // kernel instantiation FG = true, which is what implements it):
+  //   kModeFusedGate    q and k are raw projections, L2-normalised here per
+  //                     (token, head) (q / max(||q||, 1e-6)); g holds gate
+  //                     logits x, whose decay factor is exp(max(log sigmoid(x),
+  //                     lower_bound)) = max(sigmoid(x), exp_lb); beta holds
+  //                     logits b, used as sigmoid(b).
   uint32_t mode;
   float* outf;
   int64_t outf_st;
+  float exp_lb;            // exp(lower_bound), kModeFusedGate only
 };
-constexpr uint32_t kModeZeroV = 1u, kModeIdentityInit = 2u, kModeOutF32 = 4u;
+constexpr uint32_t kModeZeroV = 1u, kModeIdentityInit = 2u, kModeOutF32 = 4u, kModeFusedGate = 8u;
+constexpr float kNormEps2 = 1e-12f;  // (1e-6)^2: the norm floor of the fused normalisation, squared
 
 struct TensorMaps {
   CUtensorMap q, k, g, v;
 };
 
-template <int NS>
+// FG: the fused gate preprocessing (kModeFusedGate) is compiled in; the
+// plain kernel carries none of its code.
+template <int NS, bool FG>
 __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
     kda_fwd_kernel(const Params p, const __grid_constant__ TensorMaps tm) {
   constexpr int NSLICE = D / NS;   // CTAs per (sequence, head) = cluster size
@@ -450,6 +462,7 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
       mbar_wait(&sh.raw_full[rs], rph);
 
       // ---- raw inputs of this thread (rows past the sequence end masked)
+      constexpr bool fused = FG;
       float2 e[8], kv[8], qv[8];
 #pragma unroll
       for (int jj = 0; jj < 8; ++jj) {
@@ -458,13 +471,51 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
         const float2 gg = *reinterpret_cast<const float2*>(&rw.g[i][c0]);
         const __nv_bfloat162 kk = *reinterpret_cast<const __nv_bfloat162*>(&rw.k[i][c0]);
         const __nv_bfloat162 qq = *reinterpret_cast<const __nv_bfloat162*>(&rw.q[i][c0]);
-        e[jj] = ok ? make_float2(__expf(gg.x), __expf(gg.y)) : make_float2(1.f, 1.f);
+        float2 ee;
+        if constexpr (fused) {  // exp(max(log sigmoid(x), lb)) = max(sigmoid(x), exp(lb))
+          ee = make_float2(fmaxf(__fdividef(1.f, 1.f + __expf(-gg.x)), p.exp_lb),
+                           fmaxf(__fdividef(1.f, 1.f + __expf(-gg.y)), p.exp_lb));
+        } else {
+          ee = make_float2(__expf(gg.x), __expf(gg.y));
+        }
+        e[jj] = ok ? ee : make_float2(1.f, 1.f);
         kv[jj] = ok ? __bfloat1622float2(kk) : make_float2(0.f, 0.f);
         qv[jj] = ok ? __bfloat1622float2(qq) : make_float2(0.f, 0.f);
       }
       float bv = 0.f;
-      if (gt < C) bv = gt < m ? rw.beta[gt] : 0.f;
+      if (gt < C) {
+        const float b = rw.beta[gt];
+        bv = gt < m ? (fused ? __fdividef(1.f, 1.f + __expf(-b)) : b) : 0.f;
+      }
       mbar_arrive_warp(&sh.raw_empty[rs]);
+      // fused preprocessing: this warp's partial squared norms of its 8
+      // tokens' q and k (its 64 channels), reduced over the warp by a
+      // butterfly that halves the values each step: afterwards lane pair
+      // (l, l ^ 1) holds value 8 (l >> 4 & 1) + 4 (l >> 3 & 1) + 2 (l >> 2 & 1)
+      // + (l >> 1 & 1) of [q0..q7, k0..k7]
+      if constexpr (fused) {
+        float sv[16];
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          sv[jj] = fmaf(qv[jj].x, qv[jj].x, qv[jj].y * qv[jj].y);
+          sv[8 + jj] = fmaf(kv[jj].x, kv[jj].x, kv[jj].y * kv[jj].y);
+        }
+#pragma unroll
+        for (int w = 8, off = 16; w >= 1; w >>= 1, off >>= 1) {
+          const bool upper = (lane & off) != 0;
+#pragma unroll
+          for (int x = 0; x < w; ++x) {
+            const float send = upper ? sv[x] : sv[w + x];
+            const float got = __shfl_xor_sync(0xffffffffu, send, off);
+            sv[x] = (upper ? sv[w + x] : sv[x]) + got;
+          }
+        }
+        sv[0] += __shfl_xor_sync(0xffffffffu, sv[0], 1);
+        if ((lane & 1) == 0) {
+          const int idx = 8 * ((lane >> 4) & 1) + 4 * ((lane >> 3) & 1) + 2 * ((lane >> 2) & 1) + ((lane >> 1) & 1);
+          sh.gnorm[j & 1][gate_warp_index(warp)][idx] = sv[0];
+        }
+      }
 
       // ---- decay products: this half's total, exchanged with the other half
       float2 P = make_float2(1.f, 1.f);
@@ -478,6 +529,20 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
       if (gt < C) st.beta[gt] = bv;
       named_bar(BAR_GATE, NGATE * 32);
       const float2 Po = sh.gprod[j & 1][th ^ 1][cp];
+      if constexpr (fused) {  // full norms of this half's tokens: this warp's 64 channels + the partner warp's
+        const int wi = gate_warp_index(warp);
+        const float* a = sh.gnorm[j & 1][wi];
+        const float* b = sh.gnorm[j & 1][wi ^ 1];
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const float rq = rsqrtf(fmaxf(a[jj] + b[jj], kNormEps2));
+          const float rk = rsqrtf(fmaxf(a[8 + jj] + b[8 + jj], kNormEps2));
+          qv[jj].x *= rq;
+          qv[jj].y *= rq;
+          kv[jj].x *= rk;
+          kv[jj].y *= rk;
+        }
+      }
       // E before this half (1 for the first half), F after it (1 for the second)
       float2 E = th ? Po : make_float2(1.f, 1.f);
       float2 F = th ? make_float2(1.f, 1.f) : Po;

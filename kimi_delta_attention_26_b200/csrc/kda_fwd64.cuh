@@ -442,15 +442,28 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NTHREADS, 1)
           bulk_g2s(sm + C_KT, slot + SL_KT, 16384u, &bar.l_full);
           return true;
         };
+        // last early / late load issued, and last whose landing this warp saw
+        int ei = -1, li = -1, seen = -1;
         bool ok = load_early(0);
+        if (ok) ei = 0;
         for (int n = 0; n < nch && ok && !*abort_flag; ++n) {
           ok = load_late(n);
-          if (ok && n + 1 < nch) ok = load_early(n + 1);
+          if (ok) li = n;
+          if (ok && n + 1 < nch) {
+            ok = load_early(n + 1);
+            if (ok) ei = n + 1;
+          }
           // the slot's bytes have landed: give it back to its operand CTA
           if (ok) ok = wait_cta(&bar.e_full[n & 1], (n >> 1) & 1, abort_flag) && wait_cta(&bar.l_full, n & 1, abort_flag);
+          if (ok) seen = n;
           if (ok) mbar_arrive_remote_relaxed(&bar.slot_free[n % RING], 1u + static_cast<uint32_t>(n % NPROD));
         }
         if (!ok) *abort_flag = 1;
+        // After an abort, copies this warp issued may still be landing in
+        // shared memory. They read global memory only, so they complete: wait
+        // for each (bounded, not abortable) before the CTA may exit.
+        for (int i = seen + 1; i <= ei; ++i) mbar_wait(&bar.e_full[i & 1], (i >> 1) & 1);
+        for (int i = seen + 1; i <= li; ++i) mbar_wait(&bar.l_full, i & 1);
       }
     } else if (warp < 8) {
       // ======================================================= readout warps
@@ -573,6 +586,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NTHREADS, 1)
     float* gt = reinterpret_cast<float*>(sm + P_GT);          // [4][128] block totals
     float* bet = reinterpret_cast<float*>(sm + P_GT + 2048);  // [64] beta
     if (warp == WARP_LOAD) {
+      int issued = -1;  // last raw chunk whose loads this warp issued
       for (int j = 0; j < nmine && !*abort_flag; ++j) {
         const int c = pr + NPROD * j;
         const int64_t cs = t0 + static_cast<int64_t>(c) * CH;
@@ -580,6 +594,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NTHREADS, 1)
           *abort_flag = 1;
           break;
         }
+        issued = j;
         if (lane == 0) {
           mbar_arrive_expect_tx(&bar.raw_full, 16384u + 16384u + 32768u);
           const int tok = static_cast<int>(cs);
@@ -595,6 +610,10 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
         cp_async_arrive(&bar.raw_full);
       }
+      // the last issued chunk's copies (global reads, so they complete) have
+      // landed before the CTA may exit, also after an abort; earlier chunks'
+      // phases completed before raw_empty let the next one be issued
+      if (issued >= 0) mbar_wait(&bar.raw_full, issued & 1);
     } else if (warp == WARP_MMA) {
       if (lane == 0) {
         bool ok = true;

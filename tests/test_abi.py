@@ -16,7 +16,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 KDA_OK, KDA_ERR_NULL, KDA_ERR_SHAPE, KDA_ERR_ALIGN = 0, 1, 2, 3
 KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_CAPACITY = 4, 5, 6
-KDA_ERR_DTYPE, KDA_ERR_STRIDE, KDA_ERR_DEVICE = 7, 8, 9
+KDA_ERR_DTYPE, KDA_ERR_STRIDE, KDA_ERR_DEVICE, KDA_ERR_VALUE = 7, 8, 9, 10
 BF16, F32, I32 = 1, 2, 3
 
 
@@ -76,11 +76,11 @@ def test_exports_every_declared_symbol(lib):
 
 def test_abi_version_and_status_strings(lib):
     lib.kda_abi_version.restype = ctypes.c_int32
-    assert lib.kda_abi_version() == 3
+    assert lib.kda_abi_version() == 4
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_status_string.argtypes = [ctypes.c_int]
-    texts = {lib.kda_status_string(code) for code in range(10)}
-    assert len(texts) == 10 and b"unknown status" not in texts
+    texts = {lib.kda_status_string(code) for code in range(11)}
+    assert len(texts) == 11 and b"unknown status" not in texts
     assert lib.kda_status_string(99) == b"unknown status"
 
 
@@ -317,3 +317,26 @@ def test_decode_accepts_a_small_pool_with_indices(lib):
     c = DecodeCall(B=4, H=2, P=2)
     assert c.run(lib, idx=0x70000) in (KDA_ERR_CUDA, KDA_ERR_UNSUPPORTED)
     assert c.run(lib) == KDA_ERR_SHAPE
+
+
+# ------------------------------------------------------------ fused gate
+def test_fused_rejects_lower_bound_and_bad_tensors(lib):
+    P = ctypes.POINTER(Desc)
+    lib.kda_fwd_fused.argtypes = [P, P, P, P, P, ctypes.c_float, ctypes.c_float, ctypes.c_void_p, ctypes.c_int32,
+                                  P, P, P, ctypes.c_void_p]
+    lib.kda_fwd_fused.restype = ctypes.c_int
+    c = Call()
+
+    def run(lb, **over):
+        t = dict(c.t)
+        t.update(over)
+        ref = {k: (None if d is None else ctypes.byref(d)) for k, d in t.items()}
+        return lib.kda_fwd_fused(ref["q"], ref["k"], ref["v"], ref["g"], ref["beta"], 1.0, lb, c.cu, 1, ref["init"],
+                                 ref["out"], ref["fin"], None)
+
+    for lb in (-5.5, 0.0, 0.5, float("nan"), float("-inf")):
+        assert run(lb) == KDA_ERR_VALUE, lb
+    assert run(-5.0, q=None) == KDA_ERR_NULL
+    assert run(-5.0, g=desc(0x40000, BF16, [64, 2, 128])) == KDA_ERR_DTYPE
+    assert run(-2.0, beta=desc(0x50000, F32, [64, 3])) == KDA_ERR_SHAPE
+    assert run(-1.0, k=desc(0x20000, BF16, [64, 2, 128], [256, 128, 2])) == KDA_ERR_STRIDE

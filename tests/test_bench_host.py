@@ -44,13 +44,31 @@ def test_recorded_traffic_only_for_matching_code(bench, tmp_path, monkeypatch):
     prof = tmp_path / "profiles" / "kda_fwd_w.md"
     sha = bench.kernel_source_sha()
     _profile(prof, sha, 1234)
-    assert bench.recorded_traffic("w") == 1234.0
+    assert bench.recorded_traffic("kda_fwd_w") == 1234.0
     # a comment-only edit keeps the counters valid
     src.write_text("// header\n__global__ void k() {\n  int x = 1;\n}\n")
     assert bench.kernel_source_sha() == sha
-    assert bench.recorded_traffic("w") == 1234.0
+    assert bench.recorded_traffic("kda_fwd_w") == 1234.0
     # a code edit makes them stale
     src.write_text("__global__ void k() { int x = 2; }\n")
-    assert bench.recorded_traffic("w") is None
+    assert bench.recorded_traffic("kda_fwd_w") is None
     # no summary for the workload: nothing to report
-    assert bench.recorded_traffic("other") is None
+    assert bench.recorded_traffic("kda_fwd_other") is None
+
+
+def test_recorded_traffic_hashes_only_the_named_sources(bench, tmp_path, monkeypatch):
+    csrc = tmp_path / "csrc"
+    csrc.mkdir()
+    (csrc / "a.cuh").write_text("int a = 1;\n")
+    (csrc / "b.cuh").write_text("int b = 1;\n")
+    monkeypatch.setattr(bench, "CSRC", str(csrc))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (tmp_path / "profiles").mkdir()
+    sha = bench.kernel_source_sha(["a.cuh"])
+    with open(tmp_path / "profiles" / "kda_decode_w.md", "w") as f:
+        f.write(f"traffic_bytes_per_launch = 99\nkernel_sources = a.cuh\nkernel_source_sha256 = {sha}\n")
+    assert bench.recorded_traffic("kda_decode_w") == 99.0
+    (csrc / "b.cuh").write_text("int b = 2;\n")    # another kernel's source: still valid
+    assert bench.recorded_traffic("kda_decode_w") == 99.0
+    (csrc / "a.cuh").write_text("int a = 2;\n")    # its own source: stale
+    assert bench.recorded_traffic("kda_decode_w") is None
