@@ -57,6 +57,11 @@ def _load():
             lib.kda_oracle_unit_lower_inverse.restype = ctypes.c_int
             lib.kda_oracle_preprocess.argtypes = [P, P, P, P, i64, i32, i32, f64, f64, P, P, P, P]
             lib.kda_oracle_preprocess.restype = ctypes.c_int
+            bw_args = [P, P, P, P, P, i64, i32, i32, i32, P, i32, f64, P, P, P, P, P, P, P, P, P, i32]
+            lib.kda_oracle_backward_bf16.argtypes = bw_args
+            lib.kda_oracle_backward_bf16.restype = ctypes.c_int
+            lib.kda_oracle_backward_f64.argtypes = bw_args
+            lib.kda_oracle_backward_f64.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -173,3 +178,34 @@ def scan_raw_inputs(inp, lower_bound=-5.0, **kw):
     v = bf16_bits_to_f32(inp.v).astype(np.float64)
     init = None if inp.initial_state is None else inp.initial_state.astype(np.float64)
     return scan(qh, kh, v, g, beta, inp.cu_seqlens, inp.scale, init, **kw)
+
+
+def backward(q, k, v, g, beta, cu_seqlens, scale, dout, initial_state=None, dfinal=None, *, nthreads=0):
+    """Gradients of sum(dout * o) + sum(dfinal * S_final) with respect to q, k,
+    v, g, beta and the initial state (reverse mode of the token recurrence).
+
+    Inputs as for ``scan`` (bf16 bit patterns with float32 g/beta/states and
+    bf16-bit ``dout``, or all float64). Returns a dict of float64 arrays
+    ``dq, dk, dv, dg, dbeta, dinit`` (``dinit`` None without an initial state).
+    """
+    lib = _load()
+    bf16 = np.asarray(q).dtype == np.uint16
+    vt = np.uint16 if bf16 else np.float64
+    gt = np.float32 if bf16 else np.float64
+    q, k, v, dout = _c(q, vt), _c(k, vt), _c(v, vt), _c(dout, vt)
+    g, beta = _c(g, gt), _c(beta, gt)
+    init, dfin = _c(initial_state, gt), _c(dfinal, gt)
+    cu = _c(cu_seqlens, np.int32)
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    nseq = cu.shape[0] - 1
+    res = {"dq": np.zeros((T, H, dk)), "dk": np.zeros((T, H, dk)), "dv": np.zeros((T, H, dv)),
+           "dg": np.zeros((T, H, dk)), "dbeta": np.zeros((T, H)),
+           "dinit": np.zeros((nseq, H, dk, dv)) if initial_state is not None else None}
+    fn = lib.kda_oracle_backward_bf16 if bf16 else lib.kda_oracle_backward_f64
+    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), T, H, dk, dv, _ptr(cu), nseq, float(scale), _ptr(init),
+            _ptr(dout), _ptr(dfin), _ptr(res["dq"]), _ptr(res["dk"]), _ptr(res["dv"]), _ptr(res["dg"]),
+            _ptr(res["dbeta"]), _ptr(res["dinit"]), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle backward rejected its arguments (code {rc})")
+    return res

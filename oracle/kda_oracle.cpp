@@ -40,6 +40,10 @@
 //                             forward substitution or by the Neumann/doubling
 //                             product (page "Kimi K3 开源满月…", section
 //                             "KDA 内核到底难在哪": L^16 = 0 for 16x16 L).
+//   kda_oracle_backward_*  -- the reverse-mode derivative of the recurrence
+//                             (gradients of q, k, v, g, beta and the initial
+//                             state for given output and final-state
+//                             gradients), token by token.
 //   kda_oracle_preprocess  -- the gate preprocessing that precedes the
 //                             recurrence in a layer: q, k L2-normalised per
 //                             (token, head); g = max(log sigmoid(x), lower_bound)
@@ -343,6 +347,160 @@ void chunked_one(const double* q, const double* k, const double* v, const double
   if (fin) std::memcpy(fin, S.data(), sizeof(double) * dk * dv);
 }
 
+// ------------------------------------------------------------------ backward
+// Reverse-mode derivative of the token recurrence for one (sequence, head).
+// Per token t (S_{t-1} -> S_t), with S' = Diag(exp g) S_{t-1}, u = v - S'^T k:
+//   S_t = S' + beta k u^T = (I - beta k k^T) S' + beta k v^T,  o_t = scale S_t^T q.
+// Walking t backwards with L = dLoss/dS_t (the final-state gradient at t = T):
+//   L   += scale q dO^T            dq = scale S_t dO
+//   lk   = L^T k                   dv = beta lk,   dbeta = lk . u
+//   dk   = beta L u - beta S' lk   (through the write and through u = v - S'^T k)
+//   dS'  = L - beta k lk^T         dg_r = sum_c dS'_rc S'_rc
+//   L    = Diag(exp g) dS'         (dLoss/dS_{t-1}); at the start, d initial state = L.
+// The states of a sequence are recomputed segment by segment from checkpoints
+// taken every kCheckpoint tokens of a first forward pass.
+template <class TV, class TG>
+struct BackwardProblem {
+  const TV* q;
+  const TV* k;
+  const TV* v;
+  const TG* g;
+  const TG* beta;
+  int64_t T;
+  int32_t H, dk, dv;
+  const int32_t* cu;
+  int32_t nseq;
+  double scale;
+  const TG* init;    // [nseq, H, dk, dv] or nullptr
+  const TV* dout;    // [T, H, dv]
+  const TG* dfin;    // [nseq, H, dk, dv] or nullptr
+  double *dq, *dk_out, *dv_out, *dg, *dbeta;  // [T, H, dk], [T, H, dk], [T, H, dv], [T, H, dk], [T, H]
+  double* dinit;     // [nseq, H, dk, dv] or nullptr
+};
+
+constexpr int kCheckpoint = 64;
+
+template <class TV, class TG>
+void backward_one(const BackwardProblem<TV, TG>& P, int seq, int h) {
+  const int dk = P.dk, dv = P.dv, H = P.H;
+  const int64_t t0 = P.cu[seq], t1 = P.cu[seq + 1], len = t1 - t0;
+  const size_t SS = static_cast<size_t>(dk) * dv;
+  const size_t so = (static_cast<size_t>(seq) * H + h) * SS;
+  auto kat = [&](int64_t t, int r) { return widen(P.k[(static_cast<size_t>(t) * H + h) * dk + r]); };
+  auto qat = [&](int64_t t, int r) { return widen(P.q[(static_cast<size_t>(t) * H + h) * dk + r]); };
+  auto vat = [&](int64_t t, int c) { return widen(P.v[(static_cast<size_t>(t) * H + h) * dv + c]); };
+  auto gat = [&](int64_t t, int r) { return widen(P.g[(static_cast<size_t>(t) * H + h) * dk + r]); };
+  auto bat = [&](int64_t t) { return widen(P.beta[static_cast<size_t>(t) * H + h]); };
+  // one forward step S <- (I - b k k^T) Diag(exp g) S + b k v^T (the scan's arithmetic)
+  std::vector<double> kS(dv);
+  auto step = [&](std::vector<double>& S, int64_t t) {
+    for (int r = 0; r < dk; ++r) {
+      const double d = std::exp(gat(t, r));
+      for (int c = 0; c < dv; ++c) S[r * dv + c] *= d;
+    }
+    for (int c = 0; c < dv; ++c) kS[c] = 0.0;
+    for (int r = 0; r < dk; ++r)
+      for (int c = 0; c < dv; ++c) kS[c] += kat(t, r) * S[r * dv + c];
+    const double b = bat(t);
+    for (int r = 0; r < dk; ++r)
+      for (int c = 0; c < dv; ++c) S[r * dv + c] += b * kat(t, r) * (vat(t, c) - kS[c]);
+  };
+  std::vector<double> S(SS, 0.0);
+  if (P.init)
+    for (size_t i = 0; i < SS; ++i) S[i] = widen(P.init[so + i]);
+  const int64_t nck = len / kCheckpoint + 1;
+  std::vector<double> ck(static_cast<size_t>(nck) * SS);
+  for (int64_t t = t0; t < t1; ++t) {
+    if ((t - t0) % kCheckpoint == 0) std::copy(S.begin(), S.end(), ck.begin() + ((t - t0) / kCheckpoint) * SS);
+    step(S, t);
+  }
+  std::vector<double> L(SS, 0.0), Sp(SS), lk(dv), u(dv);
+  if (P.dfin)
+    for (size_t i = 0; i < SS; ++i) L[i] = widen(P.dfin[so + i]);
+  std::vector<double> seg(static_cast<size_t>(kCheckpoint + 1) * SS);
+  for (int64_t m = (len - 1) / kCheckpoint; m >= 0 && len > 0; --m) {
+    const int64_t ts = t0 + m * kCheckpoint, te = std::min<int64_t>(ts + kCheckpoint, t1);
+    // seg[j] = the state before token ts + j (j = 0 .. te - ts)
+    std::copy(ck.begin() + m * SS, ck.begin() + (m + 1) * SS, seg.begin());
+    for (int64_t t = ts; t < te; ++t) {
+      const size_t j = static_cast<size_t>(t - ts);
+      std::copy(seg.begin() + j * SS, seg.begin() + (j + 1) * SS, seg.begin() + (j + 1) * SS);
+      std::vector<double> tmp(seg.begin() + (j + 1) * SS, seg.begin() + (j + 2) * SS);
+      step(tmp, t);
+      std::copy(tmp.begin(), tmp.end(), seg.begin() + (j + 1) * SS);
+    }
+    for (int64_t t = te - 1; t >= ts; --t) {
+      const size_t j = static_cast<size_t>(t - ts);
+      const double* Sprev = &seg[j * SS];
+      const double* St = &seg[(j + 1) * SS];
+      const size_t rk = (static_cast<size_t>(t) * H + h) * dk, rv = (static_cast<size_t>(t) * H + h) * dv;
+      const double b = bat(t);
+      // output t: L += scale q dO^T, dq = scale S_t dO
+      for (int r = 0; r < dk; ++r) {
+        double acc = 0.0;
+        for (int c = 0; c < dv; ++c) {
+          const double dov = widen(P.dout[rv + c]);
+          L[r * dv + c] += P.scale * qat(t, r) * dov;
+          acc += St[r * dv + c] * dov;
+        }
+        P.dq[rk + r] = P.scale * acc;
+      }
+      // S' = Diag(exp g) S_{t-1}, u = v - S'^T k
+      for (int r = 0; r < dk; ++r) {
+        const double d = std::exp(gat(t, r));
+        for (int c = 0; c < dv; ++c) Sp[r * dv + c] = d * Sprev[r * dv + c];
+      }
+      for (int c = 0; c < dv; ++c) {
+        double w = 0.0, l = 0.0;
+        for (int r = 0; r < dk; ++r) {
+          w += Sp[r * dv + c] * kat(t, r);
+          l += L[r * dv + c] * kat(t, r);
+        }
+        u[c] = vat(t, c) - w;
+        lk[c] = l;
+      }
+      double db = 0.0;
+      for (int c = 0; c < dv; ++c) {
+        P.dv_out[rv + c] = b * lk[c];
+        db += lk[c] * u[c];
+      }
+      P.dbeta[static_cast<size_t>(t) * H + h] = db;
+      for (int r = 0; r < dk; ++r) {
+        double lu = 0.0, sl = 0.0;
+        for (int c = 0; c < dv; ++c) {
+          lu += L[r * dv + c] * u[c];
+          sl += Sp[r * dv + c] * lk[c];
+        }
+        P.dk_out[rk + r] = b * lu - b * sl;
+      }
+      // dS' = L - b k lk^T; dg; L <- Diag(exp g) dS'
+      for (int r = 0; r < dk; ++r) {
+        const double kr = kat(t, r), d = std::exp(gat(t, r));
+        double dgr = 0.0;
+        for (int c = 0; c < dv; ++c) {
+          const double dsp = L[r * dv + c] - b * kr * lk[c];
+          dgr += dsp * Sp[r * dv + c];
+          L[r * dv + c] = d * dsp;
+        }
+        P.dg[rk + r] = dgr;
+      }
+    }
+  }
+  if (P.dinit)
+    for (size_t i = 0; i < SS; ++i) P.dinit[so + i] = L[i];
+}
+
+template <class TV, class TG>
+int run_backward(const BackwardProblem<TV, TG>& P, int32_t nthreads) {
+  int rc = check_common(P.T, P.H, P.dk, P.dv, P.cu, P.nseq, 0, P.dv);
+  if (rc) return rc;
+  if (!P.dout || !P.dq || !P.dk_out || !P.dv_out || !P.dg || !P.dbeta) return 1;
+  parallel_for(static_cast<int64_t>(P.nseq) * P.H, nthreads, [&](int64_t i) {
+    backward_one(P, static_cast<int>(i / P.H), static_cast<int>(i % P.H));
+  });
+  return 0;
+}
+
 }  // namespace
 
 extern "C" {
@@ -445,6 +603,34 @@ int kda_oracle_preprocess(const uint16_t* q, const uint16_t* k, const float* x, 
       beta_out[static_cast<size_t>(t) * H + h] = 1.0 / (1.0 + std::exp(-bv));
     }
   return 0;
+}
+
+// Derivatives of the loss sum(dout * o) + sum(dfin * S_final) with respect to
+// q, k, v, g, beta and the initial state (reverse mode of the token
+// recurrence; see backward_one). Library-format inputs (bf16 bits for q, k, v
+// and dout; float32 for g, beta, init and dfin); every output fp64.
+// init, dfin and dinit may be NULL (zero initial state / no final-state
+// gradient / not written).
+int kda_oracle_backward_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* g,
+                             const float* beta, int64_t T, int32_t H, int32_t dk, int32_t dv, const int32_t* cu,
+                             int32_t nseq, double scale, const float* init, const uint16_t* dout, const float* dfin,
+                             double* dq, double* dkk, double* dvv, double* dg, double* dbeta, double* dinit,
+                             int32_t nthreads) {
+  if (!q || !k || !v || !g || !beta) return 1;
+  BackwardProblem<uint16_t, float> P{q, k, v, g, beta, T, H, dk, dv, cu, nseq, scale, init, dout, dfin,
+                                     dq, dkk, dvv, dg, dbeta, dinit};
+  return run_backward(P, nthreads);
+}
+
+// Same with every input in fp64.
+int kda_oracle_backward_f64(const double* q, const double* k, const double* v, const double* g, const double* beta,
+                            int64_t T, int32_t H, int32_t dk, int32_t dv, const int32_t* cu, int32_t nseq,
+                            double scale, const double* init, const double* dout, const double* dfin, double* dq,
+                            double* dkk, double* dvv, double* dg, double* dbeta, double* dinit, int32_t nthreads) {
+  if (!q || !k || !v || !g || !beta) return 1;
+  BackwardProblem<double, double> P{q, k, v, g, beta, T, H, dk, dv, cu, nseq, scale, init, dout, dfin,
+                                    dq, dkk, dvv, dg, dbeta, dinit};
+  return run_backward(P, nthreads);
 }
 
 int kda_oracle_abi_version(void) { return 1; }

@@ -31,6 +31,11 @@ P10 gate preprocessing (preprocess): unit norms per (token, head) over the
     wrong branch of the stable form; the lower bound clamps exactly where
     log sigmoid falls below it; agreement with the generator's gates and
     betas computed from the same draws.
+P11 backward: the reverse-mode gradients of q, k, v, g, beta and the initial
+    state equal central finite differences of the (pinned) forward scan, per
+    coordinate and along random directions -> every term of the hand-derived
+    reverse recurrence (a dropped term, a wrong sign or transpose shows as a
+    gradient mismatch).
 """
 import json
 import os
@@ -387,3 +392,67 @@ def test_p10_preprocessed_scan_matches_generator_scan(oracle_mod):
     o2, f2 = oracle_mod.scan_inputs(inp)
     assert np.linalg.norm(o1 - o2) / np.linalg.norm(o2) < 1e-2
     assert np.linalg.norm(f1 - f2) / np.linalg.norm(f2) < 1e-2
+
+
+# ----------------------------------------------------------------------------- P11
+def _loss(oracle_mod, args, dout, dfin):
+    q, k, v, g, beta, cu, S0, scale = args
+    o, f = oracle_mod.scan(q, k, v, g, beta, cu, scale, S0)
+    return float(np.sum(o * dout) + np.sum(f * dfin))
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_p11_backward_equals_finite_differences(oracle_mod, seed):
+    lens, H, dk, dv = [5, 0, 9, 1], 2, 6, 5
+    q, k, v, g, beta, cu, S0 = _rand_f64(lens, H, dk, dv, 70 + seed, gmin=-2.0, init=True)
+    scale = 0.7
+    rng = np.random.default_rng(80 + seed)
+    dout = rng.standard_normal(v.shape)
+    dfin = rng.standard_normal(S0.shape)
+    gr = oracle_mod.backward(q, k, v, g, beta, cu, scale, dout, S0, dfin)
+    base = [q, k, v, g, beta, cu, S0, scale]
+    names = {"dq": 0, "dk": 1, "dv": 2, "dg": 3, "dbeta": 4, "dinit": 6}
+    h = 1e-6
+    for name, idx in names.items():
+        x = base[idx]
+        # a handful of single coordinates
+        flat = rng.choice(x.size, size=min(6, x.size), replace=False)
+        for f in flat:
+            plus = [a.copy() if isinstance(a, np.ndarray) else a for a in base]
+            minus = [a.copy() if isinstance(a, np.ndarray) else a for a in base]
+            plus[idx].flat[f] += h
+            minus[idx].flat[f] -= h
+            fd = (_loss(oracle_mod, plus, dout, dfin) - _loss(oracle_mod, minus, dout, dfin)) / (2 * h)
+            an = gr[name].flat[f]
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(fd)), (name, f, fd, an)
+        # one random direction over all coordinates
+        d = rng.standard_normal(x.shape)
+        plus = [a.copy() if isinstance(a, np.ndarray) else a for a in base]
+        minus = [a.copy() if isinstance(a, np.ndarray) else a for a in base]
+        plus[idx] = plus[idx] + h * d
+        minus[idx] = minus[idx] - h * d
+        fd = (_loss(oracle_mod, plus, dout, dfin) - _loss(oracle_mod, minus, dout, dfin)) / (2 * h)
+        an = float(np.sum(gr[name] * d))
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(fd)), (name, "direction", fd, an)
+
+
+def test_p11_backward_long_sequence_crosses_checkpoints(oracle_mod):
+    """The oracle recomputes states from checkpoints every 64 tokens; a
+    sequence over several checkpoints gives the finite-difference gradients."""
+    lens, H, dk, dv = [150], 1, 4, 3
+    q, k, v, g, beta, cu, S0 = _rand_f64(lens, H, dk, dv, 90, gmin=-0.3, init=True)
+    rng = np.random.default_rng(91)
+    dout = rng.standard_normal(v.shape)
+    dfin = rng.standard_normal(S0.shape)
+    gr = oracle_mod.backward(q, k, v, g, beta, cu, 0.5, dout, S0, dfin)
+    base = [q, k, v, g, beta, cu, S0, 0.5]
+    h = 1e-6
+    for name, idx in {"dk": 1, "dg": 3, "dinit": 6}.items():
+        d = rng.standard_normal(base[idx].shape)
+        plus = list(base)
+        minus = list(base)
+        plus[idx] = base[idx] + h * d
+        minus[idx] = base[idx] - h * d
+        fd = (_loss(oracle_mod, plus, dout, dfin) - _loss(oracle_mod, minus, dout, dfin)) / (2 * h)
+        an = float(np.sum(gr[name] * d))
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(fd)), (name, fd, an)
