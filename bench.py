@@ -44,7 +44,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 CSRC = os.path.join(ROOT, "kimi_delta_attention_26_b200", "csrc")
 KERNEL_SOURCES = [os.path.join(CSRC, f)
                   for f in ("kda_prims.cuh", "kda_fwd16.cuh", "kda_fwd64.cuh", "kda_split.cuh", "kda_decode.cuh",
-                            "kda_api.cu")]
+                            "kda_bwd.cuh", "kda_api.cu")]
 
 
 def log(*a):
@@ -465,6 +465,48 @@ def fused_entry(kda, dev, stream, steps: int):
             "algorithmic_bytes_per_launch": roof["algorithmic_bytes_per_launch"]}
 
 
+# The backward's algorithmic work per token and head: one forward step
+# (decay, S'^T k, write: 5 flops per state element) and one reverse step
+# (20 flops per state element: the rank-1 updates and reductions of the
+# reverse recurrence) over the 128 x 128 state. Its bytes: the inputs, dO,
+# and the fp32 gradients of q, k, v, g and beta.
+BWD_FLOPS_PER_TOKHEAD = 25 * D * D
+BWD_BYTES_PER_TOKHEAD = 3 * D * 2 + D * 4 + 4 + D * 2 + 4 * D * 4 + 4
+# fp32 FMA issue of the CUDA cores: 148 SMs x 128 lanes x 2 flops per cycle at
+# the 1965 MHz maximum SM clock (the backward's rank-1 updates run there)
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def bwd_entry(kda, dev, stream, steps: int):
+    """kda_bwd on the Kimi-Linear-shaped workload (T=8192, H=32) with a random
+    output gradient: device time per launch (inputs larger than L2 with the
+    gradients) and its roofline on the fp32 CUDA cores."""
+    import torch
+
+    wl = kda_inputs.workload(2)
+    inp = wl.make()
+    t = lambda a: torch.from_numpy(a).to(dev)
+    q, k, v = (t(x).view(torch.bfloat16) for x in (inp.q, inp.k, inp.v))
+    g, beta = t(inp.g), t(inp.beta)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7)
+    dout = torch.randn(q.shape, device=dev, generator=gen).bfloat16()
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    launch = lambda: kda.kda_bwd(q, k, v, g, beta, dout, inp.scale, stream=stream)
+    ms_l = time_launches(launch, steps, 3, stream, flush, dev)
+    ms = sum(ms_l) / len(ms_l)
+    units = work_units(inp)
+    tflops = units * BWD_FLOPS_PER_TOKHEAD / (ms * 1e-3) / 1e12
+    gbs = units * BWD_BYTES_PER_TOKHEAD / (ms * 1e-3) / 1e9
+    return {"workload": wl.name + " (gradients of q, k, v, g, beta)", "ms": ms,
+            "value": units / (ms * 1e-3) / 1e6, "unit": UNIT,
+            "roofline": {"bound": "alu", "achieved": tflops, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+                         "frac": tflops / FP32_ALU_TFLOPS,
+                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz",
+                         "algorithmic_flops_per_launch": units * BWD_FLOPS_PER_TOKHEAD},
+            "gbs": gbs}
+
+
 # ---------------------------------------------------------------------- kda
 def run_kda(args):
     import torch
@@ -598,6 +640,7 @@ def run_kda(args):
             line["per_config"] = per_config_table(kda, dev, stream, min(args.steps, 20), (0, 64))
             line["decode"] = decode_entry(kda, dev, stream, min(args.steps, 20))
             line["fused_gate"] = fused_entry(kda, dev, stream, min(args.steps, 20))
+            line["backward"] = bwd_entry(kda, dev, stream, min(args.steps, 5))
         print(json.dumps(line), flush=True)
     if ws > 1:
         dist.barrier()

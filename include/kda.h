@@ -277,6 +277,40 @@ kda_status_t kda_decode(const kda_tensor_t* q, const kda_tensor_t* k, const kda_
                         const kda_tensor_t* state, const int32_t* state_indices,
                         const kda_tensor_t* out, void* stream);
 
+/*
+ * kda_bwd -- gradients of the prefill (training): for a loss with gradient
+ * dout = dLoss/do (and dfinal_state = dLoss/dS_final), the gradients of q, k,
+ * v, g, beta and the initial state.
+ *
+ * The sources name only a Triton implementation that trains (page "Moonshot
+ * AI … FlashKDA … (kucoin)"); this is the plain reverse-mode derivative of the
+ * recurrence above, token by token:
+ *   L = dLoss/dS_t;  L += scale q_t dO_t^T;  dq_t = scale S_t dO_t;
+ *   with S' = Diag(exp g_t) S_{t-1}, u = v_t - S'^T k_t, lk = L^T k_t:
+ *   dv_t = beta_t lk, dbeta_t = lk . u, dk_t = beta_t (L u - S' lk),
+ *   dS' = L - beta_t k_t lk^T, dg_t = rowsum(dS' * S'), L <- Diag(exp g_t) dS'.
+ *
+ * Inputs: q, k, v, g, beta, scale, cu_seqlens, num_seqs, initial_state as for
+ * kda_fwd (same layouts, strides and preconditions); dout bf16 [T, H, 128]
+ * (strides as for kda_fwd's inputs); dfinal_state fp32 [N, H, 128, 128]
+ * contiguous or NULL (zero).
+ * Outputs (fp32, contiguous, written in full): dq, dk, dv, dg [T, H, 128];
+ * dbeta [T, H]; dinitial_state [N, H, 128, 128] or NULL (not written). The
+ * gradient of g is for the natural-log decay itself.
+ * Scratch from the pool: a state checkpoint every 4 tokens and per-slice
+ * partial sums, about T x H x (4 x 64 KiB / 4 + 12 KiB) bytes. Results are
+ * deterministic. Runs on the CUDA cores (rank-1 updates token by token): much
+ * slower than kda_fwd. Errors as for kda_fwd; nothing is enqueued on any
+ * error. Returns KDA_OK once the work is enqueued.
+ */
+kda_status_t kda_bwd(const kda_tensor_t* q, const kda_tensor_t* k, const kda_tensor_t* v,
+                     const kda_tensor_t* g, const kda_tensor_t* beta, float scale,
+                     const int32_t* cu_seqlens, int32_t num_seqs, const kda_tensor_t* initial_state,
+                     const kda_tensor_t* dout, const kda_tensor_t* dfinal_state,
+                     const kda_tensor_t* dq, const kda_tensor_t* dk, const kda_tensor_t* dv,
+                     const kda_tensor_t* dg, const kda_tensor_t* dbeta,
+                     const kda_tensor_t* dinitial_state, void* stream);
+
 /* Human-readable text of a status code (static storage, never NULL). */
 const char* kda_status_string(kda_status_t status);
 

@@ -14,7 +14,7 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["kda_fwd", "kda_fwd_fused", "kda_decode", "library_path", "wait_timeouts", "device_status", "set_slice_columns", "set_path",
+__all__ = ["kda_fwd", "kda_fwd_fused", "kda_decode", "kda_bwd", "library_path", "wait_timeouts", "device_status", "set_slice_columns", "set_path",
            "set_time_split", "describe", "KDAError", "HEAD_DIM"]
 
 HEAD_DIM = 128
@@ -79,6 +79,8 @@ _lib.kda_set_time_split.argtypes = [ctypes.c_int32]
 _lib.kda_set_time_split.restype = ctypes.c_int
 _lib.kda_fwd_fused.argtypes = [_T, _T, _T, _T, _T, ctypes.c_float, ctypes.c_float, _P, ctypes.c_int32, _T, _T, _T, _P]
 _lib.kda_fwd_fused.restype = ctypes.c_int
+_lib.kda_bwd.argtypes = [_T, _T, _T, _T, _T, ctypes.c_float, _P, ctypes.c_int32, _T, _T, _T, _T, _T, _T, _T, _T, _T, _P]
+_lib.kda_bwd.restype = ctypes.c_int
 _lib.kda_decode.argtypes = [_T, _T, _T, _T, _T, ctypes.c_float, _T, _P, _T, _P]
 _lib.kda_decode.restype = ctypes.c_int
 
@@ -272,3 +274,45 @@ def kda_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tenso
     if rc != 0:
         raise KDAError(rc)
     return out
+
+
+def kda_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, beta: torch.Tensor,
+            dout: torch.Tensor, scale: Optional[float] = None, cu_seqlens: Optional[torch.Tensor] = None,
+            initial_state: Optional[torch.Tensor] = None, dfinal_state: Optional[torch.Tensor] = None,
+            stream: Optional[torch.cuda.Stream] = None):
+    """Gradients of the prefill (see ``include/kda.h``): returns a dict of fp32
+    tensors ``dq, dk, dv, dg`` [T, H, 128], ``dbeta`` [T, H] and
+    ``dinitial_state`` [N, H, 128, 128], for the output gradient ``dout``
+    (bf16 [T, H, 128]) and the final-state gradient ``dfinal_state``
+    (fp32 [N, H, 128, 128] or None)."""
+    if q.dim() != 3:
+        raise ValueError("q must be [T, H, 128]")
+    T, H, d = q.shape
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("kda_bwd runs on CUDA tensors only")
+    N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    _check(dout, "dout", torch.bfloat16, (T, H, d), dev)
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32, (N + 1,), dev, contiguous=True)
+    if initial_state is not None:
+        _check(initial_state, "initial_state", torch.float32, (N, H, d, d), dev, contiguous=True)
+    if dfinal_state is not None:
+        _check(dfinal_state, "dfinal_state", torch.float32, (N, H, d, d), dev, contiguous=True)
+    grads = {n: torch.empty((T, H, d), dtype=torch.float32, device=dev) for n in ("dq", "dk", "dv", "dg")}
+    grads["dbeta"] = torch.empty((T, H), dtype=torch.float32, device=dev)
+    grads["dinitial_state"] = torch.empty((N, H, d, d), dtype=torch.float32, device=dev)
+    if scale is None:
+        scale = d ** -0.5
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    ts = (q, k, v, g, beta, initial_state, dout, dfinal_state, grads["dq"], grads["dk"], grads["dv"], grads["dg"],
+          grads["dbeta"], grads["dinitial_state"])
+    descs = [describe(t) for t in ts]
+    r = [None if x is None else x[0] for x in descs]
+    with torch.cuda.device(dev):
+        rc = _lib.kda_bwd(r[0], r[1], r[2], r[3], r[4], ctypes.c_float(scale), _ptr(cu_seqlens), N, r[5], r[6], r[7],
+                          r[8], r[9], r[10], r[11], r[12], r[13], ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise KDAError(rc)
+    return grads

@@ -10,7 +10,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SOURCES = [os.path.join(PKG, "csrc", "kda_api.cu")]
 HEADERS = [os.path.join(ROOT, "include", "kda.h"), os.path.abspath(__file__)] + [
-    os.path.join(PKG, "csrc", f) for f in ("kda_prims.cuh", "kda_fwd16.cuh", "kda_fwd64.cuh", "kda_split.cuh", "kda_decode.cuh")]
+    os.path.join(PKG, "csrc", f) for f in ("kda_prims.cuh", "kda_fwd16.cuh", "kda_fwd64.cuh", "kda_split.cuh", "kda_decode.cuh",
+                                            "kda_bwd.cuh")]
 LIB = os.path.join(PKG, "libkda.so")
 
 NVCC_FLAGS = [

@@ -12,6 +12,7 @@
 #include "kda_fwd64.cuh"
 #include "kda_split.cuh"
 #include "kda_decode.cuh"
+#include "kda_bwd.cuh"
 
 #include <algorithm>
 #include <atomic>
@@ -178,13 +179,31 @@ std::atomic<void*> g_noalloc_ring_addr[kMaxDevices];
 std::atomic<int> g_slice_columns{0};  // 16-token path: 0 chooses per call, 16 or 32 forces
 std::atomic<int> g_path{0};           // 0 (the default path), 16 or 64
 
-template <int NS>
-cudaError_t set_smem16() {
-  cudaError_t e = cudaFuncSetAttribute(kda::kda_fwd_kernel<NS, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(sizeof(kda::Shared<NS>)));
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(kda::kda_fwd_kernel<NS, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+// The 16-token kernel's instantiations: value slice NS, fused gate FG and
+// launch mode MODE (the time split's modes run only with 32-column slices).
+constexpr uint32_t kSplitL = kda::kModeOutF32;                          // second half from zero
+constexpr uint32_t kSplitM = kda::kModeZeroV | kda::kModeIdentityInit;  // second half's map
+
+template <int NS, bool FG, uint32_t MODE>
+cudaError_t set_smem_one() {
+  return cudaFuncSetAttribute(kda::kda_fwd_kernel<NS, FG, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(sizeof(kda::Shared<NS>)));
+}
+
+cudaError_t set_smem16() {
+  cudaError_t e;
+  if ((e = set_smem_one<16, false, 0>()) != cudaSuccess || (e = set_smem_one<16, true, 0>()) != cudaSuccess ||
+      (e = set_smem_one<32, false, 0>()) != cudaSuccess || (e = set_smem_one<32, true, 0>()) != cudaSuccess ||
+      (e = set_smem_one<32, false, kSplitL>()) != cudaSuccess ||
+      (e = set_smem_one<32, true, kSplitL>()) != cudaSuccess ||
+      (e = set_smem_one<32, false, kSplitM>()) != cudaSuccess || (e = set_smem_one<32, true, kSplitM>()) != cudaSuccess)
+    return e;
+  return cudaSuccess;
+}
+
+template <int NS, bool FG, uint32_t MODE>
+void launch_one(const kda::Params& p, const kda::TensorMaps& tm, int H, int N, cudaStream_t stream) {
+  kda::kda_fwd_kernel<NS, FG, MODE><<<dim3(kda::D / NS, H, N), kda::NTHREADS, sizeof(kda::Shared<NS>), stream>>>(p, tm);
 }
 
 // Capability check and kernel attributes for `dev` (current), once.
@@ -206,10 +225,12 @@ kda_status_t check_device(int dev) {
   }
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return cuda_fail(e);
-  if ((e = set_smem16<32>()) != cudaSuccess) return cuda_fail(e);
-  if ((e = set_smem16<16>()) != cudaSuccess) return cuda_fail(e);
+  if ((e = set_smem16()) != cudaSuccess) return cuda_fail(e);
   if ((e = cudaFuncSetAttribute(kda::split::split_correct_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(kda::split::SMEM_BYTES))) != cudaSuccess)
+    return cuda_fail(e);
+  if ((e = cudaFuncSetAttribute(kda::bwd::kda_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(kda::bwd::SMEM_BYTES))) != cudaSuccess)
     return cuda_fail(e);
   if ((e = cudaFuncSetAttribute(kda::c64::kda_fwd64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(kda::c64::SMEM_BYTES))) != cudaSuccess)
@@ -222,7 +243,7 @@ kda_status_t check_device(int dev) {
   cfg.blockDim = dim3(kda::NTHREADS, 1, 1);
   cfg.dynamicSmemBytes = sizeof(kda::Shared<32>);
   int clusters = 0;
-  if ((e = cudaOccupancyMaxActiveClusters(&clusters, kda::kda_fwd_kernel<32, false>, &cfg)) != cudaSuccess)
+  if ((e = cudaOccupancyMaxActiveClusters(&clusters, kda::kda_fwd_kernel<32, false, 0>, &cfg)) != cudaSuccess)
     return cuda_fail(e);
   g_max_clusters32[dev] = clusters;
   g_num_sms[dev] = sms;
@@ -321,7 +342,6 @@ kda_status_t launch16(const Problem& P, unsigned char* ring, int dev, cudaStream
   p.out_sh = P.out.sh;
   p.H = P.num_heads;
   p.scale = P.scale;
-  p.mode = mode | (P.fused ? kda::kModeFusedGate : 0u);
   p.exp_lb = P.exp_lb;
   p.outf = outf;
   p.outf_st = static_cast<int64_t>(P.num_heads) * kda::D;
@@ -339,15 +359,22 @@ kda_status_t launch16(const Problem& P, unsigned char* ring, int dev, cudaStream
         (st = encode_3d(&tm.v, P.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.T, H, ns, kda::C, NONE)) != KDA_OK)
       return st;
   }
-  const dim3 grid16(kda::D / 16, P.num_heads, P.num_seqs), grid32(kda::D / 32, P.num_heads, P.num_seqs);
-  if (ns == 16 && P.fused) {
-    kda::kda_fwd_kernel<16, true><<<grid16, kda::NTHREADS, sizeof(kda::Shared<16>), stream>>>(p, tm);
-  } else if (ns == 16) {
-    kda::kda_fwd_kernel<16, false><<<grid16, kda::NTHREADS, sizeof(kda::Shared<16>), stream>>>(p, tm);
-  } else if (P.fused) {
-    kda::kda_fwd_kernel<32, true><<<grid32, kda::NTHREADS, sizeof(kda::Shared<32>), stream>>>(p, tm);
+  const int H = P.num_heads, N = P.num_seqs;
+  if (mode != 0 && ns != 32) return KDA_ERR_UNSUPPORTED;  // not reached: the split forces 32 columns
+  if (mode == 0 && ns == 16) {
+    if (P.fused) launch_one<16, true, 0>(p, tm, H, N, stream);
+    else launch_one<16, false, 0>(p, tm, H, N, stream);
+  } else if (mode == 0) {
+    if (P.fused) launch_one<32, true, 0>(p, tm, H, N, stream);
+    else launch_one<32, false, 0>(p, tm, H, N, stream);
+  } else if (mode == kSplitL) {
+    if (P.fused) launch_one<32, true, kSplitL>(p, tm, H, N, stream);
+    else launch_one<32, false, kSplitL>(p, tm, H, N, stream);
+  } else if (mode == kSplitM) {
+    if (P.fused) launch_one<32, true, kSplitM>(p, tm, H, N, stream);
+    else launch_one<32, false, kSplitM>(p, tm, H, N, stream);
   } else {
-    kda::kda_fwd_kernel<32, false><<<grid32, kda::NTHREADS, sizeof(kda::Shared<32>), stream>>>(p, tm);
+    return KDA_ERR_UNSUPPORTED;
   }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
@@ -490,19 +517,28 @@ kda_status_t launch16_split(const Problem& P, int dev, cudaStream_t stream) {
     for (int i = 0; i < 2 && st == KDA_OK; ++i)
       if ((e = cudaStreamWaitEvent(side[i], ev[0], 0)) != cudaSuccess) st = cuda_fail(e);
     if (st == KDA_OK) st = launch16(A, rings, dev, stream, 0, nullptr, 32);
-    if (st == KDA_OK) st = launch16(L, rings + ring_b, dev, side[0], kda::kModeOutF32, oloc, 32);
-    if (st == KDA_OK)
-      st = launch16(M, rings + 2 * ring_b, dev, side[1], kda::kModeZeroV | kda::kModeIdentityInit, nullptr, 32);
+    if (st == KDA_OK) st = launch16(L, rings + ring_b, dev, side[0], kSplitL, oloc, 32);
+    if (st == KDA_OK) st = launch16(M, rings + 2 * ring_b, dev, side[1], kSplitM, nullptr, 32);
     for (int i = 0; i < 2 && st == KDA_OK; ++i) {
       if ((e = cudaEventRecord(ev[1 + i], side[i])) != cudaSuccess) st = cuda_fail(e);
       else if ((e = cudaStreamWaitEvent(stream, ev[1 + i], 0)) != cudaSuccess) st = cuda_fail(e);
     }
     if (st == KDA_OK) {
-      // persistent: about two CTAs per SM in all, each staging its head's S_a once
+      // persistent: one CTA per SM in all, each staging its head's S_a once
       const int64_t tiles = (T1 + sp::TOK - 1) / sp::TOK;
-      const int64_t per_head = std::max<int64_t>(1, std::min<int64_t>(tiles, 2 * g_num_sms[dev] / H));
-      sp::split_correct_kernel<<<dim3(static_cast<unsigned>(per_head), H), sp::NTHREADS, sp::SMEM_BYTES, stream>>>(
-          oloc, om, sa, static_cast<__nv_bfloat16*>(P.out.data) + Ta * P.out.st, P.out.st, P.out.sh, T1, H);
+      const int64_t per_head = std::max<int64_t>(1, std::min<int64_t>(tiles, g_num_sms[dev] / H));
+      sp::CorrectMaps cm;
+      std::memset(&cm, 0, sizeof(cm));
+      const TokView vom{om, static_cast<int64_t>(H) * kda::D, kda::D};
+      const TokView vol{oloc, static_cast<int64_t>(H) * kda::D, kda::D};
+      constexpr auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
+      if ((st = load_encoder()) == KDA_OK &&
+          (st = encode_3d(&cm.om, vom, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, T1, H, 64, sp::TOK, SW)) == KDA_OK &&
+          (st = encode_3d(&cm.oloc, vol, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, T1, H, 32, sp::TOK, SW)) == KDA_OK)
+        sp::split_correct_kernel<<<dim3(static_cast<unsigned>(per_head), H), sp::NTHREADS, sp::SMEM_BYTES, stream>>>(
+            cm, sa, static_cast<__nv_bfloat16*>(P.out.data) + Ta * P.out.st, P.out.st, P.out.sh, T1);
+    }
+    if (st == KDA_OK) {
       if (P.fin) sp::split_state_kernel<<<dim3(kda::D / 16, H), 128, 0, stream>>>(mm, sa, bm, P.fin);
       if ((e = cudaGetLastError()) != cudaSuccess) st = cuda_fail(e);
     }
@@ -642,6 +678,91 @@ kda_status_t kda_decode(const kda_tensor_t* q, const kda_tensor_t* k, const kda_
                                 static_cast<cudaStream_t>(stream)>>>(p);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
+  return KDA_OK;
+}
+
+kda_status_t kda_bwd(const kda_tensor_t* q, const kda_tensor_t* k, const kda_tensor_t* v, const kda_tensor_t* g,
+                     const kda_tensor_t* beta, float scale, const int32_t* cu_seqlens, int32_t num_seqs,
+                     const kda_tensor_t* initial_state, const kda_tensor_t* dout, const kda_tensor_t* dfinal_state,
+                     const kda_tensor_t* dq, const kda_tensor_t* dk, const kda_tensor_t* dv, const kda_tensor_t* dg,
+                     const kda_tensor_t* dbeta, const kda_tensor_t* dinitial_state, void* stream) {
+  g_last_cuda_error[0] = '\0';
+  if (!dout || !dq || !dk || !dv || !dg || !dbeta) return KDA_ERR_NULL;
+  // inputs as for kda_fwd (dout in the place of out: bf16 [T, H, 128])
+  Problem P;
+  kda_status_t st =
+      check_args(q, k, v, g, beta, scale, cu_seqlens, num_seqs, initial_state, dout, dfinal_state, &P);
+  if (st != KDA_OK) return st;
+  const int64_t T = P.T, H = P.num_heads, N = P.num_seqs;
+  // gradients: fp32, contiguous
+  auto contiguous = [&](const kda_tensor_t* t, bool inner) -> kda_status_t {
+    if (t->dtype != KDA_F32) return KDA_ERR_DTYPE;
+    if (t->ndim != (inner ? 3 : 2) || t->shape[0] != T || t->shape[1] != H || (inner && t->shape[2] != KDA_HEAD_DIM))
+      return KDA_ERR_SHAPE;
+    if (T == 0) return KDA_OK;
+    if (inner ? (t->stride[2] != 1 || t->stride[1] != KDA_HEAD_DIM || (T > 1 && t->stride[0] != H * KDA_HEAD_DIM))
+              : (t->stride[1] != 1 || (T > 1 && t->stride[0] != H)))
+      return KDA_ERR_STRIDE;
+    if (!t->data) return KDA_ERR_NULL;
+    if (!aligned16(t->data)) return KDA_ERR_ALIGN;
+    return KDA_OK;
+  };
+  if ((st = contiguous(dq, true)) != KDA_OK || (st = contiguous(dk, true)) != KDA_OK ||
+      (st = contiguous(dv, true)) != KDA_OK || (st = contiguous(dg, true)) != KDA_OK ||
+      (st = contiguous(dbeta, false)) != KDA_OK)
+    return st;
+  if ((st = check_state(dinitial_state, N, H)) != KDA_OK) return st;
+  int dev = 0;
+  if ((st = prologue(&dev)) != KDA_OK) return st;
+  if ((st = prepare_pool(dev)) != KDA_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  namespace b = kda::bwd;
+  const size_t ck_bytes = round256(static_cast<size_t>(T / b::BLK + N + 1) * H * b::NSLICE * 32 * b::SLOT * 4);
+  const size_t part_bytes = round256(static_cast<size_t>(b::NSLICE) * T * H * kda::D * 4);
+  const size_t pb_bytes = round256(static_cast<size_t>(b::NSLICE) * T * H * 4);
+  void* scratch = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(&scratch, ck_bytes + 3 * part_bytes + pb_bytes, g_pool[dev].load(), cs);
+  if (e != cudaSuccess) return cuda_fail(e);
+  unsigned char* sb = static_cast<unsigned char*>(scratch);
+  b::Params p;
+  p.q = static_cast<const __nv_bfloat16*>(P.q.data);
+  p.k = static_cast<const __nv_bfloat16*>(P.k.data);
+  p.v = static_cast<const __nv_bfloat16*>(P.v.data);
+  p.dout = static_cast<const __nv_bfloat16*>(P.out.data);
+  p.g = static_cast<const float*>(P.g.data);
+  p.beta = static_cast<const float*>(P.beta.data);
+  p.cu = P.cu;
+  p.init = P.init;
+  p.dfin = P.fin;
+  p.dv = static_cast<float*>(dv->data);
+  p.dinit = dinitial_state ? static_cast<float*>(dinitial_state->data) : nullptr;
+  p.ck = reinterpret_cast<float*>(sb);
+  p.pq = reinterpret_cast<float*>(sb + ck_bytes);
+  p.pk = reinterpret_cast<float*>(sb + ck_bytes + part_bytes);
+  p.pg = reinterpret_cast<float*>(sb + ck_bytes + 2 * part_bytes);
+  p.pb = reinterpret_cast<float*>(sb + ck_bytes + 3 * part_bytes);
+  p.T = T;
+  p.q_st = P.q.st; p.q_sh = P.q.sh;
+  p.k_st = P.k.st; p.k_sh = P.k.sh;
+  p.v_st = P.v.st; p.v_sh = P.v.sh;
+  p.o_st = P.out.st; p.o_sh = P.out.sh;
+  p.g_st = P.g.st; p.g_sh = P.g.sh;
+  p.b_st = P.beta.st; p.b_sh = P.beta.sh;
+  p.H = static_cast<int>(H);
+  p.scale = scale;
+  b::kda_bwd_kernel<<<dim3(b::NSLICE / b::WARPS, static_cast<unsigned>(H), static_cast<unsigned>(N)), b::NTHREADS,
+                      b::SMEM_BYTES, cs>>>(p);
+  if (T > 0) {
+    const int64_t n4 = T * H * kda::D / 4, nb = T * H;
+    const int64_t blocks = std::min<int64_t>((n4 + 255) / 256, 8 * static_cast<int64_t>(g_num_sms[dev]));
+    b::kda_bwd_reduce_kernel<<<static_cast<unsigned>(blocks), 256, 0, cs>>>(
+        p.pq, p.pk, p.pg, p.pb, static_cast<float*>(dq->data), static_cast<float*>(dk->data),
+        static_cast<float*>(dg->data), static_cast<float*>(dbeta->data), n4, nb);
+  }
+  e = cudaGetLastError();
+  const cudaError_t ef = cudaFreeAsync(scratch, cs);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (ef != cudaSuccess) return cuda_fail(ef);
   return KDA_OK;
 }
 

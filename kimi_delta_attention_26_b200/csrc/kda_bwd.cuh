@@ -1,0 +1,427 @@
+// kda_bwd.cuh -- backward pass of the Kimi Delta Attention recurrence
+// (gradients of q, k, v, g, beta and the initial state), token by token.
+//
+// Per (sequence, head), with S' = Diag(exp g_t) S_{t-1} and u = v_t - S'^T k_t:
+//   S_t = S' + beta k u^T,   o_t = scale S_t^T q_t.
+// Walking the tokens backwards with L = dLoss/dS_t (the final-state gradient
+// at the end of the sequence):
+//   L   += scale q dO^T            dq = scale S_t dO
+//   lk   = L^T k                   dv = beta lk,   dbeta = lk . u
+//   dk   = beta (L u - S' lk)
+//   dS'  = L - beta k lk^T         dg_r = sum_c dS'_rc S'_rc
+//   L    = Diag(exp g) dS'         (and at the start, d initial state = L).
+// (The recurrence of page "Kimi K3 开源满月…", section "KDA 内核到底难在哪";
+// the pages name only a Triton implementation that trains, page "Moonshot AI …
+// FlashKDA … (kucoin)".)
+//
+// Work decomposition. Value columns evolve independently, so one warp owns
+// 16 value columns of one (sequence, head): lane l holds key rows 4l..4l+3 of
+// S and of L for those columns (64 + 64 fp32 registers). dv and the initial-
+// state gradient are column-local and written directly; dq, dk, dg and dbeta
+// sum over all 128 columns, so every warp writes its partial sums and a second
+// kernel adds the eight slices in a fixed order (deterministic results).
+// States are needed backwards in time: a first forward pass stores the state
+// every 4 tokens to global scratch; each 4-token block is then recomputed
+// from its checkpoint into lane-private shared memory and walked backwards.
+// Reductions over the keys (S'^T k, L^T k) are warp reduce-scatters followed
+// by gathers. This is the plain token-level form: every step is a rank-1
+// update, so it runs on the CUDA cores, not the tensor cores. The chain of
+// steps is serial, so every global load is taken off it: each block's token
+// inputs and checkpoint are copied into shared memory (cp.async) while the
+// previous block is being processed.
+
+#pragma once
+
+#include "kda_prims.cuh"
+
+namespace kda {
+namespace bwd {
+
+constexpr int NCOL = 8;               // value columns per warp
+constexpr int LOGC = 3;               // log2(NCOL)
+constexpr int NSLICE = D / NCOL;      // warps per (sequence, head)
+constexpr int BLK = 4;                // tokens per checkpoint block
+constexpr int WARPS = 2;              // warps per CTA (two slices of one head)
+constexpr int NF4 = NCOL;             // float4 of one lane's share of a state (4 keys x NCOL columns)
+static_assert(NCOL == (1 << LOGC) && NCOL % 8 == 0 && NCOL <= 16, "column slice");
+constexpr int NTHREADS = 32 * WARPS;
+constexpr int SLOT = 4 * NCOL;        // floats of one lane's share of a state
+
+// One token's inputs as the warp reads them from shared memory: this lane's
+// 4 keys of k, q (bf16) and g; the warp's 16 value columns of v and dO; beta.
+struct __align__(16) TokSmem {
+  uint2 k[32], q[32];
+  float4 g[32];
+  uint4 v[NCOL / 8], o[NCOL / 8];
+  float b;
+  float pad[3];
+};
+// Per warp: the block's states (BLK x 8 KB), two checkpoint buffers and two
+// token-block buffers (the block in use and the one being fetched).
+constexpr uint32_t STATE_BYTES = 32 * SLOT * 4;
+constexpr uint32_t WARP_SMEM = BLK * STATE_BYTES + 2 * STATE_BYTES + 2 * BLK * sizeof(TokSmem);
+constexpr uint32_t SMEM_BYTES = WARPS * WARP_SMEM;
+
+struct Params {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const __nv_bfloat16* dout;
+  const float* g;
+  const float* beta;
+  const int32_t* cu;       // may be null: one sequence [0, T)
+  const float* init;       // [N, H, 128, 128] or null
+  const float* dfin;       // [N, H, 128, 128] or null
+  float* dv;               // [T, H, 128]
+  float* dinit;            // [N, H, 128, 128] or null
+  float* pq;               // partials [NSLICE][T][H][128] of dq, dk, dg; [NSLICE][T][H] of dbeta
+  float* pk;
+  float* pg;
+  float* pb;
+  float* ck;               // checkpoints [(T / 4 + N + 1)][H][NSLICE][16 float4 of a lane][32 lanes]
+  int64_t T;
+  int64_t q_st, q_sh, k_st, k_sh, v_st, v_sh, o_st, o_sh, g_st, g_sh, b_st, b_sh;  // element strides
+  int H;
+  float scale;
+};
+
+// Sum over the 32 lanes of each of NCOL per-lane values; every lane gets all
+// NCOL sums. Reduce-scatter over lane bits 4, 3, ... (each step halves the
+// values a lane keeps), then plain butterflies over the remaining lane bits,
+// then a gather from a lane that holds each sum.
+__device__ __forceinline__ void allreduce(float (&x)[NCOL]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int w = NCOL / 2, off = 16; w >= 1; w >>= 1, off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      const float send = upper ? x[i] : x[w + i];
+      const float got = __shfl_xor_sync(0xffffffffu, send, off);
+      x[i] = (upper ? x[w + i] : x[i]) + got;
+    }
+  }
+  float mine = x[0];
+#pragma unroll
+  for (int off = 16 >> LOGC; off >= 1; off >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, off);
+  // lane l holds the sum of value (l >> (5 - LOGC))
+#pragma unroll
+  for (int c = 0; c < NCOL; ++c) x[c] = __shfl_sync(0xffffffffu, mine, c << (5 - LOGC));
+}
+
+struct Token {
+  float k[4], q[4], e[4];   // this lane's 4 keys
+  float v[NCOL], o[NCOL];   // the warp's value columns (v, dO)
+  float b;
+};
+
+__device__ __forceinline__ void cp16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp8(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Issue the copies of tokens [tb, tb + n) into buf (lane-specific parts by
+// every lane, the shared v / dO / beta by lanes 0-4).
+__device__ __forceinline__ void fetch_tokens(const Params& p, int64_t tb, int n, int h, int r0, int c0, int lane,
+                                             TokSmem* buf) {
+  for (int s = 0; s < n; ++s) {
+    const int64_t t = tb + s;
+    TokSmem& x = buf[s];
+    cp8(&x.k[lane], p.k + t * p.k_st + h * p.k_sh + r0);
+    cp8(&x.q[lane], p.q + t * p.q_st + h * p.q_sh + r0);
+    cp16(&x.g[lane], p.g + t * p.g_st + h * p.g_sh + r0);
+    constexpr int NV = NCOL / 8;  // 16-byte chunks of a row of the slice
+    if (lane < NV) cp16(&x.v[lane], p.v + t * p.v_st + h * p.v_sh + c0 + 8 * lane);
+    else if (lane < 2 * NV) cp16(&x.o[lane - NV], p.dout + t * p.o_st + h * p.o_sh + c0 + 8 * (lane - NV));
+    else if (lane == 2 * NV) cp_async4(&x.b, p.beta + t * p.b_st + h * p.b_sh, 4u);
+  }
+}
+
+__device__ __forceinline__ void read_token(const TokSmem& s, int lane, Token& x) {
+  const uint2 kk = s.k[lane], qq = s.q[lane];
+  const float4 gg = s.g[lane];
+  x.k[0] = __uint_as_float(kk.x << 16); x.k[1] = __uint_as_float(kk.x & 0xffff0000u);
+  x.k[2] = __uint_as_float(kk.y << 16); x.k[3] = __uint_as_float(kk.y & 0xffff0000u);
+  x.q[0] = __uint_as_float(qq.x << 16); x.q[1] = __uint_as_float(qq.x & 0xffff0000u);
+  x.q[2] = __uint_as_float(qq.y << 16); x.q[3] = __uint_as_float(qq.y & 0xffff0000u);
+  x.e[0] = __expf(gg.x); x.e[1] = __expf(gg.y); x.e[2] = __expf(gg.z); x.e[3] = __expf(gg.w);
+#pragma unroll
+  for (int half = 0; half < NCOL / 8; ++half) {
+    const uint4 vv = s.v[half], oo = s.o[half];
+    const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w}, ow[4] = {oo.x, oo.y, oo.z, oo.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x.v[8 * half + 2 * i] = __uint_as_float(vw[i] << 16);
+      x.v[8 * half + 2 * i + 1] = __uint_as_float(vw[i] & 0xffff0000u);
+      x.o[8 * half + 2 * i] = __uint_as_float(ow[i] << 16);
+      x.o[8 * half + 2 * i + 1] = __uint_as_float(ow[i] & 0xffff0000u);
+    }
+  }
+  x.b = s.b;
+}
+
+// One forward step S <- S' + beta k (v - S'^T k)^T on this lane's 4 x 16 share.
+__device__ __forceinline__ void step_forward(float (&S)[4][NCOL], const Token& x) {
+  float w[NCOL];
+#pragma unroll
+  for (int c = 0; c < NCOL; ++c) {
+    S[0][c] *= x.e[0];
+    S[1][c] *= x.e[1];
+    S[2][c] *= x.e[2];
+    S[3][c] *= x.e[3];
+    w[c] = fmaf(x.k[3], S[3][c], fmaf(x.k[2], S[2][c], fmaf(x.k[1], S[1][c], x.k[0] * S[0][c])));
+  }
+  allreduce(w);
+#pragma unroll
+  for (int c = 0; c < NCOL; ++c) {
+    const float bu = x.b * (x.v[c] - w[c]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) S[i][c] = fmaf(x.k[i], bu, S[i][c]);
+  }
+}
+
+// Grid (NSLICE / WARPS, H, N): warp w of CTA x owns value columns
+// NCOL (WARPS x + w) .. + NCOL - 1 of head y, sequence z.
+__global__ void __launch_bounds__(NTHREADS) kda_bwd_kernel(const Params p) {
+  extern __shared__ __align__(16) unsigned char smem_b[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int slice = WARPS * blockIdx.x + warp;
+  const int h = blockIdx.y, seq = blockIdx.z, H = p.H;
+  const int r0 = 4 * lane, c0 = NCOL * slice;
+  int64_t t0 = 0, t1 = p.T;
+  if (p.cu) {
+    check_bounds(p.cu, seq, gridDim.z, p.T);
+    t0 = p.cu[seq];
+    t1 = p.cu[seq + 1];
+    t0 = t0 < 0 ? 0 : (t0 > p.T ? p.T : t0);
+    t1 = t1 < t0 ? t0 : (t1 > p.T ? p.T : t1);
+  }
+  const int64_t len = t1 - t0;
+  const int64_t nblk = (len + BLK - 1) / BLK;
+  const size_t state_off = (static_cast<size_t>(seq) * H + h) * D * D;
+  // A lane's share of a state is NF4 float4 (key row i, columns 4 c4 .. +3 at
+  // element i NCOL / 4 + c4); the 32 lanes' element e are adjacent, so every
+  // access of a warp touches 512 contiguous bytes (conflict-free in shared
+  // memory).
+  // Checkpoint j of this warp: block index t0 / 4 + seq + j (the ranges of
+  // different sequences are disjoint and end below T / 4 + N + 1).
+  auto ck_ptr = [&](int64_t j) {
+    const int64_t blk = t0 / BLK + seq + j;
+    return reinterpret_cast<float4*>(p.ck + ((static_cast<size_t>(blk) * H + h) * NSLICE + slice) * (32 * SLOT)) +
+           lane;
+  };
+  unsigned char* wsm = smem_b + warp * WARP_SMEM;
+  float4* const st_base = reinterpret_cast<float4*>(wsm) + lane;                       // BLK states
+  float4* const ckb_base = reinterpret_cast<float4*>(wsm + BLK * STATE_BYTES) + lane;  // 2 checkpoint buffers
+  TokSmem* const tok_base = reinterpret_cast<TokSmem*>(wsm + (BLK + 2) * STATE_BYTES);  // 2 x BLK tokens
+  auto st_ptr = [&](int j) { return st_base + j * NF4 * 32; };
+  auto ckb_ptr = [&](int64_t j) { return ckb_base + (j & 1) * NF4 * 32; };
+  auto tok_ptr = [&](int64_t j) { return tok_base + (j & 1) * BLK; };
+  auto block_len = [&](int64_t j) {
+    const int64_t tb = t0 + j * BLK;
+    return static_cast<int>((tb + BLK < t1) ? BLK : t1 - tb);
+  };
+
+  // ---- forward pass: the state before every 4-token block
+  float S[4][NCOL];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int c = 0; c < NCOL; ++c)
+      S[i][c] = p.init ? p.init[state_off + static_cast<size_t>(r0 + i) * D + c0 + c] : 0.f;
+  if (nblk > 0) fetch_tokens(p, t0, block_len(0), h, r0, c0, lane, tok_ptr(0));
+  cp_commit();
+  for (int64_t j = 0; j < nblk; ++j) {
+    // next block's inputs in flight while this one runs
+    if (j + 1 < nblk) fetch_tokens(p, t0 + (j + 1) * BLK, block_len(j + 1), h, r0, c0, lane, tok_ptr(j + 1));
+    cp_commit();
+    float4* dst = ck_ptr(j);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int c4 = 0; c4 < NCOL / 4; ++c4)
+        dst[(i * (NCOL / 4) + c4) * 32] = make_float4(S[i][4 * c4], S[i][4 * c4 + 1], S[i][4 * c4 + 2], S[i][4 * c4 + 3]);
+    cp_wait<1>();
+    __syncwarp();
+    const TokSmem* tk = tok_ptr(j);
+    const int n = block_len(j);
+    for (int s = 0; s < n; ++s) {
+      Token x;
+      read_token(tk[s], lane, x);
+      step_forward(S, x);
+    }
+    __syncwarp();  // every lane is done with this buffer before it is refilled
+  }
+  cp_wait<0>();
+  // the checkpoints were written by this warp's own lanes: make them visible to
+  // the cp.async reads below
+  __threadfence_block();
+  __syncwarp();
+
+  // ---- backward pass
+  float L[4][NCOL];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int c = 0; c < NCOL; ++c)
+      L[i][c] = p.dfin ? p.dfin[state_off + static_cast<size_t>(r0 + i) * D + c0 + c] : 0.f;
+  const size_t pslice = static_cast<size_t>(slice) * static_cast<size_t>(p.T) * H;
+  auto fetch_block = [&](int64_t j) {
+    const float4* src = ck_ptr(j);
+    float4* dst = ckb_ptr(j);
+#pragma unroll
+    for (int e = 0; e < NF4; ++e) cp16(dst + e * 32, src + e * 32);
+    fetch_tokens(p, t0 + j * BLK, block_len(j), h, r0, c0, lane, tok_ptr(j));
+  };
+  if (nblk > 0) fetch_block(nblk - 1);
+  cp_commit();
+  for (int64_t j = nblk - 1; j >= 0; --j) {
+    const int64_t tb = t0 + j * BLK;
+    const int n = block_len(j);
+    if (j > 0) fetch_block(j - 1);
+    cp_commit();
+    cp_wait<1>();
+    __syncwarp();
+    const TokSmem* tk = tok_ptr(j);
+    // states before each token of the block: st[0] = checkpoint, st[i] after i steps
+    {
+      const float4* src = ckb_ptr(j);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int c4 = 0; c4 < NCOL / 4; ++c4) {
+          const float4 v4 = src[(i * (NCOL / 4) + c4) * 32];
+          S[i][4 * c4] = v4.x;
+          S[i][4 * c4 + 1] = v4.y;
+          S[i][4 * c4 + 2] = v4.z;
+          S[i][4 * c4 + 3] = v4.w;
+        }
+    }
+    for (int s = 0; s < n; ++s) {
+      float4* dst = st_ptr(s);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int c4 = 0; c4 < NCOL / 4; ++c4)
+          dst[(i * (NCOL / 4) + c4) * 32] = make_float4(S[i][4 * c4], S[i][4 * c4 + 1], S[i][4 * c4 + 2], S[i][4 * c4 + 3]);
+      if (s + 1 < n) {
+        Token x;
+        read_token(tk[s], lane, x);
+        step_forward(S, x);
+      }
+    }
+    for (int s = n - 1; s >= 0; --s) {
+      const int64_t t = tb + s;
+      Token x;
+      read_token(tk[s], lane, x);
+      // S' = Diag(exp g) S_{t-1} (from the block's stored state), reusing S
+      const float4* src = st_ptr(s);
+      float w[NCOL], lk[NCOL];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int c4 = 0; c4 < NCOL / 4; ++c4) {
+          const float4 v4 = src[(i * (NCOL / 4) + c4) * 32];
+          S[i][4 * c4] = v4.x * x.e[i];
+          S[i][4 * c4 + 1] = v4.y * x.e[i];
+          S[i][4 * c4 + 2] = v4.z * x.e[i];
+          S[i][4 * c4 + 3] = v4.w * x.e[i];
+        }
+      // L += scale q dO^T; partial sums over this lane's keys of S'^T k and L^T k
+#pragma unroll
+      for (int c = 0; c < NCOL; ++c) {
+        const float so = p.scale * x.o[c];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) L[i][c] = fmaf(x.q[i], so, L[i][c]);
+        w[c] = fmaf(x.k[3], S[3][c], fmaf(x.k[2], S[2][c], fmaf(x.k[1], S[1][c], x.k[0] * S[0][c])));
+        lk[c] = fmaf(x.k[3], L[3][c], fmaf(x.k[2], L[2][c], fmaf(x.k[1], L[1][c], x.k[0] * L[0][c])));
+      }
+      allreduce(w);
+      allreduce(lk);
+      float u[NCOL], db = 0.f;
+#pragma unroll
+      for (int c = 0; c < NCOL; ++c) {
+        u[c] = x.v[c] - w[c];
+        db = fmaf(lk[c], u[c], db);
+      }
+      // column-local: dv = beta lk (lane c writes column c)
+      float dvc = 0.f;
+#pragma unroll
+      for (int c = 0; c < NCOL; ++c) dvc = (lane == c) ? x.b * lk[c] : dvc;
+      if (lane < NCOL) p.dv[(static_cast<size_t>(t) * H + h) * D + c0 + lane] = dvc;
+      if (lane == 0) p.pb[pslice + static_cast<size_t>(t) * H + h] = db;
+      // per key (this lane's 4): dq, dk, dg; then L <- Diag(exp g) dS'
+      float dq[4], dk[4], dg[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float aq = 0.f, lu = 0.f, sl = 0.f, ag = 0.f;
+        const float bk = x.b * x.k[i];
+#pragma unroll
+        for (int c = 0; c < NCOL; ++c) {
+          const float st = fmaf(bk, u[c], S[i][c]);  // S_t = S' + beta k u^T
+          aq = fmaf(st, x.o[c], aq);
+          lu = fmaf(L[i][c], u[c], lu);
+          sl = fmaf(S[i][c], lk[c], sl);
+          const float dsp = fmaf(-bk, lk[c], L[i][c]);
+          ag = fmaf(dsp, S[i][c], ag);
+          L[i][c] = x.e[i] * dsp;
+        }
+        dq[i] = p.scale * aq;
+        dk[i] = x.b * (lu - sl);
+        dg[i] = ag;
+      }
+      const size_t po = (pslice + static_cast<size_t>(t) * H + h) * D + r0;
+      *reinterpret_cast<float4*>(p.pq + po) = make_float4(dq[0], dq[1], dq[2], dq[3]);
+      *reinterpret_cast<float4*>(p.pk + po) = make_float4(dk[0], dk[1], dk[2], dk[3]);
+      *reinterpret_cast<float4*>(p.pg + po) = make_float4(dg[0], dg[1], dg[2], dg[3]);
+    }
+    __syncwarp();  // every lane is done with this block's buffers before they are refilled
+  }
+  cp_wait<0>();
+  if (p.dinit) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int c = 0; c < NCOL; ++c) p.dinit[state_off + static_cast<size_t>(r0 + i) * D + c0 + c] = L[i][c];
+  }
+}
+
+// dq, dk, dg = the sum of the eight slices' partials, in slice order; dbeta
+// likewise. n4 = T * H * 128 / 4 float4 groups, nb = T * H.
+__global__ void __launch_bounds__(256) kda_bwd_reduce_kernel(const float* __restrict__ pq, const float* __restrict__ pk,
+                                                             const float* __restrict__ pg, const float* __restrict__ pb,
+                                                             float* dq, float* dk, float* dg, float* dbeta, int64_t n4,
+                                                             int64_t nb) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a, c = a;
+#pragma unroll
+    for (int s = 0; s < NSLICE; ++s) {
+      const float4 x = reinterpret_cast<const float4*>(pq)[s * n4 + i];
+      const float4 y = reinterpret_cast<const float4*>(pk)[s * n4 + i];
+      const float4 z = reinterpret_cast<const float4*>(pg)[s * n4 + i];
+      a.x += x.x; a.y += x.y; a.z += x.z; a.w += x.w;
+      b.x += y.x; b.y += y.y; b.z += y.z; b.w += y.w;
+      c.x += z.x; c.y += z.y; c.z += z.z; c.w += z.w;
+    }
+    reinterpret_cast<float4*>(dq)[i] = a;
+    reinterpret_cast<float4*>(dk)[i] = b;
+    reinterpret_cast<float4*>(dg)[i] = c;
+  }
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nb; i += stride) {
+    float a = 0.f;
+#pragma unroll
+    for (int s = 0; s < NSLICE; ++s) a += pb[s * nb + i];
+    dbeta[i] = a;
+  }
+}
+
+}  // namespace bwd
+}  // namespace kda

@@ -174,35 +174,32 @@ struct Params {
   int64_t out_st, out_sh;    // element strides of out over tokens and heads
   int32_t H;
   float scale;
-  // Launch modes of the time-split prefill (0 for a plain call):
-  //   kModeZeroV        the value tensor reads as zero (v is not loaded);
-  //   kModeIdentityInit every (sequence, head) starts from the 128 x 128
-  //                     identity (value column c = key c), which turns the
-  //                     final state into the segment's transition map;
-  //   kModeOutF32       o is written in fp32 to outf [T, H, 128] (token
-  //                     stride outf_st) instead of bf16 to out.
-  // Input mode of the fused preprocessing (any call; set together with the
-  // kernel instantiation FG = true, which is what implements it):
-  //   kModeFusedGate    q and k are raw projections, L2-normalised here per
-  //                     (token, head) (q / max(||q||, 1e-6)); g holds gate
-  //                     logits x, whose decay factor is exp(max(log sigmoid(x),
-  //                     lower_bound)) = max(sigmoid(x), exp_lb); beta holds
-  //                     logits b, used as sigmoid(b).
-  uint32_t mode;
-  float* outf;
-  int64_t outf_st;
-  float exp_lb;            // exp(lower_bound), kModeFusedGate only
+  float* outf;             // fp32 outputs [T, H, 128] (kModeOutF32 only)
+  int64_t outf_st;         // token stride of outf
+  float exp_lb;            // exp(lower_bound) (fused gate preprocessing only)
 };
-constexpr uint32_t kModeZeroV = 1u, kModeIdentityInit = 2u, kModeOutF32 = 4u, kModeFusedGate = 8u;
+// Launch modes of the time-split prefill (a template argument of the kernel;
+// 0 for a plain call):
+//   kModeZeroV        the value tensor reads as zero (v is not loaded);
+//   kModeIdentityInit every (sequence, head) starts from the 128 x 128
+//                     identity (value column c = key c), which turns the
+//                     final state into the segment's transition map;
+//   kModeOutF32       o is written in fp32 to outf (token stride outf_st)
+//                     instead of bf16 to out.
+constexpr uint32_t kModeZeroV = 1u, kModeIdentityInit = 2u, kModeOutF32 = 4u;
 constexpr float kNormEps2 = 1e-12f;  // (1e-6)^2: the norm floor of the fused normalisation, squared
 
 struct TensorMaps {
   CUtensorMap q, k, g, v;
 };
 
-// FG: the fused gate preprocessing (kModeFusedGate) is compiled in; the
-// plain kernel carries none of its code.
-template <int NS, bool FG>
+// FG: the fused gate preprocessing is compiled in: q and k are raw
+// projections, L2-normalised here per (token, head) (q / max(||q||, 1e-6));
+// g holds gate logits x, whose decay factor is exp(max(log sigmoid(x),
+// lower_bound)) = max(sigmoid(x), exp_lb); beta holds logits b, used as
+// sigmoid(b). MODE: the launch mode above. The plain kernel (FG = false,
+// MODE = 0) carries the code of neither.
+template <int NS, bool FG, uint32_t MODE>
 __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
     kda_fwd_kernel(const Params p, const __grid_constant__ TensorMaps tm) {
   constexpr int NSLICE = D / NS;   // CTAs per (sequence, head) = cluster size
@@ -279,7 +276,7 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
       for (int e = 0; e < 4; ++e) {
         const int key = 8 * u + 2 * tq + (e & 1);
         const int col = dv0 + cv + gq + 8 * (e >> 1);
-        sacc[u][e] = (p.mode & kModeIdentityInit) ? (key == col ? 1.f : 0.f)
+        sacc[u][e] = (MODE & kModeIdentityInit) ? (key == col ? 1.f : 0.f)
                      : p.init ? __ldg(p.init + sbase + static_cast<size_t>(key) * D + col) : 0.f;
       }
 
@@ -310,7 +307,7 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
       float xa[2][4], xb[2][4] = {};
       {
         uint32_t vt[4];
-        if (p.mode & kModeZeroV) {
+        if constexpr ((MODE & kModeZeroV) != 0u) {
           vt[0] = vt[1] = vt[2] = vt[3] = 0u;
         } else {
           ldsm_x4_t(vt, &st.v[(lane & 7) + ((lane >> 3) & 1) * 8][cv + (lane >> 4) * 8]);
@@ -400,7 +397,7 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
       }
       // the stage is no longer read by this warp
       mbar_arrive_warp(&sh.c_empty[s]);
-      if (p.mode & kModeOutF32) {
+      if constexpr ((MODE & kModeOutF32) != 0u) {
         // fp32 O: lane (gq, tq) of tile nt holds columns gq (+8) x tokens
         // 8nt + 2tq (+1)
         float* fbase = p.outf + static_cast<int64_t>(h) * D + dv0 + cv + gq;
@@ -411,23 +408,23 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
             const int tok = 8 * nt + 2 * tq + (e & 1);
             if (tok < m) fbase[(cs + tok) * p.outf_st + 8 * (e >> 1)] = (oa[nt][e] + ob[nt][e]) * p.scale;
           }
-        continue;
-      }
-      // ---- store O: an 8x8 transpose per tile turns (column, token pair) into
-      // (token, column pair)
-      uint32_t r[2][2];
+      } else {
+        // ---- store O: an 8x8 transpose per tile turns (column, token pair)
+        // into (token, column pair)
+        uint32_t r[2][2];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        r[nt][0] = movmatrix_t(pack_bf16((oa[nt][0] + ob[nt][0]) * p.scale, (oa[nt][1] + ob[nt][1]) * p.scale));
-        r[nt][1] = movmatrix_t(pack_bf16((oa[nt][2] + ob[nt][2]) * p.scale, (oa[nt][3] + ob[nt][3]) * p.scale));
-      }
+        for (int nt = 0; nt < 2; ++nt) {
+          r[nt][0] = movmatrix_t(pack_bf16((oa[nt][0] + ob[nt][0]) * p.scale, (oa[nt][1] + ob[nt][1]) * p.scale));
+          r[nt][1] = movmatrix_t(pack_bf16((oa[nt][2] + ob[nt][2]) * p.scale, (oa[nt][3] + ob[nt][3]) * p.scale));
+        }
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int tok = 8 * nt + gq;
-        if (tok < m) {
-          __nv_bfloat16* dst = out_base + (cs + tok) * out_st;
-          *reinterpret_cast<uint32_t*>(dst) = r[nt][0];
-          *reinterpret_cast<uint32_t*>(dst + 8) = r[nt][1];
+        for (int nt = 0; nt < 2; ++nt) {
+          const int tok = 8 * nt + gq;
+          if (tok < m) {
+            __nv_bfloat16* dst = out_base + (cs + tok) * out_st;
+            *reinterpret_cast<uint32_t*>(dst) = r[nt][0];
+            *reinterpret_cast<uint32_t*>(dst + 8) = r[nt][1];
+          }
         }
       }
     }
@@ -717,9 +714,9 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
         mbar_wait(&sh.c_empty[s], ph ^ 1u);
         mbar_wait_cl(&sh.ready[slot], static_cast<uint32_t>(n / RING) & 1u);
         fence_proxy_async_global();
-        mbar_arrive_expect_tx(&sh.c_full[s], (p.mode & kModeZeroV) ? kSlotBytes : chain_bytes<NS>());
+        mbar_arrive_expect_tx(&sh.c_full[s], (MODE & kModeZeroV) ? kSlotBytes : chain_bytes<NS>());
         bulk_g2s(&st.ops, ring + static_cast<size_t>(slot) * kSlotBytes, kSlotBytes, &sh.c_full[s]);
-        if (!(p.mode & kModeZeroV)) tma_load_3d(&st.v[0][0], &tm.v, dv0, h, tok, &sh.c_full[s]);
+        if constexpr ((MODE & kModeZeroV) == 0u) tma_load_3d(&st.v[0][0], &tm.v, dv0, h, tok, &sh.c_full[s]);
       }
     }
   }

@@ -23,26 +23,55 @@
 namespace kda {
 namespace split {
 
-constexpr int TOK = 64;         // tokens per tile of the correction
+constexpr int TOK = 32;         // tokens per tile (one pipeline stage)
+constexpr int NSTAGE = 4;       // tiles in flight per CTA
 constexpr int BP = D + 8;       // padded bf16 row pitch of the S_a tile (conflict-free ldmatrix)
-constexpr int NTHREADS = 256;   // 8 warps: 4 token tiles x 2 column halves
-constexpr uint32_t SMEM_BYTES = D * BP * 2u;
+constexpr int NCOMPUTE = 8;     // warps 0-7: 2 token halves x 4 column quarters; warp 8 issues the loads
+constexpr int NTHREADS = 32 * (NCOMPUTE + 1);
+// One stage: o_M as two 128-byte-swizzled boxes [32 tokens][64 bf16] and
+// o_loc as four boxes [32 tokens][32 fp32]; every box is 4 KB.
+constexpr uint32_t BOX_BYTES = TOK * 128u;
+constexpr uint32_t STAGE_BYTES = 6u * BOX_BYTES;
+constexpr uint32_t SA_OFF = NSTAGE * STAGE_BYTES;                      // S_a tile, bf16 [128 key][BP]
+constexpr uint32_t BAR_OFF = SA_OFF + D * BP * 2u;
+constexpr uint32_t SMEM_BYTES = BAR_OFF + 2u * NSTAGE * 8u + 1024u;   // + alignment slack
+static_assert((D * BP * 2u) % 8u == 0u, "barrier alignment");
+
+struct CorrectMaps {
+  CUtensorMap om, oloc;
+};
+
+// Byte offset of 16-byte chunk `c` of row `r` in a box written by TMA with
+// 128-byte swizzling (rows of 128 bytes, chunk index XOR row mod 8).
+__device__ __forceinline__ uint32_t sw128(int r, int c) { return static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4)); }
 
 // o[t] = bf16(o_loc[t] + S_a^T o_M[t]) for the tokens of the second half.
-// Grid (n, H), persistent over 64-token tiles: each CTA stages its head's S_a
+// Grid (n, H), persistent over 32-token tiles: each CTA stages its head's S_a
 // once, as one bf16 tile (the precision in which the chain itself feeds the
 // state to its products), and walks tiles blockIdx.x, blockIdx.x + n, ...
-// o_M is bf16 [T1, H, 128], o_loc fp32 [T1, H, 128]. Each warp issues all
-// loads of a tile (its o_M fragments and o_loc values) before its products.
-__global__ void __launch_bounds__(NTHREADS) split_correct_kernel(const float* __restrict__ oloc,
-                                                                 const __nv_bfloat16* __restrict__ om,
+// o_M is bf16 [T1, H, 128], o_loc fp32 [T1, H, 128], both read through TMA
+// into a 4-stage ring of shared memory so that enough bytes are in flight to
+// stream them at HBM speed.
+__global__ void __launch_bounds__(NTHREADS) split_correct_kernel(const __grid_constant__ CorrectMaps tm,
                                                                  const float* __restrict__ sa, __nv_bfloat16* out,
-                                                                 int64_t out_st, int64_t out_sh, int64_t T1, int H) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  __nv_bfloat16* bs = reinterpret_cast<__nv_bfloat16*>(smem_raw);   // [128 key][BP]
+                                                                 int64_t out_st, int64_t out_sh, int64_t T1) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __nv_bfloat16* bs = reinterpret_cast<__nv_bfloat16*>(sm + SA_OFF);
+  unsigned long long* full = reinterpret_cast<unsigned long long*>(sm + BAR_OFF);
+  unsigned long long* empty = full + NSTAGE;
   const int h = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int gq = lane >> 2, tq = lane & 3;
+  const int ntiles = static_cast<int>((T1 + TOK - 1) / TOK);
+  const int first = blockIdx.x, step = gridDim.x;
+  const int mine = first < ntiles ? (ntiles - first + step - 1) / step : 0;
+  if (tid == 0) {
+    for (int i = 0; i < NSTAGE; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], NCOMPUTE);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
   const float* S = sa + static_cast<size_t>(h) * D * D;
   for (int i = tid; i < D * D / 4; i += NTHREADS) {
     const int key = (4 * i) / D, col = (4 * i) % D;
@@ -53,53 +82,64 @@ __global__ void __launch_bounds__(NTHREADS) split_correct_kernel(const float* __
     *reinterpret_cast<uint2*>(bs + key * BP + col) = pk;
   }
   __syncthreads();
-  const int mt = warp & 3, nh = warp >> 2;
-  const size_t rstride = static_cast<size_t>(H) * D;  // o_loc and o_M rows
-  for (int64_t t0 = static_cast<int64_t>(blockIdx.x) * TOK; t0 < T1; t0 += static_cast<int64_t>(gridDim.x) * TOK) {
-    const int64_t row0 = t0 + 16 * mt + gq, row1 = row0 + 8;
-    const bool v0 = row0 < T1, v1 = row1 < T1;
-    const uint32_t* a0p = reinterpret_cast<const uint32_t*>(om + static_cast<size_t>(row0) * rstride + h * D);
-    const uint32_t* a1p = reinterpret_cast<const uint32_t*>(om + static_cast<size_t>(row1) * rstride + h * D);
-    const float* l0p = oloc + static_cast<size_t>(row0) * rstride + static_cast<size_t>(h) * D + 64 * nh + 2 * tq;
-    const float* l1p = oloc + static_cast<size_t>(row1) * rstride + static_cast<size_t>(h) * D + 64 * nh + 2 * tq;
-    uint32_t a[D / 16][4];
-    float2 l[8][2];
-#pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      const int kw = 8 * ks + tq;  // 32-bit word of keys 16 ks + 2 tq (+1)
-      a[ks][0] = v0 ? a0p[kw] : 0u;
-      a[ks][1] = v1 ? a1p[kw] : 0u;
-      a[ks][2] = v0 ? a0p[kw + 4] : 0u;
-      a[ks][3] = v1 ? a1p[kw + 4] : 0u;
-    }
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      l[nt][0] = v0 ? *reinterpret_cast<const float2*>(l0p + 8 * nt) : make_float2(0.f, 0.f);
-      l[nt][1] = v1 ? *reinterpret_cast<const float2*>(l1p + 8 * nt) : make_float2(0.f, 0.f);
-    }
-    float acc[8][4] = {};
-#pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-#pragma unroll
-      for (int np = 0; np < 4; ++np) {  // pairs of 8-column tiles
-        const int c = 64 * nh + 16 * np;
-        uint32_t b[4];
-        ldsm_x4_t(b, bs + (16 * ks + (lane & 7) + ((lane >> 3) & 1) * 8) * BP + c + (lane >> 4) * 8);
-        mma(acc[2 * np], a[ks], b[0], b[1]);
-        mma(acc[2 * np + 1], a[ks], b[2], b[3]);
+  if (warp == NCOMPUTE) {
+    // ---- loads: tile j of this CTA into stage j % NSTAGE
+    if (lane == 0) {
+      for (int j = 0; j < mine; ++j) {
+        const int st = j % NSTAGE;
+        if (j >= NSTAGE) mbar_wait(&empty[st], ((j / NSTAGE) - 1) & 1);
+        const int tok = (first + j * step) * TOK;
+        unsigned char* dst = sm + st * STAGE_BYTES;
+        mbar_arrive_expect_tx(&full[st], STAGE_BYTES);
+        tma_load_3d(dst, &tm.om, 0, h, tok, &full[st]);
+        tma_load_3d(dst + BOX_BYTES, &tm.om, 64, h, tok, &full[st]);
+        for (int b = 0; b < 4; ++b) tma_load_3d(dst + (2 + b) * BOX_BYTES, &tm.oloc, 32 * b, h, tok, &full[st]);
       }
     }
-    // epilogue: + o_loc, one rounding to bf16
+    return;
+  }
+  const int th = warp & 1, cq = warp >> 1;  // token half, column quarter (32 value columns)
+  const int gq = lane >> 2, tq = lane & 3;
+  for (int j = 0; j < mine; ++j) {
+    const int st = j % NSTAGE;
+    mbar_wait(&full[st], (j / NSTAGE) & 1);
+    const unsigned char* stage = sm + st * STAGE_BYTES;
+    float acc[4][4] = {};
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const int col = 64 * nh + 8 * nt + 2 * tq;
-      if (v0)
-        *reinterpret_cast<uint32_t*>(out + row0 * out_st + static_cast<int64_t>(h) * out_sh + col) =
-            pack_bf16(l[nt][0].x + acc[nt][0], l[nt][0].y + acc[nt][1]);
-      if (v1)
-        *reinterpret_cast<uint32_t*>(out + row1 * out_st + static_cast<int64_t>(h) * out_sh + col) =
-            pack_bf16(l[nt][1].x + acc[nt][2], l[nt][1].y + acc[nt][3]);
+    for (int ks = 0; ks < D / 16; ++ks) {
+      // A: 16 tokens x 16 keys of o_M (box ks / 4, chunks 2 (ks % 4) and +1)
+      uint32_t a[4];
+      const int r = 16 * th + (lane & 15);
+      ldsm_x4(a, stage + (ks >> 2) * BOX_BYTES + sw128(r, 2 * (ks & 3) + (lane >> 4)));
+#pragma unroll
+      for (int np = 0; np < 2; ++np) {  // pairs of 8-column tiles of this warp's 32 columns
+        const int c = 32 * cq + 16 * np;
+        uint32_t b[4];
+        ldsm_x4_t(b, bs + (16 * ks + (lane & 7) + ((lane >> 3) & 1) * 8) * BP + c + (lane >> 4) * 8);
+        mma(acc[2 * np], a, b[0], b[1]);
+        mma(acc[2 * np + 1], a, b[2], b[3]);
+      }
     }
+    // epilogue: + o_loc (box cq of the stage), one rounding to bf16
+    const unsigned char* lbox = stage + (2 + cq) * BOX_BYTES;
+    const int64_t tok0 = static_cast<int64_t>(first + j * step) * TOK + 16 * th;
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int r = 16 * th + gq + 8 * hr;
+      const int64_t row = tok0 + gq + 8 * hr;
+      float2 l[4];
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt)
+        l[nt] = *reinterpret_cast<const float2*>(lbox + sw128(r, 2 * nt + (tq >> 1)) + 8 * (tq & 1));
+      if (row < T1) {
+        __nv_bfloat16* o = out + row * out_st + static_cast<int64_t>(h) * out_sh + 32 * cq + 2 * tq;
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+          *reinterpret_cast<uint32_t*>(o + 8 * nt) =
+              pack_bf16(l[nt].x + acc[nt][2 * hr], l[nt].y + acc[nt][2 * hr + 1]);
+      }
+    }
+    mbar_arrive_warp(&empty[st]);
   }
 }
 

@@ -340,3 +340,42 @@ def test_fused_rejects_lower_bound_and_bad_tensors(lib):
     assert run(-5.0, g=desc(0x40000, BF16, [64, 2, 128])) == KDA_ERR_DTYPE
     assert run(-2.0, beta=desc(0x50000, F32, [64, 3])) == KDA_ERR_SHAPE
     assert run(-1.0, k=desc(0x20000, BF16, [64, 2, 128], [256, 128, 2])) == KDA_ERR_STRIDE
+
+
+# -------------------------------------------------------------- backward
+def test_bwd_rejects_bad_arguments(lib):
+    P = ctypes.POINTER(Desc)
+    lib.kda_bwd.argtypes = [P, P, P, P, P, ctypes.c_float, ctypes.c_void_p, ctypes.c_int32, P, P, P, P, P, P, P, P, P,
+                            ctypes.c_void_p]
+    lib.kda_bwd.restype = ctypes.c_int
+    T, H = 64, 2
+    base = {
+        "q": desc(0x10000, BF16, [T, H, 128]), "k": desc(0x20000, BF16, [T, H, 128]),
+        "v": desc(0x30000, BF16, [T, H, 128]), "g": desc(0x40000, F32, [T, H, 128]),
+        "beta": desc(0x50000, F32, [T, H]), "init": None, "dout": desc(0x60000, BF16, [T, H, 128]), "dfin": None,
+        "dq": desc(0x100000, F32, [T, H, 128]), "dk": desc(0x200000, F32, [T, H, 128]),
+        "dv": desc(0x300000, F32, [T, H, 128]), "dg": desc(0x400000, F32, [T, H, 128]),
+        "dbeta": desc(0x500000, F32, [T, H]), "dinit": None,
+    }
+
+    def run(**over):
+        t = dict(base)
+        t.update(over)
+        r = {n: (None if d is None else ctypes.byref(d)) for n, d in t.items()}
+        return lib.kda_bwd(r["q"], r["k"], r["v"], r["g"], r["beta"], 1.0, 0x70000, 1, r["init"], r["dout"], r["dfin"],
+                           r["dq"], r["dk"], r["dv"], r["dg"], r["dbeta"], r["dinit"], None)
+
+    for name in ("q", "dout", "dq", "dk", "dv", "dg", "dbeta"):
+        assert run(**{name: None}) == KDA_ERR_NULL, name
+    assert run(dout=desc(0x60000, F32, [T, H, 128])) == KDA_ERR_DTYPE
+    assert run(dq=desc(0x100000, BF16, [T, H, 128])) == KDA_ERR_DTYPE
+    assert run(dbeta=desc(0x500000, BF16, [T, H])) == KDA_ERR_DTYPE
+    assert run(dk=desc(0x200000, F32, [T, H, 64])) == KDA_ERR_SHAPE
+    assert run(dbeta=desc(0x500000, F32, [T, H + 1])) == KDA_ERR_SHAPE
+    assert run(dout=desc(0x60000, BF16, [T + 1, H, 128])) == KDA_ERR_SHAPE
+    # gradients must be contiguous; dout may be strided like the inputs
+    assert run(dg=desc(0x400000, F32, [T, H, 128], [H * 256, 256, 1])) == KDA_ERR_STRIDE
+    assert run(dbeta=desc(0x500000, F32, [T, H], [2 * H, 2])) == KDA_ERR_STRIDE
+    assert run(dq=desc(0x100004, F32, [T, H, 128])) == KDA_ERR_ALIGN
+    assert run(dinit=desc(0x600000, F32, [1, H, 128, 64])) == KDA_ERR_SHAPE
+    assert run(dfin=desc(0x600000, BF16, [1, H, 128, 128])) == KDA_ERR_DTYPE
