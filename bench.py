@@ -477,14 +477,15 @@ BWD_BYTES_PER_TOKHEAD = 3 * D * 2 + D * 4 + 4 + D * 2 + 4 * D * 4 + 4
 FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
-def bwd_entry(kda, dev, stream, steps: int):
-    """kda_bwd on the Kimi-Linear-shaped workload (T=8192, H=32) with a random
-    output gradient: device time per launch (inputs larger than L2 with the
-    gradients) and its roofline on the fp32 CUDA cores."""
+def bwd_entry(kda, dev, stream, steps: int, tokens: int = 8192):
+    """kda_bwd on the Kimi-Linear-shaped workload (T=8192, H=32; `tokens`
+    shortens it, for profiling captures) with a random output gradient: device
+    time per launch (L2 flushed between launches) and its roofline on the fp32
+    CUDA cores."""
     import torch
 
     wl = kda_inputs.workload(2)
-    inp = wl.make()
+    inp = kda_inputs.make_inputs([tokens], wl.num_heads, wl.seed) if tokens != wl.total_tokens else wl.make()
     t = lambda a: torch.from_numpy(a).to(dev)
     q, k, v = (t(x).view(torch.bfloat16) for x in (inp.q, inp.k, inp.v))
     g, beta = t(inp.g), t(inp.beta)
@@ -498,7 +499,8 @@ def bwd_entry(kda, dev, stream, steps: int):
     units = work_units(inp)
     tflops = units * BWD_FLOPS_PER_TOKHEAD / (ms * 1e-3) / 1e12
     gbs = units * BWD_BYTES_PER_TOKHEAD / (ms * 1e-3) / 1e9
-    return {"workload": wl.name + " (gradients of q, k, v, g, beta)", "ms": ms,
+    name = wl.name if tokens == wl.total_tokens else f"fixed_T{tokens}_H{wl.num_heads}"
+    return {"workload": name + " (gradients of q, k, v, g, beta)", "ms": ms,
             "value": units / (ms * 1e-3) / 1e6, "unit": UNIT,
             "roofline": {"bound": "alu", "achieved": tflops, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
                          "frac": tflops / FP32_ALU_TFLOPS,
@@ -524,9 +526,14 @@ def run_kda(args):
     import kimi_delta_attention_26_b200 as kda
 
     kda.set_path(args.path)
-    if args.only_decode:
+    if args.only:
+        st = torch.cuda.current_stream(dev)
         if rank == 0:
-            print(json.dumps(decode_entry(kda, dev, torch.cuda.current_stream(dev), args.steps)), flush=True)
+            if args.only == "backward":
+                res = bwd_entry(kda, dev, st, args.steps, args.bwd_tokens)
+            else:
+                res = {"decode": decode_entry, "fused": fused_entry}[args.only](kda, dev, st, args.steps)
+            print(json.dumps(res), flush=True)
         if ws > 1:
             dist.barrier()
             dist.destroy_process_group()
@@ -659,8 +666,11 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip the per-workload table (every workload, both kernel paths)")
-    ap.add_argument("--only-decode", action="store_true",
-                    help="time only the decode step (256 requests, H=32) and print its JSON object")
+    ap.add_argument("--only", choices=["decode", "fused", "backward"],
+                    help="time only that entry (decode step, fused-preprocessing prefill or backward) and print its "
+                         "JSON object")
+    ap.add_argument("--bwd-tokens", type=int, default=8192,
+                    help="sequence length of the backward entry (H=32); shorter for profiling captures")
     ap.add_argument("--path", type=int, default=0, choices=[0, 16, 64],
                     help="kernel: 0 = library default (16-token chunks on mma.sync, time split where it wins), "
                          "16 = 16-token chunks, 64 = 64-token chunks on tcgen05")

@@ -84,3 +84,28 @@ def test_bwd_full_size_uniform_varlen(kda, oracle_mod):
     inp = kda_inputs.workload(3).make()
     _grads(kda, oracle_mod, inp, 105, "bwd 8x1024 H=32 (full)")
     assert kda.device_status(reset=True) == 0
+
+
+@pytest.mark.parametrize("fill", [-5.0, 0.0])
+def test_bwd_gate_extremes(kda, oracle_mod, fill):
+    inp = kda_inputs.make_inputs([50, 9], 2, seed=106, random_initial_state=True)
+    inp.g[:] = fill
+    _grads(kda, oracle_mod, inp, 107, f"bwd g={fill}")
+
+
+def test_bwd_strided_views_bitwise_equal_contiguous(kda):
+    """q, k, v as slices of one fused projection and dout as a head-major view
+    give the same bits as contiguous tensors."""
+    import torch
+
+    inp = kda_inputs.make_inputs([130, 21], 3, seed=108, random_initial_state=True)
+    d = H.to_device(inp)
+    dout = torch.randn((inp.total_tokens, 3, 128), device="cuda").bfloat16()
+    ref = kda.kda_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], dout, inp.scale, d["cu_seqlens"], d["initial_state"])
+    fused = torch.cat([d["q"], d["k"], d["v"]], dim=2)
+    dout_hm = dout.transpose(0, 1).contiguous().transpose(0, 1)
+    got = kda.kda_bwd(fused[:, :, :128], fused[:, :, 128:256], fused[:, :, 256:], d["g"], d["beta"], dout_hm,
+                      inp.scale, d["cu_seqlens"], d["initial_state"])
+    torch.cuda.synchronize()
+    for n in ref:
+        assert torch.equal(ref[n], got[n]), n

@@ -136,3 +136,38 @@ def test_decode_full_size_workload(kda, oracle_mod):
     torch.cuda.synchronize()
     H.assert_parity(out, state, o_ref, f_ref, label="decode B=256 H=32 (full)")
     assert kda.device_status(reset=True) == 0
+
+
+@pytest.mark.parametrize("fill", [-5.0, 0.0])
+def test_decode_gate_extremes_and_no_write(kda, oracle_mod, fill):
+    """g at the lower bound or at 0 everywhere; then beta = 0 (the state only
+    decays and the output reads it)."""
+    import torch
+
+    inp = kda_inputs.make_inputs([1] * 19, 2, seed=65, random_initial_state=True)
+    inp.g[:] = fill
+    for beta0 in (False, True):
+        if beta0:
+            inp.beta[:] = 0.0
+        o_ref, f_ref = oracle_mod.scan_inputs(inp)
+        t = _step_inputs(inp, slice(None))
+        state = torch.from_numpy(inp.initial_state).cuda()
+        out = kda.kda_decode(t["q"], t["k"], t["v"], t["g"], t["beta"], state, scale=inp.scale)
+        torch.cuda.synchronize()
+        H.assert_parity(out, state, o_ref, f_ref, label=f"decode g={fill} beta0={beta0}")
+
+
+def test_decode_reversed_slot_order(kda):
+    """A permutation of the pool (request b uses slot B - 1 - b) gives the same
+    bits as the identity order on the permuted states."""
+    import torch
+
+    inp = kda_inputs.make_inputs([1] * 12, 3, seed=66, random_initial_state=True)
+    t = _step_inputs(inp, slice(None))
+    s0 = torch.from_numpy(inp.initial_state).cuda()
+    pool = s0.flip(0).contiguous()
+    idx = torch.arange(11, -1, -1, dtype=torch.int32, device="cuda")
+    o1 = kda.kda_decode(t["q"], t["k"], t["v"], t["g"], t["beta"], s0, scale=inp.scale)
+    o2 = kda.kda_decode(t["q"], t["k"], t["v"], t["g"], t["beta"], pool, scale=inp.scale, state_indices=idx)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(pool.flip(0), s0)

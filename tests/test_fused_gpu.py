@@ -101,3 +101,20 @@ def test_fused_full_size_kimi_linear_shape(kda, oracle_mod):
     inp = wl.make(raw=True)
     _check(kda, oracle_mod, inp, "fused T=8192 H=32", col_ranges=[(8, 16), (40, 48), (72, 80), (104, 112)])
     assert kda.wait_timeouts(reset=True) == 0
+
+
+def test_fused_heavy_clamp_and_strided_projection(kda, oracle_mod):
+    """lower_bound = -0.5 clamps most gates; raw q, k, v as slices of one fused
+    projection give the same bits as contiguous tensors."""
+    import torch
+
+    inp = kda_inputs.make_inputs([120, 33], 2, seed=83, raw=True, random_initial_state=True)
+    _check(kda, oracle_mod, inp, "fused lb=-0.5", lower_bound=-0.5)
+    d = _raw_device(inp)
+    ref = kda.kda_fwd_fused(d["q"], d["k"], d["v"], d["g"], d["beta"], inp.scale, -0.5, cu_seqlens=d["cu_seqlens"],
+                            initial_state=d["initial_state"])
+    proj = torch.cat([d["q"], d["k"], d["v"]], dim=2)
+    got = kda.kda_fwd_fused(proj[:, :, :128], proj[:, :, 128:256], proj[:, :, 256:], d["g"], d["beta"], inp.scale, -0.5,
+                            cu_seqlens=d["cu_seqlens"], initial_state=d["initial_state"])
+    torch.cuda.synchronize()
+    assert torch.equal(ref[0], got[0]) and torch.equal(ref[1], got[1])
