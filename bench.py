@@ -644,10 +644,18 @@ def run_kda(args):
         if ws == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(inp, args.cpu_seconds)
         if ws == 1 and not args.no_per_config:
-            line["per_config"] = per_config_table(kda, dev, stream, min(args.steps, 20), (0, 64))
-            line["decode"] = decode_entry(kda, dev, stream, min(args.steps, 20))
-            line["fused_gate"] = fused_entry(kda, dev, stream, min(args.steps, 20))
-            line["backward"] = bwd_entry(kda, dev, stream, min(args.steps, 5))
+            # the extra entries never cost the headline line: a failure is recorded in its place
+            extras = [("per_config", lambda: per_config_table(kda, dev, stream, min(args.steps, 20), (0, 64))),
+                      ("decode", lambda: decode_entry(kda, dev, stream, min(args.steps, 20))),
+                      ("fused_gate", lambda: fused_entry(kda, dev, stream, min(args.steps, 20))),
+                      ("backward", lambda: bwd_entry(kda, dev, stream, min(args.steps, 5)))]
+            for key, fn in extras:
+                try:
+                    line[key] = fn()
+                except Exception as e:  # reported, not hidden: the value names the failure
+                    log(f"{key} entry failed: {e!r}")
+                    line[key] = {"error": repr(e)}
+                    kda.set_path(args.path)
         print(json.dumps(line), flush=True)
     if ws > 1:
         dist.barrier()
