@@ -298,9 +298,9 @@ kda_status_t kda_decode(const kda_tensor_t* q, const kda_tensor_t* k, const kda_
  * dbeta [T, H]; dinitial_state [N, H, 128, 128] or NULL (not written). The
  * gradient of g is for the natural-log decay itself.
  * Scratch from the pool: a state checkpoint every 4 tokens (16 KiB per token
- * and head) and per-slice partial sums of dq, dk, dg (24 KiB per token and
- * head), about 41 KB per token and head in all (T = 8192, H = 32: 11 GB).
- * Results are deterministic. Runs on the CUDA cores (rank-1 updates token by token): much
+ * and head) and four partial sums of dq, dk, dg (6 KiB per token and head),
+ * about 23 KB per token and head in all (T = 8192, H = 32: 6 GB). Results
+ * are deterministic. Runs on the CUDA cores (rank-1 updates token by token): much
  * slower than kda_fwd. Errors as for kda_fwd; nothing is enqueued on any
  * error. Returns KDA_OK once the work is enqueued.
  */

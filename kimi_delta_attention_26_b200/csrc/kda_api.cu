@@ -475,9 +475,10 @@ size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 // helper streams; then o = o_loc + S_a^T o_M and S_T = M S_a + B.
 kda_status_t launch16_split(const Problem& P, int dev, cudaStream_t stream) {
   namespace sp = kda::split;
-  // The zero-start run writes fp32 outputs and runs ~6 % slower per token than
-  // the first half, so the first half takes ~51.6 % of the tokens (measured).
-  const int64_t T = P.T, Ta = (T * 33 / 64) & ~static_cast<int64_t>(kda::C - 1), T1 = T - Ta;
+  // Measured on B200 (T = 131072, H = 8), the first half runs ~4 % slower per
+  // token than the zero-start run of the second half (the identity run, with
+  // v = 0, is faster still), so the first half takes ~49 % of the tokens.
+  const int64_t T = P.T, Ta = (T * 63 / 128) & ~static_cast<int64_t>(kda::C - 1), T1 = T - Ta;
   const int H = P.num_heads;
   const size_t st_bytes = round256(static_cast<size_t>(H) * kda::D * kda::D * 4);
   const size_t o_bytes = round256(static_cast<size_t>(T1) * H * kda::D * 4);     // o_loc, fp32
@@ -718,8 +719,8 @@ kda_status_t kda_bwd(const kda_tensor_t* q, const kda_tensor_t* k, const kda_ten
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   namespace b = kda::bwd;
   const size_t ck_bytes = round256(static_cast<size_t>(T / b::BLK + N + 1) * H * b::NSLICE * 32 * b::SLOT * 4);
-  const size_t part_bytes = round256(static_cast<size_t>(b::NSLICE) * T * H * kda::D * 4);
-  const size_t pb_bytes = round256(static_cast<size_t>(b::NSLICE) * T * H * 4);
+  const size_t part_bytes = round256(static_cast<size_t>(b::NPART) * T * H * kda::D * 4);
+  const size_t pb_bytes = round256(static_cast<size_t>(b::NPART) * T * H * 4);
   void* scratch = nullptr;
   cudaError_t e = cudaMallocFromPoolAsync(&scratch, ck_bytes + 3 * part_bytes + pb_bytes, g_pool[dev].load(), cs);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -750,8 +751,8 @@ kda_status_t kda_bwd(const kda_tensor_t* q, const kda_tensor_t* k, const kda_ten
   p.b_st = P.beta.st; p.b_sh = P.beta.sh;
   p.H = static_cast<int>(H);
   p.scale = scale;
-  b::kda_bwd_kernel<<<dim3(b::NSLICE / b::WARPS, static_cast<unsigned>(H), static_cast<unsigned>(N)), b::NTHREADS,
-                      b::SMEM_BYTES, cs>>>(p);
+  b::kda_bwd_kernel<<<dim3(b::NPART, static_cast<unsigned>(H), static_cast<unsigned>(N)), b::NTHREADS, b::SMEM_BYTES,
+                      cs>>>(p);
   if (T > 0) {
     const int64_t n4 = T * H * kda::D / 4, nb = T * H;
     const int64_t blocks = std::min<int64_t>((n4 + 255) / 256, 8 * static_cast<int64_t>(g_num_sms[dev]));

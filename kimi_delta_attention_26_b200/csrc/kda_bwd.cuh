@@ -37,30 +37,38 @@
 namespace kda {
 namespace bwd {
 
-constexpr int NCOL = 8;               // value columns per warp
-constexpr int LOGC = 3;               // log2(NCOL)
+constexpr int NCOL = 4;               // value columns per warp
+constexpr int LOGC = 2;               // log2(NCOL)
 constexpr int NSLICE = D / NCOL;      // warps per (sequence, head)
 constexpr int BLK = 4;                // tokens per checkpoint block
-constexpr int WARPS = 2;              // warps per CTA (two slices of one head)
-constexpr int NF4 = NCOL;             // float4 of one lane's share of a state (4 keys x NCOL columns)
-static_assert(NCOL == (1 << LOGC) && NCOL % 8 == 0 && NCOL <= 16, "column slice");
+constexpr int WARPS = 8;              // warps per CTA: 32 value columns of one head
+constexpr int NPART = NSLICE / WARPS; // CTAs per (sequence, head) = partial sums per gradient
+constexpr int CCOL = NCOL * WARPS;    // value columns per CTA
 constexpr int NTHREADS = 32 * WARPS;
 constexpr int SLOT = 4 * NCOL;        // floats of one lane's share of a state
+constexpr int NF4 = NCOL;             // float4 of one lane's share of a state (4 keys x NCOL columns)
+static_assert(NCOL == (1 << LOGC) && NCOL == 4, "the token layout below assumes 4 columns per warp");
 
-// One token's inputs as the warp reads them from shared memory: this lane's
-// 4 keys of k, q (bf16) and g; the warp's 16 value columns of v and dO; beta.
+// One token's inputs for the CTA: k, q (bf16) and g for all 128 keys, v and dO
+// for the CTA's 32 value columns, beta.
 struct __align__(16) TokSmem {
-  uint2 k[32], q[32];
-  float4 g[32];
-  uint4 v[NCOL / 8], o[NCOL / 8];
+  __nv_bfloat16 k[D], q[D];
+  float g[D];
+  __nv_bfloat16 v[CCOL], o[CCOL];
   float b;
   float pad[3];
 };
-// Per warp: the block's states (BLK x 8 KB), two checkpoint buffers and two
-// token-block buffers (the block in use and the one being fetched).
+constexpr int TOK_CHUNKS = (2 * D * 2 + D * 4 + 2 * CCOL * 2) / 16;  // 16-byte copies per token (beta apart)
+
+// Shared memory: per warp the block's states and two checkpoint buffers; per
+// CTA two token-block buffers and the per-token partial sums of the 8 warps.
 constexpr uint32_t STATE_BYTES = 32 * SLOT * 4;
-constexpr uint32_t WARP_SMEM = BLK * STATE_BYTES + 2 * STATE_BYTES + 2 * BLK * sizeof(TokSmem);
-constexpr uint32_t SMEM_BYTES = WARPS * WARP_SMEM;
+constexpr uint32_t WARP_SMEM = BLK * STATE_BYTES + 2 * STATE_BYTES;
+constexpr uint32_t TOK_OFF = WARPS * WARP_SMEM;
+constexpr uint32_t RED_OFF = TOK_OFF + 2 * BLK * sizeof(TokSmem);
+constexpr uint32_t RED_BYTES = BLK * 3 * WARPS * 32 * 16;   // [token][dq, dk, dg][warp][lane] float4
+constexpr uint32_t REDB_OFF = RED_OFF + RED_BYTES;
+constexpr uint32_t SMEM_BYTES = REDB_OFF + BLK * WARPS * 4;
 
 struct Params {
   const __nv_bfloat16* q;
@@ -74,11 +82,11 @@ struct Params {
   const float* dfin;       // [N, H, 128, 128] or null
   float* dv;               // [T, H, 128]
   float* dinit;            // [N, H, 128, 128] or null
-  float* pq;               // partials [NSLICE][T][H][128] of dq, dk, dg; [NSLICE][T][H] of dbeta
+  float* pq;               // partials [NPART][T][H][128] of dq, dk, dg; [NPART][T][H] of dbeta
   float* pk;
   float* pg;
   float* pb;
-  float* ck;               // checkpoints [(T / 4 + N + 1)][H][NSLICE][16 float4 of a lane][32 lanes]
+  float* ck;               // checkpoints [(T / 4 + N + 1)][H][NSLICE][NF4 float4 of a lane][32 lanes]
   int64_t T;
   int64_t q_st, q_sh, k_st, k_sh, v_st, v_sh, o_st, o_sh, g_st, g_sh, b_st, b_sh;  // element strides
   int H;
@@ -118,52 +126,53 @@ struct Token {
 __device__ __forceinline__ void cp16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp8(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
 __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Issue the copies of tokens [tb, tb + n) into buf (lane-specific parts by
-// every lane, the shared v / dO / beta by lanes 0-4).
-__device__ __forceinline__ void fetch_tokens(const Params& p, int64_t tb, int n, int h, int r0, int c0, int lane,
-                                             TokSmem* buf) {
-  for (int s = 0; s < n; ++s) {
+// Issue the copies of tokens [tb, tb + n) into buf, spread over the CTA's
+// threads: per token TOK_CHUNKS 16-byte pieces (k, q, g rows of head h; v and
+// dO of the CTA's columns cc0 ..) and beta.
+__device__ __forceinline__ void fetch_tokens(const Params& p, int64_t tb, int n, int h, int cc0, TokSmem* buf) {
+  constexpr int PER = TOK_CHUNKS + 1;
+  for (int i = threadIdx.x; i < n * PER; i += NTHREADS) {
+    const int s = i / PER, c = i % PER;
     const int64_t t = tb + s;
     TokSmem& x = buf[s];
-    cp8(&x.k[lane], p.k + t * p.k_st + h * p.k_sh + r0);
-    cp8(&x.q[lane], p.q + t * p.q_st + h * p.q_sh + r0);
-    cp16(&x.g[lane], p.g + t * p.g_st + h * p.g_sh + r0);
-    constexpr int NV = NCOL / 8;  // 16-byte chunks of a row of the slice
-    if (lane < NV) cp16(&x.v[lane], p.v + t * p.v_st + h * p.v_sh + c0 + 8 * lane);
-    else if (lane < 2 * NV) cp16(&x.o[lane - NV], p.dout + t * p.o_st + h * p.o_sh + c0 + 8 * (lane - NV));
-    else if (lane == 2 * NV) cp_async4(&x.b, p.beta + t * p.b_st + h * p.b_sh, 4u);
+    if (c < 16) {
+      cp16(&x.k[8 * c], p.k + t * p.k_st + h * p.k_sh + 8 * c);
+    } else if (c < 32) {
+      cp16(&x.q[8 * (c - 16)], p.q + t * p.q_st + h * p.q_sh + 8 * (c - 16));
+    } else if (c < 64) {
+      cp16(&x.g[4 * (c - 32)], p.g + t * p.g_st + h * p.g_sh + 4 * (c - 32));
+    } else if (c < 68) {
+      cp16(&x.v[8 * (c - 64)], p.v + t * p.v_st + h * p.v_sh + cc0 + 8 * (c - 64));
+    } else if (c < 72) {
+      cp16(&x.o[8 * (c - 68)], p.dout + t * p.o_st + h * p.o_sh + cc0 + 8 * (c - 68));
+    } else {
+      cp_async4(&x.b, p.beta + t * p.b_st + h * p.b_sh, 4u);
+    }
   }
 }
+static_assert(TOK_CHUNKS == 72, "fetch_tokens' chunk map");
 
-__device__ __forceinline__ void read_token(const TokSmem& s, int lane, Token& x) {
-  const uint2 kk = s.k[lane], qq = s.q[lane];
-  const float4 gg = s.g[lane];
+__device__ __forceinline__ void read_token(const TokSmem& s, int lane, int warp, Token& x) {
+  const uint2 kk = *reinterpret_cast<const uint2*>(&s.k[4 * lane]);
+  const uint2 qq = *reinterpret_cast<const uint2*>(&s.q[4 * lane]);
+  const float4 gg = *reinterpret_cast<const float4*>(&s.g[4 * lane]);
+  const uint2 vv = *reinterpret_cast<const uint2*>(&s.v[NCOL * warp]);
+  const uint2 oo = *reinterpret_cast<const uint2*>(&s.o[NCOL * warp]);
   x.k[0] = __uint_as_float(kk.x << 16); x.k[1] = __uint_as_float(kk.x & 0xffff0000u);
   x.k[2] = __uint_as_float(kk.y << 16); x.k[3] = __uint_as_float(kk.y & 0xffff0000u);
   x.q[0] = __uint_as_float(qq.x << 16); x.q[1] = __uint_as_float(qq.x & 0xffff0000u);
   x.q[2] = __uint_as_float(qq.y << 16); x.q[3] = __uint_as_float(qq.y & 0xffff0000u);
   x.e[0] = __expf(gg.x); x.e[1] = __expf(gg.y); x.e[2] = __expf(gg.z); x.e[3] = __expf(gg.w);
-#pragma unroll
-  for (int half = 0; half < NCOL / 8; ++half) {
-    const uint4 vv = s.v[half], oo = s.o[half];
-    const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w}, ow[4] = {oo.x, oo.y, oo.z, oo.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      x.v[8 * half + 2 * i] = __uint_as_float(vw[i] << 16);
-      x.v[8 * half + 2 * i + 1] = __uint_as_float(vw[i] & 0xffff0000u);
-      x.o[8 * half + 2 * i] = __uint_as_float(ow[i] << 16);
-      x.o[8 * half + 2 * i + 1] = __uint_as_float(ow[i] & 0xffff0000u);
-    }
-  }
+  x.v[0] = __uint_as_float(vv.x << 16); x.v[1] = __uint_as_float(vv.x & 0xffff0000u);
+  x.v[2] = __uint_as_float(vv.y << 16); x.v[3] = __uint_as_float(vv.y & 0xffff0000u);
+  x.o[0] = __uint_as_float(oo.x << 16); x.o[1] = __uint_as_float(oo.x & 0xffff0000u);
+  x.o[2] = __uint_as_float(oo.y << 16); x.o[3] = __uint_as_float(oo.y & 0xffff0000u);
   x.b = s.b;
 }
 
@@ -187,14 +196,14 @@ __device__ __forceinline__ void step_forward(float (&S)[4][NCOL], const Token& x
   }
 }
 
-// Grid (NSLICE / WARPS, H, N): warp w of CTA x owns value columns
+// Grid (NPART, H, N): warp w of CTA x owns value columns
 // NCOL (WARPS x + w) .. + NCOL - 1 of head y, sequence z.
 __global__ void __launch_bounds__(NTHREADS) kda_bwd_kernel(const Params p) {
   extern __shared__ __align__(16) unsigned char smem_b[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int slice = WARPS * blockIdx.x + warp;
+  const int part = blockIdx.x, slice = WARPS * part + warp;
   const int h = blockIdx.y, seq = blockIdx.z, H = p.H;
-  const int r0 = 4 * lane, c0 = NCOL * slice;
+  const int r0 = 4 * lane, c0 = NCOL * slice, cc0 = CCOL * part;
   int64_t t0 = 0, t1 = p.T;
   if (p.cu) {
     check_bounds(p.cu, seq, gridDim.z, p.T);
@@ -206,10 +215,9 @@ __global__ void __launch_bounds__(NTHREADS) kda_bwd_kernel(const Params p) {
   const int64_t len = t1 - t0;
   const int64_t nblk = (len + BLK - 1) / BLK;
   const size_t state_off = (static_cast<size_t>(seq) * H + h) * D * D;
-  // A lane's share of a state is NF4 float4 (key row i, columns 4 c4 .. +3 at
-  // element i NCOL / 4 + c4); the 32 lanes' element e are adjacent, so every
-  // access of a warp touches 512 contiguous bytes (conflict-free in shared
-  // memory).
+  // A lane's share of a state is NF4 float4 (key row i, columns c0 .. c0 + 3 at
+  // element i); the 32 lanes' element e are adjacent, so every access of a
+  // warp touches 512 contiguous bytes (conflict-free in shared memory).
   // Checkpoint j of this warp: block index t0 / 4 + seq + j (the ranges of
   // different sequences are disjoint and end below T / 4 + N + 1).
   auto ck_ptr = [&](int64_t j) {
@@ -220,13 +228,29 @@ __global__ void __launch_bounds__(NTHREADS) kda_bwd_kernel(const Params p) {
   unsigned char* wsm = smem_b + warp * WARP_SMEM;
   float4* const st_base = reinterpret_cast<float4*>(wsm) + lane;                       // BLK states
   float4* const ckb_base = reinterpret_cast<float4*>(wsm + BLK * STATE_BYTES) + lane;  // 2 checkpoint buffers
-  TokSmem* const tok_base = reinterpret_cast<TokSmem*>(wsm + (BLK + 2) * STATE_BYTES);  // 2 x BLK tokens
+  TokSmem* const tok_base = reinterpret_cast<TokSmem*>(smem_b + TOK_OFF);               // 2 x BLK tokens (CTA)
+  float4* const red = reinterpret_cast<float4*>(smem_b + RED_OFF);                      // [tok][3][warp][lane]
+  float* const redb = reinterpret_cast<float*>(smem_b + REDB_OFF);                      // [tok][warp]
   auto st_ptr = [&](int j) { return st_base + j * NF4 * 32; };
   auto ckb_ptr = [&](int64_t j) { return ckb_base + (j & 1) * NF4 * 32; };
   auto tok_ptr = [&](int64_t j) { return tok_base + (j & 1) * BLK; };
   auto block_len = [&](int64_t j) {
     const int64_t tb = t0 + j * BLK;
     return static_cast<int>((tb + BLK < t1) ? BLK : t1 - tb);
+  };
+  auto store_state = [&](float4* dst, const float (&S)[4][NCOL]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dst[i * 32] = make_float4(S[i][0], S[i][1], S[i][2], S[i][3]);
+  };
+  auto load_state = [&](const float4* src, float (&S)[4][NCOL]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 v4 = src[i * 32];
+      S[i][0] = v4.x;
+      S[i][1] = v4.y;
+      S[i][2] = v4.z;
+      S[i][3] = v4.w;
+    }
   };
 
   // ---- forward pass: the state before every 4-token block
@@ -236,34 +260,29 @@ __global__ void __launch_bounds__(NTHREADS) kda_bwd_kernel(const Params p) {
 #pragma unroll
     for (int c = 0; c < NCOL; ++c)
       S[i][c] = p.init ? p.init[state_off + static_cast<size_t>(r0 + i) * D + c0 + c] : 0.f;
-  if (nblk > 0) fetch_tokens(p, t0, block_len(0), h, r0, c0, lane, tok_ptr(0));
+  if (nblk > 0) fetch_tokens(p, t0, block_len(0), h, cc0, tok_ptr(0));
   cp_commit();
   for (int64_t j = 0; j < nblk; ++j) {
-    // next block's inputs in flight while this one runs
-    if (j + 1 < nblk) fetch_tokens(p, t0 + (j + 1) * BLK, block_len(j + 1), h, r0, c0, lane, tok_ptr(j + 1));
+    // the next block's inputs are in flight while this one runs
+    if (j + 1 < nblk) fetch_tokens(p, t0 + (j + 1) * BLK, block_len(j + 1), h, cc0, tok_ptr(j + 1));
     cp_commit();
-    float4* dst = ck_ptr(j);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int c4 = 0; c4 < NCOL / 4; ++c4)
-        dst[(i * (NCOL / 4) + c4) * 32] = make_float4(S[i][4 * c4], S[i][4 * c4 + 1], S[i][4 * c4 + 2], S[i][4 * c4 + 3]);
+    store_state(ck_ptr(j), S);
     cp_wait<1>();
-    __syncwarp();
+    __syncthreads();
     const TokSmem* tk = tok_ptr(j);
     const int n = block_len(j);
     for (int s = 0; s < n; ++s) {
       Token x;
-      read_token(tk[s], lane, x);
+      read_token(tk[s], lane, warp, x);
       step_forward(S, x);
     }
-    __syncwarp();  // every lane is done with this buffer before it is refilled
+    __syncthreads();  // every warp is done with this buffer before it is refilled
   }
   cp_wait<0>();
-  // the checkpoints were written by this warp's own lanes: make them visible to
-  // the cp.async reads below
+  // this warp's own checkpoints (each lane reads back what it wrote) are
+  // ordered before the copies below
   __threadfence_block();
-  __syncwarp();
+  __syncthreads();
 
   // ---- backward pass
   float L[4][NCOL];
@@ -272,13 +291,13 @@ __global__ void __launch_bounds__(NTHREADS) kda_bwd_kernel(const Params p) {
 #pragma unroll
     for (int c = 0; c < NCOL; ++c)
       L[i][c] = p.dfin ? p.dfin[state_off + static_cast<size_t>(r0 + i) * D + c0 + c] : 0.f;
-  const size_t pslice = static_cast<size_t>(slice) * static_cast<size_t>(p.T) * H;
+  const size_t ppart = static_cast<size_t>(part) * static_cast<size_t>(p.T) * H;
   auto fetch_block = [&](int64_t j) {
     const float4* src = ck_ptr(j);
     float4* dst = ckb_ptr(j);
 #pragma unroll
     for (int e = 0; e < NF4; ++e) cp16(dst + e * 32, src + e * 32);
-    fetch_tokens(p, t0 + j * BLK, block_len(j), h, r0, c0, lane, tok_ptr(j));
+    fetch_tokens(p, t0 + j * BLK, block_len(j), h, cc0, tok_ptr(j));
   };
   if (nblk > 0) fetch_block(nblk - 1);
   cp_commit();
@@ -288,58 +307,33 @@ __global__ void __launch_bounds__(NTHREADS) kda_bwd_kernel(const Params p) {
     if (j > 0) fetch_block(j - 1);
     cp_commit();
     cp_wait<1>();
-    __syncwarp();
+    __syncthreads();
     const TokSmem* tk = tok_ptr(j);
-    // states before each token of the block: st[0] = checkpoint, st[i] after i steps
-    {
-      const float4* src = ckb_ptr(j);
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int c4 = 0; c4 < NCOL / 4; ++c4) {
-          const float4 v4 = src[(i * (NCOL / 4) + c4) * 32];
-          S[i][4 * c4] = v4.x;
-          S[i][4 * c4 + 1] = v4.y;
-          S[i][4 * c4 + 2] = v4.z;
-          S[i][4 * c4 + 3] = v4.w;
-        }
-    }
+    // states before each token of the block: st[0] = checkpoint, st[s] after s steps
+    load_state(ckb_ptr(j), S);
     for (int s = 0; s < n; ++s) {
-      float4* dst = st_ptr(s);
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int c4 = 0; c4 < NCOL / 4; ++c4)
-          dst[(i * (NCOL / 4) + c4) * 32] = make_float4(S[i][4 * c4], S[i][4 * c4 + 1], S[i][4 * c4 + 2], S[i][4 * c4 + 3]);
+      store_state(st_ptr(s), S);
       if (s + 1 < n) {
         Token x;
-        read_token(tk[s], lane, x);
+        read_token(tk[s], lane, warp, x);
         step_forward(S, x);
       }
     }
     for (int s = n - 1; s >= 0; --s) {
       const int64_t t = tb + s;
       Token x;
-      read_token(tk[s], lane, x);
-      // S' = Diag(exp g) S_{t-1} (from the block's stored state), reusing S
-      const float4* src = st_ptr(s);
+      read_token(tk[s], lane, warp, x);
+      // S' = Diag(exp g) S_{t-1} (from the block's stored state)
+      load_state(st_ptr(s), S);
       float w[NCOL], lk[NCOL];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int c4 = 0; c4 < NCOL / 4; ++c4) {
-          const float4 v4 = src[(i * (NCOL / 4) + c4) * 32];
-          S[i][4 * c4] = v4.x * x.e[i];
-          S[i][4 * c4 + 1] = v4.y * x.e[i];
-          S[i][4 * c4 + 2] = v4.z * x.e[i];
-          S[i][4 * c4 + 3] = v4.w * x.e[i];
-        }
-      // L += scale q dO^T; partial sums over this lane's keys of S'^T k and L^T k
 #pragma unroll
       for (int c = 0; c < NCOL; ++c) {
         const float so = p.scale * x.o[c];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) L[i][c] = fmaf(x.q[i], so, L[i][c]);
+        for (int i = 0; i < 4; ++i) {
+          S[i][c] *= x.e[i];
+          L[i][c] = fmaf(x.q[i], so, L[i][c]);  // L += scale q dO^T
+        }
         w[c] = fmaf(x.k[3], S[3][c], fmaf(x.k[2], S[2][c], fmaf(x.k[1], S[1][c], x.k[0] * S[0][c])));
         lk[c] = fmaf(x.k[3], L[3][c], fmaf(x.k[2], L[2][c], fmaf(x.k[1], L[1][c], x.k[0] * L[0][c])));
       }
@@ -356,7 +350,7 @@ __global__ void __launch_bounds__(NTHREADS) kda_bwd_kernel(const Params p) {
 #pragma unroll
       for (int c = 0; c < NCOL; ++c) dvc = (lane == c) ? x.b * lk[c] : dvc;
       if (lane < NCOL) p.dv[(static_cast<size_t>(t) * H + h) * D + c0 + lane] = dvc;
-      if (lane == 0) p.pb[pslice + static_cast<size_t>(t) * H + h] = db;
+      if (lane == 0) redb[s * WARPS + warp] = db;
       // per key (this lane's 4): dq, dk, dg; then L <- Diag(exp g) dS'
       float dq[4], dk[4], dg[4];
 #pragma unroll
@@ -377,12 +371,30 @@ __global__ void __launch_bounds__(NTHREADS) kda_bwd_kernel(const Params p) {
         dk[i] = x.b * (lu - sl);
         dg[i] = ag;
       }
-      const size_t po = (pslice + static_cast<size_t>(t) * H + h) * D + r0;
-      *reinterpret_cast<float4*>(p.pq + po) = make_float4(dq[0], dq[1], dq[2], dq[3]);
-      *reinterpret_cast<float4*>(p.pk + po) = make_float4(dk[0], dk[1], dk[2], dk[3]);
-      *reinterpret_cast<float4*>(p.pg + po) = make_float4(dg[0], dg[1], dg[2], dg[3]);
+      red[((s * 3 + 0) * WARPS + warp) * 32 + lane] = make_float4(dq[0], dq[1], dq[2], dq[3]);
+      red[((s * 3 + 1) * WARPS + warp) * 32 + lane] = make_float4(dk[0], dk[1], dk[2], dk[3]);
+      red[((s * 3 + 2) * WARPS + warp) * 32 + lane] = make_float4(dg[0], dg[1], dg[2], dg[3]);
     }
-    __syncwarp();  // every lane is done with this block's buffers before they are refilled
+    __syncthreads();
+    // the CTA's partial sums of the block's tokens: 8 warps added in order
+    for (int i = threadIdx.x; i < n * 3 * 32; i += NTHREADS) {
+      const int s = i / 96, v = (i / 32) % 3, l = i % 32;
+      float4 a = red[((s * 3 + v) * WARPS) * 32 + l];
+#pragma unroll
+      for (int w2 = 1; w2 < WARPS; ++w2) {
+        const float4 b = red[((s * 3 + v) * WARPS + w2) * 32 + l];
+        a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+      }
+      float* const o = v == 0 ? p.pq : (v == 1 ? p.pk : p.pg);
+      *reinterpret_cast<float4*>(o + (ppart + static_cast<size_t>(tb + s) * H + h) * D + 4 * l) = a;
+    }
+    if (threadIdx.x < n) {
+      float a = 0.f;
+#pragma unroll
+      for (int w2 = 0; w2 < WARPS; ++w2) a += redb[threadIdx.x * WARPS + w2];
+      p.pb[ppart + static_cast<size_t>(tb + threadIdx.x) * H + h] = a;
+    }
+    __syncthreads();  // the block's buffers are free for refilling
   }
   cp_wait<0>();
   if (p.dinit) {
@@ -393,8 +405,8 @@ __global__ void __launch_bounds__(NTHREADS) kda_bwd_kernel(const Params p) {
   }
 }
 
-// dq, dk, dg = the sum of the eight slices' partials, in slice order; dbeta
-// likewise. n4 = T * H * 128 / 4 float4 groups, nb = T * H.
+// dq, dk, dg = the sum of the NPART partials, in order; dbeta likewise.
+// n4 = T * H * 128 / 4 float4 groups, nb = T * H.
 __global__ void __launch_bounds__(256) kda_bwd_reduce_kernel(const float* __restrict__ pq, const float* __restrict__ pk,
                                                              const float* __restrict__ pg, const float* __restrict__ pb,
                                                              float* dq, float* dk, float* dg, float* dbeta, int64_t n4,
@@ -403,7 +415,7 @@ __global__ void __launch_bounds__(256) kda_bwd_reduce_kernel(const float* __rest
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a, c = a;
 #pragma unroll
-    for (int s = 0; s < NSLICE; ++s) {
+    for (int s = 0; s < NPART; ++s) {
       const float4 x = reinterpret_cast<const float4*>(pq)[s * n4 + i];
       const float4 y = reinterpret_cast<const float4*>(pk)[s * n4 + i];
       const float4 z = reinterpret_cast<const float4*>(pg)[s * n4 + i];
@@ -418,7 +430,7 @@ __global__ void __launch_bounds__(256) kda_bwd_reduce_kernel(const float* __rest
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nb; i += stride) {
     float a = 0.f;
 #pragma unroll
-    for (int s = 0; s < NSLICE; ++s) a += pb[s * nb + i];
+    for (int s = 0; s < NPART; ++s) a += pb[s * nb + i];
     dbeta[i] = a;
   }
 }
