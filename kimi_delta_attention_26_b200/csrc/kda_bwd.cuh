@@ -176,23 +176,60 @@ __device__ __forceinline__ void read_token(const TokSmem& s, int lane, int warp,
   x.b = s.b;
 }
 
-// One forward step S <- S' + beta k (v - S'^T k)^T on this lane's 4 x 16 share.
-__device__ __forceinline__ void step_forward(float (&S)[4][NCOL], const Token& x) {
-  float w[NCOL];
+// Packed fp32 pairs (the two value columns 2j, 2j + 1 of a lane's key row):
+// one f32x2 instruction does both, halving the issue count of the rank-1
+// updates.
+__device__ __forceinline__ unsigned long long pk2(float2 v) {
+  return (static_cast<unsigned long long>(__float_as_uint(v.y)) << 32) | __float_as_uint(v.x);
+}
+__device__ __forceinline__ float2 up2(unsigned long long r) {
+  return make_float2(__uint_as_float(static_cast<uint32_t>(r)), __uint_as_float(static_cast<uint32_t>(r >> 32)));
+}
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {  // a * b + c
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(pk2(a)), "l"(pk2(b)), "l"(pk2(c)));
+  return up2(r);
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  unsigned long long r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk2(a)), "l"(pk2(b)));
+  return up2(r);
+}
+__device__ __forceinline__ float2 dup(float a) { return make_float2(a, a); }
+
+// A lane's share of a state: key rows 4l + i (i < 4) x the warp's 4 columns,
+// as two column pairs.
+using Share = float2[4][2];
+
+// sum_i k_i X[i][.] over this lane's 4 keys, for both column pairs
+__device__ __forceinline__ void key_dot(const Token& x, const Share& X, float (&out)[NCOL]) {
 #pragma unroll
-  for (int c = 0; c < NCOL; ++c) {
-    S[0][c] *= x.e[0];
-    S[1][c] *= x.e[1];
-    S[2][c] *= x.e[2];
-    S[3][c] *= x.e[3];
-    w[c] = fmaf(x.k[3], S[3][c], fmaf(x.k[2], S[2][c], fmaf(x.k[1], S[1][c], x.k[0] * S[0][c])));
+  for (int j = 0; j < 2; ++j) {
+    float2 a = fmul2(dup(x.k[0]), X[0][j]);
+    a = ffma2(dup(x.k[1]), X[1][j], a);
+    a = ffma2(dup(x.k[2]), X[2][j], a);
+    a = ffma2(dup(x.k[3]), X[3][j], a);
+    out[2 * j] = a.x;
+    out[2 * j + 1] = a.y;
   }
+}
+
+// One forward step S <- S' + beta k (v - S'^T k)^T on this lane's share.
+__device__ __forceinline__ void step_forward(Share& S, const Token& x) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    S[i][0] = fmul2(dup(x.e[i]), S[i][0]);
+    S[i][1] = fmul2(dup(x.e[i]), S[i][1]);
+  }
+  float w[NCOL];
+  key_dot(x, S, w);
   allreduce(w);
+  const float2 bu[2] = {make_float2(x.b * (x.v[0] - w[0]), x.b * (x.v[1] - w[1])),
+                        make_float2(x.b * (x.v[2] - w[2]), x.b * (x.v[3] - w[3]))};
 #pragma unroll
-  for (int c = 0; c < NCOL; ++c) {
-    const float bu = x.b * (x.v[c] - w[c]);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) S[i][c] = fmaf(x.k[i], bu, S[i][c]);
+  for (int i = 0; i < 4; ++i) {
+    S[i][0] = ffma2(dup(x.k[i]), bu[0], S[i][0]);
+    S[i][1] = ffma2(dup(x.k[i]), bu[1], S[i][1]);
   }
 }
 
@@ -238,28 +275,32 @@ __global__ void __launch_bounds__(NTHREADS) kda_bwd_kernel(const Params p) {
     const int64_t tb = t0 + j * BLK;
     return static_cast<int>((tb + BLK < t1) ? BLK : t1 - tb);
   };
-  auto store_state = [&](float4* dst, const float (&S)[4][NCOL]) {
+  auto store_state = [&](float4* dst, const Share& S) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) dst[i * 32] = make_float4(S[i][0], S[i][1], S[i][2], S[i][3]);
+    for (int i = 0; i < 4; ++i) dst[i * 32] = make_float4(S[i][0].x, S[i][0].y, S[i][1].x, S[i][1].y);
   };
-  auto load_state = [&](const float4* src, float (&S)[4][NCOL]) {
+  auto load_state = [&](const float4* src, Share& S) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const float4 v4 = src[i * 32];
-      S[i][0] = v4.x;
-      S[i][1] = v4.y;
-      S[i][2] = v4.z;
-      S[i][3] = v4.w;
+      S[i][0] = make_float2(v4.x, v4.y);
+      S[i][1] = make_float2(v4.z, v4.w);
+    }
+  };
+  // an fp32 [N, H, 128, 128] state's share of this lane (or zeros)
+  auto load_global = [&](const float* base, Share& S) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 v4 = base ? *reinterpret_cast<const float4*>(base + state_off + static_cast<size_t>(r0 + i) * D + c0)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+      S[i][0] = make_float2(v4.x, v4.y);
+      S[i][1] = make_float2(v4.z, v4.w);
     }
   };
 
   // ---- forward pass: the state before every 4-token block
-  float S[4][NCOL];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int c = 0; c < NCOL; ++c)
-      S[i][c] = p.init ? p.init[state_off + static_cast<size_t>(r0 + i) * D + c0 + c] : 0.f;
+  Share S;
+  load_global(p.init, S);
   if (nblk > 0) fetch_tokens(p, t0, block_len(0), h, cc0, tok_ptr(0));
   cp_commit();
   for (int64_t j = 0; j < nblk; ++j) {
@@ -285,12 +326,8 @@ __global__ void __launch_bounds__(NTHREADS) kda_bwd_kernel(const Params p) {
   __syncthreads();
 
   // ---- backward pass
-  float L[4][NCOL];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int c = 0; c < NCOL; ++c)
-      L[i][c] = p.dfin ? p.dfin[state_off + static_cast<size_t>(r0 + i) * D + c0 + c] : 0.f;
+  Share L;
+  load_global(p.dfin, L);
   const size_t ppart = static_cast<size_t>(part) * static_cast<size_t>(p.T) * H;
   auto fetch_block = [&](int64_t j) {
     const float4* src = ck_ptr(j);
@@ -323,20 +360,20 @@ __global__ void __launch_bounds__(NTHREADS) kda_bwd_kernel(const Params p) {
       const int64_t t = tb + s;
       Token x;
       read_token(tk[s], lane, warp, x);
-      // S' = Diag(exp g) S_{t-1} (from the block's stored state)
+      // S' = Diag(exp g) S_{t-1} (from the block's stored state); L += scale q dO^T
       load_state(st_ptr(s), S);
-      float w[NCOL], lk[NCOL];
+      const float2 so[2] = {make_float2(p.scale * x.o[0], p.scale * x.o[1]),
+                            make_float2(p.scale * x.o[2], p.scale * x.o[3])};
 #pragma unroll
-      for (int c = 0; c < NCOL; ++c) {
-        const float so = p.scale * x.o[c];
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          S[i][c] *= x.e[i];
-          L[i][c] = fmaf(x.q[i], so, L[i][c]);  // L += scale q dO^T
+        for (int j = 0; j < 2; ++j) {
+          S[i][j] = fmul2(dup(x.e[i]), S[i][j]);
+          L[i][j] = ffma2(dup(x.q[i]), so[j], L[i][j]);
         }
-        w[c] = fmaf(x.k[3], S[3][c], fmaf(x.k[2], S[2][c], fmaf(x.k[1], S[1][c], x.k[0] * S[0][c])));
-        lk[c] = fmaf(x.k[3], L[3][c], fmaf(x.k[2], L[2][c], fmaf(x.k[1], L[1][c], x.k[0] * L[0][c])));
-      }
+      float w[NCOL], lk[NCOL];
+      key_dot(x, S, w);
+      key_dot(x, L, lk);
       allreduce(w);
       allreduce(lk);
       float u[NCOL], db = 0.f;
@@ -352,24 +389,27 @@ __global__ void __launch_bounds__(NTHREADS) kda_bwd_kernel(const Params p) {
       if (lane < NCOL) p.dv[(static_cast<size_t>(t) * H + h) * D + c0 + lane] = dvc;
       if (lane == 0) redb[s * WARPS + warp] = db;
       // per key (this lane's 4): dq, dk, dg; then L <- Diag(exp g) dS'
+      const float2 u2[2] = {make_float2(u[0], u[1]), make_float2(u[2], u[3])};
+      const float2 lk2[2] = {make_float2(lk[0], lk[1]), make_float2(lk[2], lk[3])};
+      const float2 o2[2] = {make_float2(x.o[0], x.o[1]), make_float2(x.o[2], x.o[3])};
       float dq[4], dk[4], dg[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        float aq = 0.f, lu = 0.f, sl = 0.f, ag = 0.f;
         const float bk = x.b * x.k[i];
+        float2 aq = make_float2(0.f, 0.f), lu = aq, sl = aq, ag = aq;
 #pragma unroll
-        for (int c = 0; c < NCOL; ++c) {
-          const float st = fmaf(bk, u[c], S[i][c]);  // S_t = S' + beta k u^T
-          aq = fmaf(st, x.o[c], aq);
-          lu = fmaf(L[i][c], u[c], lu);
-          sl = fmaf(S[i][c], lk[c], sl);
-          const float dsp = fmaf(-bk, lk[c], L[i][c]);
-          ag = fmaf(dsp, S[i][c], ag);
-          L[i][c] = x.e[i] * dsp;
+        for (int j = 0; j < 2; ++j) {
+          const float2 st = ffma2(dup(bk), u2[j], S[i][j]);   // S_t = S' + beta k u^T
+          aq = ffma2(st, o2[j], aq);
+          lu = ffma2(L[i][j], u2[j], lu);
+          sl = ffma2(S[i][j], lk2[j], sl);
+          const float2 dsp = ffma2(dup(-bk), lk2[j], L[i][j]);
+          ag = ffma2(dsp, S[i][j], ag);
+          L[i][j] = fmul2(dup(x.e[i]), dsp);
         }
-        dq[i] = p.scale * aq;
-        dk[i] = x.b * (lu - sl);
-        dg[i] = ag;
+        dq[i] = p.scale * (aq.x + aq.y);
+        dk[i] = x.b * ((lu.x + lu.y) - (sl.x + sl.y));
+        dg[i] = ag.x + ag.y;
       }
       red[((s * 3 + 0) * WARPS + warp) * 32 + lane] = make_float4(dq[0], dq[1], dq[2], dq[3]);
       red[((s * 3 + 1) * WARPS + warp) * 32 + lane] = make_float4(dk[0], dk[1], dk[2], dk[3]);
@@ -400,8 +440,8 @@ __global__ void __launch_bounds__(NTHREADS) kda_bwd_kernel(const Params p) {
   if (p.dinit) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int c = 0; c < NCOL; ++c) p.dinit[state_off + static_cast<size_t>(r0 + i) * D + c0 + c] = L[i][c];
+      *reinterpret_cast<float4*>(p.dinit + state_off + static_cast<size_t>(r0 + i) * D + c0) =
+          make_float4(L[i][0].x, L[i][0].y, L[i][1].x, L[i][1].y);
   }
 }
 
