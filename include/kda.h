@@ -49,7 +49,7 @@ extern "C" {
 #endif
 
 #define KDA_HEAD_DIM 128
-#define KDA_ABI_VERSION 4
+#define KDA_ABI_VERSION 5
 
 typedef enum kda_status {
   KDA_OK = 0,
@@ -221,6 +221,25 @@ kda_status_t kda_set_path(int32_t path);
  * setting is then unchanged).
  */
 kda_status_t kda_set_slice_columns(int32_t columns);
+
+/*
+ * kda_set_schedule -- how the 16-token path maps (sequence, head) pairs onto
+ * clusters.
+ *   mode 1: one cluster per pair; the hardware starts each cluster when an
+ *           earlier one has finished.
+ *   mode 2: G persistent clusters, G = the number the device holds at once,
+ *           capped at `clusters` when that is > 0, and at the number of pairs;
+ *           cluster c runs the pairs c, c + G, c + 2G, ... (pair = sequence *
+ *           num_heads + head) back to back, the next pair's operands being
+ *           prepared while the previous one's last chunks run. A small cap
+ *           makes every cluster take many pairs (testing).
+ *   mode 0 (default): 2 with no cap when the pairs outnumber the resident
+ *           clusters, else 1 (`clusters` is ignored).
+ * Each pair's arithmetic is the same either way, so the results are bitwise
+ * identical. Process-wide. Returns KDA_ERR_SHAPE for any other mode or a
+ * negative `clusters` (the setting is then unchanged).
+ */
+kda_status_t kda_set_schedule(int32_t mode, int32_t clusters);
 
 /*
  * kda_set_time_split -- the time-split prefill of kda_fwd (16-token path).

@@ -77,6 +77,8 @@ _lib.kda_set_path.argtypes = [ctypes.c_int32]
 _lib.kda_set_path.restype = ctypes.c_int
 _lib.kda_set_time_split.argtypes = [ctypes.c_int32]
 _lib.kda_set_time_split.restype = ctypes.c_int
+_lib.kda_set_schedule.argtypes = [ctypes.c_int32, ctypes.c_int32]
+_lib.kda_set_schedule.restype = ctypes.c_int
 _lib.kda_fwd_fused.argtypes = [_T, _T, _T, _T, _T, ctypes.c_float, ctypes.c_float, _P, ctypes.c_int32, _T, _T, _T, _P]
 _lib.kda_fwd_fused.restype = ctypes.c_int
 _lib.kda_bwd.argtypes = [_T, _T, _T, _T, _T, ctypes.c_float, _P, ctypes.c_int32, _T, _T, _T, _T, _T, _T, _T, _T, _T, _P]
@@ -127,6 +129,16 @@ def set_time_split(mode: int) -> None:
     """Time-split prefill of one long sequence (16-token path): 0 automatic
     (default), 1 never, 2 whenever possible. Process-wide."""
     rc = _lib.kda_set_time_split(int(mode))
+    if rc != 0:
+        raise KDAError(rc)
+
+
+def set_schedule(mode: int, clusters: int = 0) -> None:
+    """Mapping of (sequence, head) pairs onto clusters (16-token path): 0
+    automatic (default), 1 one cluster per pair, 2 persistent clusters taking
+    the pairs round robin (at most `clusters` of them when > 0). Process-wide;
+    results are bitwise the same."""
+    rc = _lib.kda_set_schedule(int(mode), int(clusters))
     if rc != 0:
         raise KDAError(rc)
 

@@ -171,6 +171,7 @@ std::mutex g_setup_mutex;                      // guards first-call setup of eve
 std::atomic<int> g_device_ready[kMaxDevices];  // 0 unknown, 1 ready, -1 unsupported
 int g_num_sms[kMaxDevices];
 int g_max_clusters32[kMaxDevices];  // co-resident 4-CTA clusters of the 32-column kernel
+int g_max_clusters16[kMaxDevices];  // co-resident 8-CTA clusters of the 16-column kernel
 // Library-private stream-ordered pool for the scratch rings. It keeps freed
 // memory (release threshold = max), so steady-state calls never map memory
 // and the process's default pool is left untouched.
@@ -178,6 +179,8 @@ std::atomic<cudaMemPool_t> g_pool[kMaxDevices];
 std::atomic<void*> g_noalloc_ring_addr[kMaxDevices];
 std::atomic<int> g_slice_columns{0};  // 16-token path: 0 chooses per call, 16 or 32 forces
 std::atomic<int> g_path{0};           // 0 (the default path), 16 or 64
+std::atomic<int> g_schedule{0};       // 16-token path: 0 automatic, 1 one cluster per pair, 2 persistent
+std::atomic<int> g_sched_clusters{0};  // persistent clusters: 0 as many as are resident, else at most this
 
 // The 16-token kernel's instantiations: value slice NS, fused gate FG and
 // launch mode MODE (the time split's modes run only with 32-column slices).
@@ -201,9 +204,12 @@ cudaError_t set_smem16() {
   return cudaSuccess;
 }
 
+// Grid (D / NS, gy, gz): gy * gz clusters, cluster c taking the (sequence,
+// head) items c, c + gy * gz, ...
 template <int NS, bool FG, uint32_t MODE>
-void launch_one(const kda::Params& p, const kda::TensorMaps& tm, int H, int N, cudaStream_t stream) {
-  kda::kda_fwd_kernel<NS, FG, MODE><<<dim3(kda::D / NS, H, N), kda::NTHREADS, sizeof(kda::Shared<NS>), stream>>>(p, tm);
+void launch_one(const kda::Params& p, const kda::TensorMaps& tm, int gy, int gz, cudaStream_t stream) {
+  kda::kda_fwd_kernel<NS, FG, MODE><<<dim3(kda::D / NS, gy, gz), kda::NTHREADS, sizeof(kda::Shared<NS>), stream>>>(p,
+                                                                                                              tm);
 }
 
 // Capability check and kernel attributes for `dev` (current), once.
@@ -235,8 +241,8 @@ kda_status_t check_device(int dev) {
   if ((e = cudaFuncSetAttribute(kda::c64::kda_fwd64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(kda::c64::SMEM_BYTES))) != cudaSuccess)
     return cuda_fail(e);
-  // How many clusters of the 32-column kernel the GPU holds at once: clusters
-  // are placed whole inside one GPC, so this can be below SMs / 4.
+  // How many clusters of the 16-token kernel the GPU holds at once: clusters
+  // are placed whole inside one GPC, so this can be below SMs / cluster size.
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3(kda::D / 32, 1, 1);
@@ -246,6 +252,11 @@ kda_status_t check_device(int dev) {
   if ((e = cudaOccupancyMaxActiveClusters(&clusters, kda::kda_fwd_kernel<32, false, 0>, &cfg)) != cudaSuccess)
     return cuda_fail(e);
   g_max_clusters32[dev] = clusters;
+  cfg.gridDim = dim3(kda::D / 16, 1, 1);
+  cfg.dynamicSmemBytes = sizeof(kda::Shared<16>);
+  if ((e = cudaOccupancyMaxActiveClusters(&clusters, kda::kda_fwd_kernel<16, false, 0>, &cfg)) != cudaSuccess)
+    return cuda_fail(e);
+  g_max_clusters16[dev] = clusters;
   g_num_sms[dev] = sms;
   g_device_ready[dev].store(1, std::memory_order_release);
   return KDA_OK;
@@ -341,6 +352,7 @@ kda_status_t launch16(const Problem& P, unsigned char* ring, int dev, cudaStream
   p.out_st = P.out.st;
   p.out_sh = P.out.sh;
   p.H = P.num_heads;
+  p.N = P.num_seqs;
   p.scale = P.scale;
   p.exp_lb = P.exp_lb;
   p.outf = outf;
@@ -361,18 +373,33 @@ kda_status_t launch16(const Problem& P, unsigned char* ring, int dev, cudaStream
   }
   const int H = P.num_heads, N = P.num_seqs;
   if (mode != 0 && ns != 32) return KDA_ERR_UNSUPPORTED;  // not reached: the split forces 32 columns
+  // One cluster per (sequence, head) item, or, when the items outnumber the
+  // clusters the device holds at once, that many persistent clusters that
+  // take the items round robin (each cluster's next item then starts filling
+  // its pipeline while the previous one drains).
+  int gy = H, gz = N;
+  {
+    const int64_t items = static_cast<int64_t>(N) * H;
+    int resident = ns == 32 ? g_max_clusters32[dev] : g_max_clusters16[dev];
+    const int sched = g_schedule.load(), cap = g_sched_clusters.load();
+    if (sched == 2 && cap > 0 && cap < resident) resident = cap;
+    if (resident > 0 && items > 1 && (sched == 2 || (sched == 0 && items > resident))) {
+      gy = static_cast<int>(items < resident ? items : resident);
+      gz = 1;
+    }
+  }
   if (mode == 0 && ns == 16) {
-    if (P.fused) launch_one<16, true, 0>(p, tm, H, N, stream);
-    else launch_one<16, false, 0>(p, tm, H, N, stream);
+    if (P.fused) launch_one<16, true, 0>(p, tm, gy, gz, stream);
+    else launch_one<16, false, 0>(p, tm, gy, gz, stream);
   } else if (mode == 0) {
-    if (P.fused) launch_one<32, true, 0>(p, tm, H, N, stream);
-    else launch_one<32, false, 0>(p, tm, H, N, stream);
+    if (P.fused) launch_one<32, true, 0>(p, tm, gy, gz, stream);
+    else launch_one<32, false, 0>(p, tm, gy, gz, stream);
   } else if (mode == kSplitL) {
-    if (P.fused) launch_one<32, true, kSplitL>(p, tm, H, N, stream);
-    else launch_one<32, false, kSplitL>(p, tm, H, N, stream);
+    if (P.fused) launch_one<32, true, kSplitL>(p, tm, gy, gz, stream);
+    else launch_one<32, false, kSplitL>(p, tm, gy, gz, stream);
   } else if (mode == kSplitM) {
-    if (P.fused) launch_one<32, true, kSplitM>(p, tm, H, N, stream);
-    else launch_one<32, false, kSplitM>(p, tm, H, N, stream);
+    if (P.fused) launch_one<32, true, kSplitM>(p, tm, gy, gz, stream);
+    else launch_one<32, false, kSplitM>(p, tm, gy, gz, stream);
   } else {
     return KDA_ERR_UNSUPPORTED;
   }
@@ -776,6 +803,13 @@ kda_status_t kda_set_path(int32_t path) {
 kda_status_t kda_set_time_split(int32_t mode) {
   if (mode < 0 || mode > 2) return KDA_ERR_SHAPE;
   g_split.store(mode);
+  return KDA_OK;
+}
+
+kda_status_t kda_set_schedule(int32_t mode, int32_t clusters) {
+  if (mode < 0 || mode > 2 || clusters < 0) return KDA_ERR_SHAPE;
+  g_schedule.store(mode);
+  g_sched_clusters.store(clusters);
   return KDA_OK;
 }
 

@@ -173,6 +173,7 @@ struct Params {
   int64_t beta_st, beta_sh;  // element strides of beta over tokens and heads
   int64_t out_st, out_sh;    // element strides of out over tokens and heads
   int32_t H;
+  int32_t N;               // sequences (items are the N * H (sequence, head) pairs)
   float scale;
   float* outf;             // fp32 outputs [T, H, 128] (kModeOutF32 only)
   int64_t outf_st;         // token stride of outf
@@ -216,22 +217,37 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
   const int tq = lane & 3;   // fragment column pair
 
   const int rank = blockIdx.x;  // value slice = rank inside the cluster
-  const int h = blockIdx.y;
-  const int seq = blockIdx.z;
   const int dv0 = rank * NS;
   const int H = p.H;
   const int64_t T = p.T;
 
-  int64_t t0 = 0, t1 = T;
-  if (p.cu) {
-    t0 = p.cu[seq];
-    t1 = p.cu[seq + 1];
-    t0 = t0 < 0 ? 0 : (t0 > T ? T : t0);
-    t1 = t1 < t0 ? t0 : (t1 > T ? T : t1);
-  }
-  const int nch = static_cast<int>((t1 - t0 + C - 1) / C);
-  const int nprod = nch > rank ? (nch - rank + NSLICE - 1) / NSLICE : 0;  // chunks this CTA produces
-  unsigned char* ring = p.ring + (static_cast<size_t>(seq) * H + h) * RING * kSlotBytes;
+  // Work items are the (sequence, head) pairs, item = seq * H + h. A cluster
+  // takes items first, first + stride, ...: one item with the grid
+  // (NSLICE, H, N); several, back to back, with the persistent grid
+  // (NSLICE, G, 1), so that an item's pipeline fill overlaps the previous
+  // item's tail. Every pipeline counter (stages, ring slots, chunk ownership)
+  // runs over all the chunks of the cluster's items, in order.
+  const int nitems = p.N * H;
+  const int first = static_cast<int>(blockIdx.z * gridDim.y + blockIdx.y);
+  const int stride = static_cast<int>(gridDim.y * gridDim.z);
+  // (seq, h) of an item and its token range; returns its number of chunks
+  auto item_at = [&](int it, int& seq, int& h, int64_t& t0, int64_t& t1) -> int {
+    seq = it / H;
+    h = it - seq * H;
+    t0 = 0;
+    t1 = T;
+    if (p.cu) {
+      t0 = p.cu[seq];
+      t1 = p.cu[seq + 1];
+      t0 = t0 < 0 ? 0 : (t0 > T ? T : t0);
+      t1 = t1 < t0 ? t0 : (t1 > T ? T : t1);
+    }
+    return static_cast<int>((t1 - t0 + C - 1) / C);
+  };
+  // chunk g of the cluster (counted over its items) is produced by CTA g mod NSLICE:
+  // the first chunk of an item this CTA produces, the item starting at chunk gbase
+  auto owned_first = [&](int64_t gbase) { return static_cast<int>(((rank - gbase) % NSLICE + NSLICE) % NSLICE); };
+  unsigned char* ring = p.ring + static_cast<size_t>(first) * RING * kSlotBytes;
 
   if (tid == 0) {
     for (int s = 0; s < PRSTAGE; ++s) {
@@ -266,10 +282,15 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
     // Nothing of the state leaves the registers and the warp needs no partner.
     const int cv = 16 * warp;          // first value column (slice-local)
     float sacc[16][4];
+    const int64_t out_st = p.out_st;
+    int64_t gc = 0;                    // the cluster's chunks so far
+    for (int it = first; it < nitems; it += stride) {
+    int seq, h;
+    int64_t t0, t1;
+    const int nch = item_at(it, seq, h, t0, t1);
     const size_t sbase = (static_cast<size_t>(seq) * H + h) * D * D;
     // this lane's output columns of head h; rows step by the token stride
     __nv_bfloat16* const out_base = p.out + static_cast<int64_t>(h) * p.out_sh + dv0 + cv + 2 * tq;
-    const int64_t out_st = p.out_st;
 #pragma unroll
     for (int u = 0; u < 16; ++u)
 #pragma unroll
@@ -280,8 +301,8 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
                      : p.init ? __ldg(p.init + sbase + static_cast<size_t>(key) * D + col) : 0.f;
       }
 
-    for (int n = 0; n < nch; ++n) {
-      const int s = n % CSTAGE;
+    for (int n = 0; n < nch; ++n, ++gc) {
+      const int s = static_cast<int>(gc % CSTAGE);
       const int64_t cs = t0 + static_cast<int64_t>(n) * C;
       const int m = static_cast<int>((t1 - cs) < C ? (t1 - cs) : C);
       ChainStage<NS>& st = sh.cst[s];
@@ -438,6 +459,7 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
           p.fin[sbase + static_cast<size_t>(key) * D + col] = sacc[u][e];
         }
     }
+    }  // items
   } else if (is_gate_warp(warp)) {
     // ============================================================ gate warps
     // Thread layout: channel pair cp (channels 2cp, 2cp+1), token half th
@@ -447,11 +469,16 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
     const int cp = gt & 63;
     const int th = gt >> 6;
     const int c0 = 2 * cp;
-    for (int j = 0; j < nprod; ++j) {
-      const int n = rank + NSLICE * j;
-      const int rs = j % PRSTAGE, ps = j % PSTAGE;
-      const uint32_t rph = static_cast<uint32_t>(j / PRSTAGE) & 1u;
-      const uint32_t pph = static_cast<uint32_t>(j / PSTAGE) & 1u;
+    int64_t gbase = 0, jg = 0;  // the item's first chunk; this CTA's produced chunks so far
+    for (int it = first; it < nitems; it += stride) {
+    int seq, h;
+    int64_t t0, t1;
+    const int nch = item_at(it, seq, h, t0, t1);
+    for (int n = owned_first(gbase); n < nch; n += NSLICE, ++jg) {
+      const int j = static_cast<int>(jg & 1);  // parity of the exchange buffers
+      const int rs = static_cast<int>(jg % PRSTAGE), ps = static_cast<int>(jg % PSTAGE);
+      const uint32_t rph = static_cast<uint32_t>(jg / PRSTAGE) & 1u;
+      const uint32_t pph = static_cast<uint32_t>(jg / PSTAGE) & 1u;
       const int64_t cs = t0 + static_cast<int64_t>(n) * C;
       const int m = static_cast<int>((t1 - cs) < C ? (t1 - cs) : C);
       RawStage& rw = sh.raw[rs];
@@ -566,11 +593,18 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
       fence_proxy_async_shared();
       mbar_arrive_warp(&sh.gate_done[ps]);
     }
+    gbase += nch;
+    }  // items
   } else if (warp == WARP_MMA) {
     // ============================================================= mma warp
-    for (int j = 0; j < nprod; ++j) {
-      const int ps = j % PSTAGE;
-      const uint32_t pph = static_cast<uint32_t>(j / PSTAGE) & 1u;
+    int64_t gbase = 0, jg = 0;
+    for (int it = first; it < nitems; it += stride) {
+    int seq, h;
+    int64_t t0, t1;
+    const int nch = item_at(it, seq, h, t0, t1);
+    for (int n = owned_first(gbase); n < nch; n += NSLICE, ++jg) {
+      const int ps = static_cast<int>(jg % PSTAGE);
+      const uint32_t pph = static_cast<uint32_t>(jg / PSTAGE) & 1u;
       ProdStage& st = sh.prod[ps];
       mbar_wait(&sh.gate_done[ps], pph);
       float accA[2][4] = {}, accQ[2][4] = {};
@@ -622,13 +656,15 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
       fence_proxy_async_shared();
       mbar_arrive_warp(&sh.solved[ps]);
     }
+    gbase += nch;
+    }  // items
   } else if (warp == WARP_STORE) {
     // ============================================================ store warp
-    // Up to two stores in flight: chunk j's slot is announced to the cluster
-    // once store j has completed, which is checked after store j+1 is issued.
+    // Up to two stores in flight: a chunk's slot is announced to the cluster
+    // once its store has completed, which is checked after the next store is
+    // issued (the last one after the loop).
     if (lane == 0) {
-      auto announce = [&](int jj) {
-        const int nn = rank + NSLICE * jj;
+      auto announce = [&](int64_t g, int ps) {
         // The slot's bytes were written by the bulk-copy engine and that
         // write has completed (bulk_wait above). The proxy fence makes them
         // visible to this thread's generic proxy and one cluster-scope
@@ -638,36 +674,50 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
         fence_proxy_async_global();
         asm volatile("fence.acq_rel.cluster;" ::: "memory");
         for (int c = 0; c < NSLICE; ++c)
-          mbar_arrive_remote_relaxed(&sh.ready[nn % RING], static_cast<uint32_t>(c));
-        mbar_arrive(&sh.prod_free[jj % PSTAGE]);
+          mbar_arrive_remote_relaxed(&sh.ready[g % RING], static_cast<uint32_t>(c));
+        mbar_arrive(&sh.prod_free[ps]);
       };
-      for (int j = 0; j < nprod; ++j) {
-        const int n = rank + NSLICE * j;
-        const int ps = j % PSTAGE;
-        const uint32_t pph = static_cast<uint32_t>(j / PSTAGE) & 1u;
-        const int slot = n % RING;
-        mbar_wait(&sh.solved[ps], pph);
-        // the slot's previous chunk (n - RING) has been copied by every CTA of the cluster
-        mbar_wait_cl(&sh.slot_free[slot], (static_cast<uint32_t>(n / RING) & 1u) ^ 1u);
-        fence_proxy_async_shared();
-        bulk_s2g(ring + static_cast<size_t>(slot) * kSlotBytes, &sh.prod[ps].ops, kSlotBytes);
-        if (j > 0) {
-          bulk_wait<1>();
-          announce(j - 1);
+      int64_t gbase = 0, jg = 0, prev_g = -1;
+      int prev_ps = 0;
+      for (int it = first; it < nitems; it += stride) {
+        int seq, h;
+        int64_t t0, t1;
+        const int nch = item_at(it, seq, h, t0, t1);
+        for (int n = owned_first(gbase); n < nch; n += NSLICE, ++jg) {
+          const int64_t g = gbase + n;
+          const int ps = static_cast<int>(jg % PSTAGE);
+          const uint32_t pph = static_cast<uint32_t>(jg / PSTAGE) & 1u;
+          const int slot = static_cast<int>(g % RING);
+          mbar_wait(&sh.solved[ps], pph);
+          // the slot's previous chunk (g - RING) has been copied by every CTA of the cluster
+          mbar_wait_cl(&sh.slot_free[slot], (static_cast<uint32_t>(g / RING) & 1u) ^ 1u);
+          fence_proxy_async_shared();
+          bulk_s2g(ring + static_cast<size_t>(slot) * kSlotBytes, &sh.prod[ps].ops, kSlotBytes);
+          if (prev_g >= 0) {
+            bulk_wait<1>();
+            announce(prev_g, prev_ps);
+          }
+          prev_g = g;
+          prev_ps = ps;
         }
+        gbase += nch;
       }
-      if (nprod > 0) {
+      if (prev_g >= 0) {
         bulk_wait<0>();
-        announce(nprod - 1);
+        announce(prev_g, prev_ps);
       }
     }
   } else if (warp == WARP_PLOAD) {
     // ====================================================== producer loads
     // lane 0: TMA boxes of q, k, g; lanes 1-16: beta (zero past the sequence end)
-    for (int j = 0; j < nprod; ++j) {
-      const int n = rank + NSLICE * j;
-      const int rs = j % PRSTAGE;
-      const uint32_t rph = static_cast<uint32_t>(j / PRSTAGE) & 1u;
+    int64_t gbase = 0, jg = 0;
+    for (int it = first; it < nitems; it += stride) {
+    int seq, h;
+    int64_t t0, t1;
+    const int nch = item_at(it, seq, h, t0, t1);
+    for (int n = owned_first(gbase); n < nch; n += NSLICE, ++jg) {
+      const int rs = static_cast<int>(jg % PRSTAGE);
+      const uint32_t rph = static_cast<uint32_t>(jg / PRSTAGE) & 1u;
       const int64_t cs = t0 + static_cast<int64_t>(n) * C;
       const int tok = static_cast<int>(cs);
       RawStage& rw = sh.raw[rs];
@@ -684,6 +734,8 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
         cp_async_arrive(&sh.raw_full[rs]);
       }
     }
+    gbase += nch;
+    }  // items
   } else if (warp == WARP_NOTIFY) {
     // ==================================================== stage notifications
     // Waiting on a transaction mbarrier costs the waiter ~100 cycles even when
@@ -691,33 +743,51 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
     // critical path and releases each chain warp through a hardware barrier.
     // The mbarrier acquire makes the landed bytes visible to this warp and the
     // barrier orders them before the chain warps' reads.
-    for (int n = 0; n < nch; ++n) {
-      const int s = n % CSTAGE;
-      mbar_wait(&sh.c_full[s], static_cast<uint32_t>(n / CSTAGE) & 1u);
+    int64_t gc = 0;
+    for (int it = first; it < nitems; it += stride) {
+    int seq, h;
+    int64_t t0, t1;
+    const int nch = item_at(it, seq, h, t0, t1);
+    for (int n = 0; n < nch; ++n, ++gc) {
+      const int s = static_cast<int>(gc % CSTAGE);
+      mbar_wait(&sh.c_full[s], static_cast<uint32_t>(gc / CSTAGE) & 1u);
       __syncwarp();
 #pragma unroll
       for (int w = 0; w < NCHAIN; ++w) named_bar_arrive(BAR_FULL0 + 2 * s + w, 64);
       // the ring slot has been copied here: give it back to its producer
-      if (lane == 0) mbar_arrive_remote_relaxed(&sh.slot_free[n % RING], static_cast<uint32_t>(n % NSLICE));
+      if (lane == 0)
+        mbar_arrive_remote_relaxed(&sh.slot_free[gc % RING], static_cast<uint32_t>(gc % NSLICE));
     }
+    }  // items
   } else if (warp == 9) {
-    if (lane == 0 && p.cu && rank == 0 && h == 0) check_bounds(p.cu, seq, static_cast<int>(gridDim.z), T);
+    if (lane == 0 && p.cu && rank == 0) {
+      for (int it = first; it < nitems; it += stride) {
+        const int seq = it / H;
+        if (it - seq * H == 0) check_bounds(p.cu, seq, p.N, T);
+      }
+    }
   } else if (warp == WARP_CLOAD) {
     // ====================================================== consumer loads
     if (lane == 0) {
-      for (int n = 0; n < nch; ++n) {
-        const int s = n % CSTAGE;
-        const uint32_t ph = static_cast<uint32_t>(n / CSTAGE) & 1u;
-        const int slot = n % RING;
+      int64_t gc = 0;
+      for (int it = first; it < nitems; it += stride) {
+      int seq, h;
+      int64_t t0, t1;
+      const int nch = item_at(it, seq, h, t0, t1);
+      for (int n = 0; n < nch; ++n, ++gc) {
+        const int s = static_cast<int>(gc % CSTAGE);
+        const uint32_t ph = static_cast<uint32_t>(gc / CSTAGE) & 1u;
+        const int slot = static_cast<int>(gc % RING);
         const int tok = static_cast<int>(t0 + static_cast<int64_t>(n) * C);
         ChainStage<NS>& st = sh.cst[s];
         mbar_wait(&sh.c_empty[s], ph ^ 1u);
-        mbar_wait_cl(&sh.ready[slot], static_cast<uint32_t>(n / RING) & 1u);
+        mbar_wait_cl(&sh.ready[slot], static_cast<uint32_t>(gc / RING) & 1u);
         fence_proxy_async_global();
         mbar_arrive_expect_tx(&sh.c_full[s], (MODE & kModeZeroV) ? kSlotBytes : chain_bytes<NS>());
         bulk_g2s(&st.ops, ring + static_cast<size_t>(slot) * kSlotBytes, kSlotBytes, &sh.c_full[s]);
         if constexpr ((MODE & kModeZeroV) == 0u) tma_load_3d(&st.v[0][0], &tm.v, dv0, h, tok, &sh.c_full[s]);
       }
+      }  // items
     }
   }
   // no CTA leaves while a peer may still arrive on its barriers

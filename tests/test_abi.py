@@ -76,7 +76,7 @@ def test_exports_every_declared_symbol(lib):
 
 def test_abi_version_and_status_strings(lib):
     lib.kda_abi_version.restype = ctypes.c_int32
-    assert lib.kda_abi_version() == 4
+    assert lib.kda_abi_version() == 5
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_status_string.argtypes = [ctypes.c_int]
     texts = {lib.kda_status_string(code) for code in range(11)}
@@ -131,6 +131,12 @@ def test_path_and_slice_settings_validated(lib):
         assert lib.kda_set_time_split(bad) == KDA_ERR_SHAPE
     for good in (1, 2, 0):
         assert lib.kda_set_time_split(good) == KDA_OK
+    lib.kda_set_schedule.argtypes = [ctypes.c_int32, ctypes.c_int32]
+    lib.kda_set_schedule.restype = ctypes.c_int
+    for bad in ((-1, 0), (3, 0), (16, 0), (2, -1)):
+        assert lib.kda_set_schedule(*bad) == KDA_ERR_SHAPE
+    for good in ((1, 0), (2, 3), (0, 0)):
+        assert lib.kda_set_schedule(*good) == KDA_OK
 
 
 @pytest.mark.parametrize("fn", ["kda_fwd", "kda_fwd_noalloc"])

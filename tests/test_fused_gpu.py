@@ -118,3 +118,19 @@ def test_fused_heavy_clamp_and_strided_projection(kda, oracle_mod):
                             cu_seqlens=d["cu_seqlens"], initial_state=d["initial_state"])
     torch.cuda.synchronize()
     assert torch.equal(ref[0], got[0]) and torch.equal(ref[1], got[1])
+
+
+def test_fused_persistent_schedule_bitwise(kda):
+    """Fused preprocessing with two persistent clusters taking all the pairs
+    gives the bits of one cluster per pair."""
+    import torch
+
+    inp = kda_inputs.make_inputs([200, 0, 31, 90, 16, 400], 3, seed=84, raw=True, random_initial_state=True)
+    try:
+        kda.set_schedule(1)
+        ref = run_fused(kda, inp)
+        kda.set_schedule(2, 2)
+        got = run_fused(kda, inp)
+    finally:
+        kda.set_schedule(0)
+    assert torch.equal(ref[0], got[0]) and torch.equal(ref[1], got[1])

@@ -5,7 +5,9 @@ Bars: o max-abs <= 3e-2 and rel-RMS <= 5e-3; final state rel-RMS <= 5e-3;
 segment handling bit-exact (a sequence gives the same bits alone or packed).
 
 Every behaviour test runs on each kernel variant: the 16-token path with 32-
-and 16-column value slices per CTA, and the 64-token tcgen05 path.
+and 16-column value slices per CTA, the same with a few persistent clusters
+taking all the (sequence, head) pairs round robin, and the 64-token tcgen05
+path.
 """
 import numpy as np
 import pytest
@@ -15,7 +17,9 @@ from tests import helpers as H
 
 pytestmark = pytest.mark.gpu
 
-VARIANTS = {"p16s32": (16, 32), "p16s16": (16, 16), "p64": (64, 0)}
+# path, value columns per CTA, persistent clusters (0: the default schedule)
+VARIANTS = {"p16s32": (16, 32, 0), "p16s16": (16, 16, 0), "p16s32q3": (16, 32, 3), "p16s16q2": (16, 16, 2),
+            "p64": (64, 0, 0)}
 
 
 @pytest.fixture(scope="module")
@@ -32,12 +36,14 @@ def kda():
 @pytest.fixture(params=list(VARIANTS), ids=list(VARIANTS))
 def variant(request, kda):
     """One kernel variant for the test; the library defaults are restored after."""
-    path, cols = VARIANTS[request.param]
+    path, cols, clusters = VARIANTS[request.param]
     kda.set_path(path)
     kda.set_slice_columns(cols)
+    kda.set_schedule(2 if clusters else 0, clusters)
     yield request.param
     kda.set_path(0)
     kda.set_slice_columns(0)
+    kda.set_schedule(0)
 
 
 @pytest.fixture(params=[16, 64], ids=["p16", "p64"])
@@ -292,6 +298,52 @@ def test_slice_variants_bitwise_equal(kda):
     o16, f16 = res[16]
     o32, f32 = res[32]
     assert torch.equal(o16, o32) and torch.equal(f16, f32)
+
+
+@pytest.mark.parametrize("cols", [32, 16])
+def test_persistent_schedules_bitwise_equal(kda, oracle_mod, cols):
+    """A cluster that runs several (sequence, head) pairs back to back gives
+    every pair the same bits as a cluster of its own: one cluster for all
+    pairs, a few, and as many as the device holds, on a batch of empty,
+    ragged and multi-chunk sequences; the persistent result also meets the
+    oracle."""
+    import torch
+
+    lens = [0, 300, 17, 1, 64, 0, 129, 1000, 16, 33, 250, 5]
+    inp = kda_inputs.make_inputs(lens, 5, seed=40, random_initial_state=True)
+    kda.set_path(16)
+    kda.set_slice_columns(cols)
+    try:
+        kda.set_schedule(1)
+        ref_o, ref_f = H.run_gpu(inp)
+        for cap in (1, 3, 7, 0):
+            kda.set_schedule(2, cap)
+            o, f = H.run_gpu(inp)
+            assert torch.equal(o, ref_o) and torch.equal(f, ref_f), f"{cols} columns, {cap} clusters"
+        kda.set_schedule(2, 4)
+        _check(oracle_mod, inp, f"persistent 4 clusters s{cols}")
+    finally:
+        kda.set_schedule(0)
+        kda.set_slice_columns(0)
+        kda.set_path(0)
+
+
+def test_persistent_full_size_uniform_varlen_bitwise(kda):
+    """The 8 x 1024, H = 32 batch (256 pairs, more than the device holds at
+    once): the default schedule (persistent) equals one cluster per pair."""
+    import torch
+
+    inp = kda_inputs.workload(3).make()
+    kda.set_path(16)
+    try:
+        kda.set_schedule(1)
+        ref = H.run_gpu(inp)
+        kda.set_schedule(0)
+        got = H.run_gpu(inp)
+    finally:
+        kda.set_schedule(0)
+        kda.set_path(0)
+    assert torch.equal(got[0], ref[0]) and torch.equal(got[1], ref[1])
 
 
 def test_zz_no_wait_timeouts(kda):
