@@ -8,7 +8,8 @@ fixed-size ring declared in device memory by the library instead.
 
 The GPU test calls it through the C ABI twice in a row, on different batches
 (so the second call runs on the first call's leftover scratch contents), on
-each kernel path, and checks that each result is bitwise identical to
+each kernel path and with a few persistent clusters running all the pairs,
+and checks that each result is bitwise identical to
 kda_fwd's on the same inputs: both run the same deterministic kernel, only
 the scratch memory differs. It loads the library itself, so it passes in a
 fresh process as well as after the other tests.
@@ -26,8 +27,8 @@ MAX_PAIRS = 32  # KDA_NOALLOC_MAX_PAIRS in include/kda.h
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("path", [16, 64])
-def test_noalloc_matches_kda_fwd_on_two_calls(path):
+@pytest.mark.parametrize("path,clusters", [(16, 0), (64, 0), (16, 3)])
+def test_noalloc_matches_kda_fwd_on_two_calls(path, clusters):
     import torch
 
     if not torch.cuda.is_available():
@@ -40,6 +41,9 @@ def test_noalloc_matches_kda_fwd_on_two_calls(path):
     fn.argtypes = [P, P, P, P, P, ctypes.c_float, ctypes.c_void_p, ctypes.c_int32, P, P, P, ctypes.c_void_p]
     fn.restype = ctypes.c_int
     kda.set_path(path)
+    # clusters > 0: a few persistent clusters run all the pairs, so each cluster's
+    # ring slots carry several pairs' chunks within one call
+    kda.set_schedule(2 if clusters else 0, clusters)
     try:
         batches = [
             kda_inputs.make_inputs([300, 17, 0, 129], 4, seed=71, random_initial_state=True),   # 16 pairs
@@ -61,4 +65,5 @@ def test_noalloc_matches_kda_fwd_on_two_calls(path):
             assert torch.equal(fin, ref_f), f"call {i}: state bits differ from kda_fwd"
     finally:
         kda.set_path(0)
+        kda.set_schedule(0)
     assert kda.wait_timeouts(reset=True) == 0
