@@ -30,7 +30,8 @@
 //                   signals the cluster.
 //     8     notify: (consumer) relays each landed stage to the chain warps
 //                   through hardware named barriers and returns the ring slot
-//                   to its producer.
+//                   to its producer. When NS = 16 this role runs on warp 1 (the
+//                   unused second chain warp), off the chain's sub-partition.
 //     9     bounds: records a cu_seqlens that is not a partition of [0, T)
 //                   in the device status word (rank 0 of head 0's clusters).
 //
@@ -75,12 +76,16 @@ constexpr int CSTAGE = 6;         // consumer stages (cload -> chain)
 // Warp w issues on sub-partition w mod 4. The two chain warps get partitions 0
 // and 1 with only the light load and notify warps beside them; the gate, mma
 // and store warps, which burst through ALU and shared-memory work, share
-// partitions 2 and 3. Warp 9 only checks the sequence bounds once.
+// partitions 2 and 3. Warp 9 only checks the sequence bounds once. (Measured:
+// a per-chunk helper beside a chain warp costs it time, so with one chain warp
+// the notify role moves to partition 1.)
 constexpr int MAX_CHAIN = 2;      // chain warps 0 (and 1), 16 value columns each
 constexpr int NGATE = 4;          // gate warps 2, 3, 6, 7
 constexpr int WARP_PLOAD = 4;
 constexpr int WARP_CLOAD = 5;
-constexpr int WARP_NOTIFY = 8;    // relays stage completion to the chain warps
+// relays stage completion to the chain warps
+template <int NS>
+__host__ __device__ constexpr int notify_warp() { return NS == 16 ? 1 : 8; }
 constexpr int WARP_MMA = 10;      // also solves (I + L)^{-1}
 constexpr int WARP_STORE = 11;
 constexpr int NTHREADS = 12 * 32;
@@ -88,10 +93,12 @@ __host__ __device__ constexpr bool is_gate_warp(int w) { return (w & 3) >= 2 && 
 __host__ __device__ constexpr int gate_warp_index(int w) { return (w & 1) + ((w >> 2) << 1); }
 
 // Hardware named barriers: 0 is the CTA-wide one, 1 the gate group's, and
-// 2 + 2 s + w tells chain warp w that consumer stage s has landed.
+// 2 + s tells the chain warps that consumer stage s has landed (the chain
+// warps and the notify warp meet there; one barrier for both chain warps
+// measured faster than one per warp).
 constexpr int BAR_GATE = 1;
 constexpr int BAR_FULL0 = 2;
-static_assert(BAR_FULL0 + 2 * CSTAGE <= 16, "named barrier ids");
+static_assert(BAR_FULL0 + CSTAGE <= 16, "named barrier ids");
 static_assert(RING % (D / 16) == 0, "a ring slot must always belong to the same producer CTA");
 
 // Padded row pitches: 272 B and 48 B rows keep 8-row ldmatrix reads on distinct banks.
@@ -308,7 +315,7 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
       ChainStage<NS>& st = sh.cst[s];
 
       // stage s has landed (the notify warp observed its mbarrier)
-      named_bar(BAR_FULL0 + 2 * s + warp, 64);
+      named_bar(BAR_FULL0 + s, 32 * (NCHAIN + 1));
 
       // Every product on the chain takes the register-resident operand as its
       // A fragment, so nothing on the chain needs a transpose:
@@ -736,7 +743,7 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
     }
     gbase += nch;
     }  // items
-  } else if (warp == WARP_NOTIFY) {
+  } else if (warp == notify_warp<NS>()) {
     // ==================================================== stage notifications
     // Waiting on a transaction mbarrier costs the waiter ~100 cycles even when
     // the phase completed long ago; this warp takes that cost off the chain's
@@ -752,8 +759,7 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
       const int s = static_cast<int>(gc % CSTAGE);
       mbar_wait(&sh.c_full[s], static_cast<uint32_t>(gc / CSTAGE) & 1u);
       __syncwarp();
-#pragma unroll
-      for (int w = 0; w < NCHAIN; ++w) named_bar_arrive(BAR_FULL0 + 2 * s + w, 64);
+      named_bar_arrive(BAR_FULL0 + s, 32 * (NCHAIN + 1));
       // the ring slot has been copied here: give it back to its producer
       if (lane == 0)
         mbar_arrive_remote_relaxed(&sh.slot_free[gc % RING], static_cast<uint32_t>(gc % NSLICE));
