@@ -502,11 +502,16 @@ size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 // helper streams; then o = o_loc + S_a^T o_M and S_T = M S_a + B.
 kda_status_t launch16_split(const Problem& P, int dev, cudaStream_t stream) {
   namespace sp = kda::split;
-  // Measured on B200 (T = 131072, H = 8), the first half runs ~4 % slower per
-  // token than the zero-start run of the second half (the identity run, with
-  // v = 0, is faster still), so the first half takes ~49 % of the tokens.
-  const int64_t T = P.T, Ta = (T * 63 / 128) & ~static_cast<int64_t>(kda::C - 1), T1 = T - Ta;
+  // The first half runs on 16-column slices (8-CTA clusters) when the device
+  // has room for its H clusters beside the second half's 2H 4-CTA clusters
+  // (16 H SMs in all). Measured on B200 (T = 131072, H = 8), a 16-column
+  // chain then runs ~25 % faster per chunk than the second half's fp32-output
+  // run, so the first half takes ~57 % of the tokens. On 32-column slices it
+  // runs ~4 % slower per token than that run (the identity run, with v = 0, is
+  // faster still) and takes ~49 % of them.
   const int H = P.num_heads;
+  const bool a16 = 16 * static_cast<int64_t>(H) <= g_num_sms[dev] && H <= g_max_clusters16[dev];
+  const int64_t T = P.T, Ta = (T * (a16 ? 73 : 63) / 128) & ~static_cast<int64_t>(kda::C - 1), T1 = T - Ta;
   const size_t st_bytes = round256(static_cast<size_t>(H) * kda::D * kda::D * 4);
   const size_t o_bytes = round256(static_cast<size_t>(T1) * H * kda::D * 4);     // o_loc, fp32
   const size_t om_bytes = round256(static_cast<size_t>(T1) * H * kda::D * 2);    // o_M, bf16
@@ -544,7 +549,7 @@ kda_status_t launch16_split(const Problem& P, int dev, cudaStream_t stream) {
     if ((e = cudaEventRecord(ev[0], stream)) != cudaSuccess) st = cuda_fail(e);
     for (int i = 0; i < 2 && st == KDA_OK; ++i)
       if ((e = cudaStreamWaitEvent(side[i], ev[0], 0)) != cudaSuccess) st = cuda_fail(e);
-    if (st == KDA_OK) st = launch16(A, rings, dev, stream, 0, nullptr, 32);
+    if (st == KDA_OK) st = launch16(A, rings, dev, stream, 0, nullptr, a16 ? 16 : 32);
     if (st == KDA_OK) st = launch16(L, rings + ring_b, dev, side[0], kSplitL, oloc, 32);
     if (st == KDA_OK) st = launch16(M, rings + 2 * ring_b, dev, side[1], kSplitM, nullptr, 32);
     for (int i = 0; i < 2 && st == KDA_OK; ++i) {
