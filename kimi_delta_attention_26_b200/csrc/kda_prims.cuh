@@ -107,7 +107,7 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long* m, uin
                : "memory");
 }
 
-// TMA tiled loads (no multicast). Out-of-range rows of the box are zero-filled.
+// TMA tiled loads into this CTA's own shared memory. Out-of-range rows of the box are zero-filled.
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
                                             unsigned long long* m) {
   asm volatile(
