@@ -245,12 +245,14 @@ kda_status_t kda_set_schedule(int32_t mode, int32_t clusters);
  * kda_set_time_split -- the time-split prefill of kda_fwd (16-token path).
  *
  * A batch of ONE sequence (num_seqs = 1) with few heads leaves most SMs idle:
- * each head is one serial chain. The time split runs the sequence's two
- * halves at once: the first from the initial state, the second twice in
+ * each head is one serial chain. The time split runs two parts of the
+ * sequence at once: the first from the initial state, the second twice in
  * parallel -- from the zero state, and with v = 0 from the identity, which
  * gives the map from its (not yet known) start state to its outputs and end
  * state -- and then combines them (o_t += S_a^T o_M(t), S_T = M S_a + B; the
- * recurrence is linear in its initial state). It takes extra scratch from the
+ * recurrence is linear in its initial state). The first part takes ~57 % of
+ * the tokens on 16-column slices when the device has 16 * H SMs for the three
+ * runs, else ~49 % on 32-column slices, so that the runs end together. It takes extra scratch from the
  * pool (about T/2 x H x 768 bytes plus three rings and three states) and two
  * helper streams (created once per device; the call stays ordered on
  * `stream`). Results agree with the unsplit path within the library's
