@@ -292,180 +292,180 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
     const int64_t out_st = p.out_st;
     int64_t gc = 0;                    // the cluster's chunks so far
     for (int it = first; it < nitems; it += stride) {
-    int seq, h;
-    int64_t t0, t1;
-    const int nch = item_at(it, seq, h, t0, t1);
-    const size_t sbase = (static_cast<size_t>(seq) * H + h) * D * D;
-    // this lane's output columns of head h; rows step by the token stride
-    __nv_bfloat16* const out_base = p.out + static_cast<int64_t>(h) * p.out_sh + dv0 + cv + 2 * tq;
-#pragma unroll
-    for (int u = 0; u < 16; ++u)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = 8 * u + 2 * tq + (e & 1);
-        const int col = dv0 + cv + gq + 8 * (e >> 1);
-        sacc[u][e] = (MODE & kModeIdentityInit) ? (key == col ? 1.f : 0.f)
-                     : p.init ? __ldg(p.init + sbase + static_cast<size_t>(key) * D + col) : 0.f;
-      }
-
-    for (int n = 0; n < nch; ++n, ++gc) {
-      const int s = static_cast<int>(gc % CSTAGE);
-      const int64_t cs = t0 + static_cast<int64_t>(n) * C;
-      const int m = static_cast<int>((t1 - cs) < C ? (t1 - cs) : C);
-      ChainStage<NS>& st = sh.cst[s];
-
-      // stage s has landed (the notify warp observed its mbarrier)
-      named_bar(BAR_FULL0 + s, 32 * (NCHAIN + 1));
-
-      // Every product on the chain takes the register-resident operand as its
-      // A fragment, so nothing on the chain needs a transpose:
-      //   X^T = V^T + S^T Kd^T,  Vnew^T = X^T Tb^T,  S^T <- S^T Diag(gamma) + Vnew^T Kend,
-      //   O^T = S^T Qd^T + Vnew^T Aqk^T  (times scale at the store).
-      // The products are ordered for one in-order warp on one tensor pipe: the
-      // state's own chain (X -> Vnew -> S) goes first at every step and the O
-      // products, which nothing waits for, fill the pipe while a chain result
-      // drains through conversion.
-      uint32_t bk[8][4];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) ldsm_x4(bk[t], &st.ops.kd[(lane & 7) + ((lane >> 4) << 3)][16 * t + ((lane >> 3) & 1) * 8]);
-      // ---- X^T (two accumulator chains per 8-token tile); each key tile of S
-      // is packed to bf16 (sa: the chunk-start state, also used by O) and then
-      // scaled by gamma for the update. Lane (gq, tq) of tile nt holds columns
-      // gq (+8) x tokens 8nt + 2tq (+1).
-      float xa[2][4], xb[2][4] = {};
-      {
-        uint32_t vt[4];
-        if constexpr ((MODE & kModeZeroV) != 0u) {
-          vt[0] = vt[1] = vt[2] = vt[3] = 0u;
-        } else {
-          ldsm_x4_t(vt, &st.v[(lane & 7) + ((lane >> 3) & 1) * 8][cv + (lane >> 4) * 8]);
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int nt = j & 1, e0 = 2 * (j >> 1);
-          xa[nt][e0] = __uint_as_float(vt[j] << 16);
-          xa[nt][e0 + 1] = __uint_as_float(vt[j] & 0xffff0000u);
-        }
-      }
-      uint32_t sa[8][4];
-      const float4* gp = reinterpret_cast<const float4*>(&st.ops.gam[tq][0]);
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        sa[t][0] = pack_bf16(sacc[2 * t][0], sacc[2 * t][1]);
-        sa[t][1] = pack_bf16(sacc[2 * t][2], sacc[2 * t][3]);
-        sa[t][2] = pack_bf16(sacc[2 * t + 1][0], sacc[2 * t + 1][1]);
-        sa[t][3] = pack_bf16(sacc[2 * t + 1][2], sacc[2 * t + 1][3]);
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          if (t & 1)
-            mma(xb[nt], sa[t], bk[t][2 * nt], bk[t][2 * nt + 1]);
-          else
-            mma(xa[nt], sa[t], bk[t][2 * nt], bk[t][2 * nt + 1]);
-        }
-        const float4 g4 = gp[t];
-        mul2(sacc[2 * t][0], sacc[2 * t][1], g4.x, g4.y);
-        mul2(sacc[2 * t][2], sacc[2 * t][3], g4.x, g4.y);
-        mul2(sacc[2 * t + 1][0], sacc[2 * t + 1][1], g4.z, g4.w);
-        mul2(sacc[2 * t + 1][2], sacc[2 * t + 1][3], g4.z, g4.w);
-      }
-      // ---- O^T = S^T Qd^T (chunk-start state) + Vnew^T Aqk^T, in three installments
-      float oa[2][4] = {}, ob[2][4] = {};
-      auto o_steps = [&](int t_begin, int t_end) {
-#pragma unroll
-        for (int t = t_begin; t < t_end; ++t) {
-          uint32_t bq[4];
-          ldsm_x4(bq, &st.ops.qd[(lane & 7) + ((lane >> 4) << 3)][16 * t + ((lane >> 3) & 1) * 8]);
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt) {
-            if (t & 1)
-              mma(ob[nt], sa[t], bq[2 * nt], bq[2 * nt + 1]);
-            else
-              mma(oa[nt], sa[t], bq[2 * nt], bq[2 * nt + 1]);
-          }
-        }
-      };
-      o_steps(0, 3);
-      // ---- Vnew^T = X^T Tb^T
-      uint32_t bt[4];
-      ldsm_x4(bt, &st.ops.tb[(lane & 7) + ((lane >> 4) << 3)][((lane >> 3) & 1) * 8]);
-      float vn[2][4] = {};
-      {
-        uint32_t ax[4];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          ax[2 * nt] = pack_bf16(xa[nt][0] + xb[nt][0], xa[nt][1] + xb[nt][1]);
-          ax[2 * nt + 1] = pack_bf16(xa[nt][2] + xb[nt][2], xa[nt][3] + xb[nt][3]);
-        }
-        mma(vn[0], ax, bt[0], bt[1]);
-        mma(vn[1], ax, bt[2], bt[3]);
-      }
-      // kd fragments are dead: the same registers take Kend
-#pragma unroll
-      for (int t = 0; t < 8; ++t) ldsm_x4_t(bk[t], &st.ops.ke[(lane & 7) + ((lane >> 3) & 1) * 8][16 * t + (lane >> 4) * 8]);
-      o_steps(3, 6);
-      // Vnew^T as an A fragment (rows = columns, k = tokens)
-      uint32_t av[4];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        av[2 * nt] = pack_bf16(vn[nt][0], vn[nt][1]);
-        av[2 * nt + 1] = pack_bf16(vn[nt][2], vn[nt][3]);
-      }
-      // ---- S^T <- S^T Diag(gamma) + Vnew^T Kend  (gamma applied above)
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        mma(sacc[2 * t], av, bk[t][0], bk[t][1]);
-        mma(sacc[2 * t + 1], av, bk[t][2], bk[t][3]);
-      }
-      o_steps(6, 8);
-      {
-        uint32_t ba[4];
-        ldsm_x4(ba, &st.ops.aqk[(lane & 7) + ((lane >> 4) << 3)][((lane >> 3) & 1) * 8]);
-        mma(oa[0], av, ba[0], ba[1]);
-        mma(oa[1], av, ba[2], ba[3]);
-      }
-      // the stage is no longer read by this warp
-      mbar_arrive_warp(&sh.c_empty[s]);
-      if constexpr ((MODE & kModeOutF32) != 0u) {
-        // fp32 O: lane (gq, tq) of tile nt holds columns gq (+8) x tokens
-        // 8nt + 2tq (+1)
-        float* fbase = p.outf + static_cast<int64_t>(h) * D + dv0 + cv + gq;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int tok = 8 * nt + 2 * tq + (e & 1);
-            if (tok < m) fbase[(cs + tok) * p.outf_st + 8 * (e >> 1)] = (oa[nt][e] + ob[nt][e]) * p.scale;
-          }
-      } else {
-        // ---- store O: an 8x8 transpose per tile turns (column, token pair)
-        // into (token, column pair)
-        uint32_t r[2][2];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          r[nt][0] = movmatrix_t(pack_bf16((oa[nt][0] + ob[nt][0]) * p.scale, (oa[nt][1] + ob[nt][1]) * p.scale));
-          r[nt][1] = movmatrix_t(pack_bf16((oa[nt][2] + ob[nt][2]) * p.scale, (oa[nt][3] + ob[nt][3]) * p.scale));
-        }
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          const int tok = 8 * nt + gq;
-          if (tok < m) {
-            __nv_bfloat16* dst = out_base + (cs + tok) * out_st;
-            *reinterpret_cast<uint32_t*>(dst) = r[nt][0];
-            *reinterpret_cast<uint32_t*>(dst + 8) = r[nt][1];
-          }
-        }
-      }
-    }
-    if (p.fin) {
+      int seq, h;
+      int64_t t0, t1;
+      const int nch = item_at(it, seq, h, t0, t1);
+      const size_t sbase = (static_cast<size_t>(seq) * H + h) * D * D;
+      // this lane's output columns of head h; rows step by the token stride
+      __nv_bfloat16* const out_base = p.out + static_cast<int64_t>(h) * p.out_sh + dv0 + cv + 2 * tq;
 #pragma unroll
       for (int u = 0; u < 16; ++u)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int key = 8 * u + 2 * tq + (e & 1);
           const int col = dv0 + cv + gq + 8 * (e >> 1);
-          p.fin[sbase + static_cast<size_t>(key) * D + col] = sacc[u][e];
+          sacc[u][e] = (MODE & kModeIdentityInit) ? (key == col ? 1.f : 0.f)
+                       : p.init ? __ldg(p.init + sbase + static_cast<size_t>(key) * D + col) : 0.f;
         }
-    }
+
+      for (int n = 0; n < nch; ++n, ++gc) {
+        const int s = static_cast<int>(gc % CSTAGE);
+        const int64_t cs = t0 + static_cast<int64_t>(n) * C;
+        const int m = static_cast<int>((t1 - cs) < C ? (t1 - cs) : C);
+        ChainStage<NS>& st = sh.cst[s];
+
+        // stage s has landed (the notify warp observed its mbarrier)
+        named_bar(BAR_FULL0 + s, 32 * (NCHAIN + 1));
+
+        // Every product on the chain takes the register-resident operand as its
+        // A fragment, so nothing on the chain needs a transpose:
+        //   X^T = V^T + S^T Kd^T,  Vnew^T = X^T Tb^T,  S^T <- S^T Diag(gamma) + Vnew^T Kend,
+        //   O^T = S^T Qd^T + Vnew^T Aqk^T  (times scale at the store).
+        // The products are ordered for one in-order warp on one tensor pipe: the
+        // state's own chain (X -> Vnew -> S) goes first at every step and the O
+        // products, which nothing waits for, fill the pipe while a chain result
+        // drains through conversion.
+        uint32_t bk[8][4];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) ldsm_x4(bk[t], &st.ops.kd[(lane & 7) + ((lane >> 4) << 3)][16 * t + ((lane >> 3) & 1) * 8]);
+        // ---- X^T (two accumulator chains per 8-token tile); each key tile of S
+        // is packed to bf16 (sa: the chunk-start state, also used by O) and then
+        // scaled by gamma for the update. Lane (gq, tq) of tile nt holds columns
+        // gq (+8) x tokens 8nt + 2tq (+1).
+        float xa[2][4], xb[2][4] = {};
+        {
+          uint32_t vt[4];
+          if constexpr ((MODE & kModeZeroV) != 0u) {
+            vt[0] = vt[1] = vt[2] = vt[3] = 0u;
+          } else {
+            ldsm_x4_t(vt, &st.v[(lane & 7) + ((lane >> 3) & 1) * 8][cv + (lane >> 4) * 8]);
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int nt = j & 1, e0 = 2 * (j >> 1);
+            xa[nt][e0] = __uint_as_float(vt[j] << 16);
+            xa[nt][e0 + 1] = __uint_as_float(vt[j] & 0xffff0000u);
+          }
+        }
+        uint32_t sa[8][4];
+        const float4* gp = reinterpret_cast<const float4*>(&st.ops.gam[tq][0]);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          sa[t][0] = pack_bf16(sacc[2 * t][0], sacc[2 * t][1]);
+          sa[t][1] = pack_bf16(sacc[2 * t][2], sacc[2 * t][3]);
+          sa[t][2] = pack_bf16(sacc[2 * t + 1][0], sacc[2 * t + 1][1]);
+          sa[t][3] = pack_bf16(sacc[2 * t + 1][2], sacc[2 * t + 1][3]);
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            if (t & 1)
+              mma(xb[nt], sa[t], bk[t][2 * nt], bk[t][2 * nt + 1]);
+            else
+              mma(xa[nt], sa[t], bk[t][2 * nt], bk[t][2 * nt + 1]);
+          }
+          const float4 g4 = gp[t];
+          mul2(sacc[2 * t][0], sacc[2 * t][1], g4.x, g4.y);
+          mul2(sacc[2 * t][2], sacc[2 * t][3], g4.x, g4.y);
+          mul2(sacc[2 * t + 1][0], sacc[2 * t + 1][1], g4.z, g4.w);
+          mul2(sacc[2 * t + 1][2], sacc[2 * t + 1][3], g4.z, g4.w);
+        }
+        // ---- O^T = S^T Qd^T (chunk-start state) + Vnew^T Aqk^T, in three installments
+        float oa[2][4] = {}, ob[2][4] = {};
+        auto o_steps = [&](int t_begin, int t_end) {
+#pragma unroll
+          for (int t = t_begin; t < t_end; ++t) {
+            uint32_t bq[4];
+            ldsm_x4(bq, &st.ops.qd[(lane & 7) + ((lane >> 4) << 3)][16 * t + ((lane >> 3) & 1) * 8]);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+              if (t & 1)
+                mma(ob[nt], sa[t], bq[2 * nt], bq[2 * nt + 1]);
+              else
+                mma(oa[nt], sa[t], bq[2 * nt], bq[2 * nt + 1]);
+            }
+          }
+        };
+        o_steps(0, 3);
+        // ---- Vnew^T = X^T Tb^T
+        uint32_t bt[4];
+        ldsm_x4(bt, &st.ops.tb[(lane & 7) + ((lane >> 4) << 3)][((lane >> 3) & 1) * 8]);
+        float vn[2][4] = {};
+        {
+          uint32_t ax[4];
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            ax[2 * nt] = pack_bf16(xa[nt][0] + xb[nt][0], xa[nt][1] + xb[nt][1]);
+            ax[2 * nt + 1] = pack_bf16(xa[nt][2] + xb[nt][2], xa[nt][3] + xb[nt][3]);
+          }
+          mma(vn[0], ax, bt[0], bt[1]);
+          mma(vn[1], ax, bt[2], bt[3]);
+        }
+        // kd fragments are dead: the same registers take Kend
+#pragma unroll
+        for (int t = 0; t < 8; ++t) ldsm_x4_t(bk[t], &st.ops.ke[(lane & 7) + ((lane >> 3) & 1) * 8][16 * t + (lane >> 4) * 8]);
+        o_steps(3, 6);
+        // Vnew^T as an A fragment (rows = columns, k = tokens)
+        uint32_t av[4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          av[2 * nt] = pack_bf16(vn[nt][0], vn[nt][1]);
+          av[2 * nt + 1] = pack_bf16(vn[nt][2], vn[nt][3]);
+        }
+        // ---- S^T <- S^T Diag(gamma) + Vnew^T Kend  (gamma applied above)
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          mma(sacc[2 * t], av, bk[t][0], bk[t][1]);
+          mma(sacc[2 * t + 1], av, bk[t][2], bk[t][3]);
+        }
+        o_steps(6, 8);
+        {
+          uint32_t ba[4];
+          ldsm_x4(ba, &st.ops.aqk[(lane & 7) + ((lane >> 4) << 3)][((lane >> 3) & 1) * 8]);
+          mma(oa[0], av, ba[0], ba[1]);
+          mma(oa[1], av, ba[2], ba[3]);
+        }
+        // the stage is no longer read by this warp
+        mbar_arrive_warp(&sh.c_empty[s]);
+        if constexpr ((MODE & kModeOutF32) != 0u) {
+          // fp32 O: lane (gq, tq) of tile nt holds columns gq (+8) x tokens
+          // 8nt + 2tq (+1)
+          float* fbase = p.outf + static_cast<int64_t>(h) * D + dv0 + cv + gq;
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int tok = 8 * nt + 2 * tq + (e & 1);
+              if (tok < m) fbase[(cs + tok) * p.outf_st + 8 * (e >> 1)] = (oa[nt][e] + ob[nt][e]) * p.scale;
+            }
+        } else {
+          // ---- store O: an 8x8 transpose per tile turns (column, token pair)
+          // into (token, column pair)
+          uint32_t r[2][2];
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            r[nt][0] = movmatrix_t(pack_bf16((oa[nt][0] + ob[nt][0]) * p.scale, (oa[nt][1] + ob[nt][1]) * p.scale));
+            r[nt][1] = movmatrix_t(pack_bf16((oa[nt][2] + ob[nt][2]) * p.scale, (oa[nt][3] + ob[nt][3]) * p.scale));
+          }
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            const int tok = 8 * nt + gq;
+            if (tok < m) {
+              __nv_bfloat16* dst = out_base + (cs + tok) * out_st;
+              *reinterpret_cast<uint32_t*>(dst) = r[nt][0];
+              *reinterpret_cast<uint32_t*>(dst + 8) = r[nt][1];
+            }
+          }
+        }
+      }
+      if (p.fin) {
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int key = 8 * u + 2 * tq + (e & 1);
+            const int col = dv0 + cv + gq + 8 * (e >> 1);
+            p.fin[sbase + static_cast<size_t>(key) * D + col] = sacc[u][e];
+          }
+      }
     }  // items
   } else if (is_gate_warp(warp)) {
     // ============================================================ gate warps
@@ -478,192 +478,192 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
     const int c0 = 2 * cp;
     int64_t gbase = 0, jg = 0;  // the item's first chunk; this CTA's produced chunks so far
     for (int it = first; it < nitems; it += stride) {
-    int seq, h;
-    int64_t t0, t1;
-    const int nch = item_at(it, seq, h, t0, t1);
-    for (int n = owned_first(gbase); n < nch; n += NSLICE, ++jg) {
-      const int j = static_cast<int>(jg & 1);  // parity of the exchange buffers
-      const int rs = static_cast<int>(jg % PRSTAGE), ps = static_cast<int>(jg % PSTAGE);
-      const uint32_t rph = static_cast<uint32_t>(jg / PRSTAGE) & 1u;
-      const uint32_t pph = static_cast<uint32_t>(jg / PSTAGE) & 1u;
-      const int64_t cs = t0 + static_cast<int64_t>(n) * C;
-      const int m = static_cast<int>((t1 - cs) < C ? (t1 - cs) : C);
-      RawStage& rw = sh.raw[rs];
-      ProdStage& st = sh.prod[ps];
-      mbar_wait(&sh.raw_full[rs], rph);
+      int seq, h;
+      int64_t t0, t1;
+      const int nch = item_at(it, seq, h, t0, t1);
+      for (int n = owned_first(gbase); n < nch; n += NSLICE, ++jg) {
+        const int j = static_cast<int>(jg & 1);  // parity of the exchange buffers
+        const int rs = static_cast<int>(jg % PRSTAGE), ps = static_cast<int>(jg % PSTAGE);
+        const uint32_t rph = static_cast<uint32_t>(jg / PRSTAGE) & 1u;
+        const uint32_t pph = static_cast<uint32_t>(jg / PSTAGE) & 1u;
+        const int64_t cs = t0 + static_cast<int64_t>(n) * C;
+        const int m = static_cast<int>((t1 - cs) < C ? (t1 - cs) : C);
+        RawStage& rw = sh.raw[rs];
+        ProdStage& st = sh.prod[ps];
+        mbar_wait(&sh.raw_full[rs], rph);
 
-      // ---- raw inputs of this thread (rows past the sequence end masked)
-      constexpr bool fused = FG;
-      float2 e[8], kv[8], qv[8];
-#pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
-        const int i = 8 * th + jj;
-        const bool ok = i < m;
-        const float2 gg = *reinterpret_cast<const float2*>(&rw.g[i][c0]);
-        const __nv_bfloat162 kk = *reinterpret_cast<const __nv_bfloat162*>(&rw.k[i][c0]);
-        const __nv_bfloat162 qq = *reinterpret_cast<const __nv_bfloat162*>(&rw.q[i][c0]);
-        float2 ee;
-        if constexpr (fused) {  // exp(max(log sigmoid(x), lb)) = max(sigmoid(x), exp(lb))
-          ee = make_float2(fmaxf(__fdividef(1.f, 1.f + __expf(-gg.x)), p.exp_lb),
-                           fmaxf(__fdividef(1.f, 1.f + __expf(-gg.y)), p.exp_lb));
-        } else {
-          ee = make_float2(__expf(gg.x), __expf(gg.y));
-        }
-        e[jj] = ok ? ee : make_float2(1.f, 1.f);
-        kv[jj] = ok ? __bfloat1622float2(kk) : make_float2(0.f, 0.f);
-        qv[jj] = ok ? __bfloat1622float2(qq) : make_float2(0.f, 0.f);
-      }
-      float bv = 0.f;
-      if (gt < C) {
-        const float b = rw.beta[gt];
-        bv = gt < m ? (fused ? __fdividef(1.f, 1.f + __expf(-b)) : b) : 0.f;
-      }
-      mbar_arrive_warp(&sh.raw_empty[rs]);
-      // fused preprocessing: this warp's partial squared norms of its 8
-      // tokens' q and k (its 64 channels), reduced over the warp by a
-      // butterfly that halves the values each step: afterwards lane pair
-      // (l, l ^ 1) holds value 8 (l >> 4 & 1) + 4 (l >> 3 & 1) + 2 (l >> 2 & 1)
-      // + (l >> 1 & 1) of [q0..q7, k0..k7]
-      if constexpr (fused) {
-        float sv[16];
+        // ---- raw inputs of this thread (rows past the sequence end masked)
+        constexpr bool fused = FG;
+        float2 e[8], kv[8], qv[8];
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
-          sv[jj] = fmaf(qv[jj].x, qv[jj].x, qv[jj].y * qv[jj].y);
-          sv[8 + jj] = fmaf(kv[jj].x, kv[jj].x, kv[jj].y * kv[jj].y);
+          const int i = 8 * th + jj;
+          const bool ok = i < m;
+          const float2 gg = *reinterpret_cast<const float2*>(&rw.g[i][c0]);
+          const __nv_bfloat162 kk = *reinterpret_cast<const __nv_bfloat162*>(&rw.k[i][c0]);
+          const __nv_bfloat162 qq = *reinterpret_cast<const __nv_bfloat162*>(&rw.q[i][c0]);
+          float2 ee;
+          if constexpr (fused) {  // exp(max(log sigmoid(x), lb)) = max(sigmoid(x), exp(lb))
+            ee = make_float2(fmaxf(__fdividef(1.f, 1.f + __expf(-gg.x)), p.exp_lb),
+                             fmaxf(__fdividef(1.f, 1.f + __expf(-gg.y)), p.exp_lb));
+          } else {
+            ee = make_float2(__expf(gg.x), __expf(gg.y));
+          }
+          e[jj] = ok ? ee : make_float2(1.f, 1.f);
+          kv[jj] = ok ? __bfloat1622float2(kk) : make_float2(0.f, 0.f);
+          qv[jj] = ok ? __bfloat1622float2(qq) : make_float2(0.f, 0.f);
         }
+        float bv = 0.f;
+        if (gt < C) {
+          const float b = rw.beta[gt];
+          bv = gt < m ? (fused ? __fdividef(1.f, 1.f + __expf(-b)) : b) : 0.f;
+        }
+        mbar_arrive_warp(&sh.raw_empty[rs]);
+        // fused preprocessing: this warp's partial squared norms of its 8
+        // tokens' q and k (its 64 channels), reduced over the warp by a
+        // butterfly that halves the values each step: afterwards lane pair
+        // (l, l ^ 1) holds value 8 (l >> 4 & 1) + 4 (l >> 3 & 1) + 2 (l >> 2 & 1)
+        // + (l >> 1 & 1) of [q0..q7, k0..k7]
+        if constexpr (fused) {
+          float sv[16];
 #pragma unroll
-        for (int w = 8, off = 16; w >= 1; w >>= 1, off >>= 1) {
-          const bool upper = (lane & off) != 0;
+          for (int jj = 0; jj < 8; ++jj) {
+            sv[jj] = fmaf(qv[jj].x, qv[jj].x, qv[jj].y * qv[jj].y);
+            sv[8 + jj] = fmaf(kv[jj].x, kv[jj].x, kv[jj].y * kv[jj].y);
+          }
 #pragma unroll
-          for (int x = 0; x < w; ++x) {
-            const float send = upper ? sv[x] : sv[w + x];
-            const float got = __shfl_xor_sync(0xffffffffu, send, off);
-            sv[x] = (upper ? sv[w + x] : sv[x]) + got;
+          for (int w = 8, off = 16; w >= 1; w >>= 1, off >>= 1) {
+            const bool upper = (lane & off) != 0;
+#pragma unroll
+            for (int x = 0; x < w; ++x) {
+              const float send = upper ? sv[x] : sv[w + x];
+              const float got = __shfl_xor_sync(0xffffffffu, send, off);
+              sv[x] = (upper ? sv[w + x] : sv[x]) + got;
+            }
+          }
+          sv[0] += __shfl_xor_sync(0xffffffffu, sv[0], 1);
+          if ((lane & 1) == 0) {
+            const int idx = 8 * ((lane >> 4) & 1) + 4 * ((lane >> 3) & 1) + 2 * ((lane >> 2) & 1) + ((lane >> 1) & 1);
+            sh.gnorm[j & 1][gate_warp_index(warp)][idx] = sv[0];
           }
         }
-        sv[0] += __shfl_xor_sync(0xffffffffu, sv[0], 1);
-        if ((lane & 1) == 0) {
-          const int idx = 8 * ((lane >> 4) & 1) + 4 * ((lane >> 3) & 1) + 2 * ((lane >> 2) & 1) + ((lane >> 1) & 1);
-          sh.gnorm[j & 1][gate_warp_index(warp)][idx] = sv[0];
-        }
-      }
 
-      // ---- decay products: this half's total, exchanged with the other half
-      float2 P = make_float2(1.f, 1.f);
-#pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
-        P.x *= e[jj].x;
-        P.y *= e[jj].y;
-      }
-      mbar_wait(&sh.prod_free[ps], pph ^ 1u);
-      sh.gprod[j & 1][th][cp] = P;
-      if (gt < C) st.beta[gt] = bv;
-      named_bar(BAR_GATE, NGATE * 32);
-      const float2 Po = sh.gprod[j & 1][th ^ 1][cp];
-      if constexpr (fused) {  // full norms of this half's tokens: this warp's 64 channels + the partner warp's
-        const int wi = gate_warp_index(warp);
-        const float* a = sh.gnorm[j & 1][wi];
-        const float* b = sh.gnorm[j & 1][wi ^ 1];
+        // ---- decay products: this half's total, exchanged with the other half
+        float2 P = make_float2(1.f, 1.f);
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
-          const float rq = rsqrtf(fmaxf(a[jj] + b[jj], kNormEps2));
-          const float rk = rsqrtf(fmaxf(a[8 + jj] + b[8 + jj], kNormEps2));
-          qv[jj].x *= rq;
-          qv[jj].y *= rq;
-          kv[jj].x *= rk;
-          kv[jj].y *= rk;
+          P.x *= e[jj].x;
+          P.y *= e[jj].y;
         }
-      }
-      // E before this half (1 for the first half), F after it (1 for the second)
-      float2 E = th ? Po : make_float2(1.f, 1.f);
-      float2 F = th ? make_float2(1.f, 1.f) : Po;
-      const float2 gamma = make_float2(P.x * Po.x, P.y * Po.y);
-      const float2 rg = make_float2(__frcp_rn(gamma.x), __frcp_rn(gamma.y));
+        mbar_wait(&sh.prod_free[ps], pph ^ 1u);
+        sh.gprod[j & 1][th][cp] = P;
+        if (gt < C) st.beta[gt] = bv;
+        named_bar(BAR_GATE, NGATE * 32);
+        const float2 Po = sh.gprod[j & 1][th ^ 1][cp];
+        if constexpr (fused) {  // full norms of this half's tokens: this warp's 64 channels + the partner warp's
+          const int wi = gate_warp_index(warp);
+          const float* a = sh.gnorm[j & 1][wi];
+          const float* b = sh.gnorm[j & 1][wi ^ 1];
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
-        const int i = 8 * th + jj;
-        E.x *= e[jj].x;
-        E.y *= e[jj].y;
-        *reinterpret_cast<uint32_t*>(&st.ops.kd[i][c0]) = pack_bf16(-kv[jj].x * E.x, -kv[jj].y * E.y);
-        *reinterpret_cast<uint32_t*>(&st.ops.qd[i][c0]) = pack_bf16(qv[jj].x * E.x, qv[jj].y * E.y);
-      }
+          for (int jj = 0; jj < 8; ++jj) {
+            const float rq = rsqrtf(fmaxf(a[jj] + b[jj], kNormEps2));
+            const float rk = rsqrtf(fmaxf(a[8 + jj] + b[8 + jj], kNormEps2));
+            qv[jj].x *= rq;
+            qv[jj].y *= rq;
+            kv[jj].x *= rk;
+            kv[jj].y *= rk;
+          }
+        }
+        // E before this half (1 for the first half), F after it (1 for the second)
+        float2 E = th ? Po : make_float2(1.f, 1.f);
+        float2 F = th ? make_float2(1.f, 1.f) : Po;
+        const float2 gamma = make_float2(P.x * Po.x, P.y * Po.y);
+        const float2 rg = make_float2(__frcp_rn(gamma.x), __frcp_rn(gamma.y));
 #pragma unroll
-      for (int jj = 7; jj >= 0; --jj) {
-        const int i = 8 * th + jj;
-        const float kfx = kv[jj].x * F.x, kfy = kv[jj].y * F.y;
-        *reinterpret_cast<uint32_t*>(&st.ops.ke[i][c0]) = pack_bf16(kfx, kfy);
-        *reinterpret_cast<uint32_t*>(&st.kr[i][c0]) = pack_bf16(kfx * rg.x, kfy * rg.y);
-        F.x *= e[jj].x;
-        F.y *= e[jj].y;
+        for (int jj = 0; jj < 8; ++jj) {
+          const int i = 8 * th + jj;
+          E.x *= e[jj].x;
+          E.y *= e[jj].y;
+          *reinterpret_cast<uint32_t*>(&st.ops.kd[i][c0]) = pack_bf16(-kv[jj].x * E.x, -kv[jj].y * E.y);
+          *reinterpret_cast<uint32_t*>(&st.ops.qd[i][c0]) = pack_bf16(qv[jj].x * E.x, qv[jj].y * E.y);
+        }
+#pragma unroll
+        for (int jj = 7; jj >= 0; --jj) {
+          const int i = 8 * th + jj;
+          const float kfx = kv[jj].x * F.x, kfy = kv[jj].y * F.y;
+          *reinterpret_cast<uint32_t*>(&st.ops.ke[i][c0]) = pack_bf16(kfx, kfy);
+          *reinterpret_cast<uint32_t*>(&st.kr[i][c0]) = pack_bf16(kfx * rg.x, kfy * rg.y);
+          F.x *= e[jj].x;
+          F.y *= e[jj].y;
+        }
+        if (th == 0) *reinterpret_cast<float2*>(&st.ops.gam[0][0] + gamma_index(c0)) = gamma;
+        fence_proxy_async_shared();
+        mbar_arrive_warp(&sh.gate_done[ps]);
       }
-      if (th == 0) *reinterpret_cast<float2*>(&st.ops.gam[0][0] + gamma_index(c0)) = gamma;
-      fence_proxy_async_shared();
-      mbar_arrive_warp(&sh.gate_done[ps]);
-    }
-    gbase += nch;
+      gbase += nch;
     }  // items
   } else if (warp == WARP_MMA) {
     // ============================================================= mma warp
     int64_t gbase = 0, jg = 0;
     for (int it = first; it < nitems; it += stride) {
-    int seq, h;
-    int64_t t0, t1;
-    const int nch = item_at(it, seq, h, t0, t1);
-    for (int n = owned_first(gbase); n < nch; n += NSLICE, ++jg) {
-      const int ps = static_cast<int>(jg % PSTAGE);
-      const uint32_t pph = static_cast<uint32_t>(jg / PSTAGE) & 1u;
-      ProdStage& st = sh.prod[ps];
-      mbar_wait(&sh.gate_done[ps], pph);
-      float accA[2][4] = {}, accQ[2][4] = {};
+      int seq, h;
+      int64_t t0, t1;
+      const int nch = item_at(it, seq, h, t0, t1);
+      for (int n = owned_first(gbase); n < nch; n += NSLICE, ++jg) {
+        const int ps = static_cast<int>(jg % PSTAGE);
+        const uint32_t pph = static_cast<uint32_t>(jg / PSTAGE) & 1u;
+        ProdStage& st = sh.prod[ps];
+        mbar_wait(&sh.gate_done[ps], pph);
+        float accA[2][4] = {}, accQ[2][4] = {};
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        uint32_t ak[4], aq[4], b[4];
-        ldsm_x4(ak, &st.ops.kd[lane & 15][16 * kk + (lane >> 4) * 8]);
-        ldsm_x4(aq, &st.ops.qd[lane & 15][16 * kk + (lane >> 4) * 8]);
-        ldsm_x4(b, &st.kr[(lane & 7) + ((lane >> 4) << 3)][16 * kk + ((lane >> 3) & 1) * 8]);
-        mma(accA[0], ak, b[0], b[1]);
-        mma(accA[1], ak, b[2], b[3]);
-        mma(accQ[0], aq, b[0], b[1]);
-        mma(accQ[1], aq, b[2], b[3]);
-      }
-      // accA = -A (Kd carries the sign): L = diag(beta) A = -beta_i accA
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-          const int i = gq + 8 * (e2 >> 1);
-          const int jc = 8 * nt + 2 * tq + (e2 & 1);
-          st.L[i][jc] = (jc < i) ? -st.beta[i] * accA[nt][e2] : 0.f;
-          st.ops.aqk[i][jc] = __float2bfloat16_rn((jc <= i) ? accQ[nt][e2] : 0.f);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          uint32_t ak[4], aq[4], b[4];
+          ldsm_x4(ak, &st.ops.kd[lane & 15][16 * kk + (lane >> 4) * 8]);
+          ldsm_x4(aq, &st.ops.qd[lane & 15][16 * kk + (lane >> 4) * 8]);
+          ldsm_x4(b, &st.kr[(lane & 7) + ((lane >> 4) << 3)][16 * kk + ((lane >> 3) & 1) * 8]);
+          mma(accA[0], ak, b[0], b[1]);
+          mma(accA[1], ak, b[2], b[3]);
+          mma(accQ[0], aq, b[0], b[1]);
+          mma(accQ[1], aq, b[2], b[3]);
         }
-      __syncwarp();
-      // (I + L)^{-1} on the same warp: lanes 0-15, one column each
-      if (lane < C) {
-        // column `col` of T = (I + L)^{-1}: x_i = [i == col] - sum_{m<i} L[i][m] x_m,
-        // reading each row of L with 16-byte loads that all lanes share
-        const int col = lane;
-        float xs[C];
+        // accA = -A (Kd carries the sign): L = diag(beta) A = -beta_i accA
 #pragma unroll
-        for (int i = 0; i < C; ++i) {
-          float acc0 = (i == col) ? 1.f : 0.f, acc1 = 0.f;
+        for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-          for (int m4 = 0; m4 < (i + 3) / 4; ++m4) {
-            const float4 l4 = *reinterpret_cast<const float4*>(&st.L[i][4 * m4]);
-            if (4 * m4 + 0 < i) acc0 = fmaf(-l4.x, xs[4 * m4 + 0], acc0);
-            if (4 * m4 + 1 < i) acc1 = fmaf(-l4.y, xs[4 * m4 + 1], acc1);
-            if (4 * m4 + 2 < i) acc0 = fmaf(-l4.z, xs[4 * m4 + 2], acc0);
-            if (4 * m4 + 3 < i) acc1 = fmaf(-l4.w, xs[4 * m4 + 3], acc1);
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const int i = gq + 8 * (e2 >> 1);
+            const int jc = 8 * nt + 2 * tq + (e2 & 1);
+            st.L[i][jc] = (jc < i) ? -st.beta[i] * accA[nt][e2] : 0.f;
+            st.ops.aqk[i][jc] = __float2bfloat16_rn((jc <= i) ? accQ[nt][e2] : 0.f);
           }
-          xs[i] = acc0 + acc1;
-        }
-        const float bc = st.beta[col];
+        __syncwarp();
+        // (I + L)^{-1} on the same warp: lanes 0-15, one column each
+        if (lane < C) {
+          // column `col` of T = (I + L)^{-1}: x_i = [i == col] - sum_{m<i} L[i][m] x_m,
+          // reading each row of L with 16-byte loads that all lanes share
+          const int col = lane;
+          float xs[C];
 #pragma unroll
-        for (int i = 0; i < C; ++i) st.ops.tb[i][col] = __float2bfloat16_rn(xs[i] * bc);
+          for (int i = 0; i < C; ++i) {
+            float acc0 = (i == col) ? 1.f : 0.f, acc1 = 0.f;
+#pragma unroll
+            for (int m4 = 0; m4 < (i + 3) / 4; ++m4) {
+              const float4 l4 = *reinterpret_cast<const float4*>(&st.L[i][4 * m4]);
+              if (4 * m4 + 0 < i) acc0 = fmaf(-l4.x, xs[4 * m4 + 0], acc0);
+              if (4 * m4 + 1 < i) acc1 = fmaf(-l4.y, xs[4 * m4 + 1], acc1);
+              if (4 * m4 + 2 < i) acc0 = fmaf(-l4.z, xs[4 * m4 + 2], acc0);
+              if (4 * m4 + 3 < i) acc1 = fmaf(-l4.w, xs[4 * m4 + 3], acc1);
+            }
+            xs[i] = acc0 + acc1;
+          }
+          const float bc = st.beta[col];
+#pragma unroll
+          for (int i = 0; i < C; ++i) st.ops.tb[i][col] = __float2bfloat16_rn(xs[i] * bc);
+        }
+        fence_proxy_async_shared();
+        mbar_arrive_warp(&sh.solved[ps]);
       }
-      fence_proxy_async_shared();
-      mbar_arrive_warp(&sh.solved[ps]);
-    }
-    gbase += nch;
+      gbase += nch;
     }  // items
   } else if (warp == WARP_STORE) {
     // ============================================================ store warp
@@ -719,29 +719,29 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
     // lane 0: TMA boxes of q, k, g; lanes 1-16: beta (zero past the sequence end)
     int64_t gbase = 0, jg = 0;
     for (int it = first; it < nitems; it += stride) {
-    int seq, h;
-    int64_t t0, t1;
-    const int nch = item_at(it, seq, h, t0, t1);
-    for (int n = owned_first(gbase); n < nch; n += NSLICE, ++jg) {
-      const int rs = static_cast<int>(jg % PRSTAGE);
-      const uint32_t rph = static_cast<uint32_t>(jg / PRSTAGE) & 1u;
-      const int64_t cs = t0 + static_cast<int64_t>(n) * C;
-      const int tok = static_cast<int>(cs);
-      RawStage& rw = sh.raw[rs];
-      mbar_wait(&sh.raw_empty[rs], rph ^ 1u);
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&sh.raw_full[rs], kRawBytes);
-        tma_load_3d(&rw.q[0][0], &tm.q, 0, h, tok, &sh.raw_full[rs]);
-        tma_load_3d(&rw.k[0][0], &tm.k, 0, h, tok, &sh.raw_full[rs]);
-        tma_load_3d(&rw.g[0][0], &tm.g, 0, h, tok, &sh.raw_full[rs]);
-      } else if (lane <= C) {
-        const int r = lane - 1;
-        const bool ok = cs + r < t1;
-        cp_async4(&rw.beta[r], p.beta + (ok ? (cs + r) * p.beta_st + h * p.beta_sh : 0), ok ? 4u : 0u);
-        cp_async_arrive(&sh.raw_full[rs]);
+      int seq, h;
+      int64_t t0, t1;
+      const int nch = item_at(it, seq, h, t0, t1);
+      for (int n = owned_first(gbase); n < nch; n += NSLICE, ++jg) {
+        const int rs = static_cast<int>(jg % PRSTAGE);
+        const uint32_t rph = static_cast<uint32_t>(jg / PRSTAGE) & 1u;
+        const int64_t cs = t0 + static_cast<int64_t>(n) * C;
+        const int tok = static_cast<int>(cs);
+        RawStage& rw = sh.raw[rs];
+        mbar_wait(&sh.raw_empty[rs], rph ^ 1u);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&sh.raw_full[rs], kRawBytes);
+          tma_load_3d(&rw.q[0][0], &tm.q, 0, h, tok, &sh.raw_full[rs]);
+          tma_load_3d(&rw.k[0][0], &tm.k, 0, h, tok, &sh.raw_full[rs]);
+          tma_load_3d(&rw.g[0][0], &tm.g, 0, h, tok, &sh.raw_full[rs]);
+        } else if (lane <= C) {
+          const int r = lane - 1;
+          const bool ok = cs + r < t1;
+          cp_async4(&rw.beta[r], p.beta + (ok ? (cs + r) * p.beta_st + h * p.beta_sh : 0), ok ? 4u : 0u);
+          cp_async_arrive(&sh.raw_full[rs]);
+        }
       }
-    }
-    gbase += nch;
+      gbase += nch;
     }  // items
   } else if (warp == notify_warp<NS>()) {
     // ==================================================== stage notifications
@@ -752,18 +752,18 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
     // barrier orders them before the chain warps' reads.
     int64_t gc = 0;
     for (int it = first; it < nitems; it += stride) {
-    int seq, h;
-    int64_t t0, t1;
-    const int nch = item_at(it, seq, h, t0, t1);
-    for (int n = 0; n < nch; ++n, ++gc) {
-      const int s = static_cast<int>(gc % CSTAGE);
-      mbar_wait(&sh.c_full[s], static_cast<uint32_t>(gc / CSTAGE) & 1u);
-      __syncwarp();
-      named_bar_arrive(BAR_FULL0 + s, 32 * (NCHAIN + 1));
-      // the ring slot has been copied here: give it back to its producer
-      if (lane == 0)
-        mbar_arrive_remote_relaxed(&sh.slot_free[gc % RING], static_cast<uint32_t>(gc % NSLICE));
-    }
+      int seq, h;
+      int64_t t0, t1;
+      const int nch = item_at(it, seq, h, t0, t1);
+      for (int n = 0; n < nch; ++n, ++gc) {
+        const int s = static_cast<int>(gc % CSTAGE);
+        mbar_wait(&sh.c_full[s], static_cast<uint32_t>(gc / CSTAGE) & 1u);
+        __syncwarp();
+        named_bar_arrive(BAR_FULL0 + s, 32 * (NCHAIN + 1));
+        // the ring slot has been copied here: give it back to its producer
+        if (lane == 0)
+          mbar_arrive_remote_relaxed(&sh.slot_free[gc % RING], static_cast<uint32_t>(gc % NSLICE));
+      }
     }  // items
   } else if (warp == 9) {
     if (lane == 0 && p.cu && rank == 0) {
@@ -777,22 +777,22 @@ __global__ void __cluster_dims__(D / NS, 1, 1) __launch_bounds__(NTHREADS, 1)
     if (lane == 0) {
       int64_t gc = 0;
       for (int it = first; it < nitems; it += stride) {
-      int seq, h;
-      int64_t t0, t1;
-      const int nch = item_at(it, seq, h, t0, t1);
-      for (int n = 0; n < nch; ++n, ++gc) {
-        const int s = static_cast<int>(gc % CSTAGE);
-        const uint32_t ph = static_cast<uint32_t>(gc / CSTAGE) & 1u;
-        const int slot = static_cast<int>(gc % RING);
-        const int tok = static_cast<int>(t0 + static_cast<int64_t>(n) * C);
-        ChainStage<NS>& st = sh.cst[s];
-        mbar_wait(&sh.c_empty[s], ph ^ 1u);
-        mbar_wait_cl(&sh.ready[slot], static_cast<uint32_t>(gc / RING) & 1u);
-        fence_proxy_async_global();
-        mbar_arrive_expect_tx(&sh.c_full[s], (MODE & kModeZeroV) ? kSlotBytes : chain_bytes<NS>());
-        bulk_g2s(&st.ops, ring + static_cast<size_t>(slot) * kSlotBytes, kSlotBytes, &sh.c_full[s]);
-        if constexpr ((MODE & kModeZeroV) == 0u) tma_load_3d(&st.v[0][0], &tm.v, dv0, h, tok, &sh.c_full[s]);
-      }
+        int seq, h;
+        int64_t t0, t1;
+        const int nch = item_at(it, seq, h, t0, t1);
+        for (int n = 0; n < nch; ++n, ++gc) {
+          const int s = static_cast<int>(gc % CSTAGE);
+          const uint32_t ph = static_cast<uint32_t>(gc / CSTAGE) & 1u;
+          const int slot = static_cast<int>(gc % RING);
+          const int tok = static_cast<int>(t0 + static_cast<int64_t>(n) * C);
+          ChainStage<NS>& st = sh.cst[s];
+          mbar_wait(&sh.c_empty[s], ph ^ 1u);
+          mbar_wait_cl(&sh.ready[slot], static_cast<uint32_t>(gc / RING) & 1u);
+          fence_proxy_async_global();
+          mbar_arrive_expect_tx(&sh.c_full[s], (MODE & kModeZeroV) ? kSlotBytes : chain_bytes<NS>());
+          bulk_g2s(&st.ops, ring + static_cast<size_t>(slot) * kSlotBytes, kSlotBytes, &sh.c_full[s]);
+          if constexpr ((MODE & kModeZeroV) == 0u) tma_load_3d(&st.v[0][0], &tm.v, dv0, h, tok, &sh.c_full[s]);
+        }
       }  // items
     }
   }
