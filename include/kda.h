@@ -257,7 +257,7 @@ kda_status_t kda_set_schedule(int32_t mode, int32_t clusters);
  * helper streams (created once per device; the call stays ordered on
  * `stream`). Results agree with the unsplit path within the library's
  * accuracy bounds, not bitwise.
- *   mode 0 (default): split when num_seqs = 1, T >= 8192 and the device holds
+ *   mode 0 (default): split when num_seqs = 1, T >= 4096 and the device holds
  *                     all 3 * H clusters of the three launches at once;
  *   mode 1: never;   mode 2: whenever num_seqs = 1 and T >= 32 (testing).
  * kda_fwd_noalloc never splits. Process-wide. Returns KDA_ERR_SHAPE for any

@@ -403,3 +403,25 @@ def test_time_split_agrees_with_unsplit(kda):
     mo, ms = H.metrics(o2, o1), H.metrics(f2, f1)
     assert mo["max_abs"] <= H.O_MAX_ABS and mo["rel_rms"] <= 2 * H.O_REL_RMS, mo
     assert ms["rel_rms"] <= 2 * H.S_REL_RMS, ms
+
+
+def test_time_split_automatic_from_4096_tokens(kda, oracle_mod):
+    """One sequence of 4096 tokens with few heads takes the split by default:
+    the automatic result equals the forced split bitwise, differs from the
+    unsplit run, and meets the oracle."""
+    import torch
+
+    inp = kda_inputs.make_inputs([4096], 2, seed=34, random_initial_state=True)
+    kda.set_path(16)
+    try:
+        res = {}
+        for mode in (0, 1, 2):
+            kda.set_time_split(mode)
+            res[mode] = H.run_gpu(inp)
+    finally:
+        kda.set_time_split(0)
+        kda.set_path(0)
+    assert torch.equal(res[0][0], res[2][0]) and torch.equal(res[0][1], res[2][1])
+    assert not torch.equal(res[0][0], res[1][0])
+    o_ref, f_ref = oracle_mod.scan_inputs(inp)
+    H.assert_parity(res[0][0], res[0][1], o_ref, f_ref, label="automatic split T=4096")
