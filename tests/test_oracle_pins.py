@@ -31,6 +31,11 @@ P10 gate preprocessing (preprocess): unit norms per (token, head) over the
     wrong branch of the stable form; the lower bound clamps exactly where
     log sigmoid falls below it; agreement with the generator's gates and
     betas computed from the same draws.
+P12 the time split's combination: the second part of a sequence run from a
+    start state S_a equals the same part run from zero plus S_a applied to the
+    part's transition map, o_t = o_loc(t) + S_a^T o_M(t) and S_T = M S_a + B,
+    where o_M and M come from the part run with v = 0 from the identity ->
+    which side S_a multiplies, the transpose in o, the scale inside o_M.
 P11 backward: the reverse-mode gradients of q, k, v, g, beta and the initial
     state equal central finite differences of the (pinned) forward scan, per
     coordinate and along random directions -> every term of the hand-derived
@@ -264,6 +269,30 @@ def test_p8_resume_from_final_state(oracle_mod):
         ob, fb = oracle_mod.scan(q[T1:], k[T1:], v[T1:], g[T1:], beta[T1:], np.array([0, 30 - T1], np.int32), 0.5, fa)
         assert np.array_equal(np.concatenate([oa, ob]), out)
         assert np.array_equal(fb, fin)
+
+
+# ----------------------------------------------------------------------------- P12
+@pytest.mark.parametrize("T1", [1, 9, 20])
+def test_p12_time_split_combination(oracle_mod, T1):
+    d, T, H, scale = 8, 29, 2, 0.7
+    q, k, v, g, beta, cu, S0 = _rand_f64([T], H, d, d, seed=40 + T1, init=True)
+    out, fin = oracle_mod.scan(q, k, v, g, beta, cu, scale, S0)
+    part = lambda x: np.ascontiguousarray(x[T1:])
+    cu2 = np.array([0, T - T1], np.int32)
+    # first part from the initial state
+    oa, Sa = oracle_mod.scan(q[:T1], k[:T1], v[:T1], g[:T1], beta[:T1], np.array([0, T1], np.int32), scale, S0)
+    # second part from zero, and with v = 0 from the identity (its transition map)
+    oloc, B = oracle_mod.scan(part(q), part(k), part(v), part(g), part(beta), cu2, scale, None)
+    eye = np.broadcast_to(np.eye(d), (1, H, d, d)).copy()
+    oM, M = oracle_mod.scan(part(q), part(k), np.zeros_like(part(v)), part(g), part(beta), cu2, scale, eye)
+    # combine: per head h, o_t = o_loc(t) + S_a[h]^T o_M(t); S_T = M[h] S_a[h] + B[h]
+    o2 = oloc + np.einsum("hkv,thk->thv", Sa[0], oM)
+    f2 = np.einsum("hij,hjv->hiv", M[0], Sa[0]) + B[0]
+    np.testing.assert_allclose(np.concatenate([oa, o2]), out, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(f2, fin[0], rtol=1e-10, atol=1e-12)
+    # the transposed combination is wrong (the pin distinguishes the two)
+    wrong = oloc + np.einsum("hvk,thk->thv", Sa[0], oM)
+    assert np.max(np.abs(wrong - out[T1:])) > 1e-3
 
 
 # ----------------------------------------------------------------------------- P9
