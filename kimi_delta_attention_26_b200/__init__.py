@@ -15,7 +15,7 @@ from typing import Optional, Tuple
 import torch
 
 __all__ = ["kda_fwd", "kda_fwd_fused", "kda_decode", "kda_bwd", "library_path", "wait_timeouts", "device_status", "set_slice_columns", "set_path",
-           "set_time_split", "describe", "KDAError", "HEAD_DIM"]
+           "set_time_split", "set_schedule", "describe", "KDAError", "HEAD_DIM"]
 
 HEAD_DIM = 128
 _PKG = os.path.dirname(os.path.abspath(__file__))
