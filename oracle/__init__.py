@@ -209,3 +209,109 @@ def backward(q, k, v, g, beta, cu_seqlens, scale, dout, initial_state=None, dfin
     if rc != 0:
         raise ValueError(f"oracle backward rejected its arguments (code {rc})")
     return res
+
+
+def chunked_backward(q, k, v, g, beta, cu_seqlens, scale, dout, initial_state=None, dfinal=None, *, chunk=16):
+    """The gradients ``backward`` computes, by the chunked (WY) form instead of
+    the token recurrence: the derivative of the chunked rewrite step by step.
+
+    Per chunk of C tokens, with Gamma the inclusive cumulative sum of g inside
+    the chunk, E = exp(Gamma), F = exp(Gamma_last - Gamma), gamma = E_last and
+    S the chunk-start state, the forward products are
+        A    = strictly lower part of (k E)(k / E)^T,  L = diag(beta) A,
+        M    = (I + L)^{-1},  W = M diag(beta),
+        X    = V - (k E) S,   Vnew = W X,
+        Aqk  = lower part (with the diagonal) of (q E)(k / E)^T,
+        O    = scale ((q E) S + Aqk Vnew),
+        S'   = diag(gamma) S + (k F)^T Vnew.
+    The backward walks the chunks in reverse with the adjoint state dS (the
+    gradient at S'): dVnew = (k F) dS + scale Aqk^T dO, dX = W^T dVnew, and
+    dS <- diag(gamma) dS + scale (q E)^T dO - (k E)^T dX. Inside a chunk the
+    gradients go through M (d(I + L)^{-1} = -M dL M), L = diag(beta) A and the
+    two masked products, then through the decay factors into Gamma, and a
+    reverse cumulative sum within the chunk turns dGamma into dg.
+
+    Float64 numpy (all inputs float64); returns the same dict as ``backward``.
+    Test infrastructure: the plan of a chunked backward, checked against the
+    token-level reverse recurrence.
+    """
+    q, k, v, g = (np.asarray(x, np.float64) for x in (q, k, v, g))
+    beta, dout = np.asarray(beta, np.float64), np.asarray(dout, np.float64)
+    cu = np.asarray(cu_seqlens, np.int64)
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    nseq = cu.shape[0] - 1
+    res = {"dq": np.zeros((T, H, dk)), "dk": np.zeros((T, H, dk)), "dv": np.zeros((T, H, dv)),
+           "dg": np.zeros((T, H, dk)), "dbeta": np.zeros((T, H)),
+           "dinit": np.zeros((nseq, H, dk, dv)) if initial_state is not None else None}
+    for s in range(nseq):
+        t0, t1 = int(cu[s]), int(cu[s + 1])
+        starts = list(range(t0, t1, chunk))
+        for h in range(H):
+            S = np.zeros((dk, dv)) if initial_state is None else np.array(initial_state[s, h], np.float64)
+
+            def parts(a, S):
+                b = min(a + chunk, t1)
+                kk, qq, vv, bb = k[a:b, h], q[a:b, h], v[a:b, h], beta[a:b, h]
+                Gam = np.cumsum(g[a:b, h], axis=0)
+                E = np.exp(Gam)
+                F = np.exp(Gam[-1] - Gam)
+                gam = E[-1]
+                Kd, Qd, KR, Ke = kk * E, qq * E, kk / E, kk * F
+                n = b - a
+                strict = np.tril(np.ones((n, n)), -1)
+                lower = np.tril(np.ones((n, n)))
+                A = (Kd @ KR.T) * strict
+                L = bb[:, None] * A
+                M = np.linalg.solve(np.eye(n) + L, np.eye(n))
+                W = M * bb[None, :]
+                X = vv - Kd @ S
+                Vn = W @ X
+                Aqk = (Qd @ KR.T) * lower
+                return dict(a=a, b=b, k=kk, q=qq, beta=bb, E=E, F=F, gam=gam, Kd=Kd, Qd=Qd, KR=KR, Ke=Ke,
+                            strict=strict, lower=lower, A=A, M=M, W=W, X=X, Vn=Vn, Aqk=Aqk)
+
+            # forward: the chunk-start states
+            states = []
+            for a in starts:
+                states.append(S)
+                c = parts(a, S)
+                S = c["gam"][:, None] * S + c["Ke"].T @ c["Vn"]
+            # backward over the chunks in reverse
+            dS = np.zeros((dk, dv)) if dfinal is None else np.array(dfinal[s, h], np.float64)
+            for a, S in zip(reversed(starts), reversed(states)):
+                c = parts(a, S)
+                a_, b_ = c["a"], c["b"]
+                dO = dout[a_:b_, h]
+                dVn = c["Ke"] @ dS + scale * c["Aqk"].T @ dO
+                dX = c["W"].T @ dVn
+                dW = dVn @ c["X"].T
+                dKd = -dX @ S.T
+                dQd = scale * dO @ S.T
+                dAqk = scale * (dO @ c["Vn"].T) * c["lower"]
+                dKe = c["Vn"] @ dS.T
+                dgam = np.sum(S * dS, axis=1)
+                dS_prev = c["gam"][:, None] * dS + scale * c["Qd"].T @ dO - c["Kd"].T @ dX
+                # W = M diag(beta); M = (I + L)^{-1}; L = diag(beta) A
+                dM = dW * c["beta"][None, :]
+                dbeta = np.sum(c["M"] * dW, axis=0)
+                dL = -(c["M"].T @ dM @ c["M"].T) * c["strict"]
+                dA = c["beta"][:, None] * dL
+                dbeta += np.sum(c["A"] * dL, axis=1)
+                # A = strict((k E)(k / E)^T), Aqk = lower((q E)(k / E)^T)
+                dKd += dA @ c["KR"]
+                dKR = dA.T @ c["Kd"] + dAqk.T @ c["Qd"]
+                dQd += dAqk @ c["KR"]
+                # back to k, q and Gamma (E = exp Gamma, KR = k exp(-Gamma), F = exp(Gamma_last - Gamma))
+                E, F = c["E"], c["F"]
+                res["dk"][a_:b_, h] = dKd * E + dKR / E + dKe * F
+                res["dq"][a_:b_, h] = dQd * E
+                dGam = (dKd * c["k"] + dQd * c["q"]) * E - dKR * c["KR"] - dKe * c["Ke"]
+                dGam[-1] += np.sum(dKe * c["Ke"], axis=0) + dgam * c["gam"]
+                res["dg"][a_:b_, h] = np.cumsum(dGam[::-1], axis=0)[::-1]
+                res["dv"][a_:b_, h] = dX
+                res["dbeta"][a_:b_, h] = dbeta
+                dS = dS_prev
+            if res["dinit"] is not None:
+                res["dinit"][s, h] = dS
+    return res

@@ -36,6 +36,10 @@ P12 the time split's combination: the second part of a sequence run from a
     part's transition map, o_t = o_loc(t) + S_a^T o_M(t) and S_T = M S_a + B,
     where o_M and M come from the part run with v = 0 from the identity ->
     which side S_a multiplies, the transpose in o, the scale inside o_M.
+P13 the chunked (WY-form) backward equals the token-level reverse recurrence at
+    chunk sizes 1..32 -> every term of the chunked derivative (the adjoint
+    state step, the inverse's derivative, the masks, the decay chain rule
+    and the in-chunk reverse cumulative sum).
 P11 backward: the reverse-mode gradients of q, k, v, g, beta and the initial
     state equal central finite differences of the (pinned) forward scan, per
     coordinate and along random directions -> every term of the hand-derived
@@ -293,6 +297,21 @@ def test_p12_time_split_combination(oracle_mod, T1):
     # the transposed combination is wrong (the pin distinguishes the two)
     wrong = oloc + np.einsum("hvk,thk->thv", Sa[0], oM)
     assert np.max(np.abs(wrong - out[T1:])) > 1e-3
+
+
+# ----------------------------------------------------------------------------- P13
+@pytest.mark.parametrize("chunk", [1, 5, 16, 32])
+@pytest.mark.parametrize("with_state", [False, True])
+def test_p13_chunked_backward_equals_token_backward(oracle_mod, chunk, with_state):
+    lens = [37, 0, 16, 5]
+    q, k, v, g, beta, cu, S0 = _rand_f64(lens, 2, 6, 5, seed=50 + chunk, init=with_state)
+    rng = np.random.default_rng(51)
+    dout = rng.standard_normal(v.shape)
+    dfin = rng.standard_normal((len(lens), 2, 6, 5)) if with_state else None
+    ref = oracle_mod.backward(q, k, v, g, beta, cu, 0.5, dout, S0, dfin)
+    got = oracle_mod.chunked_backward(q, k, v, g, beta, cu, 0.5, dout, S0, dfin, chunk=chunk)
+    for name in ("dq", "dk", "dv", "dg", "dbeta") + (("dinit",) if with_state else ()):
+        assert _rel(got[name], ref[name]) < 1e-10, name
 
 
 # ----------------------------------------------------------------------------- P9
